@@ -1,0 +1,325 @@
+/*
+ * oracle.c -- plain, slow CPU reference for one decode step of
+ * retention-scored, globally budgeted KV-cache eviction followed by
+ * attention over the kept entries.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline / reference leg load this library.  The product (the CUDA
+ * library librkv.so and its Python binding) never calls it, and the two share
+ * no source file, header, table or helper.
+ *
+ * What it follows (web summaries of three papers):
+ *   [DBTrimKV]  "Make Each Token Count: Towards Improving Long-Context
+ *               Performance with KV Cache Eviction"
+ *               - Methodology 2, geometric retention as future utility:
+ *                 the retention weight of token i at step t is beta_i^(t-i).
+ *               - Methodology 3, weight-tied global gate: one global budget
+ *                 M_global; all cached entries of all layers and heads are
+ *                 ranked together and the top M_global are kept.
+ *               - Methodology 4, implementation: paged layout with a
+ *                 variable-length KV sequence per head.
+ *   [TRIM-KV]   "Cache What Lasts: Token Retention for Memory-Bounded KV
+ *               Cache in LLMs", technical summary, core mechanisms 1, 2, 4:
+ *               beta in [0,1] per token, layer and head; decay beta^(t-i);
+ *               when over budget, evict the lowest beta^(t-i).
+ *   [ContourKV] "Trust the Mass: Forced Weights in KV-Cache Eviction"
+ *               - Problem definition: after selection the attention weights
+ *                 are renormalised over the kept set (forced weights).
+ *               - Methodology 2: the budget is enforced physically (ragged
+ *                 storage), not as a mask over the full cache.
+ *               - Methodology 3 / main contributions: dropped mass, the
+ *                 summed dense attention weight of the discarded keys.
+ *
+ * Readings where the pages are silent (each one is listed in the design doc):
+ *   - score s = fl32(float(t - i) * log(beta_i)), one IEEE binary32 multiply
+ *     (log beta^(t-i) = (t-i) log beta); -0 is the same score as +0;
+ *   - ties broken by ascending (layer, kv head, position);
+ *   - entries present at step t are those with position < t;
+ *   - logits use scale = 1/sqrt(D) (passed in); K/V bf16 values are widened
+ *     exactly; attention is accumulated in binary64;
+ *   - the paged layout, hole-fill compaction and free-page stack below are
+ *     this build's own specification.
+ *
+ * Build: gcc -O2 -std=c99 -ffp-contract=off -fexcess-precision=standard
+ *        -fno-fast-math -shared -fPIC (no FMA contraction: the score must be
+ *        exactly one rounded multiply).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_INPUT (-1) /* NaN log-retention, age outside [1, 2^24), bad layout */
+#define ORC_ERR_POOL (-2)  /* free-page stack empty on append */
+#define ORC_ERR_TABLE (-3) /* append past the end of a block table */
+
+/* The cache, in the layout both sides agree on.  C = B*L*H heads; head
+ * c = (b*L + l)*H + h.  Logical slot k of head c lives in physical page
+ * block_table[c*max_pages + k/P] at offset k%P. */
+typedef struct {
+    int32_t B, L, H, G, D, P;
+    int32_t n_pages, max_pages;
+    int32_t kv_f32;      /* 1: K/V stored as float; 0: bfloat16 bit patterns */
+    void *k_pool;        /* [n_pages][P][D] */
+    void *v_pool;        /* [n_pages][P][D] */
+    int32_t *pos_pool;   /* [n_pages][P] token position i */
+    float *lb_pool;      /* [n_pages][P] log retention log(beta_i) */
+    int32_t *block_table;/* [C][max_pages], -1 where no page */
+    int32_t *len;        /* [C] entries per head */
+    int32_t *free_stack; /* [n_pages] free page ids, top at free_stack[*free_top-1] */
+    int32_t *free_top;   /* scalar */
+} orc_cache;
+
+static int64_t n_heads(const orc_cache *cc) { return (int64_t)cc->B * cc->L * cc->H; }
+
+static int64_t phys_row(const orc_cache *cc, int64_t c, int32_t k) {
+    int32_t page = cc->block_table[c * cc->max_pages + k / cc->P];
+    return (int64_t)page * cc->P + k % cc->P;
+}
+
+/* Widen one stored K or V element to binary64 (bf16 -> f32 is a 16-bit shift). */
+static double kv_elem(const orc_cache *cc, const void *pool, int64_t row, int32_t d) {
+    if (cc->kv_f32) return (double)((const float *)pool)[row * cc->D + d];
+    uint32_t bits = (uint32_t)((const uint16_t *)pool)[row * cc->D + d] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* ---------------------------------------------------------------- score ---
+ * [DBTrimKV] Methodology 2 / [TRIM-KV] core mechanism 2: r_{t,i} = beta_i^(t-i).
+ * In log space log r = (t-i) * log beta_i; one binary32 multiply, round to
+ * nearest even.  The age t-i is an exact integer in [1, 2^24), so its
+ * conversion to float is exact.  -0 is returned as +0. */
+float orc_score(int32_t t, int32_t pos, float lb) {
+    float age = (float)(t - pos);
+    float s = age * lb;
+    if (s == 0.0f) s = 0.0f;
+    return s;
+}
+
+/* Validity of one entry's inputs: NaN log-retention or an age outside
+ * [1, 2^24) is refused. */
+int orc_entry_ok(int32_t t, int32_t pos, float lb) {
+    int64_t age = (int64_t)t - (int64_t)pos;
+    if (isnan(lb)) return 0;
+    if (age < 1 || age >= (1 << 24)) return 0;
+    return 1;
+}
+
+/* Element-wise orc_score / orc_entry_ok over arrays (for the pins). */
+void orc_score_many(int64_t n, const int32_t *t, const int32_t *pos, const float *lb,
+                    float *s, uint8_t *ok) {
+    for (int64_t e = 0; e < n; e++) {
+        ok[e] = (uint8_t)orc_entry_ok(t[e], pos[e], lb[e]);
+        s[e] = ok[e] ? orc_score(t[e], pos[e], lb[e]) : 0.0f;
+    }
+}
+
+/* --------------------------------------------------------------- select ---
+ * [DBTrimKV] Methodology 3: rank every cached entry of all layers and heads
+ * of a sequence by its score and keep the top M_global (per sequence).
+ * [TRIM-KV] core mechanism 4: the lowest scores are the ones evicted.
+ * Order: higher score first; equal scores by ascending (l, h, i). */
+typedef struct {
+    float s;
+    int32_t l, h, i;
+    int64_t c;
+    int32_t slot;
+} orc_entry;
+
+static int cmp_rank(const void *pa, const void *pb) {
+    const orc_entry *a = (const orc_entry *)pa, *b = (const orc_entry *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    if (a->l != b->l) return a->l < b->l ? -1 : 1;
+    if (a->h != b->h) return a->h < b->h ? -1 : 1;
+    if (a->i != b->i) return a->i < b->i ? -1 : 1;
+    return 0;
+}
+
+/* keep[c*max_pages*P + k] = 1 for kept slots (0 otherwise, also past len);
+ * kept[c] = number kept in head c.  t[b], m_global[b] per sequence. */
+int orc_select(const orc_cache *cc, const int32_t *t, const int64_t *m_global,
+               uint8_t *keep, int32_t *kept) {
+    const int64_t C = n_heads(cc);
+    const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
+    memset(keep, 0, (size_t)(C * slots_per_head));
+    for (int64_t c = 0; c < C; c++) kept[c] = 0;
+    for (int32_t b = 0; b < cc->B; b++) {
+        int64_t n = 0;
+        for (int32_t l = 0; l < cc->L; l++)
+            for (int32_t h = 0; h < cc->H; h++) n += cc->len[((int64_t)b * cc->L + l) * cc->H + h];
+        orc_entry *e = (orc_entry *)malloc((size_t)(n > 0 ? n : 1) * sizeof(orc_entry));
+        if (!e) return ORC_ERR_INPUT;
+        int64_t w = 0;
+        for (int32_t l = 0; l < cc->L; l++) {
+            for (int32_t h = 0; h < cc->H; h++) {
+                int64_t c = ((int64_t)b * cc->L + l) * cc->H + h;
+                for (int32_t k = 0; k < cc->len[c]; k++) {
+                    int64_t row = phys_row(cc, c, k);
+                    int32_t pos = cc->pos_pool[row];
+                    float lb = cc->lb_pool[row];
+                    if (!orc_entry_ok(t[b], pos, lb)) { free(e); return ORC_ERR_INPUT; }
+                    e[w].s = orc_score(t[b], pos, lb);
+                    e[w].l = l; e[w].h = h; e[w].i = pos; e[w].c = c; e[w].slot = k;
+                    w++;
+                }
+            }
+        }
+        qsort(e, (size_t)n, sizeof(orc_entry), cmp_rank);
+        int64_t m = m_global[b] < 0 ? 0 : m_global[b];
+        if (m > n) m = n;
+        for (int64_t r = 0; r < m; r++) {
+            keep[e[r].c * slots_per_head + e[r].slot] = 1;
+            kept[e[r].c] += 1;
+        }
+        free(e);
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------ attention ---
+ * [ContourKV] Problem definition: once the subset is chosen, the weights are
+ * the softmax renormalised over the kept set (forced weights):
+ *   o = sum_{j kept} exp(z_j - m) v_j / sum_{j kept} exp(z_j - m),
+ *   z_j = scale * <q, k_j>.
+ * [ContourKV] Methodology 3 / main contributions: dropped mass is the weight
+ * the discarded keys held under dense attention over every entry present
+ * before this step's eviction:
+ *   dm = sum_{j evicted} exp(z_j - M) / sum_{j all} exp(z_j - M).
+ * Query head qh = h*G + g of layer l reads KV head h (grouped-query attention
+ * with consecutive query heads per group).  q, out: [C][G][D]; lse, dm: [C][G].
+ * keep == NULL means every entry is kept.  A head with nothing kept gives
+ * o = 0 and lse = -inf; a head with no entries has dm = 0. */
+int orc_attention(const orc_cache *cc, const float *q, float scale, const uint8_t *keep,
+                  float *out, float *lse_kept, float *dropped) {
+    const int64_t C = n_heads(cc);
+    const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
+    const int32_t D = cc->D, G = cc->G;
+    int32_t max_len = 0;
+    for (int64_t c = 0; c < C; c++) if (cc->len[c] > max_len) max_len = cc->len[c];
+    double *z = (double *)malloc((size_t)(max_len > 0 ? max_len : 1) * sizeof(double));
+    double *acc = (double *)malloc((size_t)D * sizeof(double));
+    if (!z || !acc) { free(z); free(acc); return ORC_ERR_INPUT; }
+    for (int64_t c = 0; c < C; c++) {
+        const int32_t n = cc->len[c];
+        for (int32_t g = 0; g < G; g++) {
+            const float *qv = q + (c * G + g) * D;
+            for (int32_t k = 0; k < n; k++) {
+                int64_t row = phys_row(cc, c, k);
+                double dot = 0.0;
+                for (int32_t d = 0; d < D; d++) dot += (double)qv[d] * kv_elem(cc, cc->k_pool, row, d);
+                z[k] = (double)scale * dot;
+            }
+            /* dense over all entries present before eviction */
+            double m_all = -INFINITY;
+            for (int32_t k = 0; k < n; k++) if (z[k] > m_all) m_all = z[k];
+            double z_all = 0.0, z_ev = 0.0;
+            for (int32_t k = 0; k < n; k++) {
+                double p = exp(z[k] - m_all);
+                z_all += p;
+                if (keep && !keep[c * slots_per_head + k]) z_ev += p;
+            }
+            if (dropped) dropped[c * G + g] = (float)(n > 0 ? z_ev / z_all : 0.0);
+            /* forced weights over the kept set */
+            double m_k = -INFINITY;
+            int32_t n_kept = 0;
+            for (int32_t k = 0; k < n; k++) {
+                if (keep && !keep[c * slots_per_head + k]) continue;
+                n_kept++;
+                if (z[k] > m_k) m_k = z[k];
+            }
+            double zk = 0.0;
+            for (int32_t d = 0; d < D; d++) acc[d] = 0.0;
+            for (int32_t k = 0; k < n; k++) {
+                if (keep && !keep[c * slots_per_head + k]) continue;
+                double p = exp(z[k] - m_k);
+                int64_t row = phys_row(cc, c, k);
+                zk += p;
+                for (int32_t d = 0; d < D; d++) acc[d] += p * kv_elem(cc, cc->v_pool, row, d);
+            }
+            float *o = out + (c * G + g) * D;
+            for (int32_t d = 0; d < D; d++) o[d] = (float)(n_kept > 0 ? acc[d] / zk : 0.0);
+            if (lse_kept) lse_kept[c * G + g] = (float)(n_kept > 0 ? m_k + log(zk) : -INFINITY);
+        }
+    }
+    free(z);
+    free(acc);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------ compaction ---
+ * [ContourKV] Methodology 2: the kept set is stored physically (ragged
+ * storage); evicted rows are really removed.  [DBTrimKV] Methodology 4: each
+ * head keeps its own length in a paged layout.  This build's layout rule:
+ * heads in ascending c; in head c with n entries and n_new kept,
+ *   holes   = slots k < n_new that are not kept, ascending;
+ *   sources = slots k >= n_new that are kept, ascending;
+ * the j-th source's (K, V, position, log-retention) row is copied to the
+ * j-th hole; the pages at table indices [ceil(n_new/P), ceil(n/P)) are pushed
+ * onto the free stack in ascending table index, their table entries become
+ * -1, and len = n_new. */
+static void copy_row(const orc_cache *cc, int64_t dst, int64_t src) {
+    size_t esz = cc->kv_f32 ? 4 : 2;
+    memcpy((char *)cc->k_pool + dst * cc->D * esz, (char *)cc->k_pool + src * cc->D * esz, cc->D * esz);
+    memcpy((char *)cc->v_pool + dst * cc->D * esz, (char *)cc->v_pool + src * cc->D * esz, cc->D * esz);
+    cc->pos_pool[dst] = cc->pos_pool[src];
+    cc->lb_pool[dst] = cc->lb_pool[src];
+}
+
+int orc_compact(orc_cache *cc, const uint8_t *keep) {
+    const int64_t C = n_heads(cc);
+    const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
+    for (int64_t c = 0; c < C; c++) {
+        const uint8_t *f = keep + c * slots_per_head;
+        const int32_t n = cc->len[c];
+        int32_t n_new = 0;
+        for (int32_t k = 0; k < n; k++) n_new += f[k] ? 1 : 0;
+        int32_t hole = 0, src = n_new;
+        for (;;) {
+            while (hole < n_new && f[hole]) hole++;
+            while (src < n && !f[src]) src++;
+            if (hole >= n_new || src >= n) break;
+            copy_row(cc, phys_row(cc, c, hole), phys_row(cc, c, src));
+            hole++;
+            src++;
+        }
+        const int32_t keep_pages = (n_new + cc->P - 1) / cc->P;
+        const int32_t old_pages = (n + cc->P - 1) / cc->P;
+        for (int32_t pi = keep_pages; pi < old_pages; pi++) {
+            int32_t *slot = &cc->block_table[c * cc->max_pages + pi];
+            cc->free_stack[(*cc->free_top)++] = *slot;
+            *slot = -1;
+        }
+        cc->len[c] = n_new;
+    }
+    return ORC_OK;
+}
+
+/* --------------------------------------------------------------- append ---
+ * Decoding writes token t's K, V, position t and log-retention into slot
+ * len of every head, heads in ascending c.  When len is a multiple of P the
+ * head first takes a page from the top of the free stack. */
+int orc_append(orc_cache *cc, const int32_t *t, const void *k_new, const void *v_new,
+               const float *lb_new) {
+    const int64_t C = n_heads(cc);
+    const size_t esz = cc->kv_f32 ? 4 : 2;
+    for (int64_t c = 0; c < C; c++) {
+        const int32_t b = (int32_t)(c / ((int64_t)cc->L * cc->H));
+        const int32_t k = cc->len[c];
+        if (k / cc->P >= cc->max_pages) return ORC_ERR_TABLE;
+        if (k % cc->P == 0) {
+            if (*cc->free_top <= 0) return ORC_ERR_POOL;
+            cc->block_table[c * cc->max_pages + k / cc->P] = cc->free_stack[--(*cc->free_top)];
+        }
+        int64_t row = phys_row(cc, c, k);
+        memcpy((char *)cc->k_pool + row * cc->D * esz, (const char *)k_new + c * cc->D * esz, cc->D * esz);
+        memcpy((char *)cc->v_pool + row * cc->D * esz, (const char *)v_new + c * cc->D * esz, cc->D * esz);
+        cc->pos_pool[row] = t[b];
+        cc->lb_pool[row] = lb_new[c];
+        cc->len[c] = k + 1;
+    }
+    return ORC_OK;
+}
