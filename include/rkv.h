@@ -1,0 +1,239 @@
+/*
+ * rkv.h -- C ABI of librkv: one decode step of retention-scored, globally
+ * budgeted KV-cache eviction with grouped-query decode attention over the
+ * surviving ragged paged cache, on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow three web summaries of papers:
+ *   [DBTrimKV]  "Make Each Token Count: Towards Improving Long-Context
+ *               Performance with KV Cache Eviction"
+ *   [TRIM-KV]   "Cache What Lasts: Token Retention for Memory-Bounded KV
+ *               Cache in LLMs"
+ *   [ContourKV] "Trust the Mass: Forced Weights in KV-Cache Eviction"
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every call returns an int status: RKV_OK (0) or a negative RKV_ERR_*.
+ *   Host-side argument errors are reported synchronously and nothing is
+ *   enqueued.  rkv_last_error() returns a per-thread message for the last
+ *   failure on the calling thread.
+ * - Work is enqueued asynchronously on the caller's CUDA stream (`stream`
+ *   is a cudaStream_t passed as void*; NULL = legacy default stream).  No
+ *   call synchronises the device, and no call allocates or frees device
+ *   memory: the caller owns every buffer, including the workspace.
+ * - All pointers in rkv_cache_t / rkv_select_t and all array arguments are
+ *   DEVICE pointers unless a comment says "host".
+ * - Data-dependent failures found on the device (bad input values, pool
+ *   exhaustion, a timed-out grid barrier) do not abort: the kernel records
+ *   RKV_DEV_* bits in a status word inside the workspace and skips the
+ *   offending work.  rkv_device_status() returns the device address of that
+ *   word; after a nonzero status the cache contents are unspecified.
+ * - Several calls of one step share a workspace; calls on one workspace must
+ *   be ordered (same stream, or otherwise serialised).
+ *
+ * Cache layout (this library's own specification of the paged, per-head
+ * variable-length layout of [DBTrimKV] Methodology 4 and the physically
+ * enforced ragged storage of [ContourKV] Methodology 2)
+ * ---------------------------------------------------------------------
+ * C = B*L*H heads; head c = (b*L + l)*H + h.  Query head hq = h*G + g
+ * (G = Hq/H) of layer l reads KV head h.  Page size P = 16.
+ * Logical slot k (0 <= k < len[c]) of head c lives in page
+ * block_table[c*max_pages + k/16] at offset k%16; rows of a page are
+ * contiguous: k_pool + (page*16 + k%16)*D elements.  Slot order within a
+ * head is not position order.  free_stack[0 .. *free_top) holds the free
+ * pages; the top is free_stack[*free_top - 1].
+ */
+#ifndef RKV_H_
+#define RKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define RKV_API __attribute__((visibility("default")))
+#else
+#define RKV_API
+#endif
+
+/* ---- status codes (host) ---- */
+#define RKV_OK 0
+#define RKV_ERR_INVALID_ARG (-1)         /* null pointer, bad size, bad shape */
+#define RKV_ERR_UNSUPPORTED (-2)         /* valid but not built: (dtype, D, G), P != 16 */
+#define RKV_ERR_WORKSPACE_TOO_SMALL (-3) /* ws_bytes < rkv_workspace_size() */
+#define RKV_ERR_CUDA (-4)                /* a CUDA runtime call failed; see rkv_last_error() */
+#define RKV_ERR_NOT_IMPLEMENTED (-5)
+
+/* ---- device status bits (in the workspace status word) ---- */
+#define RKV_DEV_BAD_INPUT 1      /* NaN log-retention, age t-i outside [1, 2^24), position too wide */
+#define RKV_DEV_POOL_EXHAUSTED 2 /* append found the free-page stack empty */
+#define RKV_DEV_TABLE_OVERFLOW 4 /* append past max_pages of a head */
+#define RKV_DEV_TIMEOUT 8        /* a grid-wide barrier gave up after ~2 s */
+
+/* ---- element types of the K/V pools ---- */
+#define RKV_BF16 0
+#define RKV_F32 1
+
+/* The paged cache.  Every pointer is a device pointer owned by the caller.
+ *   k_pool, v_pool  [n_pages][16][D] of dtype (RKV_BF16 or RKV_F32)
+ *   pos_pool        [n_pages][16] int32, token position i of each row
+ *   lb_pool         [n_pages][16] float, log-retention log(beta_i) of each row
+ *                   (the retention gate output, [TRIM-KV] core mechanism 1)
+ *   block_table     [C][max_pages] int32, page id or -1
+ *   len             [C] int32, entries per head
+ *   free_stack      [n_pages] int32, free_top [1] int32
+ * Positions within one head must be distinct.  Pools must be 16-byte
+ * aligned (row bytes D*elt are a multiple of 16). */
+typedef struct rkv_cache {
+    void *k_pool;
+    void *v_pool;
+    int32_t *pos_pool;
+    float *lb_pool;
+    int32_t *block_table;
+    int32_t *len;
+    int32_t *free_stack;
+    int32_t *free_top;
+    int32_t B, L, H, Hq, D, P;
+    int32_t n_pages, max_pages;
+    int32_t dtype;
+} rkv_cache_t;
+
+/* Result of one selection, consumed by attention, dropped mass and
+ * compaction of the same step.  Device buffers owned by the caller:
+ *   kappa      [B] uint64   entry e of sequence b is kept iff key(e) < kappa[b]
+ *                           (key defined at rkv_score_select)
+ *   kept       [C] int32    entries of head c that are kept
+ *   n_pre      [C] int32    len[c] when the selection ran
+ *   keep_mask  [C][max_pages] uint16, bit r of word (c, p) set iff slot
+ *                           16p + r of head c is kept
+ *   plan       [C + 2] int32: plan[c] = pages freed by compaction in heads
+ *                           < c (exclusive prefix), plan[C] = total freed,
+ *                           plan[C+1] = *free_top when the selection ran */
+typedef struct rkv_select {
+    uint64_t *kappa;
+    int32_t *kept;
+    int32_t *n_pre;
+    uint16_t *keep_mask;
+    int32_t *plan;
+} rkv_select_t;
+
+/* Library version string (host, static). */
+RKV_API const char *rkv_version(void);
+
+/* Message of the last failed call on this thread (host, thread-local). */
+RKV_API const char *rkv_last_error(void);
+
+/* Bytes of workspace the calls below need for this cache shape (host only,
+ * no CUDA call).  Returns 0 if the shape is invalid. */
+RKV_API size_t rkv_workspace_size(const rkv_cache_t *cache);
+
+/* Zero the workspace (async memset on `stream`).  Call once after
+ * allocating it, and again after a nonzero device status. */
+RKV_API int rkv_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Device address of the int32 status word inside the workspace (RKV_DEV_*
+ * bits, sticky until rkv_workspace_init).  Pure pointer arithmetic. */
+RKV_API int32_t *rkv_device_status(void *ws);
+
+/* ---------------------------------------------------------------------------
+ * rkv_score_select -- score every cached entry and find the global top-M.
+ *
+ * [DBTrimKV] Methodology 2 / [TRIM-KV] core mechanism 2: the retention
+ * weight of token i at step t is beta_i^(t-i); its logarithm is taken as one
+ * IEEE binary32 multiply s = fl32(float(t - i) * lb_i) (round to nearest
+ * even; -0 counts as +0).  [DBTrimKV] Methodology 3: all entries of all
+ * layers and heads of a sequence are ranked together and the top M_global
+ * are kept ([TRIM-KV] core mechanism 4: the lowest are evicted).  Order:
+ * higher s first; equal s by ascending (l, h, i).  The 64-bit key is
+ * (order-preserving map of s) << 32 | ((l*H + h) << ib | i), ib = 32 -
+ * ceil(log2(L*H)); positions must be < 2^ib.
+ *
+ *   t         [B] int32   decode step of each sequence; entries present are
+ *                         those with position < t (age t-i in [1, 2^24))
+ *   m_global  [B] int64   budget per sequence (negative = 0)
+ *   sel       outputs (rkv_select_t), all written
+ * Errors: RKV_ERR_INVALID_ARG (shape), RKV_ERR_WORKSPACE_TOO_SMALL,
+ * RKV_ERR_UNSUPPORTED (L*H > 2^24), RKV_ERR_CUDA (launch).  Device:
+ * RKV_DEV_BAD_INPUT (entry ignored), RKV_DEV_TIMEOUT.
+ * One cooperative persistent launch (grid-wide barriers with a bounded wait).
+ */
+RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
+                             const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * rkv_paged_decode_attn -- grouped-query decode attention over the kept
+ * entries, read from the pre-compaction pages.
+ *
+ * [ContourKV] Problem definition: after selection the softmax is
+ * renormalised over the kept set (forced weights):
+ *   o[c,g] = sum_{j kept} exp(z_j) v_j / sum_{j kept} exp(z_j),
+ *   z_j = scale * <q[c,g], k_j>   (fp32 accumulation of bf16/f32 data).
+ * With `dropped` non-NULL the same pass also returns [ContourKV]
+ * Methodology 3's dropped mass (see rkv_dropped_mass).
+ *
+ *   q         [C][G][D] float (== [B][L][Hq][D])
+ *   scale     logit scale (1/sqrt(D) for standard attention)
+ *   sel       selection of this step, or NULL: every entry is kept
+ *   out       [C][G][D] float   written (0 where nothing is kept)
+ *   lse_kept  [C][G] float or NULL: natural-log sum of exp(z) over kept
+ *             entries (-inf where nothing is kept)
+ *   dropped   [C][G] float or NULL
+ * Errors: RKV_ERR_INVALID_ARG, RKV_ERR_UNSUPPORTED ((dtype, D, G) not
+ * instantiated), RKV_ERR_WORKSPACE_TOO_SMALL, RKV_ERR_CUDA.
+ */
+RKV_API int rkv_paged_decode_attn(const rkv_cache_t *cache, const float *q, float scale,
+                                  const rkv_select_t *sel, float *out, float *lse_kept,
+                                  float *dropped, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * rkv_dropped_mass -- per query head, the dense softmax weight held by the
+ * evicted entries ([ContourKV] Methodology 3 and main contributions):
+ *   dm[c,g] = sum_{j evicted} exp(z_j) / sum_{j present} exp(z_j)
+ * over every entry present before this step's eviction (K only; V is not
+ * read).  0 for a head with no entries; 1 if all of its entries are
+ * evicted.  sel must be non-NULL.
+ *   dropped   [C][G] float   written
+ * Errors as rkv_paged_decode_attn.
+ */
+RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float scale,
+                             const rkv_select_t *sel, float *dropped, void *ws, size_t ws_bytes,
+                             void *stream);
+
+/* ---------------------------------------------------------------------------
+ * rkv_compact_pages -- physically remove the evicted entries
+ * ([ContourKV] Methodology 2: ragged storage, not a mask; [DBTrimKV]
+ * Methodology 4: variable length per head).  Per head c with n = n_pre[c]
+ * and n_new = kept[c]: the j-th kept slot at or above n_new (ascending)
+ * fills the j-th non-kept slot below n_new (ascending), moving its K, V,
+ * position and log-retention; pages at table indices [ceil(n_new/16),
+ * ceil(n/16)) are pushed onto the free stack (heads in ascending c, pages in
+ * ascending table index), their table entries set to -1; len[c] = n_new;
+ * *free_top grows by the pages pushed.  Must follow rkv_score_select of the
+ * same step with no append in between.
+ * Errors: RKV_ERR_INVALID_ARG, RKV_ERR_WORKSPACE_TOO_SMALL, RKV_ERR_CUDA.
+ */
+RKV_API int rkv_compact_pages(const rkv_cache_t *cache, const rkv_select_t *sel, void *ws,
+                              size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * rkv_append -- write the decoded token of every sequence into every head:
+ * slot len[c] receives k_new[c], v_new[c], position t[b] and lb_new[c];
+ * when len[c] % 16 == 0 the head first pops a page from the top of the free
+ * stack (heads in ascending c); len[c] += 1.
+ *   t         [B] int32
+ *   k_new, v_new [C][D] of the pool dtype
+ *   lb_new    [C] float
+ * Errors: RKV_ERR_INVALID_ARG, RKV_ERR_WORKSPACE_TOO_SMALL, RKV_ERR_CUDA.
+ * Device: RKV_DEV_POOL_EXHAUSTED, RKV_DEV_TABLE_OVERFLOW (head skipped).
+ */
+RKV_API int rkv_append(const rkv_cache_t *cache, const int32_t *t, const void *k_new,
+                       const void *v_new, const float *lb_new, void *ws, size_t ws_bytes,
+                       void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RKV_H_ */

@@ -1,0 +1,286 @@
+"""Thin Python binding of librkv (include/rkv.h) for B200 (sm_100a).
+
+Argument marshalling only: every step of the hot path runs in the CUDA
+kernels of librkv.so.  PyTorch supplies device memory and streams.  There is
+no CPU fallback: if the library is missing or fails to load, every call
+raises.
+
+Entry points (same names as the C ABI, without the ``rkv_`` prefix):
+``score_select``, ``paged_decode_attn``, ``dropped_mass``, ``compact_pages``,
+``append``, ``workspace_size``, ``workspace_init``, ``device_status``,
+``version``, ``last_error``.  ``Cache``/``Selection``/``Workspace`` hold the
+tensors and build the C structs; ``step`` runs one decode step in the order
+select -> attention (+ dropped mass) -> compaction -> append.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librkv.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE_TOO_SMALL, ERR_CUDA, ERR_NOT_IMPLEMENTED = 0, -1, -2, -3, -4, -5
+DEV_BAD_INPUT, DEV_POOL_EXHAUSTED, DEV_TABLE_OVERFLOW, DEV_TIMEOUT = 1, 2, 4, 8
+BF16, F32 = 0, 1
+PAGE = 16
+
+EXPORTS = ("rkv_version", "rkv_last_error", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status",
+           "rkv_score_select", "rkv_paged_decode_attn", "rkv_dropped_mass", "rkv_compact_pages", "rkv_append")
+
+
+class RkvError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"librkv error {code}: {msg}")
+        self.code = code
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p), ("pos_pool", ctypes.c_void_p),
+                ("lb_pool", ctypes.c_void_p), ("block_table", ctypes.c_void_p), ("len", ctypes.c_void_p),
+                ("free_stack", ctypes.c_void_p), ("free_top", ctypes.c_void_p)] + [
+        (n, ctypes.c_int32) for n in ("B", "L", "H", "Hq", "D", "P", "n_pages", "max_pages", "dtype")]
+
+
+class SelectStruct(ctypes.Structure):
+    _fields_ = [("kappa", ctypes.c_void_p), ("kept", ctypes.c_void_p), ("n_pre", ctypes.c_void_p),
+                ("keep_mask", ctypes.c_void_p), ("plan", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load librkv.so (built in-tree by __graft_entry__.build()); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"librkv.so not found at {path}: build it with "
+                           "`python -m retention_scored_kv_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    CP, SP = ctypes.POINTER(CacheStruct), ctypes.POINTER(SelectStruct)
+    sig = {
+        "rkv_version": (ctypes.c_char_p, []),
+        "rkv_last_error": (ctypes.c_char_p, []),
+        "rkv_workspace_size": (SZ, [CP]),
+        "rkv_workspace_init": (I, [P, SZ, P]),
+        "rkv_device_status": (P, [P]),
+        "rkv_score_select": (I, [CP, P, P, SP, P, SZ, P]),
+        "rkv_paged_decode_attn": (I, [CP, P, ctypes.c_float, SP, P, P, P, P, SZ, P]),
+        "rkv_dropped_mass": (I, [CP, P, ctypes.c_float, SP, P, P, SZ, P]),
+        "rkv_compact_pages": (I, [CP, SP, P, SZ, P]),
+        "rkv_append": (I, [CP, P, P, P, P, P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise RkvError(rc, load().rkv_last_error().decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("librkv needs contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream: torch.cuda.Stream | None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+@dataclass
+class Cache:
+    """The paged cache (device tensors, caller-owned); layout as in rkv.h."""
+    k_pool: torch.Tensor      # [n_pages, 16, D] bf16 / f32
+    v_pool: torch.Tensor
+    pos_pool: torch.Tensor    # [n_pages, 16] int32
+    lb_pool: torch.Tensor     # [n_pages, 16] float32
+    block_table: torch.Tensor # [C, max_pages] int32
+    len: torch.Tensor         # [C] int32
+    free_stack: torch.Tensor  # [n_pages] int32
+    free_top: torch.Tensor    # [1] int32
+    B: int
+    L: int
+    H: int
+    Hq: int
+
+    @property
+    def D(self) -> int:
+        return self.k_pool.shape[-1]
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.H
+
+    @property
+    def C(self) -> int:
+        return self.B * self.L * self.H
+
+    @property
+    def n_pages(self) -> int:
+        return self.k_pool.shape[0]
+
+    @property
+    def max_pages(self) -> int:
+        return self.block_table.shape[1]
+
+    @property
+    def dtype_code(self) -> int:
+        return BF16 if self.k_pool.dtype == torch.bfloat16 else F32
+
+    @classmethod
+    def from_tensors(cls, t, B: int, L: int, H: int, Hq: int) -> "Cache":
+        return cls(t.k_pool, t.v_pool, t.pos_pool, t.lb_pool, t.block_table, t.len, t.free_stack, t.free_top,
+                   B, L, H, Hq)
+
+    def struct(self) -> CacheStruct:
+        return CacheStruct(_ptr(self.k_pool), _ptr(self.v_pool), _ptr(self.pos_pool), _ptr(self.lb_pool),
+                           _ptr(self.block_table), _ptr(self.len), _ptr(self.free_stack), _ptr(self.free_top),
+                           self.B, self.L, self.H, self.Hq, self.D, PAGE, self.n_pages, self.max_pages,
+                           self.dtype_code)
+
+
+@dataclass
+class Selection:
+    """Device outputs of score_select, consumed by the rest of the step."""
+    kappa: torch.Tensor      # [B] uint64 (stored as int64)
+    kept: torch.Tensor       # [C] int32
+    n_pre: torch.Tensor      # [C] int32
+    keep_mask: torch.Tensor  # [C, max_pages] uint16 (stored as int16)
+    plan: torch.Tensor       # [C + 2] int32
+
+    @classmethod
+    def empty(cls, cache: Cache) -> "Selection":
+        dev = cache.len.device
+        return cls(torch.zeros(cache.B, dtype=torch.int64, device=dev),
+                   torch.zeros(cache.C, dtype=torch.int32, device=dev),
+                   torch.zeros(cache.C, dtype=torch.int32, device=dev),
+                   torch.zeros(cache.C, cache.max_pages, dtype=torch.int16, device=dev),
+                   torch.zeros(cache.C + 2, dtype=torch.int32, device=dev))
+
+    def struct(self) -> SelectStruct:
+        return SelectStruct(_ptr(self.kappa), _ptr(self.kept), _ptr(self.n_pre), _ptr(self.keep_mask),
+                            _ptr(self.plan))
+
+
+class Workspace:
+    """Caller-owned scratch of librkv, sized by rkv_workspace_size."""
+
+    def __init__(self, cache: Cache, stream: torch.cuda.Stream | None = None):
+        self.nbytes = workspace_size(cache)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=cache.len.device)
+        workspace_init(self, stream)
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def status(self) -> int:
+        """RKV_DEV_* bits recorded on the device (reads one int32)."""
+        return int(self.buf[:4].view(torch.int32).item())
+
+
+def version() -> str:
+    return load().rkv_version().decode()
+
+
+def last_error() -> str:
+    return load().rkv_last_error().decode()
+
+
+def workspace_size(cache: Cache) -> int:
+    st = cache.struct()
+    n = load().rkv_workspace_size(ctypes.byref(st))
+    if n == 0:
+        raise RkvError(ERR_INVALID_ARG, last_error())
+    return n
+
+
+def workspace_init(ws: Workspace, stream=None):
+    _check(load().rkv_workspace_init(ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
+def device_status(ws: Workspace) -> int:
+    return load().rkv_device_status(ctypes.c_void_p(ws.ptr))
+
+
+def score_select(cache: Cache, t: torch.Tensor, m_global: torch.Tensor, sel: Selection, ws: Workspace,
+                 stream=None):
+    cs, ss = cache.struct(), sel.struct()
+    _check(load().rkv_score_select(ctypes.byref(cs), _ptr(t), _ptr(m_global), ctypes.byref(ss),
+                                   ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
+def paged_decode_attn(cache: Cache, q: torch.Tensor, scale: float, sel: Selection | None, out: torch.Tensor,
+                      lse: torch.Tensor | None, dropped: torch.Tensor | None, ws: Workspace, stream=None):
+    cs = cache.struct()
+    ss = ctypes.byref(sel.struct()) if sel is not None else None
+    _check(load().rkv_paged_decode_attn(ctypes.byref(cs), _ptr(q), ctypes.c_float(scale), ss, _ptr(out),
+                                        _ptr(lse), _ptr(dropped), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                        _stream(stream)))
+
+
+def dropped_mass(cache: Cache, q: torch.Tensor, scale: float, sel: Selection, dropped: torch.Tensor,
+                 ws: Workspace, stream=None):
+    cs, ss = cache.struct(), sel.struct()
+    _check(load().rkv_dropped_mass(ctypes.byref(cs), _ptr(q), ctypes.c_float(scale), ctypes.byref(ss),
+                                   _ptr(dropped), ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
+def compact_pages(cache: Cache, sel: Selection, ws: Workspace, stream=None):
+    cs, ss = cache.struct(), sel.struct()
+    _check(load().rkv_compact_pages(ctypes.byref(cs), ctypes.byref(ss), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                    _stream(stream)))
+
+
+def append(cache: Cache, t: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, lb_new: torch.Tensor,
+           ws: Workspace, stream=None):
+    cs = cache.struct()
+    _check(load().rkv_append(ctypes.byref(cs), _ptr(t), _ptr(k_new), _ptr(v_new), _ptr(lb_new),
+                             ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
+@dataclass
+class StepOutputs:
+    out: torch.Tensor      # [B, L, Hq, D] float32
+    lse: torch.Tensor      # [B, L, Hq] float32
+    dropped: torch.Tensor  # [B, L, Hq] float32
+
+    @classmethod
+    def empty(cls, cache: Cache) -> "StepOutputs":
+        dev = cache.len.device
+        return cls(torch.empty(cache.B, cache.L, cache.Hq, cache.D, dtype=torch.float32, device=dev),
+                   torch.empty(cache.B, cache.L, cache.Hq, dtype=torch.float32, device=dev),
+                   torch.empty(cache.B, cache.L, cache.Hq, dtype=torch.float32, device=dev))
+
+
+def step(cache: Cache, sel: Selection, ws: Workspace, outs: StepOutputs, *, q, t, m_global, k_new, v_new,
+         lb_new, evict: bool = True, scale: float | None = None, stream=None):
+    """One decode step: [select] -> attention + dropped mass -> [compaction] -> append.
+
+    On a non-evicting step every entry is kept and the dropped mass is 0."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(cache.D)
+    if evict:
+        score_select(cache, t, m_global, sel, ws, stream)
+        paged_decode_attn(cache, q, scale, sel, outs.out, outs.lse, outs.dropped, ws, stream)
+        compact_pages(cache, sel, ws, stream)
+    else:
+        paged_decode_attn(cache, q, scale, None, outs.out, outs.lse, outs.dropped, ws, stream)
+    append(cache, t, k_new, v_new, lb_new, ws, stream)

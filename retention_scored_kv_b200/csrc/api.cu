@@ -1,0 +1,317 @@
+// api.cu -- the C ABI of librkv (declared in include/rkv.h): argument
+// validation, workspace layout and kernel launches on the caller's stream.
+// No call allocates, frees or synchronises.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace rkv {
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    if (e == cudaErrorNotSupported) return fail(RKV_ERR_UNSUPPORTED, "%s: not supported for this shape", what);
+    return fail(RKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elt_bytes(int dtype) { return dtype == RKV_BF16 ? 2 : (dtype == RKV_F32 ? 4 : 0); }
+
+// Shape and pointer checks shared by every entry point.
+int check_cache(const rkv_cache_t *c, bool need_pools) {
+    if (!c) return fail(RKV_ERR_INVALID_ARG, "cache is NULL");
+    if (c->B <= 0 || c->L <= 0 || c->H <= 0 || c->Hq <= 0 || c->D <= 0)
+        return fail(RKV_ERR_INVALID_ARG, "B, L, H, Hq, D must be positive");
+    if (c->Hq % c->H != 0) return fail(RKV_ERR_INVALID_ARG, "Hq (%d) must be a multiple of H (%d)", c->Hq, c->H);
+    if (c->P != PAGE) return fail(RKV_ERR_UNSUPPORTED, "page size must be 16 (got %d)", c->P);
+    if (c->n_pages <= 0 || c->max_pages <= 0) return fail(RKV_ERR_INVALID_ARG, "n_pages and max_pages must be positive");
+    if ((int64_t)c->n_pages * PAGE >= (1ll << 31)) return fail(RKV_ERR_UNSUPPORTED, "n_pages*16 must be < 2^31");
+    const int64_t C = (int64_t)c->B * c->L * c->H;
+    if (C >= (1ll << 31) || C * c->max_pages >= (1ll << 40)) return fail(RKV_ERR_UNSUPPORTED, "too many heads");
+    const int eb = elt_bytes(c->dtype);
+    if (!eb) return fail(RKV_ERR_INVALID_ARG, "dtype must be RKV_BF16 or RKV_F32");
+    if ((c->D * eb) % 16 != 0) return fail(RKV_ERR_UNSUPPORTED, "row bytes D*elt must be a multiple of 16");
+    if (!c->len || !c->block_table) return fail(RKV_ERR_INVALID_ARG, "len / block_table is NULL");
+    if (need_pools) {
+        if (!c->k_pool || !c->v_pool || !c->pos_pool || !c->lb_pool || !c->free_stack || !c->free_top)
+            return fail(RKV_ERR_INVALID_ARG, "a cache pool pointer is NULL");
+        if (!aligned16(c->k_pool) || !aligned16(c->v_pool))
+            return fail(RKV_ERR_INVALID_ARG, "k_pool / v_pool must be 16-byte aligned");
+    }
+    return RKV_OK;
+}
+
+int check_sel(const rkv_select_t *s) {
+    if (!s || !s->kappa || !s->kept || !s->n_pre || !s->keep_mask || !s->plan)
+        return fail(RKV_ERR_INVALID_ARG, "selection buffers must all be non-NULL");
+    return RKV_OK;
+}
+
+int lh_bits(int64_t LH) {
+    int b = 0;
+    while ((1ll << b) < LH) b++;
+    return b;
+}
+
+// Select grid that depends only on the shape (upper bound for workspace sizing).
+constexpr int MAX_SEL_CTAS = 1024;
+
+void layout_for(const rkv_cache_t &c, int sel_groups_x_waves, WsLayout *L) {
+    const int G = c.Hq / c.H;
+    const int64_t C = (int64_t)c.B * c.L * c.H;
+    size_t off = 0;
+    auto take = [&](size_t bytes, size_t align) {
+        off = (off + align - 1) / align * align;
+        size_t at = off;
+        off += bytes;
+        return at;
+    };
+    L->status = take(4, 4);
+    L->done_compact = take(4, 4);
+    L->done_append = take(4, 4);
+    L->sel_begin = take(0, 256);
+    L->bar = take(4, 4);
+    L->more = take((size_t)c.B * NPASS * 4, 16);
+    L->hist = take((size_t)sel_groups_x_waves * NPASS * NBINS * 4, 256);
+    L->sel_end = take(0, 256);
+    L->head_cnt = take((size_t)C * 4, 256);
+    L->partial = take((size_t)MAX_ATTN_CTAS * 2 * attn_partial_rec_floats(c.D, G) * 4, 256);
+    L->total = take(0, 256);
+}
+
+int sm_count_now(int *out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    e = cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    return RKV_OK;
+}
+
+int check_ws(const rkv_cache_t *c, void *ws, size_t ws_bytes, WsLayout *L) {
+    if (!ws) return fail(RKV_ERR_INVALID_ARG, "workspace is NULL");
+    if (!aligned16(ws)) return fail(RKV_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    ws_layout(*c, L);
+    if (ws_bytes < L->total)
+        return fail(RKV_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes < %zu needed", ws_bytes, L->total);
+    return RKV_OK;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
+}
+
+}  // namespace
+
+bool ws_layout(const rkv_cache_t &c, WsLayout *out) {
+    // groups x waves of the selection grid never exceed 2*B (groups <= B)
+    layout_for(c, 2 * c.B, out);
+    return true;
+}
+
+}  // namespace rkv
+
+using namespace rkv;
+
+extern "C" {
+
+RKV_API const char *rkv_version(void) { return "librkv 0.1.0 (sm_100a)"; }
+
+RKV_API const char *rkv_last_error(void) { return g_err.c_str(); }
+
+RKV_API size_t rkv_workspace_size(const rkv_cache_t *cache) {
+    if (check_cache(cache, false) != RKV_OK) return 0;
+    WsLayout L;
+    ws_layout(*cache, &L);
+    return L.total;
+}
+
+RKV_API int rkv_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || ws_bytes == 0) return fail(RKV_ERR_INVALID_ARG, "workspace is NULL or empty");
+    cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
+    return RKV_OK;
+}
+
+RKV_API int32_t *rkv_device_status(void *ws) { return ws ? reinterpret_cast<int32_t *>(ws) : nullptr; }
+
+RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
+                             const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if ((rc = check_sel(sel))) return rc;
+    if (!t || !m_global) return fail(RKV_ERR_INVALID_ARG, "t / m_global is NULL");
+    WsLayout L;
+    if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
+    const int64_t LH = (int64_t)cache->L * cache->H;
+    const int lb = lh_bits(LH);
+    if (lb > 24) return fail(RKV_ERR_UNSUPPORTED, "L*H must be <= 2^24");
+    int sms = 0;
+    if ((rc = sm_count_now(&sms))) return rc;
+    SelectGrid g = select_grid_for(*cache, sms < MAX_SEL_CTAS ? sms : MAX_SEL_CTAS);
+    if (g.cache_pages < 0) return fail(RKV_ERR_UNSUPPORTED, "L*H too large for the selection kernel");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t used_hist = (size_t)g.waves * g.n_groups * NPASS * NBINS * 4;
+    cudaError_t e = cudaMemsetAsync(at<unsigned char>(ws, L.sel_begin), 0, (L.hist - L.sel_begin) + used_hist, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(selection scratch)");
+    SelectArgs a{};
+    a.pos_pool = cache->pos_pool;
+    a.lb_pool = cache->lb_pool;
+    a.block_table = cache->block_table;
+    a.len = cache->len;
+    a.free_top = cache->free_top;
+    a.B = cache->B;
+    a.LH = (int)LH;
+    a.C = (int)(cache->B * LH);
+    a.max_pages = cache->max_pages;
+    a.ibits = 32 - lb;
+    a.t = t;
+    a.m_global = m_global;
+    a.kappa = sel->kappa;
+    a.kept = sel->kept;
+    a.n_pre = sel->n_pre;
+    a.keep_mask = sel->keep_mask;
+    a.plan = sel->plan;
+    a.status = at<int32_t>(ws, L.status);
+    a.bar = at<uint32_t>(ws, L.bar);
+    a.more = at<uint32_t>(ws, L.more);
+    a.hist = at<uint32_t>(ws, L.hist);
+    a.n_groups = g.n_groups;
+    a.cta_per_group = g.cta_per_group;
+    a.waves = g.waves;
+    a.cache_pages = g.cache_pages;
+    e = launch_select(a, g, s);
+    if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
+    return RKV_OK;
+}
+
+static int attn_common(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
+                       float *out, float *lse, float *dropped, void *ws, size_t ws_bytes, void *stream,
+                       const char *what) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if (!q) return fail(RKV_ERR_INVALID_ARG, "%s: q is NULL", what);
+    if (!aligned16(q)) return fail(RKV_ERR_INVALID_ARG, "%s: q must be 16-byte aligned", what);
+    if (sel && !sel->keep_mask) return fail(RKV_ERR_INVALID_ARG, "%s: sel->keep_mask is NULL", what);
+    const int G = cache->Hq / cache->H;
+    if (!attn_supported(cache->dtype, cache->D, G))
+        return fail(RKV_ERR_UNSUPPORTED, "%s: (dtype %d, D %d, G %d) not built", what, cache->dtype, cache->D, G);
+    WsLayout L;
+    if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
+    int sms = 0;
+    if ((rc = sm_count_now(&sms))) return rc;
+    AttnArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.block_table = cache->block_table;
+    a.len = cache->len;
+    a.keep_mask = sel ? sel->keep_mask : nullptr;
+    a.q = q;
+    a.out = out;
+    a.lse = lse;
+    a.dropped = dropped;
+    a.status = at<int32_t>(ws, L.status);
+    a.head_cnt = at<uint32_t>(ws, L.head_cnt);
+    a.partial = at<float>(ws, L.partial);
+    a.C = cache->B * cache->L * cache->H;
+    a.max_pages = cache->max_pages;
+    a.qscale = scale * 1.4426950408889634f;
+    cudaError_t e = launch_attn(a, cache->dtype, cache->D, G, sms, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    return RKV_OK;
+}
+
+RKV_API int rkv_paged_decode_attn(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
+                                  float *out, float *lse_kept, float *dropped, void *ws, size_t ws_bytes,
+                                  void *stream) {
+    if (!out) return fail(RKV_ERR_INVALID_ARG, "rkv_paged_decode_attn: out is NULL");
+    return attn_common(cache, q, scale, sel, out, lse_kept, dropped, ws, ws_bytes, stream, "rkv_paged_decode_attn");
+}
+
+RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
+                             float *dropped, void *ws, size_t ws_bytes, void *stream) {
+    if (!dropped) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: dropped is NULL");
+    if (!sel) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: sel is NULL");
+    return attn_common(cache, q, scale, sel, nullptr, nullptr, dropped, ws, ws_bytes, stream, "rkv_dropped_mass");
+}
+
+RKV_API int rkv_compact_pages(const rkv_cache_t *cache, const rkv_select_t *sel, void *ws, size_t ws_bytes,
+                              void *stream) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if ((rc = check_sel(sel))) return rc;
+    WsLayout L;
+    if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
+    CompactArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.pos_pool = cache->pos_pool;
+    a.lb_pool = cache->lb_pool;
+    a.block_table = cache->block_table;
+    a.len = cache->len;
+    a.free_stack = cache->free_stack;
+    a.free_top = cache->free_top;
+    a.kept = sel->kept;
+    a.n_pre = sel->n_pre;
+    a.keep_mask = sel->keep_mask;
+    a.plan = sel->plan;
+    a.done = at<uint32_t>(ws, L.done_compact);
+    a.C = cache->B * cache->L * cache->H;
+    a.max_pages = cache->max_pages;
+    a.row_bytes = cache->D * elt_bytes(cache->dtype);
+    cudaError_t e = launch_compact(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "compact kernel launch");
+    return RKV_OK;
+}
+
+RKV_API int rkv_append(const rkv_cache_t *cache, const int32_t *t, const void *k_new, const void *v_new,
+                       const float *lb_new, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if (!t || !k_new || !v_new || !lb_new) return fail(RKV_ERR_INVALID_ARG, "rkv_append: an input is NULL");
+    if (!aligned16(k_new) || !aligned16(v_new))
+        return fail(RKV_ERR_INVALID_ARG, "rkv_append: k_new / v_new must be 16-byte aligned");
+    WsLayout L;
+    if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
+    AppendArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.pos_pool = cache->pos_pool;
+    a.lb_pool = cache->lb_pool;
+    a.block_table = cache->block_table;
+    a.len = cache->len;
+    a.free_stack = cache->free_stack;
+    a.free_top = cache->free_top;
+    a.t = t;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.lb_new = lb_new;
+    a.status = at<int32_t>(ws, L.status);
+    a.done = at<uint32_t>(ws, L.done_append);
+    a.C = cache->B * cache->L * cache->H;
+    a.LH = cache->L * cache->H;
+    a.max_pages = cache->max_pages;
+    a.row_bytes = cache->D * elt_bytes(cache->dtype);
+    cudaError_t e = launch_append(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append kernel launch");
+    return RKV_OK;
+}
+
+}  // extern "C"

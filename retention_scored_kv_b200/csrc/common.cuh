@@ -1,0 +1,224 @@
+// common.cuh -- device helpers shared by the librkv kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/rkv.h"
+
+namespace rkv {
+
+constexpr int PAGE = 16;           // rows per page (fixed; keep masks are uint16)
+constexpr int NPASS = 6;           // radix digits of the 64-bit key: 11,11,10 | 11,11,10
+constexpr int NBINS = 2048;        // bins of the widest digit
+constexpr int MAX_ATTN_CTAS = 512; // upper bound of the persistent attention grid
+constexpr uint32_t KEY_INVALID = 0xFFFFFFFFu;  // hi word no valid score maps to (NaN space)
+
+// ---------------------------------------------------------------- keys ----
+// Order-preserving map of a binary32 score to uint32 such that a HIGHER score
+// gives a SMALLER key (negative scores: the bit pattern itself, since larger
+// magnitude = lower score; positive scores: complement of the pattern below
+// 0x80000000).  +0 maps to 0x7FFFFFFF; -inf to 0xFF800000.  Callers
+// canonicalise -0 to +0 and reject NaN first.
+__device__ __forceinline__ uint32_t score_key_desc(float s) {
+    uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? u : (~u & 0x7FFFFFFFu);
+}
+
+// Digit p of the 64-bit key (hi:lo); widths 11,11,10 per 32-bit half.
+__device__ __forceinline__ uint32_t key_digit(uint32_t hi, uint32_t lo, int p) {
+    uint32_t w = p < 3 ? hi : lo;
+    int q = p < 3 ? p : p - 3;
+    return q == 0 ? (w >> 21) : (q == 1 ? ((w >> 10) & 0x7FFu) : (w & 0x3FFu));
+}
+__host__ __device__ __forceinline__ int digit_bits(int p) { return (p % 3 == 2) ? 10 : 11; }
+__host__ __device__ __forceinline__ int digit_shift(int p) {
+    // bit position of digit p's least significant bit within the 64-bit key
+    return (p < 3 ? 32 : 0) + (p % 3 == 0 ? 21 : (p % 3 == 1 ? 10 : 0));
+}
+
+// ------------------------------------------------------------ status ----
+__device__ __forceinline__ void set_status(int32_t *status, int32_t bits) {
+    if ((__ldcg(status) & bits) != bits) atomicOr(status, bits);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid-wide barrier for a cooperative (co-resident) grid.  `count` is a
+// monotonically increasing arrival counter zeroed before the launch; barrier
+// number `epoch` (1, 2, ...) completes when count reaches epoch*gridDim.x.
+// The wait is bounded (~2 s of globaltimer); on timeout RKV_DEV_TIMEOUT is
+// recorded and false returned, so the caller can leave the kernel.
+__device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, int32_t *status,
+                                             int *smem_flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(count, 1u);
+        const uint32_t target = epoch * gridDim.x;
+        int ok = 1;
+        if (ld_acquire_gpu(count) < target) {
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t spins = 0;
+            while (ld_acquire_gpu(count) < target) {
+                if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
+                    set_status(status, RKV_DEV_TIMEOUT);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(32);
+            }
+        }
+        __threadfence();
+        *smem_flag = ok;
+    }
+    __syncthreads();
+    return *smem_flag != 0;
+}
+
+// ------------------------------------------------ mbarrier / bulk copy ----
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase.  Every producer of the phase is in the
+// same CTA and always arrives, so the bound is a guard, not a protocol:
+// after ~2 s the wait records RKV_DEV_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (__ldcg(status) & RKV_DEV_TIMEOUT) return false;  // an earlier wait already gave up
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t spins = 0;
+    while (!mbar_try_wait(bar, parity)) {
+        if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
+            set_status(status, RKV_DEV_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// One bulk asynchronous global->shared copy through the TMA engine
+// (cp.async.bulk, no tensor map): both addresses 16-byte aligned, size a
+// multiple of 16; completion is signalled as transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------- math ----
+// Base-2 exponential on the SFU (ex2.approx: relative error ~2^-22).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Packed fp32 pair multiply-add (sm_100: fma.rn.f32x2), d = a*b + c per lane.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    uint64_t A, B, Cc, Dd;
+    asm("mov.b64 %0, {%1,%2};" : "=l"(A) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1,%2};" : "=l"(B) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1,%2};" : "=l"(Cc) : "f"(c.x), "f"(c.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(Dd) : "l"(A), "l"(B), "l"(Cc));
+    float2 d;
+    asm("mov.b64 {%0,%1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(Dd));
+    return d;
+}
+
+// bf16x2 word -> two floats (exact widening: a bf16 is the top half of an fp32).
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// ------------------------------------------------------------- scans ----
+// Block-wide exclusive scan of one uint32 per thread (blockDim.x <= 1024,
+// multiple of 32).  `scratch` holds >= 33 words.  Returns the exclusive
+// prefix; *total receives the block sum.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *scratch, uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = lane < nw ? scratch[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < nw) scratch[lane] = w;
+        if (lane == 31) scratch[32] = w;
+    }
+    __syncthreads();
+    uint32_t base = warp > 0 ? scratch[warp - 1] : 0u;
+    *total = scratch[32];
+    __syncthreads();
+    return base + x - v;
+}
+
+}  // namespace rkv
