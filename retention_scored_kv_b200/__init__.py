@@ -284,3 +284,100 @@ def step(cache: Cache, sel: Selection, ws: Workspace, outs: StepOutputs, *, q, t
     else:
         paged_decode_attn(cache, q, scale, None, outs.out, outs.lse, outs.dropped, ws, stream)
     append(cache, t, k_new, v_new, lb_new, ws, stream)
+
+
+def _align(n: int, a: int = 256) -> int:
+    return (n + a - 1) // a * a
+
+
+class StepRunner:
+    """One decode step on static device buffers, optionally captured in CUDA graphs.
+
+    Inputs live in one device buffer (q, k_new, v_new, lb_new, t, m_global) and
+    outputs in another (out, lse, dropped), so a step driven from host memory
+    costs one host-to-device copy, one graph replay (or the eager calls) and one
+    device-to-host copy.  ``in_layout`` / ``out_layout`` give each field's byte
+    offset, shape and dtype so callers can pack pinned host buffers."""
+
+    def __init__(self, cache: Cache, *, scale: float | None = None, use_graph: bool = True, stream=None):
+        self.cache = cache
+        self.scale = 1.0 / math.sqrt(cache.D) if scale is None else scale
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        dev = cache.len.device
+        kvdt = cache.k_pool.dtype
+        C, G, D, B = cache.C, cache.G, cache.D, cache.B
+        self.in_layout, off = {}, 0
+        for name, shape, dt in (("q", (B, cache.L, cache.Hq, D), torch.float32), ("k_new", (C, D), kvdt),
+                                ("v_new", (C, D), kvdt), ("lb_new", (C,), torch.float32),
+                                ("t", (B,), torch.int32), ("m_global", (B,), torch.int64)):
+            n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
+            self.in_layout[name] = (off, shape, dt)
+            off = _align(off + n)
+        self.in_bytes = off
+        self.out_layout, off = {}, 0
+        for name, shape in (("out", (B, cache.L, cache.Hq, D)), ("lse", (B, cache.L, cache.Hq)),
+                            ("dropped", (B, cache.L, cache.Hq))):
+            self.out_layout[name] = (off, shape, torch.float32)
+            off = _align(off + math.prod(shape) * 4)
+        self.out_bytes = off
+        self.inbuf = torch.zeros(self.in_bytes, dtype=torch.uint8, device=dev)
+        self.outbuf = torch.zeros(self.out_bytes, dtype=torch.uint8, device=dev)
+        self.inp = {k: self._view(self.inbuf, *v) for k, v in self.in_layout.items()}
+        o = {k: self._view(self.outbuf, *v) for k, v in self.out_layout.items()}
+        self.outs = StepOutputs(o["out"], o["lse"], o["dropped"])
+        self.sel = Selection.empty(cache)
+        self.ws = Workspace(cache, self.stream)
+        self.use_graph = use_graph
+        self.graphs: dict[bool, torch.cuda.CUDAGraph] = {}
+
+    @staticmethod
+    def _view(buf: torch.Tensor, off: int, shape, dt) -> torch.Tensor:
+        n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
+        return buf[off: off + n].view(dt).view(shape)
+
+    def pack(self, host: torch.Tensor, **fields) -> None:
+        """Write input fields into a host (pinned) uint8 buffer of in_bytes."""
+        for k, v in fields.items():
+            self._view(host, *self.in_layout[k]).copy_(v)
+
+    def unpack(self, host: torch.Tensor) -> dict:
+        return {k: self._view(host, *v) for k, v in self.out_layout.items()}
+
+    def _enqueue(self, evict: bool) -> None:
+        i = self.inp
+        step(self.cache, self.sel, self.ws, self.outs, q=i["q"], t=i["t"], m_global=i["m_global"],
+             k_new=i["k_new"], v_new=i["v_new"], lb_new=i["lb_new"], evict=evict, scale=self.scale,
+             stream=self.stream)
+
+    def capture(self) -> bool:
+        """Capture the evicting and non-evicting step; False if capture is refused."""
+        if not self.use_graph:
+            return False
+        try:
+            for evict in (True, False):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
+                    self._enqueue(evict)
+                self.graphs[evict] = g
+            return True
+        except Exception:
+            self.graphs.clear()
+            self.use_graph = False
+            return False
+
+    def run(self, evict: bool = True) -> None:
+        """Run one step on the inputs already in the static device buffer."""
+        g = self.graphs.get(evict)
+        if g is not None:
+            with torch.cuda.stream(self.stream):
+                g.replay()
+        else:
+            self._enqueue(evict)
+
+    def run_host(self, host_in: torch.Tensor, host_out: torch.Tensor, evict: bool = True) -> None:
+        """Copy packed host inputs in, run the step, copy packed outputs out (async)."""
+        with torch.cuda.stream(self.stream):
+            self.inbuf.copy_(host_in, non_blocking=True)
+        self.run(evict)
+        with torch.cuda.stream(self.stream):
+            host_out.copy_(self.outbuf, non_blocking=True)
