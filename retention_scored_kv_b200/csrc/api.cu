@@ -113,6 +113,37 @@ int check_ws(const rkv_cache_t *c, void *ws, size_t ws_bytes, WsLayout *L) {
     return RKV_OK;
 }
 
+// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry point.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int encode_pool_map(CUtensorMap *m, void *pool, int D, int n_pages) {
+    if (D % 64 != 0) return fail(RKV_ERR_UNSUPPORTED, "bf16 pools need D a multiple of 64");
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return fail(RKV_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    // the pool as [rows = n_pages*16][D/64 lines][64 columns] bf16; one box is
+    // a whole page (16 rows x D/64 lines x 64 columns) and lands in shared
+    // memory as 128-byte lines, 16-byte chunks XOR-swizzled by line mod 8
+    const cuuint32_t nline = (cuuint32_t)(D / 64);
+    const cuuint64_t dims[3] = {64, nline, (cuuint64_t)n_pages * PAGE};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)D * 2};
+    const cuuint32_t box[3] = {64, nline, PAGE};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pool, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(RKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return RKV_OK;
+}
+
 template <typename T>
 T *at(void *ws, size_t off) {
     return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
@@ -233,7 +264,12 @@ static int attn_common(const rkv_cache_t *cache, const float *q, float scale, co
     a.C = cache->B * cache->L * cache->H;
     a.max_pages = cache->max_pages;
     a.qscale = scale * 1.4426950408889634f;
-    cudaError_t e = launch_attn(a, cache->dtype, cache->D, G, sms, static_cast<cudaStream_t>(stream));
+    CUtensorMap tk{}, tv{};
+    if (attn_uses_tensor_maps(cache->dtype)) {
+        if ((rc = encode_pool_map(&tk, cache->k_pool, cache->D, cache->n_pages))) return rc;
+        if ((rc = encode_pool_map(&tv, cache->v_pool, cache->D, cache->n_pages))) return rc;
+    }
+    cudaError_t e = launch_attn(a, cache->dtype, cache->D, G, sms, static_cast<cudaStream_t>(stream), tk, tv);
     if (e != cudaSuccess) return cuda_fail(e, what);
     return RKV_OK;
 }

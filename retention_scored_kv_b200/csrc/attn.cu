@@ -6,24 +6,29 @@
 // and main contributions: the dropped mass is the dense softmax weight held
 // by the evicted keys, over every entry present before the eviction.
 //
-// Design (HBM-bound; see the roofline notes in the design document):
+// Design (HBM-bound: ~512 bytes of K/V per kept entry against 4*G*D flops):
 // * Persistent grid, one CTA per SM.  The pages of all heads (pre-compaction
 //   lengths, 16 rows each) are flattened in head order and split evenly
 //   across CTAs, so ragged per-head lengths cost no imbalance.
 // * Warp specialisation: one producer warp streams each page's K (and V when
-//   the page holds a kept row) into a multi-stage shared-memory ring with
-//   cp.async.bulk (TMA bulk copies, 16-byte aligned, mbarrier transaction
-//   counts), plus each head's queries; eight consumer warps take pages
-//   round-robin.
-// * Consumer math on CUDA cores in fp32: RL lanes share a row, each owning
-//   16-byte chunks (128-bit shared loads, conflict-free), q held in
-//   registers pre-scaled by scale*log2(e); packed f32x2 FMAs; a butterfly
-//   over the RL lanes finishes each dot product.  Online softmax in base 2
-//   with separate running maxima for kept and evicted rows; PV only for kept
-//   rows.
+//   the page holds a kept row) into a multi-stage shared-memory ring through
+//   the TMA engine (mbarrier transaction counts), plus each head's queries;
+//   eight consumer warps take pages round-robin.
+// * Math policies.  bf16 pools (MmaMath): pages arrive as 64-column tensor
+//   boxes in the 128-byte-swizzled layout; QK^T and PV run on the tensor
+//   cores as m16n8k16 bf16 MMAs with fp32 accumulation -- the G query rows of
+//   a KV head padded to 16, queries and softmax weights split into bf16
+//   high + low parts so the products keep ~fp32 accuracy; ldmatrix feeds the
+//   fragments without bank conflicts.  fp32 pools (CoreMath): CUDA-core FMAs,
+//   RL lanes per row, packed f32x2 FMAs and a butterfly per dot product.
+// * Online softmax in base 2 with separate running maxima for kept rows and
+//   for evicted rows (the latter only for the dropped mass); PV only for kept
+//   rows, and V is not fetched for pages without a kept row.
 // * Head boundaries: warps merge through shared memory; a head split across
 //   CTAs writes partial (max, sum, acc) records and the last CTA to arrive
 //   (atomic counter, no waiting) merges them -- the cross-split combine.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,13 +36,21 @@ namespace rkv {
 
 namespace {
 
-constexpr int NCW = 8;                 // consumer warps
-constexpr int ATTN_THREADS = (NCW + 1) * 32;
+#ifndef RKV_NCW
+#define RKV_NCW 8
+#endif
+#ifndef RKV_NPW
+#define RKV_NPW 2
+#endif
+constexpr int NCW = RKV_NCW;           // consumer warps
+constexpr int NPW = RKV_NPW;           // producer warps (one issuing lane each)
+constexpr int ATTN_THREADS = (NCW + NPW) * 32;
 constexpr int QR = 4;                  // query ring slots
 constexpr float LN2 = 0.69314718055994530942f;
 
+// ------------------------------------------------------------ CUDA cores ----
 template <typename T, int D, int G, bool WITH_V>
-struct Cfg {
+struct CoreMath {
     static constexpr int ROW_BYTES = D * (int)sizeof(T);
     static constexpr int CHUNKS = ROW_BYTES / 16;
     static constexpr int RL0 = (G <= 4) ? 8 : 16;
@@ -48,24 +61,401 @@ struct Cfg {
     static constexpr int RPP = 32 / RL;                       // rows per pass
     static constexpr int NPASSES = PAGE / RPP;
     static constexpr int PAGE_BYTES = PAGE * ROW_BYTES;
-    static constexpr int STAGE_BYTES = PAGE_BYTES * (WITH_V ? 2 : 1);
-    static constexpr int NST0 = 98304 / STAGE_BYTES;
-    static constexpr int NST = NST0 < 4 ? 4 : (NST0 > 16 ? 16 : NST0);
+    static constexpr int STAGE_ALIGN = 128;
+    static constexpr bool USES_TMAP = false;
+    static_assert(CHUNKS % RL == 0 && 32 % RL == 0, "lane mapping");
+
+    struct State {
+        float2 q2[G][DL / 2];
+        float mk[G], lk[G], me[G], le[G];
+        float2 acc[G][WITH_V ? DL / 2 : 1];
+    };
+
+    __device__ static void load_q(State &s, const float *qs, float qscale, int lane) {
+        const int tl = lane % RL;
+#pragma unroll
+        for (int g = 0; g < G; g++)
+#pragma unroll
+            for (int j = 0; j < CPL; j++)
+#pragma unroll
+                for (int e = 0; e < EPC; e += 2) {
+                    const int d = (tl + RL * j) * EPC + e;
+                    s.q2[g][(j * EPC + e) / 2] = make_float2(qs[g * D + d] * qscale, qs[g * D + d + 1] * qscale);
+                }
+#pragma unroll
+        for (int g = 0; g < G; g++) {
+            s.mk[g] = -INFINITY; s.lk[g] = 0.0f; s.me[g] = -INFINITY; s.le[g] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < (WITH_V ? DL / 2 : 1); i++) s.acc[g][i] = make_float2(0.0f, 0.0f);
+        }
+    }
+
+    __device__ static void widen(const uint4 &w, float2 *out) {
+        if constexpr (sizeof(T) == 2) {
+            out[0] = bf16x2_to_f2(w.x); out[1] = bf16x2_to_f2(w.y);
+            out[2] = bf16x2_to_f2(w.z); out[3] = bf16x2_to_f2(w.w);
+        } else {
+            out[0] = make_float2(__uint_as_float(w.x), __uint_as_float(w.y));
+            out[1] = make_float2(__uint_as_float(w.z), __uint_as_float(w.w));
+        }
+    }
+
+    __device__ static void page(State &s, const unsigned char *sk, const unsigned char *sv, uint32_t keepm,
+                                uint32_t evm, int lane) {
+        const int rg = lane / RL, tl = lane % RL;
+        float y[NPASSES][G];
+#pragma unroll
+        for (int ps = 0; ps < NPASSES; ps++) {
+            const int row = ps * RPP + rg;
+            const uint4 *kr = reinterpret_cast<const uint4 *>(sk + row * ROW_BYTES);
+            float2 part[G];
+#pragma unroll
+            for (int g = 0; g < G; g++) part[g] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int j = 0; j < CPL; j++) {
+                float2 kp[EPC / 2];
+                widen(kr[tl + RL * j], kp);
+#pragma unroll
+                for (int e = 0; e < EPC / 2; e++)
+#pragma unroll
+                    for (int g = 0; g < G; g++) part[g] = ffma2(s.q2[g][j * EPC / 2 + e], kp[e], part[g]);
+            }
+#pragma unroll
+            for (int g = 0; g < G; g++) {
+                float v = part[g].x + part[g].y;
+#pragma unroll
+                for (int o = 1; o < RL; o <<= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                y[ps][g] = v;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; g++) {
+            float pk = -INFINITY, pe = -INFINITY;
+#pragma unroll
+            for (int ps = 0; ps < NPASSES; ps++) {
+                const int row = ps * RPP + rg;
+                if ((keepm >> row) & 1u) pk = fmaxf(pk, y[ps][g]);
+                if ((evm >> row) & 1u) pe = fmaxf(pe, y[ps][g]);
+            }
+#pragma unroll
+            for (int o = RL; o < 32; o <<= 1) {
+                pk = fmaxf(pk, __shfl_xor_sync(0xFFFFFFFFu, pk, o));
+                pe = fmaxf(pe, __shfl_xor_sync(0xFFFFFFFFu, pe, o));
+            }
+            if (evm) {
+                const float mn = fmaxf(s.me[g], pe);
+                float sum = 0.0f;
+#pragma unroll
+                for (int ps = 0; ps < NPASSES; ps++)
+                    if ((evm >> (ps * RPP + rg)) & 1u) sum += ex2(y[ps][g] - mn);
+                s.le[g] = s.le[g] * ex2(s.me[g] - mn) + (tl == 0 ? sum : 0.0f);  // me = -inf -> 0
+                s.me[g] = mn;
+            }
+            if (keepm) {
+                const float mn = fmaxf(s.mk[g], pk);
+                const float alpha = ex2(s.mk[g] - mn);  // mk = -inf -> 0
+                if (alpha != 1.0f) {
+                    s.lk[g] *= alpha;
+                    if constexpr (WITH_V) {
+#pragma unroll
+                        for (int i = 0; i < DL / 2; i++) { s.acc[g][i].x *= alpha; s.acc[g][i].y *= alpha; }
+                    }
+                }
+                s.mk[g] = mn;
+                float sum = 0.0f;
+#pragma unroll
+                for (int ps = 0; ps < NPASSES; ps++) {
+                    const float p = ((keepm >> (ps * RPP + rg)) & 1u) ? ex2(y[ps][g] - mn) : 0.0f;
+                    y[ps][g] = p;
+                    sum += p;
+                }
+                s.lk[g] += (tl == 0) ? sum : 0.0f;
+            }
+        }
+        if constexpr (WITH_V) {
+            if (keepm) {
+#pragma unroll
+                for (int ps = 0; ps < NPASSES; ps++) {
+                    const uint4 *vr = reinterpret_cast<const uint4 *>(sv + (ps * RPP + rg) * ROW_BYTES);
+#pragma unroll
+                    for (int j = 0; j < CPL; j++) {
+                        float2 vp[EPC / 2];
+                        widen(vr[tl + RL * j], vp);
+#pragma unroll
+                        for (int g = 0; g < G; g++) {
+                            const float2 pp = make_float2(y[ps][g], y[ps][g]);
+#pragma unroll
+                            for (int e = 0; e < EPC / 2; e++)
+                                s.acc[g][j * EPC / 2 + e] = ffma2(pp, vp[e], s.acc[g][j * EPC / 2 + e]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // Warp state -> merge slot [G*D acc][mk G][lk G][me G][le G].
+    __device__ static void flush(State &s, float *slot, int lane) {
+        const int rg = lane / RL, tl = lane % RL;
+#pragma unroll
+        for (int g = 0; g < G; g++) {
+#pragma unroll
+            for (int o = RL; o < 32; o <<= 1) {
+                s.lk[g] += __shfl_xor_sync(0xFFFFFFFFu, s.lk[g], o);
+                s.le[g] += __shfl_xor_sync(0xFFFFFFFFu, s.le[g], o);
+            }
+            if constexpr (WITH_V) {
+#pragma unroll
+                for (int i = 0; i < DL / 2; i++) {
+#pragma unroll
+                    for (int o = RL; o < 32; o <<= 1) {
+                        s.acc[g][i].x += __shfl_xor_sync(0xFFFFFFFFu, s.acc[g][i].x, o);
+                        s.acc[g][i].y += __shfl_xor_sync(0xFFFFFFFFu, s.acc[g][i].y, o);
+                    }
+                }
+                if (rg == 0) {
+#pragma unroll
+                    for (int j = 0; j < CPL; j++)
+#pragma unroll
+                        for (int e = 0; e < EPC; e += 2) {
+                            const int d = (tl + RL * j) * EPC + e;
+                            slot[g * D + d] = s.acc[g][(j * EPC + e) / 2].x;
+                            slot[g * D + d + 1] = s.acc[g][(j * EPC + e) / 2].y;
+                        }
+                }
+            }
+            if (lane == 0) {
+                slot[G * D + g] = s.mk[g];
+                slot[G * D + G + g] = s.lk[g];
+                slot[G * D + 2 * G + g] = s.me[g];
+                slot[G * D + 3 * G + g] = s.le[g];
+            }
+        }
+    }
+
+    // Producer: the page's K (and V) rows are contiguous -- one bulk copy each.
+    __device__ static void issue(unsigned char *sk, bool load_v, int32_t phys, uint64_t *bar, const void *k_pool,
+                                 const void *v_pool, const CUtensorMap *, const CUtensorMap *, uint64_t pol) {
+        bulk_g2s(sk, (const unsigned char *)k_pool + (int64_t)phys * PAGE_BYTES, PAGE_BYTES, bar, pol);
+        if (load_v)
+            bulk_g2s(sk + PAGE_BYTES, (const unsigned char *)v_pool + (int64_t)phys * PAGE_BYTES, PAGE_BYTES, bar,
+                     pol);
+    }
+};
+
+// ----------------------------------------------------------- tensor cores ----
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float bf16_lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Split (x0, x1) into bf16x2 high parts and bf16x2 residuals.
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(x0, x1);
+    lo = pack_bf16(x0 - bf16_lo_f(hi), x1 - bf16_hi_f(hi));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// D(rows 0-7) += A(rows 0-7) * B for m16n8k16 bf16 -> fp32; rows 8-15 of A
+// are zero, so only c0/c1 are carried (the other two outputs are dropped).
+__device__ __forceinline__ void mma_rows8(float &c0, float &c1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+    float d2, d3;
+    const uint32_t z = 0u;
+    const float fz = 0.0f;
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%11,%12,%13};"
+        : "=f"(c0), "=f"(c1), "=f"(d2), "=f"(d3)
+        : "r"(a0), "r"(z), "r"(a2), "r"(z), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(fz), "f"(fz));
+}
+
+template <int D, int G, bool WITH_V>
+struct MmaMath {
+    static_assert(G >= 1 && G <= 8, "query rows of one KV head must fit 8 MMA rows");
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int ROW_BYTES = D * 2;
+    static constexpr int PAGE_BYTES = PAGE * ROW_BYTES;
+    static constexpr int NBOX = D / 64;          // 128-byte lines per row (64 columns each)
+    static constexpr int KSTEPS = D / 16;
+    static constexpr int NT = D / 8;             // PV n-tiles of 8 columns
+    static constexpr int STAGE_ALIGN = 1024;     // 128-byte swizzle atoms
+    static constexpr bool USES_TMAP = true;
+
+    struct State {
+        uint32_t qh[KSTEPS][2], ql[KSTEPS][2];   // A fragments a0, a2 of query row g = lane/4
+        float mk, lk, me, le;                     // stats of row g (lk, le: this lane's partial)
+        float o[WITH_V ? NT : 1][2];              // PV accumulators c0, c1 of row g
+    };
+
+    // A page lands as 16 rows x NBOX lines of 128 bytes (line L = row*NBOX +
+    // half) with the 16-byte chunks of each line XOR-swizzled by L mod 8.
+    __device__ static uint32_t swz(int r, int h, int c) {
+        const int L = r * NBOX + h;
+        return (uint32_t)(L * 128 + ((c ^ (L & 7)) << 4));
+    }
+
+    __device__ static void load_q(State &s, const float *qs, float qscale, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ks++) {
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int d = ks * 16 + h * 8 + 2 * t;
+                float x0 = 0.0f, x1 = 0.0f;
+                if (g < G) {
+                    x0 = qs[g * D + d] * qscale;
+                    x1 = qs[g * D + d + 1] * qscale;
+                }
+                split_bf16(x0, x1, s.qh[ks][h], s.ql[ks][h]);
+            }
+        }
+        s.mk = -INFINITY; s.lk = 0.0f; s.me = -INFINITY; s.le = 0.0f;
+#pragma unroll
+        for (int i = 0; i < (WITH_V ? NT : 1); i++) s.o[i][0] = s.o[i][1] = 0.0f;
+    }
+
+    __device__ static void page(State &s, const unsigned char *sk, const unsigned char *sv, uint32_t keepm,
+                                uint32_t evm, int lane) {
+        const int t = lane & 3, mi = lane >> 3, r8 = lane & 7;
+        // ---- S = Q K^T for the 16 rows of the page (two n-tiles of 8 rows) ----
+        float s0[2] = {0.0f, 0.0f}, s1[2] = {0.0f, 0.0f};
+        const uint32_t kbase = smem_u32(sk);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS; ks++) {
+            const int r = (mi >> 1) * 8 + r8, ch = (ks & 3) * 2 + (mi & 1);
+            uint32_t b[4];
+            ldsm_x4(kbase + swz(r, ks >> 2, ch), b);
+            mma_rows8(s0[0], s0[1], s.qh[ks][0], s.qh[ks][1], b[0], b[1]);
+            mma_rows8(s0[0], s0[1], s.ql[ks][0], s.ql[ks][1], b[0], b[1]);
+            mma_rows8(s1[0], s1[1], s.qh[ks][0], s.qh[ks][1], b[2], b[3]);
+            mma_rows8(s1[0], s1[1], s.ql[ks][0], s.ql[ks][1], b[2], b[3]);
+        }
+        // this lane holds row g = lane/4 at page rows j = 2t, 2t+1, 2t+8, 2t+9
+        const float y[4] = {s0[0], s0[1], s1[0], s1[1]};
+        const int jr[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+        float pk = -INFINITY, pe = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            if ((keepm >> jr[i]) & 1u) pk = fmaxf(pk, y[i]);
+            if ((evm >> jr[i]) & 1u) pe = fmaxf(pe, y[i]);
+        }
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            pk = fmaxf(pk, __shfl_xor_sync(0xFFFFFFFFu, pk, o));
+            pe = fmaxf(pe, __shfl_xor_sync(0xFFFFFFFFu, pe, o));
+        }
+        if (evm) {
+            const float mn = fmaxf(s.me, pe);
+            float sum = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                if ((evm >> jr[i]) & 1u) sum += ex2(y[i] - mn);
+            s.le = s.le * ex2(s.me - mn) + sum;  // me = -inf -> 0
+            s.me = mn;
+        }
+        if (!keepm) return;
+        const float mn = fmaxf(s.mk, pk);
+        const float alpha = ex2(s.mk - mn);  // mk = -inf -> 0
+        s.mk = mn;
+        float p[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) p[i] = ((keepm >> jr[i]) & 1u) ? ex2(y[i] - mn) : 0.0f;
+        s.lk = s.lk * alpha + (p[0] + p[1]) + (p[2] + p[3]);
+        if constexpr (WITH_V) {
+            if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+#pragma unroll
+                for (int i = 0; i < NT; i++) { s.o[i][0] *= alpha; s.o[i][1] *= alpha; }
+            }
+            uint32_t ph0, pl0, ph2, pl2;
+            split_bf16(p[0], p[1], ph0, pl0);
+            split_bf16(p[2], p[3], ph2, pl2);
+            const uint32_t vbase = smem_u32(sv);
+#pragma unroll
+            for (int np = 0; np < NT / 2; np++) {
+                const int r = (mi & 1) * 8 + r8, ch = (np & 3) * 2 + (mi >> 1);
+                uint32_t b[4];
+                ldsm_x4_t(vbase + swz(r, np >> 2, ch), b);
+                mma_rows8(s.o[2 * np][0], s.o[2 * np][1], ph0, ph2, b[0], b[1]);
+                mma_rows8(s.o[2 * np][0], s.o[2 * np][1], pl0, pl2, b[0], b[1]);
+                mma_rows8(s.o[2 * np + 1][0], s.o[2 * np + 1][1], ph0, ph2, b[2], b[3]);
+                mma_rows8(s.o[2 * np + 1][0], s.o[2 * np + 1][1], pl0, pl2, b[2], b[3]);
+            }
+        }
+    }
+
+    __device__ static void flush(State &s, float *slot, int lane) {
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) {
+            s.lk += __shfl_xor_sync(0xFFFFFFFFu, s.lk, o);
+            s.le += __shfl_xor_sync(0xFFFFFFFFu, s.le, o);
+        }
+        if (g < G) {
+            if constexpr (WITH_V) {
+#pragma unroll
+                for (int i = 0; i < NT; i++) {
+                    slot[g * D + i * 8 + 2 * t] = s.o[i][0];
+                    slot[g * D + i * 8 + 2 * t + 1] = s.o[i][1];
+                }
+            }
+            if (t == 0) {
+                slot[G * D + g] = s.mk;
+                slot[G * D + G + g] = s.lk;
+                slot[G * D + 2 * G + g] = s.me;
+                slot[G * D + 3 * G + g] = s.le;
+            }
+        }
+    }
+
+    // Producer: one 3-D tensor box (64 columns x NBOX lines x 16 rows) per
+    // page of K (and of V), 128-byte swizzled.
+    __device__ static void issue(unsigned char *sk, bool load_v, int32_t phys, uint64_t *bar, const void *,
+                                 const void *, const CUtensorMap *tk, const CUtensorMap *tv, uint64_t pol) {
+        tma_load_3d(sk, tk, 0, 0, phys * PAGE, bar, pol);
+        if (load_v) tma_load_3d(sk + PAGE_BYTES, tv, 0, 0, phys * PAGE, bar, pol);
+    }
+};
+
+// ------------------------------------------------------------- skeleton ----
+template <class M, int D, int G, bool WITH_V>
+struct Layout {
+    static constexpr int STAGE_BYTES = M::PAGE_BYTES * (WITH_V ? 2 : 1);
+#ifdef RKV_STAGE_BYTES_BUDGET
+    static constexpr int BUDGET = RKV_STAGE_BYTES_BUDGET;
+#else
+    static constexpr int BUDGET = 131072;
+#endif
+    static constexpr int NSW0 = BUDGET / (NCW * STAGE_BYTES);
+    static constexpr int NSW = NSW0 < 1 ? 1 : (NSW0 > 8 ? 8 : NSW0);   // stages per consumer warp
+    static constexpr int NST = NCW * NSW;
     static constexpr int QBYTES = G * D * 4;
     static constexpr int REC = G * (D + 4);                   // partial record floats
     static constexpr int WSLOT = G * D + 4 * G;               // per-warp merge slot floats
-    // shared-memory layout (bytes)
     static constexpr int OFF_STAGE = 0;
     static constexpr int OFF_Q = OFF_STAGE + NST * STAGE_BYTES;
     static constexpr int OFF_MERGE = OFF_Q + QR * QBYTES;
     static constexpr int OFF_META = OFF_MERGE + 2 * NCW * WSLOT * 4;
     static constexpr int OFF_BAR = (OFF_META + NST * 4 + 15) / 16 * 16;
-    static constexpr int OFF_MISC = OFF_BAR + (2 * NST + 2 * QR) * 8;
-    static constexpr int SMEM = OFF_MISC + 128;
-    static_assert(CHUNKS % RL == 0 && 32 % RL == 0, "lane mapping");
-    static_assert(ROW_BYTES % 16 == 0, "rows must be 16-byte multiples");
+    static constexpr int NBAR = 2 * NST + 2 * QR;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 128 + M::STAGE_ALIGN;  // + slack to align the stages
     static_assert(QBYTES % 16 == 0, "query block must be a 16-byte multiple");
+    static_assert(STAGE_BYTES % M::STAGE_ALIGN == 0, "stage alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
+    static_assert(NBAR <= ATTN_THREADS, "barrier init");
 };
 
 // Walks the heads this CTA owns, in order.  A head c with pages = ceil(len/16)
@@ -85,7 +475,6 @@ struct Walker {
     __device__ void init(const int32_t *len_, int C_, int64_t x1_, bool last_, int c0, int64_t pfx0) {
         len = len_; C = C_; x1 = x1_; last = last_; c = c0; pfx = pfx0; cbuf = -64; lbuf = 0;
     }
-    // Returns false when done; else the next head and its first page / pages.
     __device__ bool next(int *hc, int64_t *hpfx, int *hpages, int *hlen) {
         if (c >= C) return false;
         if (c < cbuf || c >= cbuf + 32) {
@@ -114,7 +503,6 @@ __device__ __forceinline__ int owner_of(int64_t x, int64_t TP, int n) {
     return j;
 }
 
-// Combine per-source (m_k, l_k, m_e, l_e, acc) states; m in base-2 units.
 struct Merged {
     float mk, lk, me, le;
 };
@@ -127,19 +515,27 @@ __device__ __forceinline__ float dm_of(const Merged &s) {
     return b / (a + b);
 }
 
-template <typename T, int D, int G, bool WITH_V>
-__global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
-    using CF = Cfg<T, D, G, WITH_V>;
-    extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + CF::OFF_BAR);
-    uint64_t *empty = full + CF::NST;
-    uint64_t *qfull = empty + CF::NST;
+// Pages are dealt to consumer warps round-robin (page li -> warp li % NCW);
+// each consumer warp owns a private ring of NSW stages, filled in order by
+// the producer warp serving it (warp w is served by producer w % NPW), so
+// every mbarrier has exactly one producer and one consumer and a phase is
+// never waited on before the previous phase of the same stage completed.
+template <class M, int D, int G, bool WITH_V>
+__global__ void __launch_bounds__(ATTN_THREADS, 1)
+    attn_kernel(AttnArgs a, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    using LY = Layout<M, D, G, WITH_V>;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((M::STAGE_ALIGN - (smem_u32(smem_raw) & (M::STAGE_ALIGN - 1))) &
+                                      (M::STAGE_ALIGN - 1));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + LY::OFF_BAR);  // [NCW][NSW]
+    uint64_t *empty = full + LY::NST;                                   // [NCW][NSW]
+    uint64_t *qfull = empty + LY::NST;
     uint64_t *qempty = qfull + QR;
-    uint32_t *meta = reinterpret_cast<uint32_t *>(smem + CF::OFF_META);
-    float *qring = reinterpret_cast<float *>(smem + CF::OFF_Q);
-    float *merge = reinterpret_cast<float *>(smem + CF::OFF_MERGE);
-    int *misc = reinterpret_cast<int *>(smem + CF::OFF_MISC);
-    int64_t *misc64 = reinterpret_cast<int64_t *>(smem + CF::OFF_MISC + 64);
+    uint32_t *meta = reinterpret_cast<uint32_t *>(smem + LY::OFF_META);
+    float *qring = reinterpret_cast<float *>(smem + LY::OFF_Q);
+    float *merge = reinterpret_cast<float *>(smem + LY::OFF_MERGE);
+    int *misc = reinterpret_cast<int *>(smem + LY::OFF_MISC);
+    int64_t *misc64 = reinterpret_cast<int64_t *>(smem + LY::OFF_MISC + 64);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nct = gridDim.x;
@@ -151,9 +547,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     uint32_t my_pages = 0;
     for (int c = h0; c < h1; c++) my_pages += (uint32_t)((max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE);
     if (tid == 0) misc[0] = a.C;
-    if (tid < 2 * CF::NST + 2 * QR) {
-        // full/empty: one arrival (producer / consuming warp); qfull: producer; qempty: every consumer warp
-        mbar_init(full + tid, tid >= 2 * CF::NST + QR ? NCW : 1);
+    if (tid < LY::NBAR) {
+        // full: producer; empty: the owning consumer warp; qfull: producer 0; qempty: every consumer warp
+        mbar_init(full + tid, tid >= 2 * LY::NST + QR ? NCW : 1);
+    }
+    if (M::USES_TMAP && tid == 0) {
+        prefetch_tensormap(&tmk);
+        prefetch_tensormap(&tmv);
     }
     uint32_t TPu;
     const uint32_t my_pfx = block_exclusive_scan(my_pages, scan + 64, &TPu);
@@ -179,8 +579,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     const int c_start = misc[0];
     const int64_t pfx_start = c_start < a.C ? misc64[0] : TP;
 
-    if (warp == NCW) {
-        // =============================== producer ===============================
+    if (warp >= NCW) {
+        // =============================== producers ===============================
+        const int pw = warp - NCW;
         Walker w;
         w.init(a.len, a.C, x1, last, c_start, pfx_start);
         const uint64_t pol_kv = policy_evict_first();
@@ -191,18 +592,19 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         while (w.next(&c, &pfx, &pages, &n)) {
             if (pages == 0) continue;
             const int64_t pa = max(pfx, x0), pb = min(pfx + pages, x1);
-            if (lane == 0) {
+            if (pw == 0 && lane == 0) {
                 const int slot = nq % QR;
                 mbar_wait(&qempty[slot], ((nq / QR) & 1) ^ 1, a.status);
-                mbar_arrive_expect_tx(&qfull[slot], CF::QBYTES);
-                bulk_g2s(qring + slot * G * D, a.q + (int64_t)c * G * D, CF::QBYTES, &qfull[slot], pol_q);
+                mbar_arrive_expect_tx(&qfull[slot], LY::QBYTES);
+                bulk_g2s(qring + slot * G * D, a.q + (int64_t)c * G * D, LY::QBYTES, &qfull[slot], pol_q);
             }
             nq++;
             for (int64_t base = pa; base < pb; base += 32) {
                 const int64_t i = base + lane;
                 int32_t phys = 0;
                 uint32_t m = 0;
-                if (i < pb) {
+                const bool mine = i < pb && ((int)((i - x0) % NCW)) % NPW == pw;
+                if (mine) {
                     const int64_t pidx = i - pfx;
                     phys = __ldg(a.block_table + (int64_t)c * a.max_pages + pidx);
                     const int nv = min(PAGE, n - (int)pidx * PAGE);
@@ -211,23 +613,23 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
                                                     : 0xFFFFu;
                     m = (kp & valid) | (valid << 16);
                 }
-                const int cnt = (int)min((int64_t)32, pb - base);
-                for (int j = 0; j < cnt; j++) {
+                uint32_t todo = __ballot_sync(0xFFFFFFFFu, mine);
+                while (todo) {
+                    const int j = __ffs(todo) - 1;
+                    todo &= todo - 1;
                     const int32_t pj = __shfl_sync(0xFFFFFFFFu, phys, j);
                     const uint32_t mj = __shfl_sync(0xFFFFFFFFu, m, j);
                     if (lane == 0) {
                         const int64_t li = base + j - x0;
-                        const int st = (int)(li % CF::NST);
-                        mbar_wait(&empty[st], (uint32_t)((li / CF::NST) & 1) ^ 1u, a.status);
-                        meta[st] = mj;
+                        const int cw = (int)(li % NCW);
+                        const int64_t nw = li / NCW;
+                        const int sg = cw * LY::NSW + (int)(nw % LY::NSW);
+                        mbar_wait(&empty[sg], (uint32_t)((nw / LY::NSW) & 1) ^ 1u, a.status);
+                        meta[sg] = mj;
                         const bool load_v = WITH_V && (mj & 0xFFFFu);
-                        mbar_arrive_expect_tx(&full[st], CF::PAGE_BYTES * (load_v ? 2 : 1));
-                        unsigned char *sk = smem + CF::OFF_STAGE + st * CF::STAGE_BYTES;
-                        bulk_g2s(sk, (const unsigned char *)a.k_pool + (int64_t)pj * CF::PAGE_BYTES, CF::PAGE_BYTES,
-                                 &full[st], pol_kv);
-                        if (load_v)
-                            bulk_g2s(sk + CF::PAGE_BYTES, (const unsigned char *)a.v_pool + (int64_t)pj * CF::PAGE_BYTES,
-                                     CF::PAGE_BYTES, &full[st], pol_kv);
+                        mbar_arrive_expect_tx(&full[sg], M::PAGE_BYTES * (load_v ? 2 : 1));
+                        M::issue(smem + LY::OFF_STAGE + sg * LY::STAGE_BYTES, load_v, pj, &full[sg], a.k_pool,
+                                 a.v_pool, &tmk, &tmv, pol_kv);
                     }
                     __syncwarp();
                 }
@@ -237,14 +639,13 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
     }
 
     // ================================ consumers ================================
-    constexpr int RL = CF::RL, DL = CF::DL, CPL = CF::CPL, EPC = CF::EPC, RPP = CF::RPP, NPASSES = CF::NPASSES;
-    const int rg = lane / RL, tl = lane % RL;
     Walker w;
     w.init(a.len, a.C, x1, last, c_start, pfx_start);
     int nq = 0;
     int c, pages, n;
     int64_t pfx;
     const int64_t TPl = TP;
+    typename M::State st;
 
     while (w.next(&c, &pfx, &pages, &n)) {
         if (pages == 0) {
@@ -261,226 +662,52 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
         }
         const int64_t pa = max(pfx, x0), pb = min(pfx + pages, x1);
         const bool whole = (pfx >= x0) && (pfx + pages <= x1);
-
-        // ---- this head's queries, pre-scaled to base-2 logits ----
-        float2 q2[G][DL / 2];
         {
             const int slot = nq % QR;
             mbar_wait(&qfull[slot], (nq / QR) & 1, a.status);
-            const float *qs = qring + slot * G * D;
-#pragma unroll
-            for (int g = 0; g < G; g++)
-#pragma unroll
-                for (int j = 0; j < CPL; j++)
-#pragma unroll
-                    for (int e = 0; e < EPC; e += 2) {
-                        const int d = (tl + RL * j) * EPC + e;
-                        q2[g][(j * EPC + e) / 2] = make_float2(qs[g * D + d] * a.qscale, qs[g * D + d + 1] * a.qscale);
-                    }
+            M::load_q(st, qring + slot * G * D, a.qscale, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&qempty[slot]);
         }
-        float mk[G], lk[G], me[G], le[G];
-        float2 acc[G][WITH_V ? DL / 2 : 1];
-#pragma unroll
-        for (int g = 0; g < G; g++) {
-            mk[g] = -INFINITY; lk[g] = 0.0f; me[g] = -INFINITY; le[g] = 0.0f;
-#pragma unroll
-            for (int i = 0; i < (WITH_V ? DL / 2 : 1); i++) acc[g][i] = make_float2(0.0f, 0.0f);
-        }
-
         // ---- pages of this head handled by this warp ----
         const int64_t la = pa - x0, lb = pb - x0;
-        int64_t li = la + (((int64_t)warp - la) % NCW + NCW) % NCW;
-        for (; li < lb; li += NCW) {
-            const int st = (int)(li % CF::NST);
-            mbar_wait(&full[st], (uint32_t)((li / CF::NST) & 1), a.status);
-            const uint32_t mt = meta[st];
-            const uint32_t keepm = mt & 0xFFFFu, validm = mt >> 16, evm = validm & ~keepm;
-            const unsigned char *sk = smem + CF::OFF_STAGE + st * CF::STAGE_BYTES;
-
-            // logits of this lane's rows (all-reduced over the RL lanes of a row)
-            float y[NPASSES][G];
-#pragma unroll
-            for (int ps = 0; ps < NPASSES; ps++) {
-                const int row = ps * RPP + rg;
-                const uint4 *kr = reinterpret_cast<const uint4 *>(sk + row * CF::ROW_BYTES);
-                float2 part[G];
-#pragma unroll
-                for (int g = 0; g < G; g++) part[g] = make_float2(0.0f, 0.0f);
-#pragma unroll
-                for (int j = 0; j < CPL; j++) {
-                    const uint4 wv = kr[tl + RL * j];
-                    float2 kp[EPC / 2];
-                    if constexpr (sizeof(T) == 2) {
-                        kp[0] = bf16x2_to_f2(wv.x); kp[1] = bf16x2_to_f2(wv.y);
-                        kp[2] = bf16x2_to_f2(wv.z); kp[3] = bf16x2_to_f2(wv.w);
-                    } else {
-                        kp[0] = make_float2(__uint_as_float(wv.x), __uint_as_float(wv.y));
-                        kp[1] = make_float2(__uint_as_float(wv.z), __uint_as_float(wv.w));
-                    }
-#pragma unroll
-                    for (int e = 0; e < EPC / 2; e++)
-#pragma unroll
-                        for (int g = 0; g < G; g++) part[g] = ffma2(q2[g][j * EPC / 2 + e], kp[e], part[g]);
-                }
-#pragma unroll
-                for (int g = 0; g < G; g++) {
-                    float s = part[g].x + part[g].y;
-#pragma unroll
-                    for (int o = 1; o < RL; o <<= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-                    y[ps][g] = s;
-                }
-            }
-
-            // dense stats of evicted rows, then the online softmax over kept rows
-#pragma unroll
-            for (int g = 0; g < G; g++) {
-                float pk = -INFINITY, pe = -INFINITY;
-#pragma unroll
-                for (int ps = 0; ps < NPASSES; ps++) {
-                    const int row = ps * RPP + rg;
-                    if ((keepm >> row) & 1u) pk = fmaxf(pk, y[ps][g]);
-                    if ((evm >> row) & 1u) pe = fmaxf(pe, y[ps][g]);
-                }
-#pragma unroll
-                for (int o = RL; o < 32; o <<= 1) {
-                    pk = fmaxf(pk, __shfl_xor_sync(0xFFFFFFFFu, pk, o));
-                    pe = fmaxf(pe, __shfl_xor_sync(0xFFFFFFFFu, pe, o));
-                }
-                if (evm) {
-                    const float mn = fmaxf(me[g], pe);
-                    float sum = 0.0f;
-#pragma unroll
-                    for (int ps = 0; ps < NPASSES; ps++) {
-                        const int row = ps * RPP + rg;
-                        if ((evm >> row) & 1u) sum += ex2(y[ps][g] - mn);
-                    }
-                    le[g] = le[g] * ex2(me[g] - mn) + (tl == 0 ? sum : 0.0f);  // me = -inf -> 0
-                    me[g] = mn;
-                }
-                if (keepm) {
-                    const float mn = fmaxf(mk[g], pk);
-                    const float alpha = ex2(mk[g] - mn);  // mk = -inf -> 0
-                    if (alpha != 1.0f) {
-                        lk[g] *= alpha;
-                        if constexpr (WITH_V) {
-#pragma unroll
-                            for (int i = 0; i < DL / 2; i++) { acc[g][i].x *= alpha; acc[g][i].y *= alpha; }
-                        }
-                    }
-                    mk[g] = mn;
-                    float sum = 0.0f;
-#pragma unroll
-                    for (int ps = 0; ps < NPASSES; ps++) {
-                        const int row = ps * RPP + rg;
-                        const float p = ((keepm >> row) & 1u) ? ex2(y[ps][g] - mn) : 0.0f;
-                        y[ps][g] = p;   // y now holds the kept weights
-                        sum += p;
-                    }
-                    lk[g] += (tl == 0) ? sum : 0.0f;
-                }
-            }
-
-            // PV over kept rows
-            if constexpr (WITH_V) {
-                if (keepm) {
-                    const unsigned char *sv = sk + CF::PAGE_BYTES;
-#pragma unroll
-                    for (int ps = 0; ps < NPASSES; ps++) {
-                        const int row = ps * RPP + rg;
-                        const uint4 *vr = reinterpret_cast<const uint4 *>(sv + row * CF::ROW_BYTES);
-#pragma unroll
-                        for (int j = 0; j < CPL; j++) {
-                            const uint4 wv = vr[tl + RL * j];
-                            float2 vp[EPC / 2];
-                            if constexpr (sizeof(T) == 2) {
-                                vp[0] = bf16x2_to_f2(wv.x); vp[1] = bf16x2_to_f2(wv.y);
-                                vp[2] = bf16x2_to_f2(wv.z); vp[3] = bf16x2_to_f2(wv.w);
-                            } else {
-                                vp[0] = make_float2(__uint_as_float(wv.x), __uint_as_float(wv.y));
-                                vp[1] = make_float2(__uint_as_float(wv.z), __uint_as_float(wv.w));
-                            }
-#pragma unroll
-                            for (int g = 0; g < G; g++) {
-                                const float2 pp = make_float2(y[ps][g], y[ps][g]);
-#pragma unroll
-                                for (int e = 0; e < EPC / 2; e++)
-                                    acc[g][j * EPC / 2 + e] = ffma2(pp, vp[e], acc[g][j * EPC / 2 + e]);
-                            }
-                        }
-                    }
-                }
-            }
+        for (int64_t li = la + (((int64_t)warp - la) % NCW + NCW) % NCW; li < lb; li += NCW) {
+            const int64_t nw = li / NCW;
+            const int sg = warp * LY::NSW + (int)(nw % LY::NSW);
+            mbar_wait(&full[sg], (uint32_t)((nw / LY::NSW) & 1), a.status);
+            const uint32_t mt = meta[sg];
+            const uint32_t keepm = mt & 0xFFFFu, evm = (mt >> 16) & ~keepm;
+            const unsigned char *sk = smem + LY::OFF_STAGE + sg * LY::STAGE_BYTES;
+#ifndef EXP_SKIP_MATH
+            M::page(st, sk, sk + M::PAGE_BYTES, keepm, evm, lane);
+#endif
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
+            if (lane == 0) mbar_arrive(&empty[sg]);
         }
-
-        // ---- warp state -> shared merge slot ----
         const int par = nq & 1;
-        float *ws_slot = merge + (par * NCW + warp) * CF::WSLOT;
-#pragma unroll
-        for (int g = 0; g < G; g++) {
-#pragma unroll
-            for (int o = RL; o < 32; o <<= 1) {
-                lk[g] += __shfl_xor_sync(0xFFFFFFFFu, lk[g], o);
-                le[g] += __shfl_xor_sync(0xFFFFFFFFu, le[g], o);
-            }
-            // lk/le were accumulated by lane tl == 0 of each row group only
-            if constexpr (WITH_V) {
-#pragma unroll
-                for (int i = 0; i < DL / 2; i++) {
-#pragma unroll
-                    for (int o = RL; o < 32; o <<= 1) {
-                        acc[g][i].x += __shfl_xor_sync(0xFFFFFFFFu, acc[g][i].x, o);
-                        acc[g][i].y += __shfl_xor_sync(0xFFFFFFFFu, acc[g][i].y, o);
-                    }
-                }
-                if (rg == 0) {
-#pragma unroll
-                    for (int j = 0; j < CPL; j++)
-#pragma unroll
-                        for (int e = 0; e < EPC; e += 2) {
-                            const int d = (tl + RL * j) * EPC + e;
-                            ws_slot[g * D + d] = acc[g][(j * EPC + e) / 2].x;
-                            ws_slot[g * D + d + 1] = acc[g][(j * EPC + e) / 2].y;
-                        }
-                }
-            }
-            if (lane == 0) {
-                ws_slot[G * D + g] = mk[g];
-                ws_slot[G * D + G + g] = lk[g];
-                ws_slot[G * D + 2 * G + g] = me[g];
-                ws_slot[G * D + 3 * G + g] = le[g];
-            }
-        }
+        M::flush(st, merge + (par * NCW + warp) * LY::WSLOT, lane);
         nq++;
         named_bar_sync(1, NCW * 32);
 
         // ---- merge the warps (consumer threads 0 .. NCW*32-1) ----
-        const int ctid = tid;  // consumers are warps 0..NCW-1
-        const float *mb = merge + par * NCW * CF::WSLOT;
+        const float *mb = merge + par * NCW * LY::WSLOT;
         float *rec = nullptr;
-        int slot_rec = 0;
-        if (!whole) {
-            slot_rec = (pfx < x0) ? 0 : 1;
-            rec = a.partial + ((int64_t)blockIdx.x * 2 + slot_rec) * CF::REC;
-        }
-        for (int e = ctid; e < G * D + G; e += NCW * 32) {
+        if (!whole) rec = a.partial + ((int64_t)blockIdx.x * 2 + ((pfx < x0) ? 0 : 1)) * LY::REC;
+        for (int e = tid; e < G * D + G; e += NCW * 32) {
             const bool is_stat = e >= G * D;
             const int g = is_stat ? e - G * D : e / D;
             Merged s;
             s.mk = -INFINITY; s.me = -INFINITY;
 #pragma unroll
             for (int wi = 0; wi < NCW; wi++) {
-                s.mk = fmaxf(s.mk, mb[wi * CF::WSLOT + G * D + g]);
-                s.me = fmaxf(s.me, mb[wi * CF::WSLOT + G * D + 2 * G + g]);
+                s.mk = fmaxf(s.mk, mb[wi * LY::WSLOT + G * D + g]);
+                s.me = fmaxf(s.me, mb[wi * LY::WSLOT + G * D + 2 * G + g]);
             }
             s.lk = 0.0f; s.le = 0.0f;
             float av = 0.0f;
 #pragma unroll
             for (int wi = 0; wi < NCW; wi++) {
-                const float *src = mb + wi * CF::WSLOT;
+                const float *src = mb + wi * LY::WSLOT;
                 const float mkw = src[G * D + g], mew = src[G * D + 2 * G + g];
                 const float fk = (mkw == -INFINITY) ? 0.0f : ex2(mkw - s.mk);
                 const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
@@ -511,7 +738,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
             __threadfence();
             named_bar_sync(1, NCW * 32);
             const int jf = owner_of(pfx, TPl, nct), jl = owner_of(pfx + pages - 1, TPl, nct);
-            if (ctid == 0) {
+            if (tid == 0) {
                 int ncover = 0;
                 for (int j = jf; j <= jl; j++) ncover += range_lo(j, TPl, nct) < range_lo(j + 1, TPl, nct) ? 1 : 0;
                 const uint32_t prev = atomicAdd(a.head_cnt + c, 1u);
@@ -520,21 +747,21 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
             named_bar_sync(1, NCW * 32);
             if (misc[4]) {
                 __threadfence();
-                for (int e = ctid; e < G * D + G; e += NCW * 32) {
+                for (int e = tid; e < G * D + G; e += NCW * 32) {
                     const bool is_stat = e >= G * D;
                     const int g = is_stat ? e - G * D : e / D;
                     Merged s;
                     s.mk = -INFINITY; s.me = -INFINITY; s.lk = 0.0f; s.le = 0.0f;
                     for (int j = jf; j <= jl; j++) {
                         if (!(range_lo(j, TPl, nct) < range_lo(j + 1, TPl, nct))) continue;
-                        const float *r = a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, TPl, nct)) ? 0 : 1)) * CF::REC;
+                        const float *r = a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, TPl, nct)) ? 0 : 1)) * LY::REC;
                         s.mk = fmaxf(s.mk, __ldcg(r + G * D + g));
                         s.me = fmaxf(s.me, __ldcg(r + G * D + 2 * G + g));
                     }
                     float av = 0.0f;
                     for (int j = jf; j <= jl; j++) {
                         if (!(range_lo(j, TPl, nct) < range_lo(j + 1, TPl, nct))) continue;
-                        const float *r = a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, TPl, nct)) ? 0 : 1)) * CF::REC;
+                        const float *r = a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, TPl, nct)) ? 0 : 1)) * LY::REC;
                         const float mkw = __ldcg(r + G * D + g), mew = __ldcg(r + G * D + 2 * G + g);
                         const float fk = (mkw == -INFINITY) ? 0.0f : ex2(mkw - s.mk);
                         const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
@@ -549,50 +776,57 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1) attn_kernel(AttnArgs a) {
                         if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
                     }
                 }
-                if (ctid == 0) a.head_cnt[c] = 0u;
+                if (tid == 0) a.head_cnt[c] = 0u;
             }
         }
     }
 }
 
-template <typename T, int D, int G, bool WITH_V>
-cudaError_t launch_one(const AttnArgs &a, int sm_count, cudaStream_t s) {
-    using CF = Cfg<T, D, G, WITH_V>;
-    auto *k = attn_kernel<T, D, G, WITH_V>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM);
+template <class M, int D, int G, bool WITH_V>
+cudaError_t launch_one(const AttnArgs &a, int sm_count, cudaStream_t s, const CUtensorMap &tk, const CUtensorMap &tv) {
+    using LY = Layout<M, D, G, WITH_V>;
+    auto *k = attn_kernel<M, D, G, WITH_V>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, LY::SMEM);
     if (e != cudaSuccess) return e;
-    int grid = sm_count < MAX_ATTN_CTAS ? sm_count : MAX_ATTN_CTAS;
-    k<<<grid, ATTN_THREADS, CF::SMEM, s>>>(a);
+    const int grid = sm_count < MAX_ATTN_CTAS ? sm_count : MAX_ATTN_CTAS;
+    k<<<grid, ATTN_THREADS, LY::SMEM, s>>>(a, tk, tv);
     return cudaGetLastError();
 }
 
-template <typename T, int D, int G>
-cudaError_t launch_dg(const AttnArgs &a, int sm_count, cudaStream_t s) {
-    return a.out ? launch_one<T, D, G, true>(a, sm_count, s) : launch_one<T, D, G, false>(a, sm_count, s);
+template <int DT, int D, int G>
+cudaError_t launch_dg(const AttnArgs &a, int sm_count, cudaStream_t s, const CUtensorMap &tk, const CUtensorMap &tv) {
+    if constexpr (DT == RKV_BF16) {
+        return a.out ? launch_one<MmaMath<D, G, true>, D, G, true>(a, sm_count, s, tk, tv)
+                     : launch_one<MmaMath<D, G, false>, D, G, false>(a, sm_count, s, tk, tv);
+    } else {
+        return a.out ? launch_one<CoreMath<float, D, G, true>, D, G, true>(a, sm_count, s, tk, tv)
+                     : launch_one<CoreMath<float, D, G, false>, D, G, false>(a, sm_count, s, tk, tv);
+    }
 }
 
-#define RKV_ATTN_CASES(X)                                                                              \
-    X(uint16_t, RKV_BF16, 128, 1) X(uint16_t, RKV_BF16, 128, 2) X(uint16_t, RKV_BF16, 128, 4)         \
-    X(uint16_t, RKV_BF16, 128, 7) X(uint16_t, RKV_BF16, 128, 8) X(uint16_t, RKV_BF16, 64, 1)          \
-    X(uint16_t, RKV_BF16, 64, 2) X(uint16_t, RKV_BF16, 64, 4) X(float, RKV_F32, 64, 1)                \
-    X(float, RKV_F32, 64, 2) X(float, RKV_F32, 64, 4) X(float, RKV_F32, 128, 1) X(float, RKV_F32, 128, 2) \
-    X(float, RKV_F32, 128, 4)
+#define RKV_ATTN_CASES(X)                                                                                  \
+    X(RKV_BF16, 128, 1) X(RKV_BF16, 128, 2) X(RKV_BF16, 128, 4) X(RKV_BF16, 128, 7) X(RKV_BF16, 128, 8)   \
+    X(RKV_BF16, 64, 1) X(RKV_BF16, 64, 2) X(RKV_BF16, 64, 4) X(RKV_F32, 64, 1) X(RKV_F32, 64, 2)          \
+    X(RKV_F32, 64, 4) X(RKV_F32, 128, 1) X(RKV_F32, 128, 2) X(RKV_F32, 128, 4)
 
 }  // namespace
 
 bool attn_supported(int dtype, int D, int G) {
-#define X(T, DT, DD, GG) \
+#define X(DT, DD, GG) \
     if (dtype == DT && D == DD && G == GG) return true;
     RKV_ATTN_CASES(X)
 #undef X
     return false;
 }
 
+bool attn_uses_tensor_maps(int dtype) { return dtype == RKV_BF16; }
+
 size_t attn_partial_rec_floats(int D, int G) { return (size_t)G * (D + 4); }
 
-cudaError_t launch_attn(const AttnArgs &a, int dtype, int D, int G, int sm_count, cudaStream_t s) {
-#define X(T, DT, DD, GG) \
-    if (dtype == DT && D == DD && G == GG) return launch_dg<T, DD, GG>(a, sm_count, s);
+cudaError_t launch_attn(const AttnArgs &a, int dtype, int D, int G, int sm_count, cudaStream_t s,
+                        const CUtensorMap &tk, const CUtensorMap &tv) {
+#define X(DT, DD, GG) \
+    if (dtype == DT && D == DD && G == GG) return launch_dg<DT, DD, GG>(a, sm_count, s, tk, tv);
     RKV_ATTN_CASES(X)
 #undef X
     return cudaErrorNotSupported;

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/rkv.h"
@@ -72,9 +73,13 @@ struct AttnArgs {
     int C, max_pages;
     float qscale;              // scale * log2(e)
 };
-// Returns cudaErrorNotSupported if (dtype, D, G) is not instantiated.
-cudaError_t launch_attn(const AttnArgs &a, int dtype, int D, int G, int sm_count, cudaStream_t s);
+// Returns cudaErrorNotSupported if (dtype, D, G) is not instantiated.  bf16
+// pools are read through the two tensor maps (64-column boxes of 16 rows,
+// 128-byte swizzle); fp32 pools ignore them.
+cudaError_t launch_attn(const AttnArgs &a, int dtype, int D, int G, int sm_count, cudaStream_t s,
+                        const CUtensorMap &tk, const CUtensorMap &tv);
 bool attn_supported(int dtype, int D, int G);
+bool attn_uses_tensor_maps(int dtype);
 size_t attn_partial_rec_floats(int D, int G);
 
 struct CompactArgs {
