@@ -85,11 +85,10 @@ void layout_for(const rkv_cache_t &c, int sel_groups_x_waves, WsLayout *L) {
     L->status = take(4, 4);
     L->done_compact = take(4, 4);
     L->done_append = take(4, 4);
-    L->sel_begin = take(0, 256);
-    L->bar = take(4, 4);
+    L->bar = take(4, 64);
+    L->leave = take(4, 64);
     L->more = take((size_t)c.B * NPASS * 4, 16);
     L->hist = take((size_t)sel_groups_x_waves * NPASS * NBINS * 4, 256);
-    L->sel_end = take(0, 256);
     L->head_cnt = take((size_t)C * 4, 256);
     L->partial = take((size_t)MAX_ATTN_CTAS * 2 * attn_partial_rec_floats(c.D, G) * 4, 256);
     L->total = take(0, 256);
@@ -199,9 +198,6 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
     SelectGrid g = select_grid_for(*cache, sms < MAX_SEL_CTAS ? sms : MAX_SEL_CTAS);
     if (g.cache_pages < 0) return fail(RKV_ERR_UNSUPPORTED, "L*H too large for the selection kernel");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t used_hist = (size_t)g.waves * g.n_groups * NPASS * NBINS * 4;
-    cudaError_t e = cudaMemsetAsync(at<unsigned char>(ws, L.sel_begin), 0, (L.hist - L.sel_begin) + used_hist, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(selection scratch)");
     SelectArgs a{};
     a.pos_pool = cache->pos_pool;
     a.lb_pool = cache->lb_pool;
@@ -222,13 +218,14 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
     a.plan = sel->plan;
     a.status = at<int32_t>(ws, L.status);
     a.bar = at<uint32_t>(ws, L.bar);
+    a.leave = at<uint32_t>(ws, L.leave);
     a.more = at<uint32_t>(ws, L.more);
     a.hist = at<uint32_t>(ws, L.hist);
     a.n_groups = g.n_groups;
     a.cta_per_group = g.cta_per_group;
     a.waves = g.waves;
     a.cache_pages = g.cache_pages;
-    e = launch_select(a, g, s);
+    cudaError_t e = launch_select(a, g, s);
     if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
     return RKV_OK;
 }

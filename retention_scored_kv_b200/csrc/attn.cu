@@ -40,7 +40,7 @@ namespace {
 #define RKV_NCW 8
 #endif
 #ifndef RKV_NPW
-#define RKV_NPW 2
+#define RKV_NPW 4
 #endif
 constexpr int NCW = RKV_NCW;           // consumer warps
 constexpr int NPW = RKV_NPW;           // producer warps (one issuing lane each)

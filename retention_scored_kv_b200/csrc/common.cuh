@@ -56,7 +56,7 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 }
 
 // Grid-wide barrier for a cooperative (co-resident) grid.  `count` is a
-// monotonically increasing arrival counter zeroed before the launch; barrier
+// monotonically increasing arrival counter, zero when the launch starts; barrier
 // number `epoch` (1, 2, ...) completes when count reaches epoch*gridDim.x.
 // The wait is bounded (~2 s of globaltimer); on timeout RKV_DEV_TIMEOUT is
 // recorded and false returned, so the caller can leave the kernel.
@@ -72,12 +72,11 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, in
             const uint64_t t0 = globaltimer_ns();
             uint32_t spins = 0;
             while (ld_acquire_gpu(count) < target) {
-                if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
+                if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
                     set_status(status, RKV_DEV_TIMEOUT);
                     ok = 0;
                     break;
                 }
-                __nanosleep(32);
             }
         }
         __threadfence();

@@ -15,11 +15,12 @@
 // offsets given by the per-head prefix the selection kernel computed, so the
 // result does not depend on scheduling order.
 //
-// Append: heads are split across CTAs; each CTA counts the page-needing heads
-// before its slice (len % 16 == 0), scans its own slice, pops pages from the
-// top of the stack in ascending head order, and warps copy the new rows.  The
-// last CTA to finish (atomic ticket, no waiting) bumps every length and the
-// stack top, so no CTA ever reads a length another CTA already changed.
+// Append: 32 heads per CTA; each CTA counts the page-needing heads before its
+// slice (len % 16 == 0), scans its own slice, pops pages from the top of the
+// stack in ascending head order, and warps store the new rows (loaded into
+// registers at kernel start).  The last CTA to finish (atomic ticket, no
+// waiting) bumps every length and the stack top, so no CTA ever reads a
+// length another CTA already changed.
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,30 +28,11 @@ namespace rkv {
 
 namespace {
 
-constexpr int CMP_THREADS = 256;
-constexpr int APP_THREADS = 256;
-
-__device__ __forceinline__ int64_t slot_row(const int32_t *table, int64_t c, int max_pages, int k) {
-    return (int64_t)__ldg(table + c * max_pages + k / PAGE) * PAGE + (k % PAGE);
-}
-
-// Warp-cooperative move of one row (K and V of row_bytes each, position,
-// log-retention) from physical row src to physical row dst.
-__device__ __forceinline__ void move_row(const CompactArgs &a, int64_t dst, int64_t src, int lane) {
-    const int chunks = a.row_bytes / 16;
-    uint4 *kd = reinterpret_cast<uint4 *>((unsigned char *)a.k_pool + dst * a.row_bytes);
-    const uint4 *ks = reinterpret_cast<const uint4 *>((const unsigned char *)a.k_pool + src * a.row_bytes);
-    uint4 *vd = reinterpret_cast<uint4 *>((unsigned char *)a.v_pool + dst * a.row_bytes);
-    const uint4 *vs = reinterpret_cast<const uint4 *>((const unsigned char *)a.v_pool + src * a.row_bytes);
-    for (int i = lane; i < 2 * chunks; i += 32) {
-        if (i < chunks) kd[i] = ks[i];
-        else vd[i - chunks] = vs[i - chunks];
-    }
-    if (lane == 0) {
-        a.pos_pool[dst] = a.pos_pool[src];
-        a.lb_pool[dst] = a.lb_pool[src];
-    }
-}
+constexpr int CMP_THREADS = 128;
+constexpr int CMP_PAIRS = 1024;   // hole/source pairs resolved per round
+constexpr int APP_THREADS = 128;  // 4 warps
+constexpr int APP_HEADS = 32;     // heads per append CTA (8 per warp)
+constexpr int MAX_ROW_CHUNKS = 32; // 16-byte chunks of one K (or V) row: D*elt <= 512 bytes
 
 __device__ __forceinline__ uint32_t below_bits(int w, int nn) {
     const int lo = w * PAGE;
@@ -59,135 +41,208 @@ __device__ __forceinline__ uint32_t below_bits(int w, int nn) {
     return (1u << (nn - lo)) - 1u;
 }
 
+// Block-wide exclusive scan over W words of a shared array, in place.
+__device__ void scan_words(int32_t *v, int W, uint32_t *scratch) {
+    uint32_t carry = 0;
+    for (int base = 0; base < W; base += blockDim.x) {
+        const int w = base + threadIdx.x;
+        const uint32_t x = w < W ? (uint32_t)v[w] : 0u;
+        uint32_t tot;
+        const uint32_t ex = block_exclusive_scan(x, scratch, &tot);
+        if (w < W) v[w] = (int32_t)(carry + ex);
+        carry += tot;
+    }
+    if (threadIdx.x == 0) v[W] = (int32_t)carry;
+    __syncthreads();
+}
+
+// One CTA per head.  The head's keep-mask words and block-table entries are
+// staged in shared memory with one round of independent loads; per-word hole
+// and source counts are scanned into ranks; pairs (j-th hole, j-th source) are
+// resolved in shared memory, then warps move the rows with every lane's
+// loads issued before its stores.
 __global__ void __launch_bounds__(CMP_THREADS) compact_kernel(CompactArgs a) {
     extern __shared__ __align__(16) int32_t cs[];
     __shared__ uint32_t scan[40];
+    __shared__ int2 pairs[CMP_PAIRS];
     const int64_t c = blockIdx.x;
     const int n = __ldg(a.n_pre + c), nn = __ldg(a.kept + c);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
     if (c == 0 && tid == 0) *a.free_top = __ldg(a.plan + a.C + 1) + __ldg(a.plan + a.C);
+    if (nn >= n) return;  // nothing evicted in this head (len unchanged)
     if (tid == 0) a.len[c] = nn;
-    if (nn >= n) return;  // nothing evicted in this head
 
     const int W = (n + PAGE - 1) / PAGE, Wn = (nn + PAGE - 1) / PAGE;
-    int32_t *src_pfx = cs;            // [W]
-    int32_t *hole_pfx = cs + W + 1;   // [W]
-    const uint16_t *mask = a.keep_mask + c * a.max_pages;
-    uint32_t carry_s = 0, carry_h = 0;
-    for (int base = 0; base < W; base += blockDim.x) {
-        const int w = base + tid;
-        uint32_t sc = 0, hc = 0;
-        if (w < W) {
-            const uint32_t valid = below_bits(w, n);
-            const uint32_t m = (uint32_t)__ldg(mask + w) & valid;
-            const uint32_t below = below_bits(w, nn);
-            sc = __popc(m & ~below & valid);
-            hc = __popc(~m & below & 0xFFFFu);
-        }
-        uint32_t ts, th;
-        const uint32_t es = block_exclusive_scan(sc, scan, &ts);
-        const uint32_t eh = block_exclusive_scan(hc, scan, &th);
-        if (w < W) {
-            src_pfx[w] = (int32_t)(carry_s + es);
-            hole_pfx[w] = (int32_t)(carry_h + eh);
-        }
-        carry_s += ts;
-        carry_h += th;
+    const int mp = a.max_pages;
+    int32_t *tbl = cs;                  // [W] page ids
+    uint16_t *msk = reinterpret_cast<uint16_t *>(cs + mp);   // [W] keep words (valid bits only)
+    int32_t *src_pfx = cs + mp + (mp + 1) / 2 + 1;           // [W + 1]
+    int32_t *hole_pfx = src_pfx + mp + 1;                    // [W + 1]
+    const uint16_t *mask = a.keep_mask + c * mp;
+    for (int w = tid; w < W; w += blockDim.x) {
+        tbl[w] = a.block_table[c * mp + w];
+        msk[w] = (uint16_t)((uint32_t)__ldg(mask + w) & below_bits(w, n));
     }
     __syncthreads();
+    for (int w = tid; w < W; w += blockDim.x) {
+        const uint32_t m = msk[w], below = below_bits(w, nn);
+        src_pfx[w] = __popc(m & ~below);
+        hole_pfx[w] = __popc(~m & below & 0xFFFFu);
+    }
+    __syncthreads();
+    scan_words(src_pfx, W, scan);
+    scan_words(hole_pfx, W, scan);
+    const int moves = hole_pfx[W];
+    const int chunks = a.row_bytes / 16;
 
-    // hole j <- source j
-    for (int w = warp; w < Wn; w += nwarp) {
-        const uint32_t m = (uint32_t)__ldg(mask + w) & below_bits(w, n);
-        uint32_t hb = ~m & below_bits(w, nn) & 0xFFFFu;
-        int rank = hole_pfx[w];
-        while (hb) {
-            const int bit = __ffs(hb) - 1;
-            hb &= hb - 1;
-            // word holding the rank-th source: largest w' with src_pfx[w'] <= rank
-            int lo = 0, hi = W - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (src_pfx[mid] <= rank) lo = mid; else hi = mid - 1;
+    for (int r0 = 0; r0 < moves; r0 += CMP_PAIRS) {
+        const int r1 = min(moves, r0 + CMP_PAIRS);
+        // resolve pairs with rank in [r0, r1): thread per hole word
+        for (int w = tid; w < Wn; w += blockDim.x) {
+            int rank = hole_pfx[w];
+            if (rank >= r1 || hole_pfx[w + 1] <= r0) continue;
+            uint32_t hb = ~(uint32_t)msk[w] & below_bits(w, nn) & 0xFFFFu;
+            while (hb) {
+                const int bit = __ffs(hb) - 1;
+                hb &= hb - 1;
+                if (rank >= r0 && rank < r1) {
+                    int lo = 0, hi = W - 1;  // word of the rank-th source: last w' with src_pfx[w'] <= rank
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (src_pfx[mid] <= rank) lo = mid; else hi = mid - 1;
+                    }
+                    uint32_t sb = (uint32_t)msk[lo] & ~below_bits(lo, nn);
+                    for (int i = rank - src_pfx[lo]; i > 0; i--) sb &= sb - 1;
+                    const int hslot = w * PAGE + bit, sslot = lo * PAGE + (__ffs(sb) - 1);
+                    pairs[rank - r0] = make_int2((int)((int64_t)tbl[hslot / PAGE] * PAGE + hslot % PAGE),
+                                                 (int)((int64_t)tbl[sslot / PAGE] * PAGE + sslot % PAGE));
+                }
+                rank++;
             }
-            const uint32_t sm = (uint32_t)__ldg(mask + lo) & below_bits(lo, n) & ~below_bits(lo, nn);
-            int skip = rank - src_pfx[lo];
-            uint32_t sb = sm;
-            for (int i = 0; i < skip; i++) sb &= sb - 1;
-            const int sbit = __ffs(sb) - 1;
-            const int hslot = w * PAGE + bit, sslot = lo * PAGE + sbit;
-            move_row(a, slot_row(a.block_table, c, a.max_pages, hslot), slot_row(a.block_table, c, a.max_pages, sslot),
-                     lane);
-            rank++;
         }
+        __syncthreads();
+        // move rows: each warp takes pairs; a row is K chunks then V chunks
+        for (int pi = warp; pi < r1 - r0; pi += nwarp) {
+            const int64_t dst = pairs[pi].x, src = pairs[pi].y;
+            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+            const int i0 = lane, i1 = lane + 32;
+            const uint4 *ks = reinterpret_cast<const uint4 *>((const unsigned char *)a.k_pool + src * a.row_bytes);
+            const uint4 *vs = reinterpret_cast<const uint4 *>((const unsigned char *)a.v_pool + src * a.row_bytes);
+            if (i0 < 2 * chunks) v0 = i0 < chunks ? ks[i0] : vs[i0 - chunks];
+            if (i1 < 2 * chunks) v1 = i1 < chunks ? ks[i1] : vs[i1 - chunks];
+            int32_t pos = 0;
+            float lbv = 0.0f;
+            if (lane == 0) { pos = a.pos_pool[src]; lbv = a.lb_pool[src]; }
+            uint4 *kd = reinterpret_cast<uint4 *>((unsigned char *)a.k_pool + dst * a.row_bytes);
+            uint4 *vd = reinterpret_cast<uint4 *>((unsigned char *)a.v_pool + dst * a.row_bytes);
+            if (i0 < 2 * chunks) { if (i0 < chunks) kd[i0] = v0; else vd[i0 - chunks] = v0; }
+            if (i1 < 2 * chunks) { if (i1 < chunks) kd[i1] = v1; else vd[i1 - chunks] = v1; }
+            if (lane == 0) { a.pos_pool[dst] = pos; a.lb_pool[dst] = lbv; }
+        }
+        __syncthreads();
     }
-    __syncthreads();
     // freed pages, ascending table index, at this head's offset in the stack
     const int top0 = __ldg(a.plan + a.C + 1), off = __ldg(a.plan + c);
     for (int pi = Wn + tid; pi < W; pi += blockDim.x) {
-        int32_t *e = a.block_table + c * a.max_pages + pi;
-        a.free_stack[top0 + off + (pi - Wn)] = *e;
-        *e = -1;
+        a.free_stack[top0 + off + (pi - Wn)] = tbl[pi];
+        a.block_table[c * mp + pi] = -1;
     }
 }
 
+// APP_HEADS heads per CTA.  Every independent load is issued first: the
+// lengths before this slice (pages needed by earlier heads), this slice's
+// lengths, the stack top, and the new rows themselves (into registers).
+// Pops are ranked by an exclusive scan; the last CTA to finish (atomic
+// ticket, no waiting) bumps every length and lowers the stack top.
 __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
     __shared__ uint32_t scan[40];
-    __shared__ int64_t rows[APP_THREADS];
+    __shared__ int64_t rows[APP_HEADS];
     __shared__ int last_flag;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
-    const int c0 = blockIdx.x * blockDim.x;
-    const int c = c0 + tid;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c0 = blockIdx.x * APP_HEADS;
+    const int chunks = a.row_bytes / 16;                 // <= MAX_ROW_CHUNKS
+    constexpr int HPW = APP_HEADS / (APP_THREADS / 32);  // heads per warp
     const int top = __ldcg(a.free_top);
-    // page-needing heads before this CTA's slice
     uint32_t before = 0;
     for (int cc = tid; cc < c0; cc += blockDim.x) before += (__ldcg(a.len + cc) % PAGE == 0) ? 1u : 0u;
+    int k = 0, tb = 0;
+    float lbn = 0.0f;
+    const int c = c0 + lane;
+    const bool mine = warp == 0 && c < a.C;
+    if (mine) {
+        k = __ldcg(a.len + c);
+        tb = __ldg(a.t + c / a.LH);
+        lbn = __ldg(a.lb_new + c);
+    }
+    // this warp's new rows, chunk i of head h in lane (i % 32), slot i / 32
+    uint4 buf[HPW][2];
+#pragma unroll
+    for (int h = 0; h < HPW; h++) {
+        const int64_t ch = c0 + warp * HPW + h;
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+            const int i = lane + 32 * j;
+            buf[h][j] = make_uint4(0, 0, 0, 0);
+            if (ch < a.C && i < 2 * chunks) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    (const unsigned char *)(i < chunks ? a.k_new : a.v_new) + ch * a.row_bytes);
+                buf[h][j] = __ldg(src + (i < chunks ? i : i - chunks));
+            }
+        }
+    }
     uint32_t tot_before;
     block_exclusive_scan(before, scan, &tot_before);
-    int k = 0;
-    uint32_t need = 0;
-    if (c < a.C) {
-        k = __ldcg(a.len + c);
-        need = (k % PAGE == 0) ? 1u : 0u;
+    const uint32_t need = (mine && k % PAGE == 0) ? 1u : 0u;
+    uint32_t ex = 0;
+    {
+        // exclusive scan of need over warp 0
+        uint32_t x = need;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+            if (lane >= o) x += y;
+        }
+        ex = x - need;
     }
-    uint32_t tot_local;
-    const uint32_t ex = block_exclusive_scan(need, scan, &tot_local);
-    int64_t row = -1;
-    if (c < a.C) {
-        const int pidx = k / PAGE;
-        if (pidx >= a.max_pages) {
-            set_status(a.status, RKV_DEV_TABLE_OVERFLOW);
-        } else if (need) {
-            const int idx = top - 1 - (int)(tot_before + ex);
-            if (idx < 0) {
-                set_status(a.status, RKV_DEV_POOL_EXHAUSTED);
+    if (warp == 0) {
+        int64_t row = -1;
+        if (mine) {
+            const int pidx = k / PAGE;
+            if (pidx >= a.max_pages) {
+                set_status(a.status, RKV_DEV_TABLE_OVERFLOW);
+            } else if (need) {
+                const int idx = top - 1 - (int)(tot_before + ex);
+                if (idx < 0) {
+                    set_status(a.status, RKV_DEV_POOL_EXHAUSTED);
+                } else {
+                    const int32_t page = __ldcg(a.free_stack + idx);
+                    a.block_table[(int64_t)c * a.max_pages + pidx] = page;
+                    row = (int64_t)page * PAGE + (k % PAGE);
+                }
             } else {
-                const int32_t page = __ldcg(a.free_stack + idx);
-                a.block_table[(int64_t)c * a.max_pages + pidx] = page;
-                row = (int64_t)page * PAGE + (k % PAGE);
+                row = (int64_t)__ldcg(a.block_table + (int64_t)c * a.max_pages + pidx) * PAGE + (k % PAGE);
             }
-        } else {
-            row = (int64_t)__ldcg(a.block_table + (int64_t)c * a.max_pages + pidx) * PAGE + (k % PAGE);
+            if (row >= 0) {
+                a.pos_pool[row] = tb;
+                a.lb_pool[row] = lbn;
+            }
         }
-        if (row >= 0) {
-            a.pos_pool[row] = __ldg(a.t + c / a.LH);
-            a.lb_pool[row] = __ldg(a.lb_new + c);
-        }
+        rows[lane] = row;
     }
-    rows[tid] = row;
     __syncthreads();
-    const int chunks = a.row_bytes / 16;
-    for (int h = warp; h < (int)blockDim.x; h += nwarp) {
-        const int64_t r = rows[h];
-        const int64_t ch = c0 + h;
-        if (r < 0 || ch >= a.C) continue;
-        uint4 *kd = reinterpret_cast<uint4 *>((unsigned char *)a.k_pool + r * a.row_bytes);
-        uint4 *vd = reinterpret_cast<uint4 *>((unsigned char *)a.v_pool + r * a.row_bytes);
-        const uint4 *ks = reinterpret_cast<const uint4 *>((const unsigned char *)a.k_new + ch * a.row_bytes);
-        const uint4 *vs = reinterpret_cast<const uint4 *>((const unsigned char *)a.v_new + ch * a.row_bytes);
-        for (int i = lane; i < 2 * chunks; i += 32) {
-            if (i < chunks) kd[i] = __ldg(ks + i);
-            else vd[i - chunks] = __ldg(vs + i - chunks);
+#pragma unroll
+    for (int h = 0; h < HPW; h++) {
+        const int hl = warp * HPW + h;
+        const int64_t r = rows[hl];
+        if (r < 0 || c0 + hl >= a.C) continue;
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+            const int i = lane + 32 * j;
+            if (i < 2 * chunks) {
+                uint4 *dst = reinterpret_cast<uint4 *>((unsigned char *)(i < chunks ? a.k_pool : a.v_pool) +
+                                                       r * a.row_bytes);
+                dst[i < chunks ? i : i - chunks] = buf[h][j];
+            }
         }
     }
     // last CTA to finish: every length +1, stack top lowered by the pops
@@ -199,9 +254,9 @@ __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
     __threadfence();
     uint32_t pops = 0;
     for (int cc = tid; cc < a.C; cc += blockDim.x) {
-        const int32_t n = __ldcg(a.len + cc);
-        pops += (n % PAGE == 0) ? 1u : 0u;
-        a.len[cc] = n + 1;
+        const int32_t nl = __ldcg(a.len + cc);
+        pops += (nl % PAGE == 0) ? 1u : 0u;
+        a.len[cc] = nl + 1;
     }
     uint32_t tot_pops;
     block_exclusive_scan(pops, scan, &tot_pops);
@@ -216,7 +271,10 @@ __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
 
 cudaError_t launch_compact(const CompactArgs &a, cudaStream_t s) {
     if (a.C == 0) return cudaSuccess;
-    const size_t smem = (size_t)(2 * (a.max_pages + 1)) * sizeof(int32_t);
+    // page ids, keep words, two prefix arrays
+    const size_t smem = (size_t)(a.max_pages + (a.max_pages + 1) / 2 + 1 + 2 * (a.max_pages + 1)) * sizeof(int32_t);
+    if (smem > 200 * 1024) return cudaErrorNotSupported;
+    if (a.row_bytes > 16 * MAX_ROW_CHUNKS) return cudaErrorNotSupported;
     cudaError_t e = cudaFuncSetAttribute(compact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     compact_kernel<<<a.C, CMP_THREADS, smem, s>>>(a);
@@ -225,7 +283,8 @@ cudaError_t launch_compact(const CompactArgs &a, cudaStream_t s) {
 
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
     if (a.C == 0) return cudaSuccess;
-    append_kernel<<<(a.C + APP_THREADS - 1) / APP_THREADS, APP_THREADS, 0, s>>>(a);
+    if (a.row_bytes > 16 * MAX_ROW_CHUNKS) return cudaErrorNotSupported;
+    append_kernel<<<(a.C + APP_HEADS - 1) / APP_HEADS, APP_THREADS, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -16,11 +16,10 @@ struct WsLayout {
     size_t status;        // int32, sticky RKV_DEV_* bits
     size_t done_compact;  // uint32, self-resetting completion counter
     size_t done_append;   // uint32, self-resetting completion counter
-    size_t sel_begin;     // start of the region zeroed before every selection
-    size_t bar;           // uint32 grid-barrier counter
-    size_t more;          // uint32 [waves][NPASS] continuation flags
-    size_t hist;          // uint32 [waves][NPASS][n_groups][NBINS]
-    size_t sel_end;
+    size_t bar;           // uint32 grid-barrier counter (reset by the selection's last CTA)
+    size_t leave;         // uint32 exit ticket of the selection
+    size_t more;          // uint32 [waves][NPASS] continuation flags (cleared at exit)
+    size_t hist;          // uint32 [waves][NPASS][n_groups][NBINS] (cleared at exit)
     size_t head_cnt;      // uint32 [C], attention split-head arrival counters (self-resetting)
     size_t partial;       // float [MAX_ATTN_CTAS][2][rec], attention partial states
     size_t total;
@@ -50,6 +49,7 @@ struct SelectArgs {
     int32_t *plan;
     int32_t *status;
     uint32_t *bar;
+    uint32_t *leave;
     uint32_t *more;
     uint32_t *hist;
     int n_groups, cta_per_group, waves, cache_pages;

@@ -35,7 +35,8 @@ constexpr int SEL_MAX_LH = 8192;
 struct SelSmem {
     int32_t *pfx;     // [LH + 1] page prefix of the group's sequence
     int32_t *lens;    // [LH]
-    uint32_t *hist;   // [NBINS]
+    int32_t *kc;      // [LH] kept counts of this CTA's pages, per head
+    uint32_t *hist;   // [4][NBINS] sub-histograms
     uint32_t *scan;   // [40]
     uint2 *keys;      // [cache_pages * 16]
     int *flag;        // barrier / misc flags
@@ -54,6 +55,21 @@ struct SeqState {
     int x0, x1;              // page range of this CTA within the sequence
 };
 
+#ifdef EXP_TIMING
+__device__ unsigned long long g_exp_t[64];
+__device__ unsigned long long g_exp_slow[64];
+#define EXP_STAMP(i)                                                                               \
+    do {                                                                                           \
+        if (threadIdx.x == 0) {                                                                    \
+            const unsigned long long tt = globaltimer_ns();                                        \
+            if (blockIdx.x == 0) g_exp_t[i] = tt;                                                  \
+            atomicMax(&g_exp_slow[i], tt);                                                         \
+        }                                                                                          \
+    } while (0)
+#else
+#define EXP_STAMP(i) do {} while (0)
+#endif
+
 // Head (local index) of flattened page x: largest c with pfx[c] <= x.
 __device__ __forceinline__ int page_head(const int32_t *pfx, int LH, int x) {
     int lo = 0, hi = LH - 1;
@@ -64,40 +80,109 @@ __device__ __forceinline__ int page_head(const int32_t *pfx, int LH, int x) {
     return lo;
 }
 
-// Rank key of slot (x, r) of the sequence.  Invalid slots (past len, or bad
-// input, which is also recorded) get hi = KEY_INVALID.
-__device__ __forceinline__ uint2 entry_key(const SelectArgs &a, const SelSmem &sm, const SeqState &st, int x,
-                                           int r) {
-    const int cl = page_head(sm.pfx, a.LH, x);
-    const int pidx = x - sm.pfx[cl];
-    const int k = pidx * PAGE + r;
-    uint2 key = make_uint2(KEY_INVALID, 0u);
-    if (k < sm.lens[cl]) {
-        const int64_t c = (int64_t)st.b * a.LH + cl;
-        const int32_t page = __ldg(a.block_table + c * a.max_pages + pidx);
-        const int64_t row = (int64_t)page * PAGE + r;
-        const int32_t pos = __ldg(a.pos_pool + row);
-        const float lb = __ldg(a.lb_pool + row);
-        const int64_t age = (int64_t)st.t - pos;
-        const bool bad = (lb != lb) || age < 1 || age >= (1 << 24) || pos < 0 ||
-                         (a.ibits < 32 && (uint32_t)pos >= (1u << a.ibits));
-        if (bad) {
-            set_status(a.status, RKV_DEV_BAD_INPUT);
-        } else {
-            float s = __fmul_rn((float)(int32_t)age, lb);
-            if (s == 0.0f) s = 0.0f;
-            key.x = score_key_desc(s);
-            key.y = (uint32_t)(((uint64_t)cl << a.ibits) | (uint32_t)pos);
-        }
+// Rank key of one slot from its position and log-retention.  Invalid slots
+// (past len, or bad input, which is also recorded) get hi = KEY_INVALID.
+__device__ __forceinline__ uint2 make_key(const SelectArgs &a, const SeqState &st, int cl, int32_t pos, float lb) {
+    const int64_t age = (int64_t)st.t - pos;
+    const bool bad = (lb != lb) || age < 1 || age >= (1 << 24) || pos < 0 ||
+                     (a.ibits < 32 && (uint32_t)pos >= (1u << a.ibits));
+    if (bad) {
+        set_status(a.status, RKV_DEV_BAD_INPUT);
+        return make_uint2(KEY_INVALID, 0u);
     }
-    return key;
+    float s = __fmul_rn((float)(int32_t)age, lb);
+    if (s == 0.0f) s = 0.0f;
+    return make_uint2(score_key_desc(s), (uint32_t)(((uint64_t)cl << a.ibits) | (uint32_t)pos));
 }
 
-__device__ __forceinline__ uint2 cached_key(const SelectArgs &a, const SelSmem &sm, const SeqState &st, int x,
-                                            int r) {
-    const int off = x - st.x0;
-    if (off < a.cache_pages) return sm.keys[off * PAGE + r];
-    return entry_key(a, sm, st, x, r);
+constexpr int UNR = 8;  // pages per thread per round (loads issued together)
+
+// Computes the keys of pages [xa, xb) of this CTA's range from global memory
+// and calls f(x, r, key) for each slot.  Warp w covers pages xa + 2w +
+// (lane >> 4) + 32*j; each lane owns slot r = lane & 15 of its page, so a
+// warp's two half-warps hold two whole pages.  Each round issues the block
+// table loads of UNR pages, then their position / log-retention loads, so a
+// round costs two dependent memory latencies.  Loop bounds are warp-uniform.
+template <typename F>
+__device__ __forceinline__ void keys_from_global(const SelectArgs &a, const SelSmem &sm, const SeqState &st, int xa,
+                                                 int xb_end, F &&f) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+    const int r = lane & 15;
+    const int step = 2 * nwarp;
+    int cur = -1;  // head of the previous page looked up (pages ascend per thread)
+    for (int xb = xa + 2 * warp; xb < xb_end; xb += step * UNR) {
+        int32_t pg[UNR];
+        int cl[UNR];
+        bool ld[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; u++) {
+            const int x = xb + (lane >> 4) + u * step;
+            ld[u] = false;
+            cl[u] = 0;
+            pg[u] = 0;
+            if (x < xb_end) {
+                if (cur < 0) cur = page_head(sm.pfx, a.LH, x);
+                while (cur + 1 < a.LH && sm.pfx[cur + 1] <= x) cur++;
+                cl[u] = cur;
+                const int pidx = x - sm.pfx[cur];
+                if (pidx * PAGE + r < sm.lens[cur]) {
+                    ld[u] = true;
+#ifdef EXP_NO_TABLE
+                    pg[u] = x;
+#else
+                    pg[u] = __ldg(a.block_table + ((int64_t)st.b * a.LH + cur) * a.max_pages + pidx);
+#endif
+                }
+            }
+        }
+        int32_t pos[UNR];
+        float lb[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; u++) {
+            pos[u] = 0;
+            lb[u] = 0.0f;
+            if (ld[u]) {
+                const int64_t row = (int64_t)pg[u] * PAGE + r;
+#ifdef EXP_NO_POSLB
+                pos[u] = (int32_t)(row & 0x7FFF);
+                lb[u] = -1.0f;
+#else
+                pos[u] = __ldg(a.pos_pool + row);
+                lb[u] = __ldg(a.lb_pool + row);
+#endif
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; u++) {
+            const int x = xb + (lane >> 4) + u * step;
+            f(x, r, (x < xb_end && ld[u]) ? make_key(a, st, cl[u], pos[u], lb[u]) : make_uint2(KEY_INVALID, 0u));
+        }
+    }
+}
+
+// Calls f(x, r, key) for every slot r of every page x of this CTA's range:
+// cached pages from shared memory (a flat loop, 32 keys = two pages per warp
+// per step), the rest recomputed from global memory.  With `fill` every key
+// is computed from global memory and the cacheable ones are stored.
+template <typename F>
+__device__ __forceinline__ void for_keys(const SelectArgs &a, const SelSmem &sm, const SeqState &st, bool fill,
+                                         F &&f) {
+    const int ncache = min(st.x1 - st.x0, a.cache_pages);
+    if (fill) {
+        keys_from_global(a, sm, st, st.x0, st.x1, [&](int x, int r, uint2 k) {
+            if (x - st.x0 < a.cache_pages && x < st.x1) sm.keys[(x - st.x0) * PAGE + r] = k;
+            f(x, r, k);
+        });
+        return;
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nk = ncache * PAGE;
+    for (int base = warp * 32; base < nk; base += blockDim.x) {
+        const int i = base + lane;
+        const uint2 k = i < nk ? sm.keys[i] : make_uint2(KEY_INVALID, 0u);
+        f(i < nk ? st.x0 + (i >> 4) : st.x1, i & 15, k);
+    }
+    if (st.x0 + ncache < st.x1) keys_from_global(a, sm, st, st.x0 + ncache, st.x1, f);
 }
 
 __device__ __forceinline__ bool key_matches(uint2 k, const SeqState &st) {
@@ -106,28 +191,37 @@ __device__ __forceinline__ bool key_matches(uint2 k, const SeqState &st) {
 }
 
 // Histogram digit p of this CTA's matching keys into the group's global bins.
-// When `fill` is set (phase 0) the keys are computed and cached on the way.
+// When `fill` is set (first pass) the keys are computed and cached on the way.
+// Lanes update NSUB interleaved sub-histograms (lane mod NSUB) to spread the
+// shared-memory atomics of keys that share a digit; they are summed on flush.
+constexpr int NSUB = 4;
 __device__ void hist_pass(const SelectArgs &a, const SelSmem &sm, const SeqState &st, int p, int g, int wave,
                           bool fill, bool count) {
-    for (int i = threadIdx.x; i < NBINS; i += blockDim.x) sm.hist[i] = 0u;
+    for (int i = threadIdx.x; i < NSUB * NBINS; i += blockDim.x) sm.hist[i] = 0u;
     __syncthreads();
-    const int r = threadIdx.x & 15;
-    for (int x = st.x0 + (int)(threadIdx.x >> 4); x < st.x1; x += blockDim.x >> 4) {
-        uint2 k;
-        if (fill) {
-            k = entry_key(a, sm, st, x, r);
-            const int off = x - st.x0;
-            if (off < a.cache_pages) sm.keys[off * PAGE + r] = k;
-        } else {
-            k = cached_key(a, sm, st, x, r);
-        }
-        if (count && key_matches(k, st)) atomicAdd(&sm.hist[key_digit(k.x, k.y, p)], 1u);
-    }
+    EXP_STAMP(30 + 3 * p);
+    const int lane = threadIdx.x & 31;
+    uint32_t *hsub = sm.hist + (lane & (NSUB - 1)) * NBINS;
+    for_keys(a, sm, st, fill, [&](int x, int r, uint2 k) {
+        if (!count) return;
+        const bool hit = x < st.x1 && key_matches(k, st);
+#ifdef EXP_MATCH_ANY
+        const uint32_t d = hit ? key_digit(k.x, k.y, p) : 0xFFFFFFFFu;
+        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
+        if (hit && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], (uint32_t)__popc(peers));
+#else
+        if (hit) atomicAdd(&hsub[key_digit(k.x, k.y, p)], 1u);
+#endif
+    });
+    EXP_STAMP(31 + 3 * p);
     __syncthreads();
+    EXP_STAMP(32 + 3 * p);
     if (count) {
         uint32_t *gh = a.hist + ((size_t)(wave * NPASS + p) * a.n_groups + g) * NBINS;
         for (int i = threadIdx.x; i < NBINS; i += blockDim.x) {
-            const uint32_t v = sm.hist[i];
+            uint32_t v = 0;
+#pragma unroll
+            for (int j = 0; j < NSUB; j++) v += sm.hist[j * NBINS + i];
             if (v) atomicAdd(gh + i, v);
         }
     }
@@ -137,13 +231,11 @@ __device__ void hist_pass(const SelectArgs &a, const SelSmem &sm, const SeqState
 __device__ void scan_pass(const SelectArgs &a, const SelSmem &sm, SeqState &st, int p, int g, int wave) {
     const uint32_t *gh = a.hist + ((size_t)(wave * NPASS + p) * a.n_groups + g) * NBINS;
     constexpr int PER = NBINS / SEL_THREADS;  // 4
-    uint32_t v[PER];
-    uint32_t loc = 0;
-#pragma unroll
-    for (int j = 0; j < PER; j++) {
-        v[j] = __ldcg(gh + threadIdx.x * PER + j);
-        loc += v[j];
-    }
+    const uint4 v4 = __ldcg(reinterpret_cast<const uint4 *>(gh) + threadIdx.x);
+    const uint32_t v[PER] = {v4.x, v4.y, v4.z, v4.w};
+    const uint32_t loc = v[0] + v[1] + v[2] + v[3];
+    EXP_STAMP(50 + 2 * p);
+    if (threadIdx.x == 0) sm.bcast[3] = 0u;
     uint32_t total;
     const uint32_t ex = block_exclusive_scan(loc, sm.scan, &total);
     if (ex < st.rank && st.rank <= ex + loc) {
@@ -154,13 +246,23 @@ __device__ void scan_pass(const SelectArgs &a, const SelSmem &sm, SeqState &st, 
                 sm.bcast[0] = threadIdx.x * PER + j;  // digit
                 sm.bcast[1] = st.rank - cum;          // new rank within the bucket
                 sm.bcast[2] = v[j];                   // bucket size
+                sm.bcast[3] = 1u;
             }
             cum += v[j];
         }
     }
     __syncthreads();
-    const uint32_t d = sm.bcast[0], nr = sm.bcast[1], h = sm.bcast[2];
+    const uint32_t d = sm.bcast[0], nr = sm.bcast[1], h = sm.bcast[2], found = sm.bcast[3];
     __syncthreads();
+    EXP_STAMP(51 + 2 * p);
+    if (!found) {
+        // fewer matching keys than the rank (only when entries were rejected
+        // as bad input): keep every key with the current prefix
+        if (threadIdx.x == 0) set_status(a.status, RKV_DEV_BAD_INPUT);
+        st.done = true;
+        st.kappa = (st.pk | ~st.pm) + 1ull;
+        return;
+    }
     const int sh = digit_shift(p);
     const uint64_t dm = ((1ull << digit_bits(p)) - 1ull) << sh;
     st.pk |= (uint64_t)d << sh;
@@ -172,29 +274,40 @@ __device__ void scan_pass(const SelectArgs &a, const SelSmem &sm, SeqState &st, 
     }
 }
 
-// Keep masks (warp ballots over the 16 slots of a page) and kept counts.
+// Head (local index) of a page from the key of its slot 0 (lo = cl << ib | i).
+__device__ __forceinline__ int head_of(const SelectArgs &a, const SelSmem &sm, int x, uint2 k0) {
+    if (k0.x != KEY_INVALID) return a.ibits >= 32 ? 0 : (int)(k0.y >> a.ibits);
+    return page_head(sm.pfx, a.LH, x);
+}
+
+// Keep masks (half-warp ballots over the 16 slots of a page); kept counts are
+// summed per head in shared memory and flushed with one atomic per head.
 __device__ void final_pass(const SelectArgs &a, const SelSmem &sm, const SeqState &st) {
-    const int lane = threadIdx.x & 31, r = lane & 15;
-    const int nwarp = blockDim.x >> 5, warp = threadIdx.x >> 5;
-    for (int xb = st.x0 + warp * 2; xb < st.x1; xb += nwarp * 2) {
-        const int x = xb + (lane >> 4);
-        bool keep = false;
-        if (x < st.x1) {
-            const uint2 k = cached_key(a, sm, st, x, r);
-            const uint64_t K = ((uint64_t)k.x << 32) | k.y;
-            keep = k.x != KEY_INVALID && K < st.kappa;
-        }
+    const int lane = threadIdx.x & 31;
+    for_keys(a, sm, st, false, [&](int x, int r, uint2 k) {
+        const uint64_t K = ((uint64_t)k.x << 32) | k.y;
+        const bool keep = x < st.x1 && k.x != KEY_INVALID && K < st.kappa;
         const uint32_t ball = __ballot_sync(0xFFFFFFFFu, keep);
         if (r == 0 && x < st.x1) {
             const uint32_t m16 = (ball >> (lane & 16)) & 0xFFFFu;
-            const int cl = page_head(sm.pfx, a.LH, x);
+            const int cl = head_of(a, sm, x, k);
             const int pidx = x - sm.pfx[cl];
-            const int64_t c = (int64_t)st.b * a.LH + cl;
-            a.keep_mask[c * a.max_pages + pidx] = (uint16_t)m16;
-            if (m16) atomicAdd(a.kept + c, __popc(m16));
+            a.keep_mask[((int64_t)st.b * a.LH + cl) * a.max_pages + pidx] = (uint16_t)m16;
+            if (m16) atomicAdd(&sm.kc[cl], __popc(m16));
+        }
+    });
+    EXP_STAMP(60);
+    __syncthreads();
+    EXP_STAMP(61);
+    if (st.x0 < st.x1) {
+        const int c_lo = page_head(sm.pfx, a.LH, st.x0), c_hi = page_head(sm.pfx, a.LH, st.x1 - 1);
+        for (int cl = c_lo + (int)threadIdx.x; cl <= c_hi; cl += blockDim.x) {
+            const int v = sm.kc[cl];
+            if (v) atomicAdd(a.kept + (int64_t)st.b * a.LH + cl, v);
         }
     }
 }
+
 
 __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -204,7 +317,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         sm.keys = reinterpret_cast<uint2 *>(p);
         p += (size_t)a.cache_pages * PAGE * sizeof(uint2);
         sm.hist = reinterpret_cast<uint32_t *>(p);
-        p += NBINS * sizeof(uint32_t);
+        p += 4 * NBINS * sizeof(uint32_t);
         sm.scan = reinterpret_cast<uint32_t *>(p);
         p += 40 * sizeof(uint32_t);
         sm.bcast = reinterpret_cast<uint32_t *>(p);
@@ -214,10 +327,13 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         sm.pfx = reinterpret_cast<int32_t *>(p);
         p += (size_t)(a.LH + 1) * sizeof(int32_t);
         sm.lens = reinterpret_cast<int32_t *>(p);
+        p += (size_t)a.LH * sizeof(int32_t);
+        sm.kc = reinterpret_cast<int32_t *>(p);
     }
     const int g = blockIdx.x / a.cta_per_group;
     const int rr = blockIdx.x % a.cta_per_group;
     uint32_t epoch = 0;
+    EXP_STAMP(0);
     bool alive = true;
 
     for (int wave = 0; wave < a.waves && alive; wave++) {
@@ -236,7 +352,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
                 const int cl = base + threadIdx.x;
                 int32_t n = cl < a.LH ? __ldcg(a.len + (int64_t)st.b * a.LH + cl) : 0;
                 if (n < 0) n = 0;
-                if (cl < a.LH) sm.lens[cl] = n;
+                if (cl < a.LH) { sm.lens[cl] = n; sm.kc[cl] = 0; }
                 uint32_t tot;
                 const uint32_t ex = block_exclusive_scan((uint32_t)((n + PAGE - 1) / PAGE), sm.scan, &tot);
                 if (cl < a.LH) sm.pfx[cl] = (int32_t)(carry + ex);
@@ -266,9 +382,12 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
             st.pm = 0;
             st.done = (st.m == 0) || (st.m == st.n);
             st.kappa = st.m == 0 ? 0ull : ~0ull;
+            EXP_STAMP(1);
             hist_pass(a, sm, st, 0, g, wave, /*fill=*/true, /*count=*/!st.done);
         }
+        EXP_STAMP(2);
         alive = grid_barrier(a.bar, ++epoch, a.status, sm.flag);
+        EXP_STAMP(3);
         for (int p = 0; alive; p++) {
             if (st.active && !st.done) scan_pass(a, sm, st, p, g, wave);
             if (st.active && st.done && !finalized) {
@@ -280,14 +399,37 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
                 if (rr == 0 && threadIdx.x == 0) atomicOr(a.more + wave * NPASS + p, 1u);
                 hist_pass(a, sm, st, p + 1, g, wave, false, true);
             }
+            EXP_STAMP(4 + 2 * p);
             alive = grid_barrier(a.bar, ++epoch, a.status, sm.flag);
+            EXP_STAMP(5 + 2 * p);
             if (!alive) break;
             if (__ldcg(a.more + wave * NPASS + p) == 0u) break;
         }
     }
+    if (!alive) return;
+    // Every histogram and flag read of this launch happened before the last
+    // barrier: clear them for the next launch, and let the last CTA to leave
+    // reset the barrier counter (the workspace must be re-initialised after a
+    // timed-out barrier, which skips this).
+    {
+        const size_t nh = (size_t)a.waves * NPASS * a.n_groups * NBINS;
+        for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nh; i += (size_t)gridDim.x * blockDim.x)
+            a.hist[i] = 0u;
+        for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.waves * NPASS; i += gridDim.x * blockDim.x)
+            a.more[i] = 0u;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();
+            if (atomicAdd(a.leave, 1u) == gridDim.x - 1) {
+                *a.bar = 0u;
+                *a.leave = 0u;
+                __threadfence();
+            }
+        }
+    }
     // Free-page plan over all heads (after the last barrier every kept count
     // and n_pre is final): plan[c] = pages freed in heads < c.
-    if (!alive || blockIdx.x != 0) return;
+    if (blockIdx.x != 0) return;
     uint32_t carry = 0;
     for (int base = 0; base < a.C; base += blockDim.x) {
         const int c = base + threadIdx.x;
@@ -305,9 +447,20 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         a.plan[a.C] = (int32_t)carry;
         a.plan[a.C + 1] = __ldcg(a.free_top);
     }
+    EXP_STAMP(20);
 }
 
 }  // namespace
+
+#ifdef EXP_TIMING
+extern "C" __attribute__((visibility("default"))) void exp_read_times(unsigned long long *t, unsigned long long *slow) {
+    cudaMemcpyFromSymbol(t, g_exp_t, sizeof(g_exp_t));
+    cudaMemcpyFromSymbol(slow, g_exp_slow, sizeof(g_exp_slow));
+    unsigned long long z[64] = {0};
+    cudaMemcpyToSymbol(g_exp_t, z, sizeof(z));
+    cudaMemcpyToSymbol(g_exp_slow, z, sizeof(z));
+}
+#endif
 
 int select_max_smem() { return 227 * 1024; }
 
@@ -319,7 +472,7 @@ SelectGrid select_grid_for(const rkv_cache_t &c, int sm_count) {
     g.n_groups = c.B < ctas ? c.B : ctas;
     g.cta_per_group = ctas / g.n_groups;
     g.waves = (c.B + g.n_groups - 1) / g.n_groups;
-    const int fixed = NBINS * 4 + 40 * 4 + 16 + 16 + (2 * LH + 1) * 4;
+    const int fixed = 4 * NBINS * 4 + 40 * 4 + 16 + 16 + (3 * LH + 1) * 4;
     const int avail = select_max_smem() - fixed - 1024;
     g.cache_pages = avail > 0 ? avail / (PAGE * (int)sizeof(uint2)) : 0;
     // no point caching more pages than the largest per-CTA share could hold
