@@ -128,13 +128,13 @@ int encode_pool_map(CUtensorMap *m, void *pool, int D, int n_pages) {
             return fail(RKV_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
         fn = reinterpret_cast<EncodeTiledFn>(p);
     }
-    // the pool as [rows = n_pages*16][D/64 lines][64 columns] bf16; one box is
-    // a whole page (16 rows x D/64 lines x 64 columns) and lands in shared
-    // memory as 128-byte lines, 16-byte chunks XOR-swizzled by line mod 8
-    const cuuint32_t nline = (cuuint32_t)(D / 64);
-    const cuuint64_t dims[3] = {64, nline, (cuuint64_t)n_pages * PAGE};
-    const cuuint64_t strides[2] = {128, (cuuint64_t)D * 2};
-    const cuuint32_t box[3] = {64, nline, PAGE};
+    // the pool as a 3-D tensor (64 columns, n_pages*16 rows, D/64 halves) of
+    // bf16: one box is a whole page and lands in shared memory as D/64 planes
+    // of 16 rows x 128 bytes, 16-byte chunks XOR-swizzled by line mod 8
+    const cuuint32_t nhalf = (cuuint32_t)(D / 64);
+    const cuuint64_t dims[3] = {64, (cuuint64_t)n_pages * PAGE, nhalf};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, 128};
+    const cuuint32_t box[3] = {64, PAGE, nhalf};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, pool, dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -45,6 +45,25 @@ namespace {
 constexpr int NCW = RKV_NCW;           // consumer warps
 constexpr int NPW = RKV_NPW;           // producer warps (one issuing lane each)
 constexpr int ATTN_THREADS = (NCW + NPW) * 32;
+// Register split between warpgroups (consumers: warps 0..NCW-1, producers:
+// the last NPW warps).  The block launches with LAUNCH_REGS per thread; the
+// producer warpgroup gives registers back to the consumer warpgroups:
+// NPW*32*PRODUCER_REGS + NCW*32*CONSUMER_REGS <= ATTN_THREADS*LAUNCH_REGS.
+constexpr int LAUNCH_REGS = 168;
+constexpr int PRODUCER_REGS = 56;
+constexpr int CONSUMER_REGS = 224;
+constexpr bool REG_SPLIT = (NCW % 4 == 0) && (NPW % 4 == 0);
+static_assert(!REG_SPLIT || NPW * 32 * PRODUCER_REGS + NCW * 32 * CONSUMER_REGS <= ATTN_THREADS * LAUNCH_REGS,
+              "register split exceeds the launch allocation");
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
 constexpr int QR = 4;                  // query ring slots
 constexpr float LN2 = 0.69314718055994530942f;
 
@@ -300,10 +319,12 @@ struct MmaMath {
         float o[WITH_V ? NT : 1][2];              // PV accumulators c0, c1 of row g
     };
 
-    // A page lands as 16 rows x NBOX lines of 128 bytes (line L = row*NBOX +
-    // half) with the 16-byte chunks of each line XOR-swizzled by L mod 8.
+    // A page lands as NBOX planes (64-column halves) of 16 rows x 128 bytes
+    // (line L = half*16 + row), the 16-byte chunks of each line XOR-swizzled by
+    // L mod 8 -- eight consecutive rows of one half hit eight distinct bank
+    // groups, so every 8x8 ldmatrix is conflict-free.
     __device__ static uint32_t swz(int r, int h, int c) {
-        const int L = r * NBOX + h;
+        const int L = h * PAGE + r;
         return (uint32_t)(L * 128 + ((c ^ (L & 7)) << 4));
     }
 
@@ -331,20 +352,22 @@ struct MmaMath {
                                 uint32_t evm, int lane) {
         const int t = lane & 3, mi = lane >> 3, r8 = lane & 7;
         // ---- S = Q K^T for the 16 rows of the page (two n-tiles of 8 rows) ----
-        float s0[2] = {0.0f, 0.0f}, s1[2] = {0.0f, 0.0f};
+        // four independent accumulation chains (high/low query parts x two
+        // 8-row halves of the page), summed at the end
+        float s0h[2] = {0.0f, 0.0f}, s0l[2] = {0.0f, 0.0f}, s1h[2] = {0.0f, 0.0f}, s1l[2] = {0.0f, 0.0f};
         const uint32_t kbase = smem_u32(sk);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ks++) {
             const int r = (mi >> 1) * 8 + r8, ch = (ks & 3) * 2 + (mi & 1);
             uint32_t b[4];
             ldsm_x4(kbase + swz(r, ks >> 2, ch), b);
-            mma_rows8(s0[0], s0[1], s.qh[ks][0], s.qh[ks][1], b[0], b[1]);
-            mma_rows8(s0[0], s0[1], s.ql[ks][0], s.ql[ks][1], b[0], b[1]);
-            mma_rows8(s1[0], s1[1], s.qh[ks][0], s.qh[ks][1], b[2], b[3]);
-            mma_rows8(s1[0], s1[1], s.ql[ks][0], s.ql[ks][1], b[2], b[3]);
+            mma_rows8(s0h[0], s0h[1], s.qh[ks][0], s.qh[ks][1], b[0], b[1]);
+            mma_rows8(s1h[0], s1h[1], s.qh[ks][0], s.qh[ks][1], b[2], b[3]);
+            mma_rows8(s0l[0], s0l[1], s.ql[ks][0], s.ql[ks][1], b[0], b[1]);
+            mma_rows8(s1l[0], s1l[1], s.ql[ks][0], s.ql[ks][1], b[2], b[3]);
         }
         // this lane holds row g = lane/4 at page rows j = 2t, 2t+1, 2t+8, 2t+9
-        const float y[4] = {s0[0], s0[1], s1[0], s1[1]};
+        const float y[4] = {s0h[0] + s0l[0], s0h[1] + s0l[1], s1h[0] + s1l[0], s1h[1] + s1l[1]};
         const int jr[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
         float pk = -INFINITY, pe = -INFINITY;
 #pragma unroll
@@ -420,12 +443,12 @@ struct MmaMath {
         }
     }
 
-    // Producer: one 3-D tensor box (64 columns x NBOX lines x 16 rows) per
+    // Producer: one 3-D tensor box (64 columns x 16 rows x NBOX halves) per
     // page of K (and of V), 128-byte swizzled.
     __device__ static void issue(unsigned char *sk, bool load_v, int32_t phys, uint64_t *bar, const void *,
                                  const void *, const CUtensorMap *tk, const CUtensorMap *tv, uint64_t pol) {
-        tma_load_3d(sk, tk, 0, 0, phys * PAGE, bar, pol);
-        if (load_v) tma_load_3d(sk + PAGE_BYTES, tv, 0, 0, phys * PAGE, bar, pol);
+        tma_load_3d(sk, tk, 0, phys * PAGE, 0, bar, pol);
+        if (load_v) tma_load_3d(sk + PAGE_BYTES, tv, 0, phys * PAGE, 0, bar, pol);
     }
 };
 
@@ -581,6 +604,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 
     if (warp >= NCW) {
         // =============================== producers ===============================
+        if constexpr (REG_SPLIT) setmaxnreg_dec<PRODUCER_REGS>();
         const int pw = warp - NCW;
         Walker w;
         w.init(a.len, a.C, x1, last, c_start, pfx_start);
@@ -639,6 +663,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     }
 
     // ================================ consumers ================================
+    if constexpr (REG_SPLIT) setmaxnreg_inc<CONSUMER_REGS>();
     Walker w;
     w.init(a.len, a.C, x1, last, c_start, pfx_start);
     int nq = 0;
