@@ -703,9 +703,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             const uint32_t mt = meta[sg];
             const uint32_t keepm = mt & 0xFFFFu, evm = (mt >> 16) & ~keepm;
             const unsigned char *sk = smem + LY::OFF_STAGE + sg * LY::STAGE_BYTES;
-#ifndef EXP_SKIP_MATH
             M::page(st, sk, sk + M::PAGE_BYTES, keepm, evm, lane);
-#endif
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[sg]);
         }

@@ -55,20 +55,6 @@ struct SeqState {
     int x0, x1;              // page range of this CTA within the sequence
 };
 
-#ifdef EXP_TIMING
-__device__ unsigned long long g_exp_t[64];
-__device__ unsigned long long g_exp_slow[64];
-#define EXP_STAMP(i)                                                                               \
-    do {                                                                                           \
-        if (threadIdx.x == 0) {                                                                    \
-            const unsigned long long tt = globaltimer_ns();                                        \
-            if (blockIdx.x == 0) g_exp_t[i] = tt;                                                  \
-            atomicMax(&g_exp_slow[i], tt);                                                         \
-        }                                                                                          \
-    } while (0)
-#else
-#define EXP_STAMP(i) do {} while (0)
-#endif
 
 // Head (local index) of flattened page x: largest c with pfx[c] <= x.
 __device__ __forceinline__ int page_head(const int32_t *pfx, int LH, int x) {
@@ -127,11 +113,7 @@ __device__ __forceinline__ void keys_from_global(const SelectArgs &a, const SelS
                 const int pidx = x - sm.pfx[cur];
                 if (pidx * PAGE + r < sm.lens[cur]) {
                     ld[u] = true;
-#ifdef EXP_NO_TABLE
-                    pg[u] = x;
-#else
                     pg[u] = __ldg(a.block_table + ((int64_t)st.b * a.LH + cur) * a.max_pages + pidx);
-#endif
                 }
             }
         }
@@ -143,13 +125,8 @@ __device__ __forceinline__ void keys_from_global(const SelectArgs &a, const SelS
             lb[u] = 0.0f;
             if (ld[u]) {
                 const int64_t row = (int64_t)pg[u] * PAGE + r;
-#ifdef EXP_NO_POSLB
-                pos[u] = (int32_t)(row & 0x7FFF);
-                lb[u] = -1.0f;
-#else
                 pos[u] = __ldg(a.pos_pool + row);
                 lb[u] = __ldg(a.lb_pool + row);
-#endif
             }
         }
 #pragma unroll
@@ -199,23 +176,14 @@ __device__ void hist_pass(const SelectArgs &a, const SelSmem &sm, const SeqState
                           bool fill, bool count) {
     for (int i = threadIdx.x; i < NSUB * NBINS; i += blockDim.x) sm.hist[i] = 0u;
     __syncthreads();
-    EXP_STAMP(30 + 3 * p);
     const int lane = threadIdx.x & 31;
     uint32_t *hsub = sm.hist + (lane & (NSUB - 1)) * NBINS;
     for_keys(a, sm, st, fill, [&](int x, int r, uint2 k) {
         if (!count) return;
         const bool hit = x < st.x1 && key_matches(k, st);
-#ifdef EXP_MATCH_ANY
-        const uint32_t d = hit ? key_digit(k.x, k.y, p) : 0xFFFFFFFFu;
-        const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
-        if (hit && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], (uint32_t)__popc(peers));
-#else
         if (hit) atomicAdd(&hsub[key_digit(k.x, k.y, p)], 1u);
-#endif
     });
-    EXP_STAMP(31 + 3 * p);
     __syncthreads();
-    EXP_STAMP(32 + 3 * p);
     if (count) {
         uint32_t *gh = a.hist + ((size_t)(wave * NPASS + p) * a.n_groups + g) * NBINS;
         for (int i = threadIdx.x; i < NBINS; i += blockDim.x) {
@@ -234,7 +202,6 @@ __device__ void scan_pass(const SelectArgs &a, const SelSmem &sm, SeqState &st, 
     const uint4 v4 = __ldcg(reinterpret_cast<const uint4 *>(gh) + threadIdx.x);
     const uint32_t v[PER] = {v4.x, v4.y, v4.z, v4.w};
     const uint32_t loc = v[0] + v[1] + v[2] + v[3];
-    EXP_STAMP(50 + 2 * p);
     if (threadIdx.x == 0) sm.bcast[3] = 0u;
     uint32_t total;
     const uint32_t ex = block_exclusive_scan(loc, sm.scan, &total);
@@ -254,7 +221,6 @@ __device__ void scan_pass(const SelectArgs &a, const SelSmem &sm, SeqState &st, 
     __syncthreads();
     const uint32_t d = sm.bcast[0], nr = sm.bcast[1], h = sm.bcast[2], found = sm.bcast[3];
     __syncthreads();
-    EXP_STAMP(51 + 2 * p);
     if (!found) {
         // fewer matching keys than the rank (only when entries were rejected
         // as bad input): keep every key with the current prefix
@@ -296,9 +262,7 @@ __device__ void final_pass(const SelectArgs &a, const SelSmem &sm, const SeqStat
             if (m16) atomicAdd(&sm.kc[cl], __popc(m16));
         }
     });
-    EXP_STAMP(60);
     __syncthreads();
-    EXP_STAMP(61);
     if (st.x0 < st.x1) {
         const int c_lo = page_head(sm.pfx, a.LH, st.x0), c_hi = page_head(sm.pfx, a.LH, st.x1 - 1);
         for (int cl = c_lo + (int)threadIdx.x; cl <= c_hi; cl += blockDim.x) {
@@ -333,7 +297,6 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
     const int g = blockIdx.x / a.cta_per_group;
     const int rr = blockIdx.x % a.cta_per_group;
     uint32_t epoch = 0;
-    EXP_STAMP(0);
     bool alive = true;
 
     for (int wave = 0; wave < a.waves && alive; wave++) {
@@ -382,12 +345,9 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
             st.pm = 0;
             st.done = (st.m == 0) || (st.m == st.n);
             st.kappa = st.m == 0 ? 0ull : ~0ull;
-            EXP_STAMP(1);
             hist_pass(a, sm, st, 0, g, wave, /*fill=*/true, /*count=*/!st.done);
         }
-        EXP_STAMP(2);
         alive = grid_barrier(a.bar, ++epoch, a.status, sm.flag);
-        EXP_STAMP(3);
         for (int p = 0; alive; p++) {
             if (st.active && !st.done) scan_pass(a, sm, st, p, g, wave);
             if (st.active && st.done && !finalized) {
@@ -399,9 +359,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
                 if (rr == 0 && threadIdx.x == 0) atomicOr(a.more + wave * NPASS + p, 1u);
                 hist_pass(a, sm, st, p + 1, g, wave, false, true);
             }
-            EXP_STAMP(4 + 2 * p);
             alive = grid_barrier(a.bar, ++epoch, a.status, sm.flag);
-            EXP_STAMP(5 + 2 * p);
             if (!alive) break;
             if (__ldcg(a.more + wave * NPASS + p) == 0u) break;
         }
@@ -447,20 +405,10 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         a.plan[a.C] = (int32_t)carry;
         a.plan[a.C + 1] = __ldcg(a.free_top);
     }
-    EXP_STAMP(20);
 }
 
 }  // namespace
 
-#ifdef EXP_TIMING
-extern "C" __attribute__((visibility("default"))) void exp_read_times(unsigned long long *t, unsigned long long *slow) {
-    cudaMemcpyFromSymbol(t, g_exp_t, sizeof(g_exp_t));
-    cudaMemcpyFromSymbol(slow, g_exp_slow, sizeof(g_exp_slow));
-    unsigned long long z[64] = {0};
-    cudaMemcpyToSymbol(g_exp_t, z, sizeof(z));
-    cudaMemcpyToSymbol(g_exp_slow, z, sizeof(z));
-}
-#endif
 
 int select_max_smem() { return 227 * 1024; }
 
