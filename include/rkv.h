@@ -163,6 +163,27 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
                              const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * rkv_score_select_noalloc -- rkv_score_select without a workspace argument,
+ * for callers that cannot allocate device memory themselves (for example
+ * code running where cudaMalloc is not permitted, such as inside a host
+ * callback or under an allocator they do not control).  It has no
+ * counterpart in the papers: it is a deployment convenience.  Same inputs,
+ * outputs, results and errors as rkv_score_select; its scratch (status word,
+ * barrier counters, radix histograms) is a fixed __device__ array of about
+ * 0.75 MiB inside the library, which every GPU that loads the library holds
+ * until the process exits.  Limits: at most 16 sequences (B <= 16), else
+ * RKV_ERR_UNSUPPORTED.  The first call on a device looks up that array's
+ * device address (cudaGetSymbolAddress), so make the first call on each
+ * device before any stream capture.  Each call clears the scratch it uses
+ * (an async memset on `stream`) and allocates nothing.  All calls share the
+ * one array: calls that overlap on the GPU (different streams, or other
+ * threads) race and must be serialised by the caller.  Device-side input
+ * errors are not reported by this variant (its status word is private).
+ */
+RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
+                                     const rkv_select_t *sel, void *stream);
+
+/* ---------------------------------------------------------------------------
  * rkv_paged_decode_attn -- grouped-query decode attention over the kept
  * entries, read from the pre-compaction pages.
  *

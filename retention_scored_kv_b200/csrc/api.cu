@@ -230,6 +230,67 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
     return RKV_OK;
 }
 
+// Allocation-free variant of rkv_score_select (no workspace argument): the
+// selection scratch lives in a fixed device array of the library instead.
+RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
+                                     const rkv_select_t *sel, void *stream) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if ((rc = check_sel(sel))) return rc;
+    if (!t || !m_global) return fail(RKV_ERR_INVALID_ARG, "t / m_global is NULL");
+    if (cache->B > NOALLOC_MAX_B)
+        return fail(RKV_ERR_UNSUPPORTED,
+                    "rkv_score_select_noalloc: batch %d exceeds its fixed scratch (at most %d sequences); "
+                    "use rkv_score_select with a workspace",
+                    cache->B, NOALLOC_MAX_B);
+    const int64_t LH = (int64_t)cache->L * cache->H;
+    const int lb = lh_bits(LH);
+    if (lb > 24) return fail(RKV_ERR_UNSUPPORTED, "L*H must be <= 2^24");
+    int sms = 0;
+    if ((rc = sm_count_now(&sms))) return rc;
+    const SelectGrid g = select_grid_for(*cache, sms < MAX_SEL_CTAS ? sms : MAX_SEL_CTAS);
+    if (g.waves * g.n_groups > NOALLOC_MAX_B)
+        return fail(RKV_ERR_UNSUPPORTED, "rkv_score_select_noalloc: too many sequences for its fixed scratch");
+    uint32_t *scr = nullptr;
+    const char *why = nullptr;
+    if (noalloc_scratch(&scr, &why)) return fail(RKV_ERR_CUDA, "rkv_score_select_noalloc scratch: %s", why);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // status, barrier counter, ticket, flags and this call's histograms start at zero
+    const size_t words = NOALLOC_HIST + (size_t)g.waves * g.n_groups * NPASS * NBINS;
+    cudaError_t e = cudaMemsetAsync(scr, 0, words * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(noalloc scratch)");
+    SelectArgs a{};
+    a.pos_pool = cache->pos_pool;
+    a.lb_pool = cache->lb_pool;
+    a.block_table = cache->block_table;
+    a.len = cache->len;
+    a.free_top = cache->free_top;
+    a.B = cache->B;
+    a.LH = (int)LH;
+    a.C = (int)(cache->B * LH);
+    a.max_pages = cache->max_pages;
+    a.ibits = 32 - lb;
+    a.t = t;
+    a.m_global = m_global;
+    a.kappa = sel->kappa;
+    a.kept = sel->kept;
+    a.n_pre = sel->n_pre;
+    a.keep_mask = sel->keep_mask;
+    a.plan = sel->plan;
+    a.status = reinterpret_cast<int32_t *>(scr + NOALLOC_STATUS);
+    a.bar = scr + NOALLOC_BAR;
+    a.leave = scr + NOALLOC_LEAVE;
+    a.more = scr + NOALLOC_MORE;
+    a.hist = scr + NOALLOC_HIST;
+    a.n_groups = g.n_groups;
+    a.cta_per_group = g.cta_per_group;
+    a.waves = g.waves;
+    a.cache_pages = g.cache_pages;
+    e = launch_select(a, g, s);
+    if (e != cudaSuccess) return cuda_fail(e, "select kernel launch (noalloc)");
+    return RKV_OK;
+}
+
 static int attn_common(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
                        float *out, float *lse, float *dropped, void *ws, size_t ws_bytes, void *stream,
                        const char *what) {

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/rkv.h"
+#include "common.cuh"
 
 namespace rkv {
 
@@ -55,6 +56,18 @@ struct SelectArgs {
     int n_groups, cta_per_group, waves, cache_pages;
 };
 cudaError_t launch_select(const SelectArgs &a, const SelectGrid &g, cudaStream_t s);
+
+// Fixed scratch of the allocation-free selection (a __device__ array in
+// select.cu): word offsets of its fields and its size.
+constexpr int NOALLOC_MAX_B = 16;
+constexpr int NOALLOC_MAX_DEVICES = 64;
+constexpr size_t NOALLOC_STATUS = 0, NOALLOC_BAR = 16, NOALLOC_LEAVE = 32, NOALLOC_MORE = 64;
+constexpr size_t NOALLOC_HIST = 256;  // after the flags, 1 KiB aligned
+constexpr size_t NOALLOC_WORDS = NOALLOC_HIST + (size_t)NOALLOC_MAX_B * NPASS * NBINS;
+static_assert(NOALLOC_MORE + NOALLOC_MAX_B * NPASS <= NOALLOC_HIST, "flag region");
+// Device address of that array on the current device (looked up once per
+// device); returns nonzero and sets *err on failure.
+int noalloc_scratch(uint32_t **out, const char **err);
 int select_max_smem();
 
 struct AttnArgs {

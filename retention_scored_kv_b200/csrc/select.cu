@@ -22,6 +22,8 @@
 // compaction kernel consumes.
 #include <cooperative_groups.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -407,7 +409,37 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
     }
 }
 
+// Scratch of the allocation-free selection entry point: status word, grid
+// barrier counter, exit ticket, continuation flags and radix histograms for up
+// to NOALLOC_MAX_B sequences (about 0.75 MiB).  Every GPU that loads the
+// library holds it until the process exits; all calls share it.
+static __device__ __align__(256) uint32_t g_noalloc_scratch[NOALLOC_WORDS];
+
 }  // namespace
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side name is only a stand-in, not a device address).
+int noalloc_scratch(uint32_t **out, const char **err) {
+    static std::mutex mu;
+    static uint32_t *ptrs[NOALLOC_MAX_DEVICES] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) {
+        *err = "no usable current CUDA device";
+        return -1;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            *err = cudaGetErrorString(e);
+            return -1;
+        }
+        ptrs[dev] = static_cast<uint32_t *>(p);
+    }
+    *out = ptrs[dev];
+    return 0;
+}
 
 
 int select_max_smem() { return 227 * 1024; }
