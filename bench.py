@@ -44,6 +44,12 @@ import torch  # noqa: E402
 import workloads  # noqa: E402
 
 METRIC = "evict+paged-decode steps/s"
+
+# DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of one
+# attention launch of the llama32k steady step, from the 16-layer capture in
+# profiles/attn_kernel_llama32k_16L.md scaled x2 to the full launch.  Reported
+# only while the attention kernel's sources are the ones that were captured.
+ATTN_TRAFFIC = {"sources_sha256": "6e67ee544df2f78e", "workload": "llama32k", "bytes_per_launch": 2 * 139.574528e6}
 UNIT = "steps/s"
 SAMPLE_LAYERS = 2  # CPU oracle sample: 2 of the workload's layers, time scaled by L / 2
 
@@ -363,7 +369,7 @@ def run_rkv(args, world, rank, local):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "no flush: per-step K/V working set > 126 MB L2", "graph": use_graph},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": args.traffic,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": attn_traffic(cfg, args.traffic),
                      "kernel": "attn_kernel (paged decode attention + dropped mass)",
                      "bytes_per_launch": a_bytes, "peak_source": peaks["source"]},
         "step_hbm": {"bytes_per_step": s_bytes, "achieved_gbs": s_bytes / step_s / 1e9,
@@ -400,6 +406,20 @@ def _graph_upload(graph, stream):
         lib.cudaGraphUpload(ctypes.c_void_p(graph.raw_cuda_graph_exec()), ctypes.c_void_p(stream.cuda_stream))
     except Exception:
         pass
+
+
+def attn_traffic(cfg: workloads.Config, override):
+    """ncu DRAM bytes per attention launch, or None if not measured for these sources."""
+    if override is not None:
+        return override
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("retention_scored_kv_b200/csrc/attn.cu", "retention_scored_kv_b200/csrc/common.cuh"):
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if cfg.name == ATTN_TRAFFIC["workload"] and h.hexdigest()[:16] == ATTN_TRAFFIC["sources_sha256"]:
+        return ATTN_TRAFFIC["bytes_per_launch"]
+    return None
 
 
 def _peaks() -> dict:
