@@ -87,6 +87,9 @@ void layout_for(const rkv_cache_t &c, int sel_groups_x_waves, WsLayout *L) {
     L->done_append = take(4, 4);
     L->bar = take(4, 64);
     L->leave = take(4, 64);
+    L->win = take((size_t)c.B * 16, 16);
+    L->cnt = take((size_t)c.B * 16, 16);
+    L->cand = take((size_t)c.B * WIN_CAP * 8, 16);
     L->more = take((size_t)c.B * NPASS * 4, 16);
     L->hist = take((size_t)sel_groups_x_waves * NPASS * NBINS * 4, 256);
     L->head_cnt = take((size_t)C * 4, 256);
@@ -219,6 +222,9 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
     a.status = at<int32_t>(ws, L.status);
     a.bar = at<uint32_t>(ws, L.bar);
     a.leave = at<uint32_t>(ws, L.leave);
+    a.win = at<uint32_t>(ws, L.win);
+    a.cnt = at<uint32_t>(ws, L.cnt);
+    a.cand = at<uint2>(ws, L.cand);
     a.more = at<uint32_t>(ws, L.more);
     a.hist = at<uint32_t>(ws, L.hist);
     a.n_groups = g.n_groups;
@@ -255,7 +261,9 @@ RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t,
     const char *why = nullptr;
     if (noalloc_scratch(&scr, &why)) return fail(RKV_ERR_CUDA, "rkv_score_select_noalloc scratch: %s", why);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // status, barrier counter, ticket, flags and this call's histograms start at zero
+    // status, barrier counter, ticket, flags, counters, threshold windows and
+    // this call's histograms start at zero (a cleared window means the exact
+    // radix passes run; candidates need no clearing)
     const size_t words = NOALLOC_HIST + (size_t)g.waves * g.n_groups * NPASS * NBINS;
     cudaError_t e = cudaMemsetAsync(scr, 0, words * sizeof(uint32_t), s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(noalloc scratch)");
@@ -281,6 +289,9 @@ RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t,
     a.bar = scr + NOALLOC_BAR;
     a.leave = scr + NOALLOC_LEAVE;
     a.more = scr + NOALLOC_MORE;
+    a.win = scr + NOALLOC_WIN;
+    a.cnt = scr + NOALLOC_CNT;
+    a.cand = reinterpret_cast<uint2 *>(scr + NOALLOC_CAND);
     a.hist = scr + NOALLOC_HIST;
     a.n_groups = g.n_groups;
     a.cta_per_group = g.cta_per_group;

@@ -13,6 +13,7 @@ constexpr int PAGE = 16;           // rows per page (fixed; keep masks are uint1
 constexpr int NPASS = 6;           // radix digits of the 64-bit key: 11,11,10 | 11,11,10
 constexpr int NBINS = 2048;        // bins of the widest digit
 constexpr int MAX_ATTN_CTAS = 512; // upper bound of the persistent attention grid
+constexpr int WIN_CAP = 1024;      // threshold-window candidates per sequence
 constexpr uint32_t KEY_INVALID = 0xFFFFFFFFu;  // hi word no valid score maps to (NaN space)
 
 // ---------------------------------------------------------------- keys ----

@@ -19,6 +19,9 @@ struct WsLayout {
     size_t done_append;   // uint32, self-resetting completion counter
     size_t bar;           // uint32 grid-barrier counter (reset by the selection's last CTA)
     size_t leave;         // uint32 exit ticket of the selection
+    size_t win;           // uint32 [B][4] threshold window per sequence (kept across calls)
+    size_t cnt;           // uint32 [B][4] per-call counters: keys above the window, candidates
+    size_t cand;          // uint2 [B][WIN_CAP] keys inside the window
     size_t more;          // uint32 [waves][NPASS] continuation flags (cleared at exit)
     size_t hist;          // uint32 [waves][NPASS][n_groups][NBINS] (cleared at exit)
     size_t head_cnt;      // uint32 [C], attention split-head arrival counters (self-resetting)
@@ -51,6 +54,9 @@ struct SelectArgs {
     int32_t *status;
     uint32_t *bar;
     uint32_t *leave;
+    uint32_t *win;
+    uint32_t *cnt;
+    uint2 *cand;
     uint32_t *more;
     uint32_t *hist;
     int n_groups, cta_per_group, waves, cache_pages;
@@ -62,9 +68,13 @@ cudaError_t launch_select(const SelectArgs &a, const SelectGrid &g, cudaStream_t
 constexpr int NOALLOC_MAX_B = 16;
 constexpr int NOALLOC_MAX_DEVICES = 64;
 constexpr size_t NOALLOC_STATUS = 0, NOALLOC_BAR = 16, NOALLOC_LEAVE = 32, NOALLOC_MORE = 64;
-constexpr size_t NOALLOC_HIST = 256;  // after the flags, 1 KiB aligned
-constexpr size_t NOALLOC_WORDS = NOALLOC_HIST + (size_t)NOALLOC_MAX_B * NPASS * NBINS;
-static_assert(NOALLOC_MORE + NOALLOC_MAX_B * NPASS <= NOALLOC_HIST, "flag region");
+constexpr size_t NOALLOC_WIN = 192, NOALLOC_CNT = 256;     // [MAX_B][4] each
+constexpr size_t NOALLOC_HIST = 512;  // after the flags and counters, 2 KiB aligned
+constexpr size_t NOALLOC_CAND = NOALLOC_HIST + (size_t)NOALLOC_MAX_B * NPASS * NBINS;
+constexpr size_t NOALLOC_WORDS = NOALLOC_CAND + (size_t)NOALLOC_MAX_B * WIN_CAP * 2;
+static_assert(NOALLOC_MORE + NOALLOC_MAX_B * NPASS <= NOALLOC_WIN, "flag region");
+static_assert(NOALLOC_WIN + 4 * NOALLOC_MAX_B <= NOALLOC_CNT && NOALLOC_CNT + 4 * NOALLOC_MAX_B <= NOALLOC_HIST,
+              "counter region");
 // Device address of that array on the current device (looked up once per
 // device); returns nonzero and sets *err on failure.
 int noalloc_scratch(uint32_t **out, const char **err);

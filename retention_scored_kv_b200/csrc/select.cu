@@ -55,6 +55,10 @@ struct SeqState {
     bool done;
     uint64_t kappa;          // exclusive threshold once done
     int x0, x1;              // page range of this CTA within the sequence
+    bool wv;                 // threshold window of the previous call is usable
+    uint32_t wlo, whi;       // window [wlo, whi) in score-key (hi word) space
+    int wres;                // 0 unused, 1 resolved in the window, 2 missed, 3 overflowed
+    uint32_t wn;             // candidates found in the window
 };
 
 
@@ -180,11 +184,36 @@ __device__ void hist_pass(const SelectArgs &a, const SelSmem &sm, const SeqState
     __syncthreads();
     const int lane = threadIdx.x & 31;
     uint32_t *hsub = sm.hist + (lane & (NSUB - 1)) * NBINS;
+    // first pass only: keys above the previous threshold's window are
+    // counted, keys inside it are appended to the candidate list
+    const bool win = fill && count && st.wv;
+    uint32_t above = 0;
+    uint32_t *ncand = a.cnt + (size_t)st.b * 4 + 1;
+    uint2 *cand = a.cand + (size_t)st.b * WIN_CAP;
     for_keys(a, sm, st, fill, [&](int x, int r, uint2 k) {
         if (!count) return;
         const bool hit = x < st.x1 && key_matches(k, st);
         if (hit) atomicAdd(&hsub[key_digit(k.x, k.y, p)], 1u);
+        if (win) {
+            const bool valid = x < st.x1 && k.x != KEY_INVALID;
+            above += (valid && k.x < st.wlo) ? 1u : 0u;
+            const bool in = valid && k.x >= st.wlo && k.x < st.whi;
+            const uint32_t ball = __ballot_sync(0xFFFFFFFFu, in);
+            if (ball) {
+                const int leader = __ffs(ball) - 1;
+                uint32_t base = 0;
+                if (lane == leader) base = atomicAdd(ncand, (uint32_t)__popc(ball));
+                base = __shfl_sync(0xFFFFFFFFu, base, leader);
+                const uint32_t idx = base + (uint32_t)__popc(ball & ((1u << lane) - 1u));
+                if (in && idx < WIN_CAP) cand[idx] = k;
+            }
+        }
     });
+    if (win) {
+        uint32_t tot;
+        block_exclusive_scan(above, sm.scan, &tot);
+        if (threadIdx.x == 0 && tot) atomicAdd(a.cnt + (size_t)st.b * 4, tot);
+    }
     __syncthreads();
     if (count) {
         uint32_t *gh = a.hist + ((size_t)(wave * NPASS + p) * a.n_groups + g) * NBINS;
@@ -240,6 +269,61 @@ __device__ void scan_pass(const SelectArgs &a, const SelSmem &sm, SeqState &st, 
         st.done = true;
         st.kappa = (st.pk | ~st.pm) + 1ull;
     }
+}
+
+// After the first barrier: if the previous threshold's window holds the
+// M-th key (keys above the window < M <= above + candidates, and every
+// candidate was stored), the threshold is the (M - above)-th smallest
+// candidate -- found by counting, per candidate, the candidates below it
+// (64-bit keys are distinct).  Otherwise the radix passes continue.
+__device__ void try_window(const SelectArgs &a, const SelSmem &sm, SeqState &st) {
+    if (!st.wv) return;
+    const uint32_t above = __ldcg(a.cnt + (size_t)st.b * 4), nc = __ldcg(a.cnt + (size_t)st.b * 4 + 1);
+    st.wn = nc;
+    if (nc > WIN_CAP) { st.wres = 3; return; }
+    if (!((int64_t)above < st.m && st.m <= (int64_t)above + nc)) { st.wres = 2; return; }
+    const uint32_t r = (uint32_t)(st.m - above);  // 1-based rank among the candidates
+    uint2 *cs = reinterpret_cast<uint2 *>(sm.hist);  // 4*NBINS words >= 2*WIN_CAP
+    const uint2 *cand = a.cand + (size_t)st.b * WIN_CAP;
+    for (uint32_t i = threadIdx.x; i < nc; i += blockDim.x) cs[i] = __ldcg(cand + i);
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < nc; i += blockDim.x) {
+        const uint64_t Ki = ((uint64_t)cs[i].x << 32) | cs[i].y;
+        uint32_t less = 0;
+        for (uint32_t j = 0; j < nc; j++) less += ((((uint64_t)cs[j].x << 32) | cs[j].y) < Ki) ? 1u : 0u;
+        if (less == r - 1) {
+            const uint64_t kap = Ki + 1ull;
+            sm.bcast[0] = (uint32_t)kap;
+            sm.bcast[1] = (uint32_t)(kap >> 32);
+        }
+    }
+    __syncthreads();
+    st.kappa = ((uint64_t)sm.bcast[1] << 32) | sm.bcast[0];
+    st.done = true;
+    st.wres = 1;
+    __syncthreads();
+}
+
+// Window for the next call, centred on this call's threshold score key and
+// resized by what this call saw (group leader only).
+__device__ void update_window(const SelectArgs &a, const SeqState &st) {
+    if (st.kappa == 0ull || st.kappa == ~0ull) return;  // nothing or everything kept
+    uint32_t *w = a.win + (size_t)st.b * 4;
+    const uint32_t center = (uint32_t)((st.kappa - 1ull) >> 32);
+    uint32_t hw = w[3];
+    if (hw == 0u) hw = 1u << 14;
+    if (st.wres == 1) {
+        if (st.wn > WIN_CAP / 2) hw = hw > 1u ? hw >> 1 : 1u;
+        else if (st.wn < 64u) hw = hw < (1u << 28) ? hw << 1 : hw;
+    } else if (st.wres == 2) {
+        hw = hw < (1u << 26) ? hw << 2 : (1u << 28);
+    } else if (st.wres == 3) {
+        hw = hw > 4u ? hw >> 2 : 1u;
+    }
+    w[1] = center > hw ? center - hw : 0u;
+    w[2] = center < 0xFFFFFFFFu - hw ? center + hw : 0xFFFFFFFFu;
+    w[3] = hw;
+    w[0] = 1u;
 }
 
 // Head (local index) of a page from the key of its slot 0 (lo = cl << ib | i).
@@ -298,6 +382,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
     }
     const int g = blockIdx.x / a.cta_per_group;
     const int rr = blockIdx.x % a.cta_per_group;
+    const bool single = a.n_groups == 1 && a.waves == 1;
     uint32_t epoch = 0;
     bool alive = true;
 
@@ -308,6 +393,9 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         st.done = true;
         st.kappa = 0;
         st.x0 = st.x1 = 0;
+        st.wv = false;
+        st.wres = 0;
+        st.wn = 0;
         bool finalized = false;
         if (st.active) {
             // page prefix and lengths of this sequence's heads
@@ -347,16 +435,28 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
             st.pm = 0;
             st.done = (st.m == 0) || (st.m == st.n);
             st.kappa = st.m == 0 ? 0ull : ~0ull;
+            {
+                const uint32_t *w = a.win + (size_t)st.b * 4;
+                st.wv = __ldcg(w) != 0u;
+                st.wlo = __ldcg(w + 1);
+                st.whi = __ldcg(w + 2);
+            }
             hist_pass(a, sm, st, 0, g, wave, /*fill=*/true, /*count=*/!st.done);
         }
         alive = grid_barrier(a.bar, ++epoch, a.status, sm.flag);
+        if (alive && st.active && !st.done) try_window(a, sm, st);
         for (int p = 0; alive; p++) {
             if (st.active && !st.done) scan_pass(a, sm, st, p, g, wave);
             if (st.active && st.done && !finalized) {
                 final_pass(a, sm, st);
-                if (rr == 0 && threadIdx.x == 0) a.kappa[st.b] = st.kappa;
+                if (rr == 0 && threadIdx.x == 0) {
+                    a.kappa[st.b] = st.kappa;
+                    update_window(a, st);
+                }
                 finalized = true;
             }
+            // one sequence: every CTA is resolved together, no closing barrier
+            if (single && finalized) break;
             if (st.active && !st.done) {
                 if (rr == 0 && threadIdx.x == 0) atomicOr(a.more + wave * NPASS + p, 1u);
                 hist_pass(a, sm, st, p + 1, g, wave, false, true);
@@ -367,29 +467,35 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         }
     }
     if (!alive) return;
-    // Every histogram and flag read of this launch happened before the last
-    // barrier: clear them for the next launch, and let the last CTA to leave
-    // reset the barrier counter (the workspace must be re-initialised after a
-    // timed-out barrier, which skips this).
-    {
-        const size_t nh = (size_t)a.waves * NPASS * a.n_groups * NBINS;
+    // Clear this launch's scratch for the next one.  With several groups the
+    // closing barrier has passed, so every histogram read is done and the
+    // CTAs clear slices in parallel; with one group CTAs leave without a
+    // closing barrier and the last CTA to leave (ticket) clears them.  The
+    // last CTA also resets the barrier counter and the window counters and
+    // builds the free-page plan -- every kept count is final once all CTAs
+    // have flushed and taken the ticket.  (A timed-out barrier skips this;
+    // the workspace must then be re-initialised.)
+    const size_t nh = (size_t)a.waves * NPASS * a.n_groups * NBINS;
+    if (!single) {
         for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nh; i += (size_t)gridDim.x * blockDim.x)
             a.hist[i] = 0u;
         for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < a.waves * NPASS; i += gridDim.x * blockDim.x)
             a.more[i] = 0u;
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            __threadfence();
-            if (atomicAdd(a.leave, 1u) == gridDim.x - 1) {
-                *a.bar = 0u;
-                *a.leave = 0u;
-                __threadfence();
-            }
-        }
     }
-    // Free-page plan over all heads (after the last barrier every kept count
-    // and n_pre is final): plan[c] = pages freed in heads < c.
-    if (blockIdx.x != 0) return;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        *sm.flag = atomicAdd(a.leave, 1u) == gridDim.x - 1 ? 1 : 0;
+    }
+    __syncthreads();
+    if (!*sm.flag) return;
+    __threadfence();
+    if (single) {
+        for (size_t i = threadIdx.x; i < nh; i += blockDim.x) a.hist[i] = 0u;
+        for (int i = threadIdx.x; i < a.waves * NPASS; i += blockDim.x) a.more[i] = 0u;
+    }
+    for (int i = threadIdx.x; i < 4 * a.B; i += blockDim.x) a.cnt[i] = 0u;
+    // free-page plan over all heads: plan[c] = pages freed in heads < c
     uint32_t carry = 0;
     for (int base = 0; base < a.C; base += blockDim.x) {
         const int c = base + threadIdx.x;
@@ -406,6 +512,9 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
     if (threadIdx.x == 0) {
         a.plan[a.C] = (int32_t)carry;
         a.plan[a.C + 1] = __ldcg(a.free_top);
+        *a.bar = 0u;
+        *a.leave = 0u;
+        __threadfence();
     }
 }
 

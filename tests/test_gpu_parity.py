@@ -232,3 +232,32 @@ def test_multi_step_small_evict_every_other(rkv):
                              ref["dropped"], kept_any)
         compare_state(dc, hc)
     assert ws.status() == 0
+
+
+def test_select_reuses_threshold_window_across_calls(rkv):
+    # One workspace across many calls: the previous call's threshold window is
+    # hit (similar budgets), missed (budget jumps) and overflows (dense ties);
+    # every call must match the oracle exactly.
+    cfg = workloads.small_config(L=3, H=4, G=1, D=64, B=1, T0=6000, kv_dtype="bf16")
+    rng = np.random.default_rng(31)
+    dc = _ragged(cfg, 31, rng.integers(200, 2500, size=cfg.C))
+    cache = rkv_cache(rkv, dc)
+    ws = rkv.Workspace(cache)
+    n = int(dc.len.sum())
+    budgets = [n // 2, n // 2 + 3, n // 2 - 40, n // 2 + 100, n // 5, n // 5 + 1, (9 * n) // 10, (9 * n) // 10 - 7,
+               1, n - 1, n // 3]
+    for i, m in enumerate(budgets):
+        t = 6000 + (i % 3)
+        sel = rkv.Selection.empty(cache)
+        rkv.score_select(cache, torch.tensor([t], dtype=torch.int32, device="cuda"),
+                         torch.tensor([m], dtype=torch.int64, device="cuda"), sel, ws)
+        sync()
+        _check_select(dc, sel, ws, [t], [m])
+    few = torch.tensor([-0.5, -0.25], dtype=torch.float32, device="cuda")
+    dc.lb_pool.copy_(few[torch.randint(0, 2, dc.lb_pool.shape, device="cuda")])   # many exact ties
+    for m in (n // 2, n // 2 + 1, n // 4):
+        sel = rkv.Selection.empty(cache)
+        rkv.score_select(cache, torch.tensor([6000], dtype=torch.int32, device="cuda"),
+                         torch.tensor([m], dtype=torch.int64, device="cuda"), sel, ws)
+        sync()
+        _check_select(dc, sel, ws, [6000], [m])
