@@ -169,8 +169,8 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
  * callback or under an allocator they do not control).  It has no
  * counterpart in the papers: it is a deployment convenience.  Same inputs,
  * outputs, results and errors as rkv_score_select; its scratch (status word,
- * barrier counters, radix histograms) is a fixed __device__ array of about
- * 0.75 MiB inside the library, which every GPU that loads the library holds
+ * barrier counters, radix histograms, window candidates) is a fixed __device__ array of about
+ * 0.9 MiB inside the library, which every GPU that loads the library holds
  * until the process exits.  Limits: at most 16 sequences (B <= 16), else
  * RKV_ERR_UNSUPPORTED.  The first call on a device looks up that array's
  * device address (cudaGetSymbolAddress), so make the first call on each

@@ -519,8 +519,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
 }
 
 // Scratch of the allocation-free selection entry point: status word, grid
-// barrier counter, exit ticket, continuation flags and radix histograms for up
-// to NOALLOC_MAX_B sequences (about 0.75 MiB).  Every GPU that loads the
+// barrier counter, exit ticket, continuation flags, radix histograms and window candidates for up
+// to NOALLOC_MAX_B sequences (about 0.9 MiB).  Every GPU that loads the
 // library holds it until the process exits; all calls share it.
 static __device__ __align__(256) uint32_t g_noalloc_scratch[NOALLOC_WORDS];
 
