@@ -4,6 +4,10 @@ decode attention over the kept entries (select -> attention + dropped mass
 -> compaction -> append), on synthetic Llama-3.1-8B-shaped data.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rkv|reference] [--config NAME]
+                    [--path fused|separate]
+
+--path fused (default) runs each step as one rkv_decode_step launch; separate
+runs the four entry points (select, attention, compaction, append).
 
 Default workload "llama32k": 32 layers x 8 KV heads (32 query heads, GQA 4),
 head dim 128, bf16 K/V, batch 1, 32K-token prefill, global budget
@@ -17,8 +21,9 @@ Timing: the K timed steps are one CUDA graph replay bracketed by a barrier
 and synchronize on both sides, timed with CUDA events on the launching
 stream; multi-GPU runs are independent replicas (one sequence per rank,
 "scaling": "weak") and report the maximum over ranks.  Per-kernel CUDA events
-inside the graph give each kernel's average duration; the attention kernel's
-algorithmic bytes over that duration is the roofline entry.  e2e repeats the
+inside the graph give each kernel's average duration; the dominant kernel's
+algorithmic bytes over that duration is the roofline entry (the fused step
+kernel: the whole step's bytes; separate path: the attention kernel's).  e2e repeats the
 measurement through the public API with packed pinned host inputs and
 outputs (one H2D + graph replay + one D2H per step).  cpu_baseline times the
 CPU oracle on a bounded sample of the same step (2 of 32 layers) on the host
@@ -50,6 +55,8 @@ METRIC = "evict+paged-decode steps/s"
 # profiles/attn_kernel_llama32k_16L.md scaled x2 to the full launch.  Reported
 # only while the attention kernel's sources are the ones that were captured.
 ATTN_TRAFFIC = {"sources_sha256": "6e67ee544df2f78e", "workload": "llama32k", "bytes_per_launch": 2 * 139.574528e6}
+# The same for the fused step kernel (none captured yet for its sources).
+STEP_TRAFFIC = None
 UNIT = "steps/s"
 SAMPLE_LAYERS = 2  # CPU oracle sample: 2 of the workload's layers, time scaled by L / 2
 
@@ -217,16 +224,24 @@ def run_rkv(args, world, rank, local):
     dc = workloads.prefill_cache(cfg, seed, device=dev, n_steps=total)
     cache = rkv.Cache.from_tensors(dc, cfg.B, cfg.L, cfg.H, cfg.Hq)
     stream = torch.cuda.Stream(device=dev)
-    runner = rkv.StepRunner(cache, scale=cfg.scale, stream=stream)
+    fused = args.path == "fused"
+    runner = rkv.StepRunner(cache, scale=cfg.scale, stream=stream, fused=fused)
     sel, ws, outs = runner.sel, runner.ws, runner.outs
 
     # inputs of every step, resident on the device
     per_step = [workloads.step_inputs(cfg, seed, s, dev) for s in range(total)]
+    kernel_names = ["step"] if fused else ["select", "attn", "compact", "append"]
 
     def enqueue(s, ev=None):
         inp = per_step[s]
         if not inp["evict"]:
             raise RuntimeError("bench workloads evict every step")
+        if fused:
+            rkv.decode_step(cache, inp["t"], inp["m_global"], inp["q"], cfg.scale, inp["k_new"], inp["v_new"],
+                            inp["lb_new"], sel, outs.out, outs.lse, outs.dropped, ws, stream)
+            if ev is not None:
+                ev[0].record(stream)
+            return
         rkv.score_select(cache, inp["t"], inp["m_global"], sel, ws, stream)
         if ev is not None:
             ev[0].record(stream)
@@ -297,13 +312,12 @@ def run_rkv(args, world, rank, local):
     status = ws.status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
-    kern = {"select": [], "attn": [], "compact": [], "append": []}
+    kern = {k: [] for k in kernel_names}
     for i in range(K):
         e = evs[i]
-        kern["select"].append(e[4].elapsed_time(e[0]))
-        kern["attn"].append(e[0].elapsed_time(e[1]))
-        kern["compact"].append(e[1].elapsed_time(e[2]))
-        kern["append"].append(e[2].elapsed_time(e[3]))
+        marks = [e[4]] + e[:len(kernel_names)]
+        for j, k in enumerate(kernel_names):
+            kern[k].append(marks[j].elapsed_time(marks[j + 1]))
     kern_us = {k: 1000.0 * statistics.mean(v) for k, v in kern.items()}
     clocks = clk.summary()
 
@@ -352,11 +366,18 @@ def run_rkv(args, world, rank, local):
         cpu = {"value": o["value"], "unit": UNIT, "cores": o["cores"], "kind": "oracle", "sample": o["sample"]}
 
     peaks = _peaks()
-    a_bytes = attn_bytes(cfg, n_pre, kept, pages)
-    attn_s = kern_us["attn"] * 1e-6
-    achieved = a_bytes / attn_s / 1e9
-    step_s = ms_max / K / 1000.0
     s_bytes = step_bytes(cfg, n_pre, kept, pages)
+    if fused:
+        # one launch does the whole step: its algorithmic bytes are the step's
+        a_bytes, dom_s = s_bytes, kern_us["step"] * 1e-6
+        kernel_desc = "step_kernel (selection + paged decode attention + dropped mass + compaction + append)"
+        traffic = attn_traffic(cfg, args.traffic, STEP_TRAFFIC, "step")
+    else:
+        a_bytes, dom_s = attn_bytes(cfg, n_pre, kept, pages), kern_us["attn"] * 1e-6
+        kernel_desc = "attn_kernel (paged decode attention + dropped mass)"
+        traffic = attn_traffic(cfg, args.traffic, ATTN_TRAFFIC, "attn")
+    achieved = a_bytes / dom_s / 1e9
+    step_s = ms_max / K / 1000.0
     retained = (2 if cfg.kv_dtype == "bf16" else 4) * 2 * cfg.D * kept
     line = {
         "metric": METRIC, "value": world * K / (ms_max / 1000.0), "unit": UNIT, "n_gpus": world, "steps": K,
@@ -369,14 +390,13 @@ def run_rkv(args, world, rank, local):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "no flush: per-step K/V working set > 126 MB L2", "graph": use_graph},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": attn_traffic(cfg, args.traffic),
-                     "kernel": "attn_kernel (paged decode attention + dropped mass)",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "kernel": kernel_desc,
                      "bytes_per_launch": a_bytes, "peak_source": peaks["source"]},
         "step_hbm": {"bytes_per_step": s_bytes, "achieved_gbs": s_bytes / step_s / 1e9,
                      "frac": s_bytes / step_s / 1e9 / peaks["hbm_gbs"]},
         "retained_kv": {"gbs": retained / step_s / 1e9, "frac_of_peak": retained / step_s / 1e9 / peaks["hbm_gbs"]},
         "kernels_us": kern_us, "us_per_step": 1000.0 * ms_max / K, "step0_ms": step0_ms,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * K, "clocks": clocks,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(kernel_names) * K, "clocks": clocks, "path": args.path,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -408,17 +428,30 @@ def _graph_upload(graph, stream):
         pass
 
 
-def attn_traffic(cfg: workloads.Config, override):
-    """ncu DRAM bytes per attention launch, or None if not measured for these sources."""
-    if override is not None:
-        return override
+TRAFFIC_SOURCES = {
+    "attn": ("retention_scored_kv_b200/csrc/attn.cu", "retention_scored_kv_b200/csrc/attn_core.cuh",
+             "retention_scored_kv_b200/csrc/common.cuh"),
+    "step": ("retention_scored_kv_b200/csrc/step.cu", "retention_scored_kv_b200/csrc/attn_core.cuh",
+             "retention_scored_kv_b200/csrc/common.cuh"),
+}
+
+
+def sources_sha(kind: str) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in ("retention_scored_kv_b200/csrc/attn.cu", "retention_scored_kv_b200/csrc/common.cuh"):
+    for f in TRAFFIC_SOURCES[kind]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    if cfg.name == ATTN_TRAFFIC["workload"] and h.hexdigest()[:16] == ATTN_TRAFFIC["sources_sha256"]:
-        return ATTN_TRAFFIC["bytes_per_launch"]
+    return h.hexdigest()[:16]
+
+
+def attn_traffic(cfg: workloads.Config, override, record: dict | None, kind: str):
+    """ncu DRAM bytes per launch of the dominant kernel, or None if not
+    measured for these sources and this workload."""
+    if override is not None:
+        return override
+    if record and cfg.name == record["workload"] and sources_sha(kind) == record["sources_sha256"]:
+        return record["bytes_per_launch"]
     return None
 
 
@@ -462,6 +495,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0, help="cut the workload to this many layers (profiling)")
     ap.add_argument("--cpu-steps", type=int, default=250)
+    ap.add_argument("--path", choices=["fused", "separate"], default="fused",
+                    help="fused: one rkv_decode_step launch per step; separate: the four entry points")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")

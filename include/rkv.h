@@ -102,7 +102,9 @@ typedef struct rkv_cache {
 
 /* Result of one selection, consumed by attention, dropped mass and
  * compaction of the same step.  Device buffers owned by the caller:
- *   kappa      [B] uint64   entry e of sequence b is kept iff key(e) < kappa[b]
+ *   kappa      [B] uint64   entry e of sequence b is kept iff key(e) < kappa[b];
+ *                           kappa = (largest kept key) + 1, or 0 when nothing
+ *                           and ~0 when everything is kept
  *                           (key defined at rkv_score_select)
  *   kept       [C] int32    entries of head c that are kept
  *   n_pre      [C] int32    len[c] when the selection ran
@@ -133,8 +135,12 @@ RKV_API size_t rkv_workspace_size(const rkv_cache_t *cache);
  * allocating it, and again after a nonzero device status. */
 RKV_API int rkv_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
-/* Device address of the int32 status word inside the workspace (RKV_DEV_*
- * bits, sticky until rkv_workspace_init).  Pure pointer arithmetic. */
+/* Device address of the status block inside the workspace: int32[4] =
+ *   [0] RKV_DEV_* bits (sticky until rkv_workspace_init)
+ *   [1] site of the first bounded wait that gave up (0: none), for reports
+ *   [2] rkv_decode_step calls whose selection was resolved in the threshold
+ *       window, [3] those that ran the exact selection (cumulative counters).
+ * Pure pointer arithmetic. */
 RKV_API int32_t *rkv_device_status(void *ws);
 
 /* ---------------------------------------------------------------------------
@@ -252,6 +258,46 @@ RKV_API int rkv_compact_pages(const rkv_cache_t *cache, const rkv_select_t *sel,
 RKV_API int rkv_append(const rkv_cache_t *cache, const int32_t *t, const void *k_new,
                        const void *v_new, const float *lb_new, void *ws, size_t ws_bytes,
                        void *stream);
+
+/* ---------------------------------------------------------------------------
+ * rkv_decode_step -- one whole decode step in one launch, with the results
+ * of the separate calls
+ *     m_global != NULL:  rkv_score_select -> rkv_paged_decode_attn (with
+ *                        the selection, dropped mass included) ->
+ *                        rkv_compact_pages -> rkv_append
+ *     m_global == NULL:  rkv_paged_decode_attn (every entry kept) ->
+ *                        rkv_append  (a step that evicts nothing)
+ * Selection outputs, keep masks, block tables, lengths, pools and the free
+ * stack are identical to those calls; out / lse_kept / dropped agree with
+ * them within floating-point rounding (the sums are grouped differently).
+ *
+ * Steady decoding keeps each sequence's threshold in a window inside the
+ * workspace (shared with rkv_score_select): entries whose keys fall outside
+ * the previous call's window are classified while their K/V stream through
+ * the attention, the few inside it are ranked after one grid barrier.  When
+ * the window cannot decide (first call on a workspace, a prefill-sized
+ * eviction, a sharp change of scores) the exact radix selection runs inside
+ * the same launch before the attention, so the result never depends on the
+ * window -- only the time does.
+ *
+ *   t, q, scale, out, lse_kept, dropped   as rkv_paged_decode_attn
+ *   m_global  [B] int64 or NULL   budgets, as rkv_score_select
+ *   k_new, v_new, lb_new          as rkv_append
+ *   sel       selection outputs (required when m_global != NULL; kappa,
+ *             kept, n_pre, keep_mask and plan are written)
+ * Limits: B <= 64; B*L*H <= 384 * (SM count); the (dtype, D, G) instances
+ * of rkv_paged_decode_attn; max_pages small enough for the compaction
+ * scratch in shared memory (about 14 bytes per page on top of the
+ * attention stages).  q, k_new, v_new, pos_pool and lb_pool 16-byte aligned.
+ * Errors: RKV_ERR_INVALID_ARG, RKV_ERR_UNSUPPORTED,
+ * RKV_ERR_WORKSPACE_TOO_SMALL, RKV_ERR_CUDA.  Device: RKV_DEV_BAD_INPUT,
+ * RKV_DEV_POOL_EXHAUSTED, RKV_DEV_TABLE_OVERFLOW, RKV_DEV_TIMEOUT (then
+ * re-initialise the workspace).  One cooperative launch, one CTA per SM.
+ */
+RKV_API int rkv_decode_step(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
+                            const float *q, float scale, const void *k_new, const void *v_new,
+                            const float *lb_new, const rkv_select_t *sel, float *out, float *lse_kept,
+                            float *dropped, void *ws, size_t ws_bytes, void *stream);
 
 #ifdef __cplusplus
 }

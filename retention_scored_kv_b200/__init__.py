@@ -7,10 +7,11 @@ raises.
 
 Entry points (same names as the C ABI, without the ``rkv_`` prefix):
 ``score_select``, ``paged_decode_attn``, ``dropped_mass``, ``compact_pages``,
-``append``, ``workspace_size``, ``workspace_init``, ``device_status``,
-``version``, ``last_error``.  ``Cache``/``Selection``/``Workspace`` hold the
-tensors and build the C structs; ``step`` runs one decode step in the order
-select -> attention (+ dropped mass) -> compaction -> append.
+``append``, ``decode_step``, ``workspace_size``, ``workspace_init``,
+``device_status``, ``version``, ``last_error``.  ``Cache``/``Selection``/
+``Workspace`` hold the tensors and build the C structs; ``step`` runs one
+decode step, either as the separate calls select -> attention (+ dropped
+mass) -> compaction -> append or as the single fused ``decode_step`` launch.
 """
 from __future__ import annotations
 
@@ -30,7 +31,8 @@ BF16, F32 = 0, 1
 PAGE = 16
 
 EXPORTS = ("rkv_version", "rkv_last_error", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status",
-           "rkv_score_select", "rkv_paged_decode_attn", "rkv_dropped_mass", "rkv_compact_pages", "rkv_append")
+           "rkv_score_select", "rkv_paged_decode_attn", "rkv_dropped_mass", "rkv_compact_pages", "rkv_append",
+           "rkv_decode_step")
 
 
 class RkvError(RuntimeError):
@@ -77,6 +79,7 @@ def load(path: str | None = None):
         "rkv_dropped_mass": (I, [CP, P, ctypes.c_float, SP, P, P, SZ, P]),
         "rkv_compact_pages": (I, [CP, SP, P, SZ, P]),
         "rkv_append": (I, [CP, P, P, P, P, P, SZ, P]),
+        "rkv_decode_step": (I, [CP, P, P, P, ctypes.c_float, P, P, P, SP, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -195,6 +198,12 @@ class Workspace:
         """RKV_DEV_* bits recorded on the device (reads one int32)."""
         return int(self.buf[:4].view(torch.int32).item())
 
+    def counters(self) -> dict:
+        """The device status block: bits, first timeout site, and the fused
+        steps resolved in the threshold window / by the exact selection."""
+        v = self.buf[:16].view(torch.int32).tolist()
+        return {"status": v[0], "timeout_site": v[1], "window_steps": v[2], "exact_steps": v[3]}
+
 
 def version() -> str:
     return load().rkv_version().decode()
@@ -256,6 +265,17 @@ def append(cache: Cache, t: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tens
                              ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
 
 
+def decode_step(cache: Cache, t: torch.Tensor, m_global: torch.Tensor | None, q: torch.Tensor, scale: float,
+                k_new: torch.Tensor, v_new: torch.Tensor, lb_new: torch.Tensor, sel: Selection | None,
+                out: torch.Tensor, lse: torch.Tensor | None, dropped: torch.Tensor | None, ws: Workspace,
+                stream=None):
+    cs = cache.struct()
+    ss = ctypes.byref(sel.struct()) if sel is not None else None
+    _check(load().rkv_decode_step(ctypes.byref(cs), _ptr(t), _ptr(m_global), _ptr(q), ctypes.c_float(scale),
+                                  _ptr(k_new), _ptr(v_new), _ptr(lb_new), ss, _ptr(out), _ptr(lse), _ptr(dropped),
+                                  ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
 @dataclass
 class StepOutputs:
     out: torch.Tensor      # [B, L, Hq, D] float32
@@ -271,12 +291,17 @@ class StepOutputs:
 
 
 def step(cache: Cache, sel: Selection, ws: Workspace, outs: StepOutputs, *, q, t, m_global, k_new, v_new,
-         lb_new, evict: bool = True, scale: float | None = None, stream=None):
+         lb_new, evict: bool = True, scale: float | None = None, fused: bool = False, stream=None):
     """One decode step: [select] -> attention + dropped mass -> [compaction] -> append.
 
-    On a non-evicting step every entry is kept and the dropped mass is 0."""
+    On a non-evicting step every entry is kept and the dropped mass is 0.
+    ``fused`` runs the whole step as one ``decode_step`` launch."""
     if scale is None:
         scale = 1.0 / math.sqrt(cache.D)
+    if fused:
+        decode_step(cache, t, m_global if evict else None, q, scale, k_new, v_new, lb_new, sel if evict else None,
+                    outs.out, outs.lse, outs.dropped, ws, stream)
+        return
     if evict:
         score_select(cache, t, m_global, sel, ws, stream)
         paged_decode_attn(cache, q, scale, sel, outs.out, outs.lse, outs.dropped, ws, stream)
@@ -299,8 +324,10 @@ class StepRunner:
     device-to-host copy.  ``in_layout`` / ``out_layout`` give each field's byte
     offset, shape and dtype so callers can pack pinned host buffers."""
 
-    def __init__(self, cache: Cache, *, scale: float | None = None, use_graph: bool = True, stream=None):
+    def __init__(self, cache: Cache, *, scale: float | None = None, use_graph: bool = True, fused: bool = True,
+                 stream=None):
         self.cache = cache
+        self.fused = fused
         self.scale = 1.0 / math.sqrt(cache.D) if scale is None else scale
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         dev = cache.len.device
@@ -328,6 +355,7 @@ class StepRunner:
         self.sel = Selection.empty(cache)
         self.ws = Workspace(cache, self.stream)
         self.use_graph = use_graph
+        self.capture_error: str | None = None
         self.graphs: dict[bool, torch.cuda.CUDAGraph] = {}
 
     @staticmethod
@@ -347,11 +375,15 @@ class StepRunner:
         i = self.inp
         step(self.cache, self.sel, self.ws, self.outs, q=i["q"], t=i["t"], m_global=i["m_global"],
              k_new=i["k_new"], v_new=i["v_new"], lb_new=i["lb_new"], evict=evict, scale=self.scale,
-             stream=self.stream)
+             fused=self.fused, stream=self.stream)
 
     def capture(self) -> bool:
         """Capture the evicting and non-evicting step; False if capture is refused."""
         if not self.use_graph:
+            return False
+        if self.stream == torch.cuda.default_stream(self.stream.device):
+            self.capture_error = "CUDA graphs need a non-default stream: pass stream=torch.cuda.Stream()"
+            self.use_graph = False
             return False
         try:
             for evict in (True, False):
@@ -360,7 +392,8 @@ class StepRunner:
                     self._enqueue(evict)
                 self.graphs[evict] = g
             return True
-        except Exception:
+        except Exception as ex:
+            self.capture_error = f"{type(ex).__name__}: {ex}"
             self.graphs.clear()
             self.use_graph = False
             return False

@@ -82,18 +82,36 @@ void layout_for(const rkv_cache_t &c, int sel_groups_x_waves, WsLayout *L) {
         off += bytes;
         return at;
     };
-    L->status = take(4, 4);
+    L->status = take(16, 16);  // bits, first timeout site, fused steps resolved in the window / exactly
     L->done_compact = take(4, 4);
     L->done_append = take(4, 4);
     L->bar = take(4, 64);
     L->leave = take(4, 64);
     L->win = take((size_t)c.B * 16, 16);
     L->cnt = take((size_t)c.B * 16, 16);
+    L->kmax = take((size_t)c.B * 8, 16);
     L->cand = take((size_t)c.B * WIN_CAP * 8, 16);
     L->more = take((size_t)c.B * NPASS * 4, 16);
     L->hist = take((size_t)sel_groups_x_waves * NPASS * NBINS * 4, 256);
     L->head_cnt = take((size_t)C * 4, 256);
     L->partial = take((size_t)MAX_ATTN_CTAS * 2 * attn_partial_rec_floats(c.D, G) * 4, 256);
+    // fused decode step (nothing when the batch is too large for it)
+    const int SB = c.B <= STEP_MAX_B ? c.B : 0;
+    const int64_t SC = SB ? C : 0;
+    const size_t cw = SB ? step_ctr_words(SC, SB) : 0;
+    L->step_bar = take(4, 64);
+    L->step_leave = take(4, 64);
+    L->step_parity = take(4, 64);
+    L->step_ctr = take(2 * cw * 4, 256);
+    L->ckey = take((size_t)SB * WIN_CAP * 8, 256);
+    L->cslot = take((size_t)SB * WIN_CAP * 4, 256);
+    L->cfate = take((size_t)SB * WIN_CAP * 4, 256);
+    L->cz = take((size_t)SB * WIN_CAP * G * 4, 256);
+    L->cv = take((size_t)SB * WIN_CAP * c.D * elt_bytes(c.dtype), 256);
+    L->ghist = take((size_t)NPASS * SB * NBINS * 4, 256);
+    L->hrec = take((size_t)SC * attn_partial_rec_floats(c.D, G) * 4, 256);
+    L->npre = take((size_t)SC * 4, 256);
+    L->pfx = take((size_t)(SC + 1) * 4, 256);
     L->total = take(0, 256);
 }
 
@@ -224,6 +242,7 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
     a.leave = at<uint32_t>(ws, L.leave);
     a.win = at<uint32_t>(ws, L.win);
     a.cnt = at<uint32_t>(ws, L.cnt);
+    a.kmax = at<unsigned long long>(ws, L.kmax);
     a.cand = at<uint2>(ws, L.cand);
     a.more = at<uint32_t>(ws, L.more);
     a.hist = at<uint32_t>(ws, L.hist);
@@ -291,6 +310,7 @@ RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t,
     a.more = scr + NOALLOC_MORE;
     a.win = scr + NOALLOC_WIN;
     a.cnt = scr + NOALLOC_CNT;
+    a.kmax = reinterpret_cast<unsigned long long *>(scr + NOALLOC_KMAX);
     a.cand = reinterpret_cast<uint2 *>(scr + NOALLOC_CAND);
     a.hist = scr + NOALLOC_HIST;
     a.n_groups = g.n_groups;
@@ -355,6 +375,99 @@ RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float sca
     if (!dropped) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: dropped is NULL");
     if (!sel) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: sel is NULL");
     return attn_common(cache, q, scale, sel, nullptr, nullptr, dropped, ws, ws_bytes, stream, "rkv_dropped_mass");
+}
+
+RKV_API int rkv_decode_step(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global, const float *q,
+                            float scale, const void *k_new, const void *v_new, const float *lb_new,
+                            const rkv_select_t *sel, float *out, float *lse_kept, float *dropped, void *ws,
+                            size_t ws_bytes, void *stream) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if (!t || !q || !k_new || !v_new || !lb_new || !out)
+        return fail(RKV_ERR_INVALID_ARG, "rkv_decode_step: t, q, k_new, v_new, lb_new and out must be non-NULL");
+    if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(cache->pos_pool) ||
+        !aligned16(cache->lb_pool))
+        return fail(RKV_ERR_INVALID_ARG, "rkv_decode_step: q, k_new, v_new, pos_pool and lb_pool must be 16-byte aligned");
+    if (m_global && (rc = check_sel(sel))) return rc;
+    if (cache->B > STEP_MAX_B)
+        return fail(RKV_ERR_UNSUPPORTED, "rkv_decode_step: at most %d sequences per call (B = %d)", STEP_MAX_B,
+                    cache->B);
+    const int G = cache->Hq / cache->H;
+    if (!step_supported(cache->dtype, cache->D, G))
+        return fail(RKV_ERR_UNSUPPORTED, "rkv_decode_step: (dtype %d, D %d, G %d) not built", cache->dtype, cache->D, G);
+    const int64_t LH = (int64_t)cache->L * cache->H;
+    const int lb = lh_bits(LH);
+    if (lb > 24) return fail(RKV_ERR_UNSUPPORTED, "L*H must be <= 2^24");
+    WsLayout L;
+    if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
+    int sms = 0;
+    if ((rc = sm_count_now(&sms))) return rc;
+    const int grid = sms < MAX_ATTN_CTAS ? sms : MAX_ATTN_CTAS;
+    const int64_t C = (int64_t)cache->B * LH;
+    if (C > (int64_t)STEP_HEADS_PER_CTA * grid)
+        return fail(RKV_ERR_UNSUPPORTED, "rkv_decode_step: %lld heads exceed %d per SM", (long long)C,
+                    STEP_HEADS_PER_CTA);
+    const size_t smem = step_smem_bytes(cache->dtype, cache->D, G, cache->max_pages);
+    if (smem == 0 || smem > 227 * 1024)
+        return fail(RKV_ERR_UNSUPPORTED, "rkv_decode_step: max_pages %d needs %zu bytes of shared memory",
+                    cache->max_pages, smem);
+    StepArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.pos_pool = cache->pos_pool;
+    a.lb_pool = cache->lb_pool;
+    a.block_table = cache->block_table;
+    a.len = cache->len;
+    a.free_stack = cache->free_stack;
+    a.free_top = cache->free_top;
+    a.B = cache->B;
+    a.LH = (int)LH;
+    a.C = (int)C;
+    a.max_pages = cache->max_pages;
+    a.ibits = 32 - lb;
+    a.row_bytes = cache->D * elt_bytes(cache->dtype);
+    a.t = t;
+    a.m_global = m_global;
+    a.q = q;
+    a.qscale = scale * 1.4426950408889634f;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.lb_new = lb_new;
+    a.out = out;
+    a.lse = lse_kept;
+    a.dropped = dropped;
+    if (m_global) {
+        a.kappa = sel->kappa;
+        a.kept = sel->kept;
+        a.n_pre = sel->n_pre;
+        a.keep_mask = sel->keep_mask;
+        a.plan = sel->plan;
+    }
+    a.status = at<int32_t>(ws, L.status);
+    a.bar = at<uint32_t>(ws, L.step_bar);
+    a.leave = at<uint32_t>(ws, L.step_leave);
+    a.parity = at<uint32_t>(ws, L.step_parity);
+    a.ctr = at<uint32_t>(ws, L.step_ctr);
+    a.ctr_words = (int)step_ctr_words(C, cache->B);
+    a.win = at<uint32_t>(ws, L.win);
+    a.ckey = at<uint64_t>(ws, L.ckey);
+    a.cslot = at<int32_t>(ws, L.cslot);
+    a.cfate = at<int32_t>(ws, L.cfate);
+    a.cz = at<float>(ws, L.cz);
+    a.cv = at<unsigned char>(ws, L.cv);
+    a.ghist = at<uint32_t>(ws, L.ghist);
+    a.partial = at<float>(ws, L.partial);
+    a.hrec = at<float>(ws, L.hrec);
+    a.npre = at<int32_t>(ws, L.npre);
+    a.pfx = at<int32_t>(ws, L.pfx);
+    CUtensorMap tk{}, tv{};
+    if (attn_uses_tensor_maps(cache->dtype)) {
+        if ((rc = encode_pool_map(&tk, cache->k_pool, cache->D, cache->n_pages))) return rc;
+        if ((rc = encode_pool_map(&tv, cache->v_pool, cache->D, cache->n_pages))) return rc;
+    }
+    cudaError_t e = launch_step(a, cache->dtype, cache->D, G, grid, static_cast<cudaStream_t>(stream), tk, tv);
+    if (e != cudaSuccess) return cuda_fail(e, "rkv_decode_step");
+    return RKV_OK;
 }
 
 RKV_API int rkv_compact_pages(const rkv_cache_t *cache, const rkv_select_t *sel, void *ws, size_t ws_bytes,

@@ -44,6 +44,13 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t bits) {
     if ((__ldcg(status) & bits) != bits) atomicOr(status, bits);
 }
 
+// A bounded wait that gave up: RKV_DEV_TIMEOUT in status[0] and, if no
+// earlier wait gave up, its site code in status[1].
+__device__ __forceinline__ void record_timeout(int32_t *status, int32_t site) {
+    set_status(status, RKV_DEV_TIMEOUT);
+    atomicCAS(status + 1, 0, site);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -62,7 +69,7 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 // The wait is bounded (~2 s of globaltimer); on timeout RKV_DEV_TIMEOUT is
 // recorded and false returned, so the caller can leave the kernel.
 __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, int32_t *status,
-                                             int *smem_flag) {
+                                             int *smem_flag, int32_t site = 0x100) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -74,7 +81,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, in
             uint32_t spins = 0;
             while (ld_acquire_gpu(count) < target) {
                 if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
-                    set_status(status, RKV_DEV_TIMEOUT);
+                    record_timeout(status, site + (int32_t)epoch);
                     ok = 0;
                     break;
                 }
@@ -85,6 +92,32 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, in
     }
     __syncthreads();
     return *smem_flag != 0;
+}
+
+// Threshold window kept across calls, per sequence: w[0] valid, [w[1], w[2])
+// the score-key (high word) range whose keys are ranked individually next
+// call, w[3] its half width.  Centred on this call's threshold score key and
+// resized by how this call went: wres 1 resolved in the window (wn
+// candidates: shrink above WIN_CAP/2, grow below 64), 2 missed (grow 4x),
+// 3 too many candidates (shrink 4x), 0 no window was used.  Nothing changes
+// when nothing or everything was kept (kappa 0 or ~0).
+__device__ __forceinline__ void window_next(uint32_t *w, uint64_t kappa, int wres, uint32_t wn) {
+    if (kappa == 0ull || kappa == ~0ull) return;
+    const uint32_t center = (uint32_t)((kappa - 1ull) >> 32);
+    uint32_t hw = w[3];
+    if (hw == 0u) hw = 1u << 14;
+    if (wres == 1) {
+        if (wn > WIN_CAP / 2) hw = hw > 1u ? hw >> 1 : 1u;
+        else if (wn < 64u) hw = hw < (1u << 28) ? hw << 1 : hw;
+    } else if (wres == 2) {
+        hw = hw < (1u << 26) ? hw << 2 : (1u << 28);
+    } else if (wres == 3) {
+        hw = hw > 4u ? hw >> 2 : 1u;
+    }
+    w[1] = center > hw ? center - hw : 0u;
+    w[2] = center < 0xFFFFFFFFu - hw ? center + hw : 0xFFFFFFFFu;
+    w[3] = hw;
+    w[0] = 1u;
 }
 
 // ------------------------------------------------ mbarrier / bulk copy ----
@@ -125,14 +158,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Bounded wait on an mbarrier phase.  Every producer of the phase is in the
 // same CTA and always arrives, so the bound is a guard, not a protocol:
 // after ~2 s the wait records RKV_DEV_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status, int32_t site = 1) {
     if (mbar_try_wait(bar, parity)) return true;
     if (__ldcg(status) & RKV_DEV_TIMEOUT) return false;  // an earlier wait already gave up
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
     while (!mbar_try_wait(bar, parity)) {
         if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
-            set_status(status, RKV_DEV_TIMEOUT);
+            record_timeout(status, site);
             return false;
         }
     }

@@ -20,14 +20,33 @@ struct WsLayout {
     size_t bar;           // uint32 grid-barrier counter (reset by the selection's last CTA)
     size_t leave;         // uint32 exit ticket of the selection
     size_t win;           // uint32 [B][4] threshold window per sequence (kept across calls)
-    size_t cnt;           // uint32 [B][4] per-call counters: keys above the window, candidates
+    size_t cnt;           // uint32 [B][4] per-call counters: keys above the window, candidates, window outcome
+    size_t kmax;          // uint64 [B] largest kept key (cleared at exit)
     size_t cand;          // uint2 [B][WIN_CAP] keys inside the window
     size_t more;          // uint32 [waves][NPASS] continuation flags (cleared at exit)
     size_t hist;          // uint32 [waves][NPASS][n_groups][NBINS] (cleared at exit)
     size_t head_cnt;      // uint32 [C], attention split-head arrival counters (self-resetting)
     size_t partial;       // float [MAX_ATTN_CTAS][2][rec], attention partial states
+    // fused decode step (rkv_decode_step)
+    size_t step_bar;      // uint32 grid-barrier counter (reset by the last CTA to leave)
+    size_t step_leave;    // uint32 exit ticket
+    size_t step_parity;   // uint32, which half of step_ctr this call uses (flipped at exit)
+    size_t step_ctr;      // uint32 [2][ctr_words]: per-call counters, one half zeroed while the other is used
+    size_t ckey;          // uint64 [B][WIN_CAP] keys of the window candidates
+    size_t cslot;         // int32  [B][WIN_CAP] logical slot of each candidate in its head
+    size_t cfate;         // int32  [B][WIN_CAP] 1 if the candidate is kept
+    size_t cz;            // float  [B][WIN_CAP][G] base-2 logits of each candidate
+    size_t cv;            // [B][WIN_CAP][row bytes] V row of each candidate (pool dtype)
+    size_t ghist;         // uint32 [NPASS][B][NBINS] exact-select histograms (cleared after use)
+    size_t hrec;          // float  [C][rec] state of whole heads that hold candidates
+    size_t npre;          // int32  [C] pre-step lengths
+    size_t pfx;           // int32  [C+1] page prefix of the pre-step lengths (own range of each CTA)
     size_t total;
 };
+
+// Per-call counters of the fused step: head_kept[C], head_flag[C],
+// seq[B][4] (keys above the window, candidates), misc[16] (compaction arrivals).
+inline size_t step_ctr_words(int64_t C, int B) { return (size_t)(2 * C + 4 * (int64_t)B + 16 + 63) / 64 * 64; }
 
 struct SelectGrid {
     int n_groups, cta_per_group, waves, threads, smem_bytes, cache_pages;
@@ -56,6 +75,7 @@ struct SelectArgs {
     uint32_t *leave;
     uint32_t *win;
     uint32_t *cnt;
+    unsigned long long *kmax;
     uint2 *cand;
     uint32_t *more;
     uint32_t *hist;
@@ -69,11 +89,13 @@ constexpr int NOALLOC_MAX_B = 16;
 constexpr int NOALLOC_MAX_DEVICES = 64;
 constexpr size_t NOALLOC_STATUS = 0, NOALLOC_BAR = 16, NOALLOC_LEAVE = 32, NOALLOC_MORE = 64;
 constexpr size_t NOALLOC_WIN = 192, NOALLOC_CNT = 256;     // [MAX_B][4] each
+constexpr size_t NOALLOC_KMAX = 384;                        // uint64 [MAX_B]
 constexpr size_t NOALLOC_HIST = 512;  // after the flags and counters, 2 KiB aligned
 constexpr size_t NOALLOC_CAND = NOALLOC_HIST + (size_t)NOALLOC_MAX_B * NPASS * NBINS;
 constexpr size_t NOALLOC_WORDS = NOALLOC_CAND + (size_t)NOALLOC_MAX_B * WIN_CAP * 2;
 static_assert(NOALLOC_MORE + NOALLOC_MAX_B * NPASS <= NOALLOC_WIN, "flag region");
-static_assert(NOALLOC_WIN + 4 * NOALLOC_MAX_B <= NOALLOC_CNT && NOALLOC_CNT + 4 * NOALLOC_MAX_B <= NOALLOC_HIST,
+static_assert(NOALLOC_WIN + 4 * NOALLOC_MAX_B <= NOALLOC_CNT && NOALLOC_CNT + 4 * NOALLOC_MAX_B <= NOALLOC_KMAX &&
+                  NOALLOC_KMAX + 2 * NOALLOC_MAX_B <= NOALLOC_HIST,
               "counter region");
 // Device address of that array on the current device (looked up once per
 // device); returns nonzero and sets *err on failure.
@@ -104,6 +126,59 @@ cudaError_t launch_attn(const AttnArgs &a, int dtype, int D, int G, int sm_count
 bool attn_supported(int dtype, int D, int G);
 bool attn_uses_tensor_maps(int dtype);
 size_t attn_partial_rec_floats(int D, int G);
+
+// Fused decode step: selection, attention with dropped mass, compaction and
+// append in one cooperative launch (one CTA per SM).
+constexpr int STEP_MAX_B = 64;      // sequences per call
+constexpr int STEP_HEADS_PER_CTA = 384;  // C <= this * grid
+struct StepArgs {
+    void *k_pool;
+    void *v_pool;
+    int32_t *pos_pool;
+    float *lb_pool;
+    int32_t *block_table;
+    int32_t *len;
+    int32_t *free_stack;
+    int32_t *free_top;
+    int B, LH, C, max_pages, ibits, row_bytes;
+    const int32_t *t;
+    const int64_t *m_global;   // NULL: this step evicts nothing
+    const float *q;
+    float qscale;              // scale * log2(e)
+    const void *k_new;
+    const void *v_new;
+    const float *lb_new;
+    float *out;
+    float *lse;                // may be NULL
+    float *dropped;            // may be NULL
+    uint64_t *kappa;           // selection outputs (evicting steps)
+    int32_t *kept;
+    int32_t *n_pre;
+    uint16_t *keep_mask;
+    int32_t *plan;
+    int32_t *status;
+    uint32_t *bar;
+    uint32_t *leave;
+    uint32_t *parity;
+    uint32_t *ctr;             // [2][ctr_words]
+    int ctr_words;
+    uint32_t *win;             // [B][4], shared with the selection kernel
+    uint64_t *ckey;
+    int32_t *cslot;
+    int32_t *cfate;
+    float *cz;
+    unsigned char *cv;
+    uint32_t *ghist;
+    float *partial;
+    float *hrec;
+    int32_t *npre;
+    int32_t *pfx;
+};
+bool step_supported(int dtype, int D, int G);
+// Shared memory the step kernel needs for this shape (0: not supported).
+size_t step_smem_bytes(int dtype, int D, int G, int max_pages);
+cudaError_t launch_step(const StepArgs &a, int dtype, int D, int G, int grid, cudaStream_t s,
+                        const CUtensorMap &tk, const CUtensorMap &tv);
 
 struct CompactArgs {
     void *k_pool;

@@ -43,6 +43,7 @@ struct SelSmem {
     uint2 *keys;      // [cache_pages * 16]
     int *flag;        // barrier / misc flags
     uint32_t *bcast;  // [4] broadcast words
+    unsigned long long *kmax;  // largest kept key of this CTA's pages
 };
 
 struct SeqState {
@@ -304,28 +305,6 @@ __device__ void try_window(const SelectArgs &a, const SelSmem &sm, SeqState &st)
     __syncthreads();
 }
 
-// Window for the next call, centred on this call's threshold score key and
-// resized by what this call saw (group leader only).
-__device__ void update_window(const SelectArgs &a, const SeqState &st) {
-    if (st.kappa == 0ull || st.kappa == ~0ull) return;  // nothing or everything kept
-    uint32_t *w = a.win + (size_t)st.b * 4;
-    const uint32_t center = (uint32_t)((st.kappa - 1ull) >> 32);
-    uint32_t hw = w[3];
-    if (hw == 0u) hw = 1u << 14;
-    if (st.wres == 1) {
-        if (st.wn > WIN_CAP / 2) hw = hw > 1u ? hw >> 1 : 1u;
-        else if (st.wn < 64u) hw = hw < (1u << 28) ? hw << 1 : hw;
-    } else if (st.wres == 2) {
-        hw = hw < (1u << 26) ? hw << 2 : (1u << 28);
-    } else if (st.wres == 3) {
-        hw = hw > 4u ? hw >> 2 : 1u;
-    }
-    w[1] = center > hw ? center - hw : 0u;
-    w[2] = center < 0xFFFFFFFFu - hw ? center + hw : 0xFFFFFFFFu;
-    w[3] = hw;
-    w[0] = 1u;
-}
-
 // Head (local index) of a page from the key of its slot 0 (lo = cl << ib | i).
 __device__ __forceinline__ int head_of(const SelectArgs &a, const SelSmem &sm, int x, uint2 k0) {
     if (k0.x != KEY_INVALID) return a.ibits >= 32 ? 0 : (int)(k0.y >> a.ibits);
@@ -334,11 +313,17 @@ __device__ __forceinline__ int head_of(const SelectArgs &a, const SelSmem &sm, i
 
 // Keep masks (half-warp ballots over the 16 slots of a page); kept counts are
 // summed per head in shared memory and flushed with one atomic per head.
+// The largest kept key goes to a.kmax[b]: the reported threshold is that key
+// + 1 whichever way it was found (a radix bucket kept whole only bounds it).
 __device__ void final_pass(const SelectArgs &a, const SelSmem &sm, const SeqState &st) {
     const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) *sm.kmax = 0ull;
+    __syncthreads();
+    unsigned long long kmx = 0ull;
     for_keys(a, sm, st, false, [&](int x, int r, uint2 k) {
         const uint64_t K = ((uint64_t)k.x << 32) | k.y;
         const bool keep = x < st.x1 && k.x != KEY_INVALID && K < st.kappa;
+        if (keep && K > kmx) kmx = K;
         const uint32_t ball = __ballot_sync(0xFFFFFFFFu, keep);
         if (r == 0 && x < st.x1) {
             const uint32_t m16 = (ball >> (lane & 16)) & 0xFFFFu;
@@ -348,7 +333,14 @@ __device__ void final_pass(const SelectArgs &a, const SelSmem &sm, const SeqStat
             if (m16) atomicAdd(&sm.kc[cl], __popc(m16));
         }
     });
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(0xFFFFFFFFu, kmx, o);
+        kmx = y > kmx ? y : kmx;
+    }
+    if (lane == 0 && kmx) atomicMax(sm.kmax, kmx);
     __syncthreads();
+    if (threadIdx.x == 0 && *sm.kmax) atomicMax(a.kmax + st.b, *sm.kmax);
     if (st.x0 < st.x1) {
         const int c_lo = page_head(sm.pfx, a.LH, st.x0), c_hi = page_head(sm.pfx, a.LH, st.x1 - 1);
         for (int cl = c_lo + (int)threadIdx.x; cl <= c_hi; cl += blockDim.x) {
@@ -370,6 +362,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         p += 4 * NBINS * sizeof(uint32_t);
         sm.scan = reinterpret_cast<uint32_t *>(p);
         p += 40 * sizeof(uint32_t);
+        sm.kmax = reinterpret_cast<unsigned long long *>(p);
+        p += 16;
         sm.bcast = reinterpret_cast<uint32_t *>(p);
         p += 4 * sizeof(uint32_t);
         sm.flag = reinterpret_cast<int *>(p);
@@ -450,8 +444,15 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
             if (st.active && st.done && !finalized) {
                 final_pass(a, sm, st);
                 if (rr == 0 && threadIdx.x == 0) {
-                    a.kappa[st.b] = st.kappa;
-                    update_window(a, st);
+                    // trivial budgets report kappa now; the others once every
+                    // CTA's largest kept key is in (last CTA to leave)
+                    if (st.m == 0 || st.m == st.n) {
+                        a.kappa[st.b] = st.kappa;
+                        a.cnt[(size_t)st.b * 4 + 2] = 0xFFFFFFFFu;
+                    } else {
+                        a.cnt[(size_t)st.b * 4 + 2] = (uint32_t)st.wres;
+                        a.cnt[(size_t)st.b * 4 + 3] = st.wn;
+                    }
                 }
                 finalized = true;
             }
@@ -494,6 +495,16 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         for (size_t i = threadIdx.x; i < nh; i += blockDim.x) a.hist[i] = 0u;
         for (int i = threadIdx.x; i < a.waves * NPASS; i += blockDim.x) a.more[i] = 0u;
     }
+    for (int b = threadIdx.x; b < a.B; b += blockDim.x) {
+        const uint32_t wres = __ldcg(a.cnt + (size_t)b * 4 + 2);
+        if (wres != 0xFFFFFFFFu) {
+            const uint64_t kap = __ldcg(a.kmax + b) + 1ull;
+            a.kappa[b] = kap;
+            window_next(a.win + (size_t)b * 4, kap, (int)wres, __ldcg(a.cnt + (size_t)b * 4 + 3));
+        }
+        a.kmax[b] = 0ull;
+    }
+    __syncthreads();
     for (int i = threadIdx.x; i < 4 * a.B; i += blockDim.x) a.cnt[i] = 0u;
     // free-page plan over all heads: plan[c] = pages freed in heads < c
     uint32_t carry = 0;
@@ -561,7 +572,7 @@ SelectGrid select_grid_for(const rkv_cache_t &c, int sm_count) {
     g.n_groups = c.B < ctas ? c.B : ctas;
     g.cta_per_group = ctas / g.n_groups;
     g.waves = (c.B + g.n_groups - 1) / g.n_groups;
-    const int fixed = 4 * NBINS * 4 + 40 * 4 + 16 + 16 + (3 * LH + 1) * 4;
+    const int fixed = 4 * NBINS * 4 + 40 * 4 + 16 + 16 + 16 + (3 * LH + 1) * 4;
     const int avail = select_max_smem() - fixed - 1024;
     g.cache_pages = avail > 0 ? avail / (PAGE * (int)sizeof(uint2)) : 0;
     // no point caching more pages than the largest per-CTA share could hold

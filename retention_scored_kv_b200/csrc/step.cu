@@ -1,0 +1,1379 @@
+// step.cu -- one decode step in a single cooperative launch (sm_100a):
+// retention scores and global top-M selection, paged grouped-query decode
+// attention over the kept entries with the dropped mass, compaction of the
+// kept entries and the append of the new token.
+//
+// Make Each Token Count (DBTrimKV), Methodology 2-4, and Cache What Lasts
+// (TRIM-KV), core mechanism 4: every cached entry scores (t - i) * log(beta_i),
+// the top M_global of a sequence over all layers and heads are kept, ties by
+// ascending (layer, head, position), and each head keeps its own length.
+// Trust the Mass (ContourKV), Problem definition and Methodology 2-3: the
+// softmax is renormalised over the kept keys, the dropped mass is the dense
+// weight of the evicted keys, and evicted rows are physically removed.
+//
+// The separate kernels (selection, attention, compaction, append) each pay
+// a launch and a grid ramp, and in steady decoding the selection scans only
+// ~8 bytes per entry against the ~512 bytes of K/V the attention streams.
+// This kernel folds them into one launch:
+//  * Speculative pass.  Each sequence keeps a threshold window across calls
+//    (a score-key range around the previous threshold).  The attention pass
+//    fetches every page's positions and log-retentions with its K/V, builds
+//    each entry's 64-bit rank key and classifies it: below the window's low
+//    key -> kept, at or above its high key -> evicted, inside -> candidate.
+//    Kept and evicted rows go straight into the online softmax; candidates
+//    are set aside with their logits and V row.
+//  * Resolve.  After one grid barrier, per sequence: if the keys below the
+//    window are fewer than M and the candidates reach M, the threshold is the
+//    (M - below)-th smallest candidate; each candidate's fate follows from
+//    its rank among the candidates alone.
+//  * Exact path.  Without a usable window (the prefill eviction, a miss, too
+//    many candidates) an exact radix select runs in the same launch (digits
+//    11/11/10 per 32-bit key half, per-sequence histograms behind bounded
+//    grid barriers), writes the keep masks and kept counts, and the attention
+//    pass then reads the masks.
+//  * Tail.  Heads are dealt to CTAs in contiguous chunks: heads split across
+//    CTAs or holding candidates are merged, candidate keep bits patched, each
+//    head compacted (hole-fill, freed pages pushed at the plan's offsets) and
+//    the new rows appended; a pop waits (bounded) only for a page pushed in
+//    this call.
+// Selection, keep masks, block tables, lengths and the free stack come out
+// identical to the separate calls; attention outputs agree within rounding.
+#include <cuda.h>
+
+#include "attn_core.cuh"
+#include "common.cuh"
+#include "internal.h"
+
+namespace rkv {
+
+namespace {
+
+using namespace core;
+
+constexpr int NTH = ATTN_THREADS;
+constexpr int NWARP = NTH / 32;
+constexpr int MAXB = STEP_MAX_B;
+constexpr int UNR = 4;           // pages per half-warp per round of the exact select
+constexpr int HGRP = 8;          // sequences histogrammed together in the exact select
+constexpr int CMP_PAIRS = 1024;  // hole/source pairs resolved per compaction round
+static_assert(STEP_HEADS_PER_CTA == NTH, "tail chunk = one head per thread");
+
+enum : uint32_t { SF_TRIVIAL = 1u, SF_WIN = 2u, SF_DONE = 4u };
+
+// Tail scratch (offsets in the big region).
+constexpr int T_STASH = 0;                       // int32 [5][NTH]
+constexpr int T_CL = 5 * NTH * 4;                // int32 [WIN_CAP] candidate list of one head
+constexpr int T_PAIRS = T_CL + WIN_CAP * 4;      // int2 [CMP_PAIRS]
+constexpr int T_TBL = T_PAIRS + CMP_PAIRS * 8;   // int32 [mp], src [mp+1], hole [mp+1], uint16 msk [mp]
+
+__host__ __device__ constexpr size_t tail_bytes(int mp) {
+    return (size_t)T_TBL + (size_t)mp * 4 + 2 * ((size_t)mp + 1) * 4 + (size_t)mp * 2 + 16;
+}
+constexpr size_t RADIX_BYTES = (size_t)HGRP * NBINS * 4;
+constexpr size_t RESOLVE_BYTES = (size_t)WIN_CAP * 8;
+
+// Shared memory: the fixed part (pipeline barriers, per-sequence state, scan
+// scratch) first, then the big region: attention stages, positions /
+// log-retentions, query ring, merge slots and stage metadata during an
+// attention pass; scratch of the other phases outside it.
+template <class M, int D, int G>
+struct StepLayout {
+    static constexpr int STAGE_BYTES = M::PAGE_BYTES * 2;
+    static constexpr int NSW0 = 131072 / (NCW * STAGE_BYTES);
+    static constexpr int NSW = NSW0 < 1 ? 1 : (NSW0 > 8 ? 8 : NSW0);   // stages per consumer warp
+    static constexpr int NST = NCW * NSW;
+    static constexpr int QBYTES = G * D * 4;
+    static constexpr int REC = G * (D + 4);                   // partial record floats
+    static constexpr int WSLOT = G * D + 4 * G + 4;           // merge slot: acc, mk, lk, me, le, candidates
+    static constexpr int NBAR = 2 * NST + 2 * QR;
+    static constexpr int OFF_BAR = 0;
+    static constexpr int OFF_SEQ = (NBAR * 8 + 15) / 16 * 16;
+    static constexpr int SEQ_BYTES = MAXB * (7 * 8 + 8 * 4);
+    static constexpr int OFF_SCAN = OFF_SEQ + SEQ_BYTES;      // [4][36] words
+    static constexpr int OFF_MISC = OFF_SCAN + 4 * 36 * 4;    // int [64], int64 [8]
+    static constexpr int FIXED = OFF_MISC + 64 * 4 + 8 * 8;
+    static constexpr int OFF_BIG = (FIXED + M::STAGE_ALIGN - 1) / M::STAGE_ALIGN * M::STAGE_ALIGN;
+    static constexpr int B_STAGE = 0;
+    static constexpr int B_POSLB = NST * STAGE_BYTES;         // [NST][16 positions, 16 log-retentions]
+    static constexpr int B_Q = B_POSLB + NST * 128;
+    static constexpr int B_MERGE = B_Q + QR * QBYTES;
+    static constexpr int B_META = B_MERGE + 2 * NCW * WSLOT * 4;
+    static constexpr int BIG_ATTN = B_META + NST * 4;
+    static_assert(STAGE_BYTES % M::STAGE_ALIGN == 0, "stage alignment");
+    static_assert(QBYTES % 16 == 0, "query block must be a 16-byte multiple");
+    static_assert(NBAR <= NTH, "barrier init");
+    static_assert(BIG_ATTN >= (int)RADIX_BYTES && BIG_ATTN >= (int)RESOLVE_BYTES, "scratch");
+    static size_t smem(int mp) {
+        const size_t big = tail_bytes(mp) > (size_t)BIG_ATTN ? tail_bytes(mp) : (size_t)BIG_ATTN;
+        return (size_t)OFF_BIG + big + M::STAGE_ALIGN;
+    }
+};
+
+struct Sm {
+    uint64_t *bars;
+    uint64_t *lo, *hi, *kap, *pk, *pm;  // [MAXB]
+    unsigned long long *kmx;             // [MAXB] largest kept key of this CTA's pages
+    int64_t *m;                          // [MAXB] clamped budget
+    int32_t *t;                          // [MAXB]
+    uint32_t *n, *rank, *fl, *above, *nc, *off, *wres, *spare;  // [MAXB]
+    uint32_t *scan;                      // [4][36]
+    int *misc;                           // [64]
+    int64_t *misc64;                     // [8]
+    unsigned char *big;
+};
+
+// misc slots
+enum { MS_CSTART = 0, MS_CLAST, MS_RADIX, MS_MISS, MS_BAR, MS_TOTAL, MS_FOUND, MS_DIG, MS_NR, MS_H, MS_NCL,
+       MS_ACTIVE };
+
+struct Ctx {
+    int64_t TP, x0, x1, pfx_start;
+    int c_start, c_last;
+    bool last, evict;
+    int32_t top0;
+    uint32_t par, epoch;
+    int h0, h1;
+    uint32_t my_pfx;
+    bool exact;      // the exact selection ran (its thresholds are reported in the tail)
+    int passes;      // exact-select passes run (histograms to clear)
+    int attn_runs;   // attention passes run
+    // The pipeline barriers are initialised once per launch; a later
+    // attention pass continues their phases: its page indices start after
+    // the pages of the earlier passes (pbase) and its query slots after
+    // their heads (qbase).  Producer and consumer count both alike.
+    int64_t pbase;
+    int qbase;
+    uint32_t *head_kept, *head_flag, *seqc, *arrive;
+};
+
+template <int NSCAN>
+__device__ __forceinline__ void block_scan_n(const uint32_t (&v)[NSCAN], uint32_t (&ex)[NSCAN],
+                                             uint32_t (&tot)[NSCAN], uint32_t *scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t x[NSCAN];
+#pragma unroll
+    for (int s = 0; s < NSCAN; s++) {
+        x[s] = v[s];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x[s], o);
+            if (lane >= o) x[s] += y;
+        }
+        if (lane == 31) scratch[s * 36 + warp] = x[s];
+    }
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int s = 0; s < NSCAN; s++) {
+            uint32_t w = lane < nw ? scratch[s * 36 + lane] : 0u;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+                if (lane >= o) w += y;
+            }
+            if (lane < nw) scratch[s * 36 + lane] = w;
+            if (lane == 31) scratch[s * 36 + 32] = w;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int s = 0; s < NSCAN; s++) {
+        ex[s] = (warp > 0 ? scratch[s * 36 + warp - 1] : 0u) + x[s] - v[s];
+        tot[s] = scratch[s * 36 + 32];
+    }
+    __syncthreads();
+}
+
+// Rank key of one entry: hi = order-preserving map of s = fl32(float(t - i)
+// * lb) (smaller = ranked first), lo = (l*H + h) << ibits | i.  Returns false
+// for an entry the method cannot score (NaN log-retention, age outside
+// [1, 2^24), position out of range).
+__device__ __forceinline__ bool entry_key(int32_t t, uint32_t cl, int32_t pos, float lb, int ibits, uint64_t *K) {
+    const int64_t age = (int64_t)t - pos;
+    if ((lb != lb) || age < 1 || age >= (1 << 24) || pos < 0 || (ibits < 32 && (uint32_t)pos >= (1u << ibits)))
+        return false;
+    float s = __fmul_rn((float)(int32_t)age, lb);
+    if (s == 0.0f) s = 0.0f;
+    *K = ((uint64_t)score_key_desc(s) << 32) | (uint32_t)(((uint64_t)cl << ibits) | (uint32_t)pos);
+    return true;
+}
+
+__device__ __forceinline__ uint32_t below_bits(int w, int nn) {
+    const int lo = w * PAGE;
+    if (lo + PAGE <= nn) return 0xFFFFu;
+    if (lo >= nn) return 0u;
+    return (1u << (nn - lo)) - 1u;
+}
+
+__device__ void scan_words(int32_t *v, int W, uint32_t *scratch) {
+    uint32_t carry = 0;
+    for (int base = 0; base < W; base += blockDim.x) {
+        const int w = base + threadIdx.x;
+        const uint32_t x = w < W ? (uint32_t)v[w] : 0u;
+        uint32_t tot;
+        const uint32_t ex = block_exclusive_scan(x, scratch, &tot);
+        if (w < W) v[w] = (int32_t)(carry + ex);
+        carry += tot;
+    }
+    if (threadIdx.x == 0) v[W] = (int32_t)carry;
+    __syncthreads();
+}
+
+// ------------------------------------------------------------- prologue ----
+template <class M, int D, int G>
+__device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &cx, const CUtensorMap *tmk,
+                                         const CUtensorMap *tmv) {
+    const int tid = threadIdx.x, nct = gridDim.x;
+    cx.par = __ldcg(a.parity) & 1u;
+    uint32_t *mine = a.ctr + (size_t)cx.par * a.ctr_words;
+    uint32_t *other = a.ctr + (size_t)(cx.par ^ 1u) * a.ctr_words;
+    cx.head_kept = mine;
+    cx.head_flag = mine + a.C;
+    cx.seqc = mine + 2 * (size_t)a.C;
+    cx.arrive = cx.seqc + 4 * (size_t)a.B;
+    // the other half is the next call's: clear it now
+    for (size_t i = (size_t)blockIdx.x * NTH + tid; i < (size_t)a.ctr_words; i += (size_t)nct * NTH) other[i] = 0u;
+    cx.top0 = __ldcg(a.free_top);
+    cx.evict = a.m_global != nullptr;
+    cx.epoch = 0;
+    cx.exact = false;
+    cx.passes = 0;
+    cx.attn_runs = 0;
+    cx.pbase = 0;
+    cx.qbase = 0;
+    if (tid < MAXB) sm.n[tid] = 0u;
+    if (tid < 64) sm.misc[tid] = 0;
+    if (tid == 0) {
+        sm.misc[MS_CSTART] = a.C;
+        sm.misc[MS_CLAST] = -1;
+    }
+    if (M::USES_TMAP && tid == 0) {
+        prefetch_tensormap(tmk);
+        prefetch_tensormap(tmv);
+    }
+    __syncthreads();
+    const int CS = (a.C + NTH - 1) / NTH;
+    cx.h0 = min(a.C, tid * CS);
+    cx.h1 = min(a.C, cx.h0 + CS);
+    uint32_t my_pages = 0;
+    for (int c = cx.h0; c < cx.h1; c++) {
+        const int32_t n = max(__ldcg(a.len + c), 0);
+        my_pages += (uint32_t)((n + PAGE - 1) / PAGE);
+        atomicAdd(&sm.n[c / a.LH], (uint32_t)n);
+        if (c % nct == (int)blockIdx.x) {
+            a.npre[c] = n;
+            if (cx.evict) a.n_pre[c] = n;
+        }
+    }
+    uint32_t TPu;
+    cx.my_pfx = block_exclusive_scan(my_pages, sm.scan, &TPu);
+    cx.TP = TPu;
+    cx.x0 = range_lo(blockIdx.x, cx.TP, nct);
+    cx.x1 = range_lo(blockIdx.x + 1, cx.TP, nct);
+    cx.last = blockIdx.x == nct - 1;
+    // first head of the range (first c with pfx + max(pages, 1) > x0) and
+    // the last head the range visits (last c with pfx < x1; every head for
+    // the last CTA)
+    int first = a.C, lastc = -1;
+    int64_t first_pfx = 0;
+    {
+        int64_t p = cx.my_pfx;
+        for (int c = cx.h0; c < cx.h1; c++) {
+            const int64_t pg = (max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE;
+            if (first == a.C && p + (pg > 0 ? pg : 1) > cx.x0) {
+                first = c;
+                first_pfx = p;
+            }
+            if (p < cx.x1 || cx.last) lastc = c;
+            p += pg;
+        }
+    }
+    if (first < a.C) atomicMin(&sm.misc[MS_CSTART], first);
+    if (lastc >= 0) atomicMax(&sm.misc[MS_CLAST], lastc);
+    __syncthreads();
+    if (first < a.C && first == sm.misc[MS_CSTART]) sm.misc64[0] = first_pfx;
+    // per-sequence setup
+    if (tid < a.B) {
+        const int b = tid;
+        sm.t[b] = __ldg(a.t + b);
+        const int64_t N = sm.n[b];
+        uint32_t fl = SF_TRIVIAL | SF_DONE;
+        uint64_t lo = ~0ull, hi = ~0ull, kap = ~0ull;
+        int64_t m = N;
+        if (cx.evict) {
+            const int64_t mg = __ldg(a.m_global + b);
+            m = mg < 0 ? 0 : (mg > N ? N : mg);
+            if (m == 0 || m == N) {
+                kap = m == 0 ? 0ull : ~0ull;
+                lo = hi = kap;
+            } else {
+                const uint32_t *w = a.win + (size_t)b * 4;
+                if (__ldcg(w) != 0u) {
+                    fl = SF_WIN;
+                    lo = (uint64_t)__ldcg(w + 1) << 32;
+                    hi = (uint64_t)__ldcg(w + 2) << 32;
+                } else {
+                    fl = 0u;
+                    atomicOr(&sm.misc[MS_RADIX], 1);
+                }
+                kap = 0ull;
+            }
+        }
+        sm.m[b] = m;
+        sm.fl[b] = fl;
+        sm.lo[b] = lo;
+        sm.hi[b] = hi;
+        sm.kap[b] = kap;
+        sm.wres[b] = 0u;
+        sm.above[b] = 0u;
+        sm.nc[b] = 0u;
+    }
+    __syncthreads();
+    cx.c_start = sm.misc[MS_CSTART];
+    cx.c_last = sm.misc[MS_CLAST];
+    cx.pfx_start = cx.c_start < a.C ? sm.misc64[0] : cx.TP;
+}
+
+// -------------------------------------------------------- attention pass ----
+// Pages are dealt to consumer warps round-robin (page li -> warp li % NCW);
+// each consumer warp owns a private ring filled in order by producer warp
+// (warp % NPW), so every mbarrier has one producer and one consumer.  SPEC
+// classifies entries against the sequences' windows; otherwise the keep
+// masks come from memory (or every entry is kept when nothing is evicted).
+template <class M, int D, int G, bool SPEC>
+__device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &cx, const CUtensorMap *tmk,
+                                          const CUtensorMap *tmv) {
+    using LY = StepLayout<M, D, G>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint64_t *full = sm.bars, *empty = full + LY::NST, *qfull = empty + LY::NST, *qempty = qfull + QR;
+    unsigned char *stage = sm.big + LY::B_STAGE;
+    unsigned char *poslb = sm.big + LY::B_POSLB;
+    float *qring = reinterpret_cast<float *>(sm.big + LY::B_Q);
+    float *merge = reinterpret_cast<float *>(sm.big + LY::B_MERGE);
+    uint32_t *meta = reinterpret_cast<uint32_t *>(sm.big + LY::B_META);
+    __syncthreads();
+    if (cx.attn_runs == 0) {
+        if (tid < LY::NBAR) {
+            // full: producer; empty: the owning consumer warp; qfull: producer 0; qempty: every consumer warp
+            mbar_init(full + tid, tid >= 2 * LY::NST + QR ? NCW : 1);
+        }
+        fence_mbar_init();
+        __syncthreads();
+    }
+    const int64_t pb0 = cx.pbase;
+    // timeout site codes: 0x10 (speculative pass) / 0x20 (mask pass) + wait kind
+    const int32_t site = SPEC ? 0x10 : 0x20;
+    cx.attn_runs++;
+    const bool masks = !SPEC && cx.evict;
+
+    if (warp >= NCW) {
+        // =============================== producers ===============================
+        if constexpr (REG_SPLIT) setmaxnreg_dec<PRODUCER_REGS>();
+        const int pw = warp - NCW;
+        Walker w;
+        w.init(a.len, a.C, cx.x1, cx.last, cx.c_start, cx.pfx_start);
+        const uint64_t pol_kv = policy_evict_first();
+        const uint64_t pol_keep = policy_evict_last();
+        int nq = cx.qbase;
+        int c, pages, n;
+        int64_t pfx;
+        while (w.next(&c, &pfx, &pages, &n)) {
+            if (pages == 0) continue;
+            const int64_t pa = max(pfx, cx.x0), pb = min(pfx + pages, cx.x1);
+            if (pw == 0 && lane == 0) {
+                const int slot = nq % QR;
+                mbar_wait(&qempty[slot], ((nq / QR) & 1) ^ 1, a.status, site + 1);
+                mbar_arrive_expect_tx(&qfull[slot], LY::QBYTES);
+                bulk_g2s(qring + slot * G * D, a.q + (int64_t)c * G * D, LY::QBYTES, &qfull[slot], pol_keep);
+            }
+            nq++;
+            for (int64_t base = pa; base < pb; base += 32) {
+                const int64_t i = base + lane;
+                int32_t phys = 0;
+                uint32_t m = 0;
+                const bool mine = i < pb && ((int)((i - cx.x0 + pb0) % NCW)) % NPW == pw;
+                if (mine) {
+                    const int64_t pidx = i - pfx;
+                    phys = __ldg(a.block_table + (int64_t)c * a.max_pages + pidx);
+                    const int nv = min(PAGE, n - (int)pidx * PAGE);
+                    const uint32_t valid = nv >= PAGE ? 0xFFFFu : ((1u << nv) - 1u);
+                    const uint32_t kp =
+                        masks ? (uint32_t)__ldcg(a.keep_mask + (int64_t)c * a.max_pages + pidx) : 0xFFFFu;
+                    m = SPEC ? (valid << 16) : ((kp & valid) | (valid << 16));
+                }
+                uint32_t todo = __ballot_sync(0xFFFFFFFFu, mine);
+                while (todo) {
+                    const int j = __ffs(todo) - 1;
+                    todo &= todo - 1;
+                    const int32_t pj = __shfl_sync(0xFFFFFFFFu, phys, j);
+                    const uint32_t mj = __shfl_sync(0xFFFFFFFFu, m, j);
+                    if (lane == 0) {
+                        const int64_t li = base + j - cx.x0 + pb0;
+                        const int cw = (int)(li % NCW);
+                        const int64_t nw = li / NCW;
+                        const int sg = cw * LY::NSW + (int)(nw % LY::NSW);
+                        mbar_wait(&empty[sg], (uint32_t)((nw / LY::NSW) & 1) ^ 1u, a.status, site + 2);
+                        meta[sg] = mj;
+                        const bool load_v = SPEC || (mj & 0xFFFFu);
+                        mbar_arrive_expect_tx(&full[sg], M::PAGE_BYTES * (load_v ? 2 : 1) + (SPEC ? 128u : 0u));
+                        M::issue(stage + sg * LY::STAGE_BYTES, load_v, pj, &full[sg], a.k_pool, a.v_pool, tmk, tmv,
+                                 pol_kv);
+                        if (SPEC) {
+                            bulk_g2s(poslb + sg * 128, a.pos_pool + (int64_t)pj * PAGE, 64, &full[sg], pol_keep);
+                            bulk_g2s(poslb + sg * 128 + 64, a.lb_pool + (int64_t)pj * PAGE, 64, &full[sg], pol_keep);
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        cx.qbase = nq;
+    } else {
+        // ================================ consumers ================================
+        if constexpr (REG_SPLIT) setmaxnreg_inc<CONSUMER_REGS>();
+        Walker w;
+        w.init(a.len, a.C, cx.x1, cx.last, cx.c_start, cx.pfx_start);
+        int nq = cx.qbase;
+        int c, pages, n;
+        int64_t pfx;
+        typename M::State st;
+        while (w.next(&c, &pfx, &pages, &n)) {
+            if (pages == 0) {
+                // a head with no entries: o = 0, lse = -inf, dropped = 0
+                if (warp == 0) {
+                    for (int e = lane; e < G * D; e += 32) a.out[(int64_t)c * G * D + e] = 0.0f;
+                    if (lane < G) {
+                        if (a.lse) a.lse[(int64_t)c * G + lane] = -INFINITY;
+                        if (a.dropped) a.dropped[(int64_t)c * G + lane] = 0.0f;
+                    }
+                }
+                continue;
+            }
+            const int64_t pa = max(pfx, cx.x0), pb = min(pfx + pages, cx.x1);
+            const bool whole = (pfx >= cx.x0) && (pfx + pages <= cx.x1);
+            {
+                const int slot = nq % QR;
+                mbar_wait(&qfull[slot], (nq / QR) & 1, a.status, site + 3);
+                M::load_q(st, qring + slot * G * D, a.qscale, lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qempty[slot]);
+            }
+            int b = 0;
+            uint32_t cl = 0;
+            uint64_t wlo = 0, whi = 0;
+            int32_t tb = 0;
+            if constexpr (SPEC) {
+                b = c / a.LH;
+                cl = (uint32_t)(c - b * a.LH);
+                wlo = sm.lo[b];
+                whi = sm.hi[b];
+                tb = sm.t[b];
+            }
+            uint32_t kc = 0, ncw = 0;
+            // virtual page index v = li + pb0 (this pass's pages follow the earlier passes')
+            const int64_t la = pa - cx.x0 + pb0, lb = pb - cx.x0 + pb0;
+            for (int64_t v = la + (((int64_t)warp - la) % NCW + NCW) % NCW; v < lb; v += NCW) {
+                const int64_t li = v - pb0;
+                const int64_t nw = v / NCW;
+                const int sg = warp * LY::NSW + (int)(nw % LY::NSW);
+                mbar_wait(&full[sg], (uint32_t)((nw / LY::NSW) & 1), a.status, site + 4);
+                const uint32_t mt = meta[sg];
+                const unsigned char *sk = stage + sg * LY::STAGE_BYTES;
+                uint32_t keepm, evm, candm = 0u, cbase = 0u;
+                float *zdst = nullptr;
+                int zcap = 0;
+                if constexpr (SPEC) {
+                    const uint32_t valid = mt >> 16;
+                    const int r = lane & 15;
+                    const unsigned char *pl = poslb + sg * 128;
+                    const int32_t pos = reinterpret_cast<const int32_t *>(pl)[r];
+                    const float lbv = reinterpret_cast<const float *>(pl + 64)[r];
+                    bool kept = false, cand = false, bad = false;
+                    uint64_t K = 0ull;
+                    if ((valid >> r) & 1u) {
+                        bad = !entry_key(tb, cl, pos, lbv, a.ibits, &K);
+                        kept = !bad && K < wlo;
+                        cand = !bad && !kept && K < whi;
+                    }
+                    keepm = __ballot_sync(0xFFFFFFFFu, kept) & 0xFFFFu;
+                    candm = __ballot_sync(0xFFFFFFFFu, cand) & 0xFFFFu;
+                    if (__ballot_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, RKV_DEV_BAD_INPUT);
+                    evm = valid & ~keepm & ~candm;
+                    const int64_t pidx = li + cx.x0 - pfx;
+                    if (lane == 0) a.keep_mask[(int64_t)c * a.max_pages + pidx] = (uint16_t)keepm;
+                    kc += (uint32_t)__popc(keepm);
+                    if (candm) {
+                        if (lane == 0) {
+                            cbase = atomicAdd(cx.seqc + (size_t)b * 4 + 1, (uint32_t)__popc(candm));
+                            atomicOr(cx.head_flag + c, 1u);
+                        }
+                        cbase = __shfl_sync(0xFFFFFFFFu, cbase, 0);
+                        if (lane < 16 && cand) {
+                            const uint32_t idx = cbase + (uint32_t)__popc(candm & ((1u << r) - 1u));
+                            if (idx < (uint32_t)WIN_CAP) {
+                                a.ckey[(size_t)b * WIN_CAP + idx] = K;
+                                a.cslot[(size_t)b * WIN_CAP + idx] = (int32_t)(pidx * PAGE + r);
+                            }
+                        }
+                        zdst = a.cz + ((size_t)b * WIN_CAP + cbase) * G;
+                        zcap = cbase < (uint32_t)WIN_CAP ? (int)(WIN_CAP - cbase) : 0;
+                        ncw += (uint32_t)__popc(candm);
+                    }
+                } else {
+                    keepm = mt & 0xFFFFu;
+                    evm = (mt >> 16) & ~keepm;
+                }
+                M::template page<SPEC>(st, sk, sk + M::PAGE_BYTES, keepm, evm, lane, candm, zdst, zcap);
+                if constexpr (SPEC) {
+                    if (candm) {
+                        // set the candidates' V rows aside
+                        uint32_t bits = candm;
+                        uint32_t k = cbase;
+                        while (bits) {
+                            const int j = __ffs(bits) - 1;
+                            bits &= bits - 1;
+                            if (k < (uint32_t)WIN_CAP)
+                                M::copy_row(sk + M::PAGE_BYTES, j, a.cv + ((size_t)b * WIN_CAP + k) * a.row_bytes, lane);
+                            k++;
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[sg]);
+            }
+            if constexpr (SPEC) {
+                if (lane == 0 && kc) {
+                    atomicAdd(cx.head_kept + c, kc);
+                    atomicAdd(cx.seqc + (size_t)b * 4, kc);
+                }
+            }
+            const int par = nq & 1;
+            float *slot = merge + (par * NCW + warp) * LY::WSLOT;
+            M::flush(st, slot, lane);
+            if (lane == 0) slot[G * D + 4 * G] = (float)ncw;
+            nq++;
+            named_bar_sync(1, NCW * 32);
+
+            // ---- merge the warps (consumer threads) ----
+            const float *mb = merge + par * NCW * LY::WSLOT;
+            float hc = 0.0f;
+#pragma unroll
+            for (int wi = 0; wi < NCW; wi++) hc += mb[wi * LY::WSLOT + G * D + 4 * G];
+            // whole head without candidates: final; else a record for the tail
+            const int dest = whole ? (hc > 0.0f ? 1 : 0) : 2;
+            float *rec = dest == 1 ? a.hrec + (int64_t)c * LY::REC
+                                   : a.partial + ((int64_t)blockIdx.x * 2 + ((pfx < cx.x0) ? 0 : 1)) * LY::REC;
+            for (int e = tid; e < G * D + G; e += NCW * 32) {
+                const bool is_stat = e >= G * D;
+                const int g = is_stat ? e - G * D : e / D;
+                Merged s;
+                s.mk = -INFINITY;
+                s.me = -INFINITY;
+#pragma unroll
+                for (int wi = 0; wi < NCW; wi++) {
+                    s.mk = fmaxf(s.mk, mb[wi * LY::WSLOT + G * D + g]);
+                    s.me = fmaxf(s.me, mb[wi * LY::WSLOT + G * D + 2 * G + g]);
+                }
+                s.lk = 0.0f;
+                s.le = 0.0f;
+                float av = 0.0f;
+#pragma unroll
+                for (int wi = 0; wi < NCW; wi++) {
+                    const float *src = mb + wi * LY::WSLOT;
+                    const float mkw = src[G * D + g], mew = src[G * D + 2 * G + g];
+                    const float fk = (mkw == -INFINITY) ? 0.0f : ex2(mkw - s.mk);
+                    const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
+                    s.lk += src[G * D + G + g] * fk;
+                    s.le += src[G * D + 3 * G + g] * fe;
+                    if (!is_stat) av += src[e] * fk;
+                }
+                if (dest == 0) {
+                    if (!is_stat) {
+                        a.out[(int64_t)c * G * D + e] = s.lk > 0.0f ? av / s.lk : 0.0f;
+                    } else {
+                        if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
+                        if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
+                    }
+                } else if (!is_stat) {
+                    rec[e] = av;
+                } else {
+                    rec[G * D + g] = s.mk;
+                    rec[G * D + G + g] = s.lk;
+                    rec[G * D + 2 * G + g] = s.me;
+                    rec[G * D + 3 * G + g] = s.le;
+                }
+            }
+            if (dest == 1 && tid == 0) atomicOr(cx.head_flag + c, 2u);
+        }
+        cx.qbase = nq;
+        if constexpr (REG_SPLIT) setmaxnreg_dec<LAUNCH_REGS>();
+    }
+    cx.pbase = pb0 + (cx.x1 - cx.x0);
+    __syncthreads();
+    if (warp >= NCW) {
+        if constexpr (REG_SPLIT) setmaxnreg_inc<LAUNCH_REGS>();
+    }
+}
+
+// --------------------------------------------------------------- resolve ----
+// After the speculative pass: per sequence, is the M-th key inside the
+// window with every candidate stored?  If so every candidate's fate is its
+// rank among the candidates (keys are distinct), counted by the CTA that owns
+// its slice; kept candidates are added to their head's kept count and the
+// M-th key gives the exclusive threshold.  Returns false if any sequence
+// missed (the exact path runs instead).
+__device__ bool resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
+    const int tid = threadIdx.x, nct = gridDim.x;
+    if (tid < a.B) {
+        const int b = tid;
+        if (!(sm.fl[b] & SF_TRIVIAL)) {
+            const uint32_t above = __ldcg(cx.seqc + (size_t)b * 4), nc = __ldcg(cx.seqc + (size_t)b * 4 + 1);
+            const int64_t m = sm.m[b];
+            const bool hit = nc <= (uint32_t)WIN_CAP && (int64_t)above < m && m <= (int64_t)above + nc;
+            sm.above[b] = above;
+            sm.nc[b] = hit ? nc : 0u;
+            // window outcome, used to resize it even if another sequence
+            // sends the call down the exact path
+            sm.wres[b] = hit ? 1u : (nc > (uint32_t)WIN_CAP ? 3u : 2u);
+            if (!hit) atomicOr(&sm.misc[MS_MISS], 1);
+        }
+    }
+    __syncthreads();
+    if (sm.misc[MS_MISS]) return false;
+    if (tid == 0) {
+        uint32_t o = 0;
+        for (int b = 0; b < a.B; b++) {
+            sm.off[b] = o;
+            o += sm.nc[b];
+        }
+        sm.misc[MS_TOTAL] = (int)o;
+    }
+    __syncthreads();
+    const int64_t total = sm.misc[MS_TOTAL];
+    const int64_t s0 = (int64_t)blockIdx.x * total / nct, s1 = (int64_t)(blockIdx.x + 1) * total / nct;
+    uint64_t *keys = reinterpret_cast<uint64_t *>(sm.big);
+    for (int b = 0; b < a.B; b++) {
+        const int64_t ob = sm.off[b], nb = sm.nc[b];
+        const int64_t jlo = max(s0, ob) - ob, jhi = min(s1, ob + nb) - ob;
+        if (jlo >= jhi) continue;
+        for (int i = tid; i < nb; i += NTH) keys[i] = __ldcg(a.ckey + (size_t)b * WIN_CAP + i);
+        __syncthreads();
+        const uint32_t r = (uint32_t)(sm.m[b] - (int64_t)sm.above[b]);  // 1-based
+        for (int64_t j = jlo + tid; j < jhi; j += NTH) {
+            const uint64_t K = keys[j];
+            uint32_t less = 0;
+            for (int i = 0; i < nb; i++) less += keys[i] < K ? 1u : 0u;
+            const bool kept = less < r;
+            a.cfate[(size_t)b * WIN_CAP + j] = kept ? 1 : 0;
+            if (kept) {
+                const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
+                atomicAdd(cx.head_kept + (int64_t)b * a.LH + cl, 1u);
+            }
+            if (less == r - 1) {
+                const uint64_t kap = K + 1ull;
+                a.kappa[b] = kap;
+                window_next(a.win + (size_t)b * 4, kap, 1, (uint32_t)nb);
+            }
+        }
+        __syncthreads();
+    }
+    if (blockIdx.x == 0 && tid < a.B && (sm.fl[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap[tid];
+    return true;
+}
+
+// --------------------------------------------------------- exact select ----
+// Calls f(c, pidx, r, K, ok) for slot r of every page of this CTA's range
+// (c = -1 past the range end), half a warp per page, UNR pages per half-warp
+// per round with their loads issued together.  Heads are found through the
+// range's page prefix in a.pfx.  Loop bounds are warp-uniform.
+template <typename F>
+__device__ __forceinline__ void for_range_keys(const StepArgs &a, const Sm &sm, const Ctx &cx, F &&f) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r = lane & 15;
+    constexpr int STEP = 2 * NWARP;
+    int cur = -1;
+    for (int64_t xb = cx.x0 + 2 * warp; xb < cx.x1; xb += (int64_t)STEP * UNR) {
+        int32_t pg[UNR];
+        int hc[UNR], pidx[UNR];
+        bool ld[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; u++) {
+            const int64_t x = xb + (lane >> 4) + (int64_t)u * STEP;
+            ld[u] = false;
+            hc[u] = -1;
+            pidx[u] = 0;
+            pg[u] = 0;
+            if (x < cx.x1) {
+                if (cur < 0) {
+                    int lo = cx.c_start, hi = cx.c_last;  // last c with pfx[c] <= x
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (a.pfx[mid] <= x) lo = mid; else hi = mid - 1;
+                    }
+                    cur = lo;
+                }
+                while (cur < cx.c_last && a.pfx[cur + 1] <= x) cur++;
+                hc[u] = cur;
+                pidx[u] = (int)(x - a.pfx[cur]);
+                if (pidx[u] * PAGE + r < max(__ldcg(a.len + cur), 0)) {
+                    ld[u] = true;
+                    pg[u] = __ldcg(a.block_table + (int64_t)cur * a.max_pages + pidx[u]);
+                }
+            }
+        }
+        int32_t pos[UNR];
+        float lbv[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; u++) {
+            pos[u] = 0;
+            lbv[u] = 0.0f;
+            if (ld[u]) {
+                pos[u] = __ldcg(a.pos_pool + (int64_t)pg[u] * PAGE + r);
+                lbv[u] = __ldcg(a.lb_pool + (int64_t)pg[u] * PAGE + r);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; u++) {
+            uint64_t K = 0ull;
+            bool ok = false;
+            if (ld[u]) {
+                const int b = hc[u] / a.LH;
+                ok = entry_key(sm.t[b], (uint32_t)(hc[u] - b * a.LH), pos[u], lbv[u], a.ibits, &K);
+                if (!ok) set_status(a.status, RKV_DEV_BAD_INPUT);
+            }
+            f(hc[u], pidx[u], r, K, ok);
+        }
+    }
+}
+
+// This call's largest kept key of sequence b (uint64 in the counter half).
+__device__ __forceinline__ unsigned long long *kmax_of(const Ctx &cx, int b) {
+    return reinterpret_cast<unsigned long long *>(cx.seqc + (size_t)b * 4 + 2);
+}
+
+// Digit p of sequence b's threshold from its completed global histogram
+// (every CTA computes the same result).
+__device__ void scan_digit(const StepArgs &a, const Sm &sm, int b, int p) {
+    const int tid = threadIdx.x;
+    constexpr int PER = (NBINS + NTH - 1) / NTH;
+    const uint32_t *gh = a.ghist + ((size_t)p * a.B + b) * NBINS;
+    uint32_t v[PER], loc = 0;
+#pragma unroll
+    for (int j = 0; j < PER; j++) {
+        const int i = tid * PER + j;
+        v[j] = i < NBINS ? __ldcg(gh + i) : 0u;
+        loc += v[j];
+    }
+    if (tid == 0) sm.misc[MS_FOUND] = 0;
+    uint32_t total;
+    const uint32_t ex = block_exclusive_scan(loc, sm.scan, &total);
+    const uint32_t rank = sm.rank[b];
+    if (ex < rank && rank <= ex + loc) {
+        uint32_t cum = ex;
+#pragma unroll
+        for (int j = 0; j < PER; j++) {
+            if (cum < rank && rank <= cum + v[j]) {
+                sm.misc[MS_DIG] = tid * PER + j;
+                sm.misc[MS_NR] = (int)(rank - cum);
+                sm.misc[MS_H] = (int)v[j];
+                sm.misc[MS_FOUND] = 1;
+            }
+            cum += v[j];
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        if (!sm.misc[MS_FOUND]) {
+            // fewer matching keys than the rank (entries rejected as bad input)
+            set_status(a.status, RKV_DEV_BAD_INPUT);
+            sm.fl[b] |= SF_DONE;
+            sm.kap[b] = (sm.pk[b] | ~sm.pm[b]) + 1ull;
+        } else {
+            const int sh = digit_shift(p);
+            const uint64_t d = (uint64_t)sm.misc[MS_DIG];
+            sm.pk[b] |= d << sh;
+            sm.pm[b] |= ((1ull << digit_bits(p)) - 1ull) << sh;
+            sm.rank[b] = (uint32_t)sm.misc[MS_NR];
+            if ((uint32_t)sm.misc[MS_H] == sm.rank[b] || p == NPASS - 1) {
+                sm.fl[b] |= SF_DONE;
+                sm.kap[b] = (sm.pk[b] | ~sm.pm[b]) + 1ull;
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// Exact threshold of every non-trivial sequence by radix passes over this
+// CTA's page range, then keep masks and kept counts for every page of it.
+__device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    {
+        // page prefix of the heads this CTA's range visits, for page -> head
+        int64_t p = cx.my_pfx;
+        for (int c = cx.h0; c < cx.h1; c++) {
+            if (c >= cx.c_start && c <= cx.c_last + 1) a.pfx[c] = (int32_t)p;
+            p += (max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE;
+        }
+        if (tid == 0 && cx.c_last + 1 == a.C) a.pfx[a.C] = (int32_t)cx.TP;
+    }
+    cx.exact = true;
+    if (tid < a.B && !(sm.fl[tid] & SF_TRIVIAL)) {
+        sm.fl[tid] &= ~SF_DONE;
+        sm.rank[tid] = (uint32_t)sm.m[tid];
+        sm.pk[tid] = 0ull;
+        sm.pm[tid] = 0ull;
+    }
+    if (tid < MAXB) sm.kmx[tid] = 0ull;
+    __syncthreads();
+    const int b_first = cx.c_start < a.C ? cx.c_start / a.LH : 0;
+    const int b_last = cx.c_last >= 0 ? cx.c_last / a.LH : -1;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sm.big);
+    for (int p = 0; p < NPASS; p++) {
+        if (tid == 0) {
+            int act = 0;
+            for (int b = 0; b < a.B; b++) act |= (sm.fl[b] & SF_DONE) ? 0 : 1;
+            sm.misc[MS_ACTIVE] = act;
+        }
+        __syncthreads();
+        if (!sm.misc[MS_ACTIVE]) break;
+        cx.passes = p + 1;
+        for (int g0 = b_first; g0 <= b_last; g0 += HGRP) {
+            const int g1 = min(b_last + 1, g0 + HGRP);
+            for (int i = tid; i < (g1 - g0) * NBINS; i += NTH) hist[i] = 0u;
+            __syncthreads();
+            for_range_keys(a, sm, cx, [&](int c, int, int, uint64_t K, bool ok) {
+                if (!ok) return;
+                const int b = c / a.LH;
+                if (b < g0 || b >= g1 || (sm.fl[b] & SF_DONE) || ((K ^ sm.pk[b]) & sm.pm[b]) != 0ull) return;
+                atomicAdd(&hist[(b - g0) * NBINS + key_digit((uint32_t)(K >> 32), (uint32_t)K, p)], 1u);
+            });
+            __syncthreads();
+            for (int i = tid; i < (g1 - g0) * NBINS; i += NTH) {
+                const uint32_t v = hist[i];
+                const int b = g0 + i / NBINS;
+                if (v) atomicAdd(a.ghist + ((size_t)p * a.B + b) * NBINS + (i % NBINS), v);
+            }
+            __syncthreads();
+        }
+        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return false;
+        for (int b = 0; b < a.B; b++)
+            if (!(sm.fl[b] & SF_DONE)) scan_digit(a, sm, b, p);
+    }
+    // keep masks (half-warp ballots), kept counts and the largest kept key of
+    // each sequence (the reported threshold is that key + 1: a radix bucket
+    // kept whole only bounds it)
+    int kb = -1;
+    unsigned long long km = 0ull;
+    for_range_keys(a, sm, cx, [&](int c, int pidx, int r, uint64_t K, bool ok) {
+        const int b = c >= 0 ? c / a.LH : 0;
+        const bool keep = ok && K < sm.kap[b];
+        if (keep) {
+            if (b != kb) {
+                if (kb >= 0) atomicMax(sm.kmx + kb, km);
+                kb = b;
+                km = K;
+            } else if (K > km) {
+                km = K;
+            }
+        }
+        const uint32_t ball = __ballot_sync(0xFFFFFFFFu, keep);
+        if (r == 0 && c >= 0) {
+            const uint32_t m16 = (ball >> (lane & 16)) & 0xFFFFu;
+            a.keep_mask[(int64_t)c * a.max_pages + pidx] = (uint16_t)m16;
+            if (m16) atomicAdd(cx.head_kept + c, (uint32_t)__popc(m16));
+        }
+    });
+    if (kb >= 0) atomicMax(sm.kmx + kb, km);
+    __syncthreads();
+    if (tid < a.B && sm.kmx[tid]) atomicMax(kmax_of(cx, tid), sm.kmx[tid]);
+    if (blockIdx.x == 0 && tid < a.B && (sm.fl[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap[tid];
+    __syncthreads();
+    return true;
+}
+
+// ------------------------------------------------------------------ tail ----
+template <class M>
+__device__ __forceinline__ float row_elt(const unsigned char *row, int d) {
+    if constexpr (M::ROW_BYTES / M::DIM == 2) {
+        return __uint_as_float((uint32_t)__ldcg(reinterpret_cast<const unsigned short *>(row) + d) << 16);
+    } else {
+        return __ldcg(reinterpret_cast<const float *>(row) + d);
+    }
+}
+
+// Merge of a head's partial states: the records of the CTAs its pages span
+// (or the record of the one CTA that held candidates of it) and its
+// candidates, each kept (logit z, weight 1, value v) or evicted (logit z).
+template <class M, int D, int G>
+__device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int64_t pfx, int jf, int jl,
+                             uint32_t flag, bool cands) {
+    using LY = StepLayout<M, D, G>;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nct = gridDim.x;
+    const int b = c / a.LH;
+    const int cl = c - b * a.LH;
+    int32_t *clist = reinterpret_cast<int32_t *>(sm.big + T_CL);
+    int ncl = 0;
+    if (cands) {
+        if (warp == 0) {
+            const int nb = (int)sm.nc[b];
+            int cnt = 0;
+            for (int base = 0; base < nb; base += 32) {
+                const int i = base + lane;
+                bool mine = false;
+                if (i < nb) {
+                    const uint64_t K = __ldcg(a.ckey + (size_t)b * WIN_CAP + i);
+                    mine = (a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits)) == cl;
+                }
+                const uint32_t ball = __ballot_sync(0xFFFFFFFFu, mine);
+                if (mine) clist[cnt + __popc(ball & ((1u << lane) - 1u))] = i;
+                cnt += __popc(ball);
+            }
+            if (lane == 0) sm.misc[MS_NCL] = cnt;
+        }
+        __syncthreads();
+        ncl = sm.misc[MS_NCL];
+    }
+    const bool split = jf != jl;
+    const size_t cb = (size_t)b * WIN_CAP;
+    for (int e = tid; e < G * D + G; e += NTH) {
+        const bool is_stat = e >= G * D;
+        const int g = is_stat ? e - G * D : e / D;
+        Merged s;
+        s.mk = -INFINITY;
+        s.me = -INFINITY;
+        if (split) {
+            for (int j = jf; j <= jl; j++) {
+                if (!(range_lo(j, cx.TP, nct) < range_lo(j + 1, cx.TP, nct))) continue;
+                const float *r = a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, cx.TP, nct)) ? 0 : 1)) * LY::REC;
+                s.mk = fmaxf(s.mk, __ldcg(r + G * D + g));
+                s.me = fmaxf(s.me, __ldcg(r + G * D + 2 * G + g));
+            }
+        } else if (flag & 2u) {
+            const float *r = a.hrec + (int64_t)c * LY::REC;
+            s.mk = fmaxf(s.mk, __ldcg(r + G * D + g));
+            s.me = fmaxf(s.me, __ldcg(r + G * D + 2 * G + g));
+        }
+        for (int i = 0; i < ncl; i++) {
+            const size_t idx = cb + clist[i];
+            const float z = __ldcg(a.cz + idx * G + g);
+            if (__ldcg(a.cfate + idx)) s.mk = fmaxf(s.mk, z); else s.me = fmaxf(s.me, z);
+        }
+        s.lk = 0.0f;
+        s.le = 0.0f;
+        float av = 0.0f;
+        auto add = [&](const float *r) {
+            const float mkw = __ldcg(r + G * D + g), mew = __ldcg(r + G * D + 2 * G + g);
+            const float fk = (mkw == -INFINITY) ? 0.0f : ex2(mkw - s.mk);
+            const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
+            s.lk += __ldcg(r + G * D + G + g) * fk;
+            s.le += __ldcg(r + G * D + 3 * G + g) * fe;
+            if (!is_stat) av += __ldcg(r + e) * fk;
+        };
+        if (split) {
+            for (int j = jf; j <= jl; j++) {
+                if (!(range_lo(j, cx.TP, nct) < range_lo(j + 1, cx.TP, nct))) continue;
+                add(a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, cx.TP, nct)) ? 0 : 1)) * LY::REC);
+            }
+        } else if (flag & 2u) {
+            add(a.hrec + (int64_t)c * LY::REC);
+        }
+        for (int i = 0; i < ncl; i++) {
+            const size_t idx = cb + clist[i];
+            const float z = __ldcg(a.cz + idx * G + g);
+            if (__ldcg(a.cfate + idx)) {
+                const float w = ex2(z - s.mk);
+                s.lk += w;
+                if (!is_stat) av += w * row_elt<M>(a.cv + idx * a.row_bytes, e - g * D);
+            } else {
+                s.le += ex2(z - s.me);
+            }
+        }
+        if (!is_stat) {
+            a.out[(int64_t)c * G * D + e] = s.lk > 0.0f ? av / s.lk : 0.0f;
+        } else {
+            if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
+            if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
+        }
+    }
+    if (cands && tid == 0) {
+        for (int i = 0; i < ncl; i++) {
+            const size_t idx = cb + clist[i];
+            if (__ldcg(a.cfate + idx)) {
+                const int slot = __ldcg(a.cslot + idx);
+                uint16_t *wd = a.keep_mask + (int64_t)c * a.max_pages + slot / PAGE;
+                *wd = (uint16_t)(*wd | (1u << (slot % PAGE)));
+            }
+        }
+    }
+    __syncthreads();
+}
+
+// Hole-fill compaction of head c (n entries, nn kept): the j-th non-kept
+// slot below nn takes the j-th kept slot at or above nn; pages past
+// ceil(nn/16) go to the free stack at this head's plan offset.
+__device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int n, int nn, int32_t off) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int mp = a.max_pages;
+    int32_t *tbl = reinterpret_cast<int32_t *>(sm.big + T_TBL);
+    int32_t *src_pfx = tbl + mp;
+    int32_t *hole_pfx = src_pfx + mp + 1;
+    uint16_t *msk = reinterpret_cast<uint16_t *>(hole_pfx + mp + 1);
+    int2 *pairs = reinterpret_cast<int2 *>(sm.big + T_PAIRS);
+    const int W = (n + PAGE - 1) / PAGE, Wn = (nn + PAGE - 1) / PAGE;
+    const int64_t cm = (int64_t)c * mp;
+    for (int w = tid; w < W; w += NTH) {
+        tbl[w] = __ldcg(a.block_table + cm + w);
+        const uint32_t m = (uint32_t)__ldcg(a.keep_mask + cm + w) & below_bits(w, n);
+        msk[w] = (uint16_t)m;
+        const uint32_t below = below_bits(w, nn);
+        src_pfx[w] = __popc(m & ~below);
+        hole_pfx[w] = __popc(~m & below & 0xFFFFu);
+    }
+    __syncthreads();
+    scan_words(src_pfx, W, sm.scan);
+    scan_words(hole_pfx, W, sm.scan);
+    const int moves = min(hole_pfx[W], src_pfx[W]);
+    const int chunks = a.row_bytes / 16;
+    for (int r0 = 0; r0 < moves; r0 += CMP_PAIRS) {
+        const int r1 = min(moves, r0 + CMP_PAIRS);
+        for (int w = tid; w < Wn; w += NTH) {
+            int rank = hole_pfx[w];
+            if (rank >= r1 || hole_pfx[w + 1] <= r0) continue;
+            uint32_t hb = ~(uint32_t)msk[w] & below_bits(w, nn) & 0xFFFFu;
+            while (hb) {
+                const int bit = __ffs(hb) - 1;
+                hb &= hb - 1;
+                if (rank >= r0 && rank < r1) {
+                    int lo = 0, hi = W - 1;  // word of the rank-th source: last w' with src_pfx[w'] <= rank
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (src_pfx[mid] <= rank) lo = mid; else hi = mid - 1;
+                    }
+                    uint32_t sb = (uint32_t)msk[lo] & ~below_bits(lo, nn);
+                    for (int i = rank - src_pfx[lo]; i > 0; i--) sb &= sb - 1;
+                    const int hslot = w * PAGE + bit, sslot = lo * PAGE + (__ffs(sb) - 1);
+                    pairs[rank - r0] = make_int2((int)((int64_t)tbl[hslot / PAGE] * PAGE + hslot % PAGE),
+                                                 (int)((int64_t)tbl[sslot / PAGE] * PAGE + sslot % PAGE));
+                }
+                rank++;
+            }
+        }
+        __syncthreads();
+        for (int pi = warp; pi < r1 - r0; pi += NWARP) {
+            const int64_t dst = pairs[pi].x, src = pairs[pi].y;
+            const int i0 = lane, i1 = lane + 32;
+            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+            const uint4 *ks = reinterpret_cast<const uint4 *>((const unsigned char *)a.k_pool + src * a.row_bytes);
+            const uint4 *vs = reinterpret_cast<const uint4 *>((const unsigned char *)a.v_pool + src * a.row_bytes);
+            if (i0 < 2 * chunks) v0 = i0 < chunks ? __ldcg(ks + i0) : __ldcg(vs + i0 - chunks);
+            if (i1 < 2 * chunks) v1 = i1 < chunks ? __ldcg(ks + i1) : __ldcg(vs + i1 - chunks);
+            int32_t pos = 0;
+            float lbv = 0.0f;
+            if (lane == 0) {
+                pos = __ldcg(a.pos_pool + src);
+                lbv = __ldcg(a.lb_pool + src);
+            }
+            uint4 *kd = reinterpret_cast<uint4 *>((unsigned char *)a.k_pool + dst * a.row_bytes);
+            uint4 *vd = reinterpret_cast<uint4 *>((unsigned char *)a.v_pool + dst * a.row_bytes);
+            if (i0 < 2 * chunks) {
+                if (i0 < chunks) kd[i0] = v0; else vd[i0 - chunks] = v0;
+            }
+            if (i1 < 2 * chunks) {
+                if (i1 < chunks) kd[i1] = v1; else vd[i1 - chunks] = v1;
+            }
+            if (lane == 0) {
+                a.pos_pool[dst] = pos;
+                a.lb_pool[dst] = lbv;
+            }
+        }
+        __syncthreads();
+    }
+    for (int pi = Wn + tid; pi < W; pi += NTH) {
+        a.free_stack[cx.top0 + off + (pi - Wn)] = tbl[pi];
+        a.block_table[cm + pi] = -1;
+    }
+    __syncthreads();
+}
+
+// Bounded wait until every CTA has finished its compactions (pushes).
+__device__ bool wait_pushes(const StepArgs &a, const Ctx &cx) {
+    const uint32_t target = gridDim.x;
+    if (ld_acquire_gpu(cx.arrive) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t spins = 0;
+    while (ld_acquire_gpu(cx.arrive) < target) {
+        if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
+            record_timeout(a.status, 0x200);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Append of the new token to head c (one warp): slot k (the post-compaction
+// length) takes K, V, position t and log-retention; a page is popped when k
+// is a multiple of 16 (the pop-th pop of this call, ascending head order).
+__device__ void append_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int k, int pop, uint32_t pushes) {
+    const int lane = threadIdx.x & 31;
+    const int chunks = a.row_bytes / 16;
+    const int i0 = lane, i1 = lane + 32;
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    const uint4 *kn = reinterpret_cast<const uint4 *>((const unsigned char *)a.k_new + (int64_t)c * a.row_bytes);
+    const uint4 *vn = reinterpret_cast<const uint4 *>((const unsigned char *)a.v_new + (int64_t)c * a.row_bytes);
+    if (i0 < 2 * chunks) v0 = i0 < chunks ? __ldg(kn + i0) : __ldg(vn + i0 - chunks);
+    if (i1 < 2 * chunks) v1 = i1 < chunks ? __ldg(kn + i1) : __ldg(vn + i1 - chunks);
+    int64_t row = -1;
+    if (lane == 0) {
+        const int pidx = k / PAGE;
+        if (pidx >= a.max_pages) {
+            set_status(a.status, RKV_DEV_TABLE_OVERFLOW);
+        } else if (k % PAGE == 0) {
+            const int idx = cx.top0 + (int)pushes - 1 - pop;
+            if (idx < 0) {
+                set_status(a.status, RKV_DEV_POOL_EXHAUSTED);
+            } else if (idx < cx.top0 || wait_pushes(a, cx)) {
+                const int32_t page = __ldcg(a.free_stack + idx);
+                a.block_table[(int64_t)c * a.max_pages + pidx] = page;
+                row = (int64_t)page * PAGE;
+            }
+        } else {
+            row = (int64_t)__ldcg(a.block_table + (int64_t)c * a.max_pages + pidx) * PAGE + (k % PAGE);
+        }
+        if (row >= 0) {
+            a.pos_pool[row] = sm.t[c / a.LH];
+            a.lb_pool[row] = __ldg(a.lb_new + c);
+        }
+        a.len[c] = k + 1;
+    }
+    row = __shfl_sync(0xFFFFFFFFu, row, 0);
+    if (row >= 0) {
+        uint4 *kd = reinterpret_cast<uint4 *>((unsigned char *)a.k_pool + row * a.row_bytes);
+        uint4 *vd = reinterpret_cast<uint4 *>((unsigned char *)a.v_pool + row * a.row_bytes);
+        if (i0 < 2 * chunks) {
+            if (i0 < chunks) kd[i0] = v0; else vd[i0 - chunks] = v0;
+        }
+        if (i1 < 2 * chunks) {
+            if (i1 < chunks) kd[i1] = v1; else vd[i1 - chunks] = v1;
+        }
+    }
+}
+
+template <class M, int D, int G>
+__device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) {
+    const int tid = threadIdx.x, warp = tid >> 5, nct = gridDim.x;
+    const int C = a.C;
+    const int hc0 = (int)((int64_t)blockIdx.x * C / nct), hc1 = (int)((int64_t)(blockIdx.x + 1) * C / nct);
+    int32_t *st_npre = reinterpret_cast<int32_t *>(sm.big + T_STASH);
+    int32_t *st_nnew = st_npre + NTH, *st_pfx = st_nnew + NTH, *st_plan = st_pfx + NTH, *st_pop = st_plan + NTH;
+    // exact-select histograms are no longer read by anyone: clear them
+    if (cx.passes > 0) {
+        const size_t nh = (size_t)cx.passes * a.B * NBINS;
+        for (size_t i = (size_t)blockIdx.x * NTH + tid; i < nh; i += (size_t)nct * NTH) a.ghist[i] = 0u;
+    }
+    // per head: pre-step pages, freed pages, pops -- prefixes over all heads
+    uint32_t carry[3] = {0u, 0u, 0u};
+    for (int base = 0; base < C; base += NTH) {
+        const int c = base + tid;
+        int32_t np = 0, nn = 0;
+        uint32_t v[3] = {0u, 0u, 0u};
+        if (c < C) {
+            np = __ldcg(a.npre + c);
+            nn = cx.evict ? (int32_t)__ldcg(cx.head_kept + c) : np;
+            v[0] = (uint32_t)((np + PAGE - 1) / PAGE);
+            v[1] = cx.evict ? v[0] - (uint32_t)((nn + PAGE - 1) / PAGE) : 0u;
+            v[2] = (nn % PAGE == 0) ? 1u : 0u;
+        }
+        uint32_t ex[3], tot[3];
+        block_scan_n<3>(v, ex, tot, sm.scan);
+        if (c >= hc0 && c < hc1) {
+            const int k = c - hc0;
+            st_npre[k] = np;
+            st_nnew[k] = nn;
+            st_pfx[k] = (int32_t)(carry[0] + ex[0]);
+            st_plan[k] = (int32_t)(carry[1] + ex[1]);
+            st_pop[k] = (int32_t)(carry[2] + ex[2]);
+        }
+#pragma unroll
+        for (int s = 0; s < 3; s++) carry[s] += tot[s];
+    }
+    const uint32_t pushes = carry[1], pops = carry[2];
+    __syncthreads();
+    if (cx.evict) {
+        for (int k = tid; k < hc1 - hc0; k += NTH) {
+            a.kept[hc0 + k] = st_nnew[k];
+            a.plan[hc0 + k] = st_plan[k];
+        }
+    }
+    if (cx.exact && blockIdx.x == 0 && tid < a.B && !(sm.fl[tid] & SF_TRIVIAL)) {
+        // thresholds of the exact selection: largest kept key + 1 (every CTA's
+        // final pass is complete), and the window for the next call
+        const uint64_t kap = __ldcg(kmax_of(cx, tid)) + 1ull;
+        a.kappa[tid] = kap;
+        window_next(a.win + (size_t)tid * 4, kap, (int)sm.wres[tid], sm.nc[tid]);
+    }
+    if (blockIdx.x == nct - 1 && tid == 0) {
+        if (cx.evict) {
+            a.plan[C] = (int32_t)pushes;
+            a.plan[C + 1] = cx.top0;
+        }
+        const int nt = cx.top0 + (int)pushes - (int)pops;
+        *a.free_top = nt < 0 ? 0 : nt;
+    }
+    // merges, keep-bit patches and compaction, head by head
+    for (int c = hc0; c < hc1; c++) {
+        const int k = c - hc0;
+        const int np = st_npre[k], nn = st_nnew[k];
+        const int pages = (np + PAGE - 1) / PAGE;
+        if (pages > 0) {
+            const int64_t pfx = st_pfx[k];
+            const int jf = owner_of(pfx, cx.TP, nct), jl = owner_of(pfx + pages - 1, cx.TP, nct);
+            const uint32_t flag = __ldcg(cx.head_flag + c);
+            const bool cands = spec && (flag & 1u);
+            if (jf != jl || (flag & 2u) || cands) combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, cands);
+        }
+        if (cx.evict && nn < np) compact_head(a, sm, cx, c, np, nn, st_plan[k]);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        atomicAdd(cx.arrive, 1u);
+    }
+    for (int k = warp; k < hc1 - hc0; k += NWARP) append_head(a, sm, cx, hc0 + k, st_nnew[k], st_pop[k], pushes);
+}
+
+// ---------------------------------------------------------------- kernel ----
+template <class M, int D, int G>
+__global__ void __launch_bounds__(NTH, 1)
+    step_kernel(StepArgs a, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
+    using LY = StepLayout<M, D, G>;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((M::STAGE_ALIGN - (smem_u32(smem_raw) & (M::STAGE_ALIGN - 1))) &
+                                      (M::STAGE_ALIGN - 1));
+    Sm sm;
+    sm.bars = reinterpret_cast<uint64_t *>(smem + LY::OFF_BAR);
+    {
+        unsigned char *p = smem + LY::OFF_SEQ;
+        sm.lo = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
+        sm.hi = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
+        sm.kap = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
+        sm.pk = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
+        sm.pm = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
+        sm.kmx = reinterpret_cast<unsigned long long *>(p); p += MAXB * 8;
+        sm.m = reinterpret_cast<int64_t *>(p); p += MAXB * 8;
+        sm.t = reinterpret_cast<int32_t *>(p); p += MAXB * 4;
+        sm.n = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
+        sm.rank = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
+        sm.fl = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
+        sm.above = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
+        sm.nc = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
+        sm.off = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
+        sm.wres = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
+    }
+    sm.spare = nullptr;
+    sm.scan = reinterpret_cast<uint32_t *>(smem + LY::OFF_SCAN);
+    sm.misc = reinterpret_cast<int *>(smem + LY::OFF_MISC);
+    sm.misc64 = reinterpret_cast<int64_t *>(smem + LY::OFF_MISC + 64 * 4);
+    sm.big = smem + LY::OFF_BIG;
+
+    Ctx cx;
+    prologue<M, D, G>(a, sm, cx, &tmk, &tmv);
+    bool spec = false;
+    if (cx.evict && !sm.misc[MS_RADIX]) {
+        attn_pass<M, D, G, true>(a, sm, cx, &tmk, &tmv);
+        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return;
+        if (resolve(a, sm, cx)) {
+            if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return;
+            spec = true;
+            if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(a.status + 2, 1);
+        } else {
+            // a window missed: drop the speculative counts, select exactly
+            for (size_t i = (size_t)blockIdx.x * NTH + threadIdx.x; i < 2 * (size_t)a.C; i += (size_t)gridDim.x * NTH)
+                cx.head_kept[i] = 0u;  // head_kept and head_flag are adjacent
+        }
+    }
+    if (!spec) {
+        if (cx.evict && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(a.status + 3, 1);
+        if (cx.evict && !exact_select(a, sm, cx)) return;
+        attn_pass<M, D, G, false>(a, sm, cx, &tmk, &tmv);
+        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return;
+    }
+    tail<M, D, G>(a, sm, cx, spec);
+    // exit ticket: the last CTA resets the barrier counter and flips the half
+    // of the per-call counters the next call uses
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(a.leave, 1u) == gridDim.x - 1) {
+            *a.bar = 0u;
+            *a.leave = 0u;
+            *a.parity = cx.par ^ 1u;
+            __threadfence();
+        }
+    }
+}
+
+template <class M, int D, int G>
+cudaError_t launch_one(const StepArgs &a, int grid, cudaStream_t s, const CUtensorMap &tk, const CUtensorMap &tv) {
+    using LY = StepLayout<M, D, G>;
+    auto *k = step_kernel<M, D, G>;
+    const size_t smem = LY::smem(a.max_pages);
+    if (smem > 227 * 1024) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NTH);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, a, tk, tv);
+}
+
+template <int DT, int D, int G>
+struct Pick;
+template <int D, int G>
+struct Pick<RKV_BF16, D, G> {
+    using M = MmaMath<D, G, true>;
+};
+template <int D, int G>
+struct Pick<RKV_F32, D, G> {
+    using M = CoreMath<float, D, G, true>;
+};
+
+#define RKV_STEP_CASES(X)                                                                                  \
+    X(RKV_BF16, 128, 1) X(RKV_BF16, 128, 2) X(RKV_BF16, 128, 4) X(RKV_BF16, 128, 7) X(RKV_BF16, 128, 8)   \
+    X(RKV_BF16, 64, 1) X(RKV_BF16, 64, 2) X(RKV_BF16, 64, 4) X(RKV_F32, 64, 1) X(RKV_F32, 64, 2)          \
+    X(RKV_F32, 64, 4) X(RKV_F32, 128, 1) X(RKV_F32, 128, 2) X(RKV_F32, 128, 4)
+
+}  // namespace
+
+bool step_supported(int dtype, int D, int G) {
+#define X(DT, DD, GG) \
+    if (dtype == DT && D == DD && G == GG) return true;
+    RKV_STEP_CASES(X)
+#undef X
+    return false;
+}
+
+size_t step_smem_bytes(int dtype, int D, int G, int max_pages) {
+#define X(DT, DD, GG) \
+    if (dtype == DT && D == DD && G == GG) return StepLayout<typename Pick<DT, DD, GG>::M, DD, GG>::smem(max_pages);
+    RKV_STEP_CASES(X)
+#undef X
+    return 0;
+}
+
+cudaError_t launch_step(const StepArgs &a, int dtype, int D, int G, int grid, cudaStream_t s,
+                        const CUtensorMap &tk, const CUtensorMap &tv) {
+#define X(DT, DD, GG) \
+    if (dtype == DT && D == DD && G == GG) return launch_one<typename Pick<DT, DD, GG>::M, DD, GG>(a, grid, s, tk, tv);
+    RKV_STEP_CASES(X)
+#undef X
+    return cudaErrorNotSupported;
+}
+
+}  // namespace rkv
