@@ -61,13 +61,33 @@ static_assert(STEP_HEADS_PER_CTA == NTH, "tail chunk = one head per thread");
 enum : uint32_t { SF_TRIVIAL = 1u, SF_WIN = 2u, SF_DONE = 4u };
 
 // Tail scratch (offsets in the big region).
-constexpr int T_STASH = 0;                       // int32 [5][NTH]
-constexpr int T_CL = 5 * NTH * 4;                // int32 [WIN_CAP] candidate list of one head
+constexpr int T_STASH = 0;                       // int32 [6][NTH]
+constexpr int T_CL = 6 * NTH * 4;                // int32 [WIN_CAP] candidate list of one head
 constexpr int T_PAIRS = T_CL + WIN_CAP * 4;      // int2 [CMP_PAIRS]
 constexpr int T_TBL = T_PAIRS + CMP_PAIRS * 8;   // int32 [mp], src [mp+1], hole [mp+1], uint16 msk [mp]
+// Per-warp scratch of the warp-level merge and compaction (used before the
+// block-wide fallbacks, which reuse the same bytes from T_TBL on).
+constexpr int RCAP = 16;    // partial records a warp merges (CTAs a head spans)
+constexpr int CCAP = 128;   // candidates of one head a warp merges
+constexpr int HCAP = 64;    // evicted entries of one head a warp compacts
+struct WarpScr {
+    const float *recp[RCAP];
+    float st[4][RCAP * 8];  // mk, lk, me, le of each record and query row
+    float fk[RCAP * 8];     // record weights 2^(mk_rec - mk)
+    float mk[8], lk[8];
+    int32_t cidx[CCAP];     // candidate indices (within the sequence's list)
+    int32_t cfate[CCAP];
+    float cz[CCAP * 8];     // logits, then weights 2^(z - mk) (0 for evicted)
+    int32_t holes[HCAP], srcs[HCAP];
+};
+constexpr int WARP_SCR = 9216;
+static_assert(sizeof(WarpScr) <= WARP_SCR, "warp scratch");
+constexpr int T_WARP = T_TBL;
 
 __host__ __device__ constexpr size_t tail_bytes(int mp) {
-    return (size_t)T_TBL + (size_t)mp * 4 + 2 * ((size_t)mp + 1) * 4 + (size_t)mp * 2 + 16;
+    const size_t cmp = (size_t)T_TBL + (size_t)mp * 4 + 2 * ((size_t)mp + 1) * 4 + (size_t)mp * 2 + 16;
+    const size_t wrp = (size_t)T_WARP + (size_t)NWARP * WARP_SCR;
+    return cmp > wrp ? cmp : wrp;
 }
 constexpr size_t RADIX_BYTES = (size_t)HGRP * NBINS * 4;
 constexpr size_t RESOLVE_BYTES = (size_t)WIN_CAP * 8;
@@ -1008,6 +1028,159 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
     __syncthreads();
 }
 
+// Warp-level merge of head c (same sources and result as combine_head):
+// lanes load every record's per-row statistics and every candidate's logits
+// in one round, lanes 0..G-1 merge them per query row, then every lane
+// accumulates EPL output elements with the records' loads issued together.
+// Returns false (nothing written) when the head has more than RCAP records
+// or CCAP candidates; the block-wide merge handles it then.
+template <class M, int D, int G>
+__device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, WarpScr &w, int c, int64_t pfx,
+                             int jf, int jl, uint32_t flag, bool cands) {
+    using LY = StepLayout<M, D, G>;
+    constexpr int GD = G * D;
+    constexpr int EPL = (GD + 31) / 32;
+    const int lane = threadIdx.x & 31, nct = gridDim.x;
+    const int b = c / a.LH;
+    const int cl = c - b * a.LH;
+    // ---- sources ----
+    int nrec = 0;
+    if (lane == 0) {
+        if (jf != jl) {
+            for (int j = jf; j <= jl; j++) {
+                const int64_t lo = range_lo(j, cx.TP, nct);
+                if (!(lo < range_lo(j + 1, cx.TP, nct))) continue;
+                if (nrec < RCAP) w.recp[nrec] = a.partial + ((int64_t)j * 2 + ((pfx < lo) ? 0 : 1)) * LY::REC;
+                nrec++;
+            }
+        } else if (flag & 2u) {
+            w.recp[0] = a.hrec + (int64_t)c * LY::REC;
+            nrec = 1;
+        }
+    }
+    nrec = __shfl_sync(0xFFFFFFFFu, nrec, 0);
+    if (nrec > RCAP) return false;
+    int ncl = 0;
+    const size_t cb = (size_t)b * WIN_CAP;
+    if (cands) {
+        const int nb = (int)sm.nc[b];
+        for (int base = 0; base < nb; base += 32) {
+            const int i = base + lane;
+            bool mine = false;
+            if (i < nb) {
+                const uint64_t K = __ldcg(a.ckey + cb + i);
+                mine = (a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits)) == cl;
+            }
+            const uint32_t ball = __ballot_sync(0xFFFFFFFFu, mine);
+            const int k = ncl + __popc(ball & ((1u << lane) - 1u));
+            if (mine && k < CCAP) w.cidx[k] = i;
+            ncl += __popc(ball);
+        }
+        if (ncl > CCAP) return false;
+    }
+    __syncwarp();
+    // ---- one round of loads: record statistics, candidate logits and fates ----
+    for (int t = lane; t < nrec * G; t += 32) {
+        const float *r = w.recp[t / G] + GD + (t % G);
+        w.st[0][t] = __ldcg(r);
+        w.st[1][t] = __ldcg(r + G);
+        w.st[2][t] = __ldcg(r + 2 * G);
+        w.st[3][t] = __ldcg(r + 3 * G);
+    }
+    for (int t = lane; t < ncl * G; t += 32) w.cz[t] = __ldcg(a.cz + (cb + w.cidx[t / G]) * G + (t % G));
+    for (int i = lane; i < ncl; i += 32) w.cfate[i] = __ldcg(a.cfate + cb + w.cidx[i]);
+    __syncwarp();
+    // ---- per query row: merged maxima, sums, lse and dropped mass ----
+    if (lane < G) {
+        const int g = lane;
+        Merged s;
+        s.mk = -INFINITY;
+        s.me = -INFINITY;
+        for (int k = 0; k < nrec; k++) {
+            s.mk = fmaxf(s.mk, w.st[0][k * G + g]);
+            s.me = fmaxf(s.me, w.st[2][k * G + g]);
+        }
+        for (int i = 0; i < ncl; i++) {
+            const float z = w.cz[i * G + g];
+            if (w.cfate[i]) s.mk = fmaxf(s.mk, z); else s.me = fmaxf(s.me, z);
+        }
+        s.lk = 0.0f;
+        s.le = 0.0f;
+        for (int k = 0; k < nrec; k++) {
+            const float mkw = w.st[0][k * G + g], mew = w.st[2][k * G + g];
+            const float fk = (mkw == -INFINITY) ? 0.0f : ex2(mkw - s.mk);
+            const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
+            w.fk[k * G + g] = fk;
+            s.lk += w.st[1][k * G + g] * fk;
+            s.le += w.st[3][k * G + g] * fe;
+        }
+        for (int i = 0; i < ncl; i++) {
+            const float z = w.cz[i * G + g];
+            if (w.cfate[i]) {
+                const float f = ex2(z - s.mk);
+                w.cz[i * G + g] = f;
+                s.lk += f;
+            } else {
+                w.cz[i * G + g] = 0.0f;
+                s.le += ex2(z - s.me);
+            }
+        }
+        w.mk[g] = s.mk;
+        w.lk[g] = s.lk;
+        if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
+        if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
+    }
+    __syncwarp();
+    // ---- outputs: EPL elements per lane, two records' loads in flight at a time ----
+    float av[EPL];
+#pragma unroll
+    for (int u = 0; u < EPL; u++) av[u] = 0.0f;
+    for (int k = 0; k < nrec; k += 2) {
+        const bool two = k + 1 < nrec;
+        float v0[EPL], v1[EPL];
+#pragma unroll
+        for (int u = 0; u < EPL; u++) {
+            const int e = lane + 32 * u;
+            v0[u] = e < GD ? __ldcg(w.recp[k] + e) : 0.0f;
+            v1[u] = (two && e < GD) ? __ldcg(w.recp[k + 1] + e) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < EPL; u++) {
+            const int e = lane + 32 * u;
+            const int g = (e < GD ? e : 0) / D;
+            av[u] += v0[u] * w.fk[k * G + g] + (two ? v1[u] * w.fk[(k + 1) * G + g] : 0.0f);
+        }
+    }
+    for (int i = 0; i < ncl; i++) {
+        if (!w.cfate[i]) continue;
+        const unsigned char *row = a.cv + (cb + w.cidx[i]) * a.row_bytes;
+#pragma unroll
+        for (int u = 0; u < EPL; u++) {
+            const int e = lane + 32 * u;
+            if (e < GD) av[u] += w.cz[i * G + e / D] * row_elt<M>(row, e % D);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < EPL; u++) {
+        const int e = lane + 32 * u;
+        if (e < GD) {
+            const float lk = w.lk[e / D];
+            a.out[(int64_t)c * GD + e] = lk > 0.0f ? av[u] / lk : 0.0f;
+        }
+    }
+    // ---- keep bits of the kept candidates (several may share a mask word) ----
+    for (int i = lane; i < ncl; i += 32) {
+        if (!w.cfate[i]) continue;
+        const int slot = __ldcg(a.cslot + cb + w.cidx[i]);
+        const int64_t idx = (int64_t)c * a.max_pages + slot / PAGE;
+        const uintptr_t addr = reinterpret_cast<uintptr_t>(a.keep_mask + idx);
+        unsigned int *word = reinterpret_cast<unsigned int *>(addr & ~(uintptr_t)3);
+        atomicOr(word, (1u << (slot % PAGE)) << ((addr & 2) ? 16 : 0));
+    }
+    __syncwarp();
+    return true;
+}
+
 // Hole-fill compaction of head c (n entries, nn kept): the j-th non-kept
 // slot below nn takes the j-th kept slot at or above nn; pages past
 // ceil(nn/16) go to the free stack at this head's plan offset.
@@ -1095,6 +1268,124 @@ __device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
     __syncthreads();
 }
 
+// Warp-level hole-fill compaction of head c (same result as compact_head)
+// for heads with at most HCAP evicted entries; returns false otherwise and
+// the block-wide compaction runs.  Keep words are read WPL per lane per round
+// (loads issued together); holes (non-kept slots below nn) and sources (kept
+// slots at or above nn) are listed in ascending order with warp scans; rows
+// move four pairs at a time with every load issued before the stores.
+__device__ bool compact_warp(const StepArgs &a, const Ctx &cx, WarpScr &w, int c, int n, int nn, int32_t off) {
+    if (n - nn > HCAP) return false;
+    constexpr int WPL = 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t cm = (int64_t)c * a.max_pages;
+    const int W = (n + PAGE - 1) / PAGE, Wn = (nn + PAGE - 1) / PAGE;
+    int nh = 0, ns = 0;
+    for (int w0 = 0; w0 < W; w0 += 32 * WPL) {
+        uint32_t m[WPL];
+#pragma unroll
+        for (int u = 0; u < WPL; u++) {
+            const int wd = w0 + 32 * u + lane;
+            m[u] = wd < W ? ((uint32_t)__ldcg(a.keep_mask + cm + wd) & below_bits(wd, n)) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < WPL; u++) {
+            if (w0 + 32 * u >= W) break;
+            const int wd = w0 + 32 * u + lane;
+            const uint32_t below = below_bits(wd, nn);
+            uint32_t hb = ~m[u] & below & 0xFFFFu, sb = m[u] & ~below;
+            const int hc = __popc(hb), sc = __popc(sb);
+            int hx = hc, sx = sc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xFFFFFFFFu, hx, o), z = __shfl_up_sync(0xFFFFFFFFu, sx, o);
+                if (lane >= o) {
+                    hx += y;
+                    sx += z;
+                }
+            }
+            const int htot = __shfl_sync(0xFFFFFFFFu, hx, 31), stot = __shfl_sync(0xFFFFFFFFu, sx, 31);
+            hx = nh + hx - hc;
+            sx = ns + sx - sc;
+            while (hb) {
+                const int bit = __ffs(hb) - 1;
+                hb &= hb - 1;
+                if (hx < HCAP) w.holes[hx] = wd * PAGE + bit;
+                hx++;
+            }
+            while (sb) {
+                const int bit = __ffs(sb) - 1;
+                sb &= sb - 1;
+                if (sx < HCAP) w.srcs[sx] = wd * PAGE + bit;
+                sx++;
+            }
+            nh += htot;
+            ns += stot;
+        }
+    }
+    __syncwarp();
+    const int moves = min(min(nh, ns), HCAP);
+    // physical rows of the pairs (table entries read before any is cleared)
+    for (int p = lane; p < moves; p += 32) {
+        const int hs = w.holes[p], ss = w.srcs[p];
+        w.holes[p] = __ldcg(a.block_table + cm + hs / PAGE) * PAGE + hs % PAGE;
+        w.srcs[p] = __ldcg(a.block_table + cm + ss / PAGE) * PAGE + ss % PAGE;
+    }
+    __syncwarp();
+    const int chunks = a.row_bytes / 16;
+    for (int p0 = 0; p0 < moves; p0 += 4) {
+        uint4 v[4][2];
+        int32_t pos = 0;
+        float lbv = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const int p = p0 + q;
+            const int64_t src = p < moves ? w.srcs[p] : 0;
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int i = lane + 32 * h;
+                v[q][h] = make_uint4(0, 0, 0, 0);
+                if (p < moves && i < 2 * chunks) {
+                    const uint4 *base = reinterpret_cast<const uint4 *>(
+                        (const unsigned char *)(i < chunks ? a.k_pool : a.v_pool) + src * a.row_bytes);
+                    v[q][h] = __ldcg(base + (i < chunks ? i : i - chunks));
+                }
+            }
+            if (lane == q && p < moves) {
+                pos = __ldcg(a.pos_pool + src);
+                lbv = __ldcg(a.lb_pool + src);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const int p = p0 + q;
+            if (p >= moves) break;
+            const int64_t dst = w.holes[p];
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int i = lane + 32 * h;
+                if (i < 2 * chunks) {
+                    uint4 *base = reinterpret_cast<uint4 *>((unsigned char *)(i < chunks ? a.k_pool : a.v_pool) +
+                                                            dst * a.row_bytes);
+                    base[i < chunks ? i : i - chunks] = v[q][h];
+                }
+            }
+            if (lane == q) {
+                a.pos_pool[dst] = pos;
+                a.lb_pool[dst] = lbv;
+            }
+        }
+    }
+    __syncwarp();
+    // freed pages, ascending table index, at this head's offset in the stack
+    for (int pi = Wn + lane; pi < W; pi += 32) {
+        a.free_stack[cx.top0 + off + (pi - Wn)] = __ldcg(a.block_table + cm + pi);
+        a.block_table[cm + pi] = -1;
+    }
+    __syncwarp();
+    return true;
+}
+
 // Bounded wait until every CTA has finished its compactions (pushes).
 __device__ bool wait_pushes(const StepArgs &a, const Ctx &cx) {
     const uint32_t target = gridDim.x;
@@ -1160,7 +1451,7 @@ __device__ void append_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int 
 
 template <class M, int D, int G>
 __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) {
-    const int tid = threadIdx.x, warp = tid >> 5, nct = gridDim.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nct = gridDim.x;
     const int C = a.C;
     const int hc0 = (int)((int64_t)blockIdx.x * C / nct), hc1 = (int)((int64_t)(blockIdx.x + 1) * C / nct);
     int32_t *st_npre = reinterpret_cast<int32_t *>(sm.big + T_STASH);
@@ -1219,19 +1510,41 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
         const int nt = cx.top0 + (int)pushes - (int)pops;
         *a.free_top = nt < 0 ? 0 : nt;
     }
-    // merges, keep-bit patches and compaction, head by head
-    for (int c = hc0; c < hc1; c++) {
-        const int k = c - hc0;
+    // merges, keep-bit patches and compaction: one warp per head; heads too
+    // large for a warp are done block-wide afterwards, one at a time
+    int32_t *st_heavy = st_pop + NTH;
+    WarpScr &wsc = *reinterpret_cast<WarpScr *>(sm.big + T_WARP + warp * WARP_SCR);
+    for (int k = warp; k < hc1 - hc0; k += NWARP) {
+        const int c = hc0 + k;
         const int np = st_npre[k], nn = st_nnew[k];
         const int pages = (np + PAGE - 1) / PAGE;
+        int heavy = 0;
         if (pages > 0) {
             const int64_t pfx = st_pfx[k];
             const int jf = owner_of(pfx, cx.TP, nct), jl = owner_of(pfx + pages - 1, cx.TP, nct);
             const uint32_t flag = __ldcg(cx.head_flag + c);
             const bool cands = spec && (flag & 1u);
-            if (jf != jl || (flag & 2u) || cands) combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, cands);
+            if ((jf != jl || (flag & 2u) || cands) &&
+                !combine_warp<M, D, G>(a, sm, cx, wsc, c, pfx, jf, jl, flag, cands))
+                heavy = 3;  // merge, then compaction (after the keep-bit patches), block-wide
         }
-        if (cx.evict && nn < np) compact_head(a, sm, cx, c, np, nn, st_plan[k]);
+        if (!(heavy & 2) && cx.evict && nn < np && !compact_warp(a, cx, wsc, c, np, nn, st_plan[k])) heavy |= 2;
+        if (lane == 0) st_heavy[k] = heavy;
+    }
+    __syncthreads();
+    for (int k = 0; k < hc1 - hc0; k++) {
+        const int heavy = st_heavy[k];
+        if (!heavy) continue;
+        const int c = hc0 + k;
+        const int np = st_npre[k], nn = st_nnew[k];
+        if (heavy & 1) {
+            const int pages = (np + PAGE - 1) / PAGE;
+            const int64_t pfx = st_pfx[k];
+            const int jf = owner_of(pfx, cx.TP, nct), jl = owner_of(pfx + pages - 1, cx.TP, nct);
+            const uint32_t flag = __ldcg(cx.head_flag + c);
+            combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, spec && (flag & 1u));
+        }
+        if ((heavy & 2) && cx.evict && nn < np) compact_head(a, sm, cx, c, np, nn, st_plan[k]);
     }
     __syncthreads();
     if (tid == 0) {
