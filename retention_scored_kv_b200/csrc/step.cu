@@ -92,6 +92,18 @@ __host__ __device__ constexpr size_t tail_bytes(int mp) {
 constexpr size_t RADIX_BYTES = (size_t)HGRP * NBINS * 4;
 constexpr size_t RESOLVE_BYTES = (size_t)WIN_CAP * 8;
 
+// Fixed part of shared memory (offsets from the 1024-aligned base, the same
+// for every instance): per-sequence state, scan scratch, flags, the CTA range
+// starts and the pipeline barriers; the big region follows at S_BIG.
+constexpr int MAX_NBAR = 2 * NCW * 8 + 2 * QR;
+constexpr int S_LO = 0, S_HI = S_LO + MAXB * 8, S_KAP = S_HI + MAXB * 8, S_PK = S_KAP + MAXB * 8,
+              S_PM = S_PK + MAXB * 8, S_KMX = S_PM + MAXB * 8, S_M = S_KMX + MAXB * 8, S_T = S_M + MAXB * 8,
+              S_N = S_T + MAXB * 4, S_RANK = S_N + MAXB * 4, S_FL = S_RANK + MAXB * 4, S_ABOVE = S_FL + MAXB * 4,
+              S_NC = S_ABOVE + MAXB * 4, S_OFF = S_NC + MAXB * 4, S_WRES = S_OFF + MAXB * 4,
+              S_SCAN = S_WRES + MAXB * 4, S_MISC = S_SCAN + 4 * 36 * 4, S_MISC64 = S_MISC + 64 * 4,
+              S_RLO = S_MISC64 + 8 * 8, S_BAR = (S_RLO + (MAX_ATTN_CTAS + 1) * 4 + 15) / 16 * 16,
+              S_BIG = (S_BAR + MAX_NBAR * 8 + 1023) / 1024 * 1024;
+
 // Shared memory: the fixed part (pipeline barriers, per-sequence state, scan
 // scratch) first, then the big region: attention stages, positions /
 // log-retentions, query ring, merge slots and stage metadata during an
@@ -106,13 +118,6 @@ struct StepLayout {
     static constexpr int REC = G * (D + 4);                   // partial record floats
     static constexpr int WSLOT = G * D + 4 * G + 4;           // merge slot: acc, mk, lk, me, le, candidates
     static constexpr int NBAR = 2 * NST + 2 * QR;
-    static constexpr int OFF_BAR = 0;
-    static constexpr int OFF_SEQ = (NBAR * 8 + 15) / 16 * 16;
-    static constexpr int SEQ_BYTES = MAXB * (7 * 8 + 8 * 4);
-    static constexpr int OFF_SCAN = OFF_SEQ + SEQ_BYTES;      // [4][36] words
-    static constexpr int OFF_MISC = OFF_SCAN + 4 * 36 * 4;    // int [64], int64 [8]
-    static constexpr int FIXED = OFF_MISC + 64 * 4 + 8 * 8;
-    static constexpr int OFF_BIG = (FIXED + M::STAGE_ALIGN - 1) / M::STAGE_ALIGN * M::STAGE_ALIGN;
     static constexpr int B_STAGE = 0;
     static constexpr int B_POSLB = NST * STAGE_BYTES;         // [NST][16 positions, 16 log-retentions]
     static constexpr int B_Q = B_POSLB + NST * 128;
@@ -121,39 +126,54 @@ struct StepLayout {
     static constexpr int BIG_ATTN = B_META + NST * 4;
     static_assert(STAGE_BYTES % M::STAGE_ALIGN == 0, "stage alignment");
     static_assert(QBYTES % 16 == 0, "query block must be a 16-byte multiple");
-    static_assert(NBAR <= NTH, "barrier init");
+    static_assert(NBAR <= NTH && NBAR <= MAX_NBAR, "barrier init");
+    static_assert(M::STAGE_ALIGN <= 1024, "big region alignment");
     static_assert(BIG_ATTN >= (int)RADIX_BYTES && BIG_ATTN >= (int)RESOLVE_BYTES, "scratch");
     static size_t smem(int mp) {
         const size_t big = tail_bytes(mp) > (size_t)BIG_ATTN ? tail_bytes(mp) : (size_t)BIG_ATTN;
-        return (size_t)OFF_BIG + big + M::STAGE_ALIGN;
+        return (size_t)S_BIG + big + 1024;
     }
 };
 
+// Shared memory through one base pointer (offsets are constants, so no
+// per-array pointers stay live across the attention pass).
 struct Sm {
-    uint64_t *bars;
-    uint64_t *lo, *hi, *kap, *pk, *pm;  // [MAXB]
-    unsigned long long *kmx;             // [MAXB] largest kept key of this CTA's pages
-    int64_t *m;                          // [MAXB] clamped budget
-    int32_t *t;                          // [MAXB]
-    uint32_t *n, *rank, *fl, *above, *nc, *off, *wres, *spare;  // [MAXB]
-    uint32_t *scan;                      // [4][36]
-    int *misc;                           // [64]
-    int64_t *misc64;                     // [8]
-    unsigned char *big;
+    unsigned char *base;
+    template <typename T>
+    __device__ __forceinline__ T *at(int off) const { return reinterpret_cast<T *>(base + off); }
+    __device__ __forceinline__ uint64_t *bars() const { return at<uint64_t>(S_BAR); }
+    __device__ __forceinline__ uint64_t *lo() const { return at<uint64_t>(S_LO); }
+    __device__ __forceinline__ uint64_t *hi() const { return at<uint64_t>(S_HI); }
+    __device__ __forceinline__ uint64_t *kap() const { return at<uint64_t>(S_KAP); }
+    __device__ __forceinline__ uint64_t *pk() const { return at<uint64_t>(S_PK); }
+    __device__ __forceinline__ uint64_t *pm() const { return at<uint64_t>(S_PM); }
+    __device__ __forceinline__ unsigned long long *kmx() const { return at<unsigned long long>(S_KMX); }
+    __device__ __forceinline__ int64_t *m() const { return at<int64_t>(S_M); }
+    __device__ __forceinline__ int32_t *t() const { return at<int32_t>(S_T); }
+    __device__ __forceinline__ uint32_t *n() const { return at<uint32_t>(S_N); }
+    __device__ __forceinline__ uint32_t *rank() const { return at<uint32_t>(S_RANK); }
+    __device__ __forceinline__ uint32_t *fl() const { return at<uint32_t>(S_FL); }
+    __device__ __forceinline__ uint32_t *above() const { return at<uint32_t>(S_ABOVE); }
+    __device__ __forceinline__ uint32_t *nc() const { return at<uint32_t>(S_NC); }
+    __device__ __forceinline__ uint32_t *off() const { return at<uint32_t>(S_OFF); }
+    __device__ __forceinline__ uint32_t *wres() const { return at<uint32_t>(S_WRES); }
+    __device__ __forceinline__ uint32_t *scan() const { return at<uint32_t>(S_SCAN); }
+    __device__ __forceinline__ int *misc() const { return at<int>(S_MISC); }
+    __device__ __forceinline__ int64_t *misc64() const { return at<int64_t>(S_MISC64); }
+    __device__ __forceinline__ int32_t *rlo() const { return at<int32_t>(S_RLO); }
+    __device__ __forceinline__ unsigned char *big() const { return base + S_BIG; }
 };
 
 // misc slots
 enum { MS_CSTART = 0, MS_CLAST, MS_RADIX, MS_MISS, MS_BAR, MS_TOTAL, MS_FOUND, MS_DIG, MS_NR, MS_H, MS_NCL,
-       MS_ACTIVE };
+       MS_ACTIVE, MS_QN, MS_QH };
 
 struct Ctx {
-    int64_t TP, x0, x1, pfx_start;
+    int32_t TP, x0, x1, pfx_start;  // flattened pages (< 2^27)
     int c_start, c_last;
     bool last, evict;
     int32_t top0;
     uint32_t par, epoch;
-    int h0, h1;
-    uint32_t my_pfx;
     bool exact;      // the exact selection ran (its thresholds are reported in the tail)
     int passes;      // exact-select passes run (histograms to clear)
     int attn_runs;   // attention passes run
@@ -161,10 +181,23 @@ struct Ctx {
     // attention pass continues their phases: its page indices start after
     // the pages of the earlier passes (pbase) and its query slots after
     // their heads (qbase).  Producer and consumer count both alike.
-    int64_t pbase;
+    int32_t pbase;
     int qbase;
-    uint32_t *head_kept, *head_flag, *seqc, *arrive;
 };
+
+// This call's half of the per-call counters: head_kept[C], head_flag[C],
+// seq[B][4], arrivals.
+__device__ __forceinline__ uint32_t *ctr_of(const StepArgs &a, const Ctx &cx) {
+    return a.ctr + (size_t)cx.par * a.ctr_words;
+}
+__device__ __forceinline__ uint32_t *head_kept_of(const StepArgs &a, const Ctx &cx) { return ctr_of(a, cx); }
+__device__ __forceinline__ uint32_t *head_flag_of(const StepArgs &a, const Ctx &cx) { return ctr_of(a, cx) + a.C; }
+__device__ __forceinline__ uint32_t *seqc_of(const StepArgs &a, const Ctx &cx) {
+    return ctr_of(a, cx) + 2 * (size_t)a.C;
+}
+__device__ __forceinline__ uint32_t *arrive_of(const StepArgs &a, const Ctx &cx) {
+    return ctr_of(a, cx) + 2 * (size_t)a.C + 4 * (size_t)a.B;
+}
 
 template <int NSCAN>
 __device__ __forceinline__ void block_scan_n(const uint32_t (&v)[NSCAN], uint32_t (&ex)[NSCAN],
@@ -239,18 +272,24 @@ __device__ void scan_words(int32_t *v, int W, uint32_t *scratch) {
     __syncthreads();
 }
 
+// CTA whose page range holds flattened page x: the largest j with
+// rlo[j] <= x (empty ranges share their start with the next one).
+__device__ __forceinline__ int owner_rlo(const int32_t *rlo, int nct, int64_t x) {
+    int lo = 0, hi = nct - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (rlo[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 // ------------------------------------------------------------- prologue ----
 template <class M, int D, int G>
 __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &cx, const CUtensorMap *tmk,
                                          const CUtensorMap *tmv) {
     const int tid = threadIdx.x, nct = gridDim.x;
     cx.par = __ldcg(a.parity) & 1u;
-    uint32_t *mine = a.ctr + (size_t)cx.par * a.ctr_words;
     uint32_t *other = a.ctr + (size_t)(cx.par ^ 1u) * a.ctr_words;
-    cx.head_kept = mine;
-    cx.head_flag = mine + a.C;
-    cx.seqc = mine + 2 * (size_t)a.C;
-    cx.arrive = cx.seqc + 4 * (size_t)a.B;
     // the other half is the next call's: clear it now
     for (size_t i = (size_t)blockIdx.x * NTH + tid; i < (size_t)a.ctr_words; i += (size_t)nct * NTH) other[i] = 0u;
     cx.top0 = __ldcg(a.free_top);
@@ -261,11 +300,11 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
     cx.attn_runs = 0;
     cx.pbase = 0;
     cx.qbase = 0;
-    if (tid < MAXB) sm.n[tid] = 0u;
-    if (tid < 64) sm.misc[tid] = 0;
+    if (tid < MAXB) sm.n()[tid] = 0u;
+    if (tid < 64) sm.misc()[tid] = 0;
     if (tid == 0) {
-        sm.misc[MS_CSTART] = a.C;
-        sm.misc[MS_CLAST] = -1;
+        sm.misc()[MS_CSTART] = a.C;
+        sm.misc()[MS_CLAST] = -1;
     }
     if (M::USES_TMAP && tid == 0) {
         prefetch_tensormap(tmk);
@@ -273,23 +312,24 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
     }
     __syncthreads();
     const int CS = (a.C + NTH - 1) / NTH;
-    cx.h0 = min(a.C, tid * CS);
-    cx.h1 = min(a.C, cx.h0 + CS);
+    const int h0 = min(a.C, tid * CS), h1 = min(a.C, h0 + CS);
     uint32_t my_pages = 0;
-    for (int c = cx.h0; c < cx.h1; c++) {
+    for (int c = h0; c < h1; c++) {
         const int32_t n = max(__ldcg(a.len + c), 0);
         my_pages += (uint32_t)((n + PAGE - 1) / PAGE);
-        atomicAdd(&sm.n[c / a.LH], (uint32_t)n);
+        atomicAdd(&sm.n()[c / a.LH], (uint32_t)n);
         if (c % nct == (int)blockIdx.x) {
             a.npre[c] = n;
             if (cx.evict) a.n_pre[c] = n;
         }
     }
     uint32_t TPu;
-    cx.my_pfx = block_exclusive_scan(my_pages, sm.scan, &TPu);
-    cx.TP = TPu;
-    cx.x0 = range_lo(blockIdx.x, cx.TP, nct);
-    cx.x1 = range_lo(blockIdx.x + 1, cx.TP, nct);
+    const uint32_t my_pfx = block_exclusive_scan(my_pages, sm.scan(), &TPu);
+    cx.TP = (int32_t)TPu;
+    cx.x0 = (int32_t)range_lo(blockIdx.x, cx.TP, nct);
+    cx.x1 = (int32_t)range_lo(blockIdx.x + 1, cx.TP, nct);
+    // every CTA's range start, once (the tail looks them up instead of dividing)
+    for (int j = tid; j <= nct; j += NTH) sm.rlo()[j] = (int32_t)range_lo(j, cx.TP, nct);
     cx.last = blockIdx.x == nct - 1;
     // first head of the range (first c with pfx + max(pages, 1) > x0) and
     // the last head the range visits (last c with pfx < x1; every head for
@@ -297,8 +337,8 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
     int first = a.C, lastc = -1;
     int64_t first_pfx = 0;
     {
-        int64_t p = cx.my_pfx;
-        for (int c = cx.h0; c < cx.h1; c++) {
+        int64_t p = my_pfx;
+        for (int c = h0; c < h1; c++) {
             const int64_t pg = (max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE;
             if (first == a.C && p + (pg > 0 ? pg : 1) > cx.x0) {
                 first = c;
@@ -308,15 +348,15 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
             p += pg;
         }
     }
-    if (first < a.C) atomicMin(&sm.misc[MS_CSTART], first);
-    if (lastc >= 0) atomicMax(&sm.misc[MS_CLAST], lastc);
+    if (first < a.C) atomicMin(&sm.misc()[MS_CSTART], first);
+    if (lastc >= 0) atomicMax(&sm.misc()[MS_CLAST], lastc);
     __syncthreads();
-    if (first < a.C && first == sm.misc[MS_CSTART]) sm.misc64[0] = first_pfx;
+    if (first < a.C && first == sm.misc()[MS_CSTART]) sm.misc64()[0] = first_pfx;
     // per-sequence setup
     if (tid < a.B) {
         const int b = tid;
-        sm.t[b] = __ldg(a.t + b);
-        const int64_t N = sm.n[b];
+        sm.t()[b] = __ldg(a.t + b);
+        const int64_t N = sm.n()[b];
         uint32_t fl = SF_TRIVIAL | SF_DONE;
         uint64_t lo = ~0ull, hi = ~0ull, kap = ~0ull;
         int64_t m = N;
@@ -334,24 +374,24 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
                     hi = (uint64_t)__ldcg(w + 2) << 32;
                 } else {
                     fl = 0u;
-                    atomicOr(&sm.misc[MS_RADIX], 1);
+                    atomicOr(&sm.misc()[MS_RADIX], 1);
                 }
                 kap = 0ull;
             }
         }
-        sm.m[b] = m;
-        sm.fl[b] = fl;
-        sm.lo[b] = lo;
-        sm.hi[b] = hi;
-        sm.kap[b] = kap;
-        sm.wres[b] = 0u;
-        sm.above[b] = 0u;
-        sm.nc[b] = 0u;
+        sm.m()[b] = m;
+        sm.fl()[b] = fl;
+        sm.lo()[b] = lo;
+        sm.hi()[b] = hi;
+        sm.kap()[b] = kap;
+        sm.wres()[b] = 0u;
+        sm.above()[b] = 0u;
+        sm.nc()[b] = 0u;
     }
     __syncthreads();
-    cx.c_start = sm.misc[MS_CSTART];
-    cx.c_last = sm.misc[MS_CLAST];
-    cx.pfx_start = cx.c_start < a.C ? sm.misc64[0] : cx.TP;
+    cx.c_start = sm.misc()[MS_CSTART];
+    cx.c_last = sm.misc()[MS_CLAST];
+    cx.pfx_start = cx.c_start < a.C ? (int32_t)sm.misc64()[0] : cx.TP;
 }
 
 // -------------------------------------------------------- attention pass ----
@@ -365,12 +405,12 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                                           const CUtensorMap *tmv) {
     using LY = StepLayout<M, D, G>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t *full = sm.bars, *empty = full + LY::NST, *qfull = empty + LY::NST, *qempty = qfull + QR;
-    unsigned char *stage = sm.big + LY::B_STAGE;
-    unsigned char *poslb = sm.big + LY::B_POSLB;
-    float *qring = reinterpret_cast<float *>(sm.big + LY::B_Q);
-    float *merge = reinterpret_cast<float *>(sm.big + LY::B_MERGE);
-    uint32_t *meta = reinterpret_cast<uint32_t *>(sm.big + LY::B_META);
+    uint64_t *full = sm.bars(), *empty = full + LY::NST, *qfull = empty + LY::NST, *qempty = qfull + QR;
+    unsigned char *stage = sm.big() + LY::B_STAGE;
+    unsigned char *poslb = sm.big() + LY::B_POSLB;
+    float *qring = reinterpret_cast<float *>(sm.big() + LY::B_Q);
+    float *merge = reinterpret_cast<float *>(sm.big() + LY::B_MERGE);
+    uint32_t *meta = reinterpret_cast<uint32_t *>(sm.big() + LY::B_META);
     __syncthreads();
     if (cx.attn_runs == 0) {
         if (tid < LY::NBAR) {
@@ -399,7 +439,7 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
         int64_t pfx;
         while (w.next(&c, &pfx, &pages, &n)) {
             if (pages == 0) continue;
-            const int64_t pa = max(pfx, cx.x0), pb = min(pfx + pages, cx.x1);
+            const int64_t pa = max(pfx, (int64_t)cx.x0), pb = min(pfx + pages, (int64_t)cx.x1);
             if (pw == 0 && lane == 0) {
                 const int slot = nq % QR;
                 mbar_wait(&qempty[slot], ((nq / QR) & 1) ^ 1, a.status, site + 1);
@@ -469,7 +509,7 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                 }
                 continue;
             }
-            const int64_t pa = max(pfx, cx.x0), pb = min(pfx + pages, cx.x1);
+            const int64_t pa = max(pfx, (int64_t)cx.x0), pb = min(pfx + pages, (int64_t)cx.x1);
             const bool whole = (pfx >= cx.x0) && (pfx + pages <= cx.x1);
             {
                 const int slot = nq % QR;
@@ -485,9 +525,9 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
             if constexpr (SPEC) {
                 b = c / a.LH;
                 cl = (uint32_t)(c - b * a.LH);
-                wlo = sm.lo[b];
-                whi = sm.hi[b];
-                tb = sm.t[b];
+                wlo = sm.lo()[b];
+                whi = sm.hi()[b];
+                tb = sm.t()[b];
             }
             uint32_t kc = 0, ncw = 0;
             // virtual page index v = li + pb0 (this pass's pages follow the earlier passes')
@@ -524,8 +564,8 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                     kc += (uint32_t)__popc(keepm);
                     if (candm) {
                         if (lane == 0) {
-                            cbase = atomicAdd(cx.seqc + (size_t)b * 4 + 1, (uint32_t)__popc(candm));
-                            atomicOr(cx.head_flag + c, 1u);
+                            cbase = atomicAdd(seqc_of(a, cx) + (size_t)b * 4 + 1, (uint32_t)__popc(candm));
+                            atomicOr(head_flag_of(a, cx) + c, 1u);
                         }
                         cbase = __shfl_sync(0xFFFFFFFFu, cbase, 0);
                         if (lane < 16 && cand) {
@@ -563,8 +603,8 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
             }
             if constexpr (SPEC) {
                 if (lane == 0 && kc) {
-                    atomicAdd(cx.head_kept + c, kc);
-                    atomicAdd(cx.seqc + (size_t)b * 4, kc);
+                    atomicAdd(head_kept_of(a, cx) + c, kc);
+                    atomicAdd(seqc_of(a, cx) + (size_t)b * 4, kc);
                 }
             }
             const int par = nq & 1;
@@ -623,7 +663,7 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                     rec[G * D + 3 * G + g] = s.le;
                 }
             }
-            if (dest == 1 && tid == 0) atomicOr(cx.head_flag + c, 2u);
+            if (dest == 1 && tid == 0) atomicOr(head_flag_of(a, cx) + c, 2u);
         }
         cx.qbase = nq;
         if constexpr (REG_SPLIT) setmaxnreg_dec<LAUNCH_REGS>();
@@ -646,58 +686,63 @@ __device__ bool resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
     const int tid = threadIdx.x, nct = gridDim.x;
     if (tid < a.B) {
         const int b = tid;
-        if (!(sm.fl[b] & SF_TRIVIAL)) {
-            const uint32_t above = __ldcg(cx.seqc + (size_t)b * 4), nc = __ldcg(cx.seqc + (size_t)b * 4 + 1);
-            const int64_t m = sm.m[b];
+        if (!(sm.fl()[b] & SF_TRIVIAL)) {
+            const uint32_t above = __ldcg(seqc_of(a, cx) + (size_t)b * 4), nc = __ldcg(seqc_of(a, cx) + (size_t)b * 4 + 1);
+            const int64_t m = sm.m()[b];
             const bool hit = nc <= (uint32_t)WIN_CAP && (int64_t)above < m && m <= (int64_t)above + nc;
-            sm.above[b] = above;
-            sm.nc[b] = hit ? nc : 0u;
+            sm.above()[b] = above;
+            sm.nc()[b] = hit ? nc : 0u;
             // window outcome, used to resize it even if another sequence
             // sends the call down the exact path
-            sm.wres[b] = hit ? 1u : (nc > (uint32_t)WIN_CAP ? 3u : 2u);
-            if (!hit) atomicOr(&sm.misc[MS_MISS], 1);
+            sm.wres()[b] = hit ? 1u : (nc > (uint32_t)WIN_CAP ? 3u : 2u);
+            if (!hit) atomicOr(&sm.misc()[MS_MISS], 1);
         }
     }
     __syncthreads();
-    if (sm.misc[MS_MISS]) return false;
+    if (sm.misc()[MS_MISS]) return false;
     if (tid == 0) {
         uint32_t o = 0;
         for (int b = 0; b < a.B; b++) {
-            sm.off[b] = o;
-            o += sm.nc[b];
+            sm.off()[b] = o;
+            o += sm.nc()[b];
         }
-        sm.misc[MS_TOTAL] = (int)o;
+        sm.misc()[MS_TOTAL] = (int)o;
     }
     __syncthreads();
-    const int64_t total = sm.misc[MS_TOTAL];
+    const int64_t total = sm.misc()[MS_TOTAL];
     const int64_t s0 = (int64_t)blockIdx.x * total / nct, s1 = (int64_t)(blockIdx.x + 1) * total / nct;
-    uint64_t *keys = reinterpret_cast<uint64_t *>(sm.big);
+    uint64_t *keys = reinterpret_cast<uint64_t *>(sm.big());
     for (int b = 0; b < a.B; b++) {
-        const int64_t ob = sm.off[b], nb = sm.nc[b];
+        const int64_t ob = sm.off()[b], nb = sm.nc()[b];
         const int64_t jlo = max(s0, ob) - ob, jhi = min(s1, ob + nb) - ob;
         if (jlo >= jhi) continue;
         for (int i = tid; i < nb; i += NTH) keys[i] = __ldcg(a.ckey + (size_t)b * WIN_CAP + i);
         __syncthreads();
-        const uint32_t r = (uint32_t)(sm.m[b] - (int64_t)sm.above[b]);  // 1-based
-        for (int64_t j = jlo + tid; j < jhi; j += NTH) {
+        const uint32_t r = (uint32_t)(sm.m()[b] - (int64_t)sm.above()[b]);  // 1-based
+        // one warp per candidate: lanes count the smaller keys in parallel
+        const int lane = tid & 31, warp = tid >> 5;
+        for (int64_t j = jlo + warp; j < jhi; j += NWARP) {
             const uint64_t K = keys[j];
             uint32_t less = 0;
-            for (int i = 0; i < nb; i++) less += keys[i] < K ? 1u : 0u;
-            const bool kept = less < r;
-            a.cfate[(size_t)b * WIN_CAP + j] = kept ? 1 : 0;
-            if (kept) {
-                const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
-                atomicAdd(cx.head_kept + (int64_t)b * a.LH + cl, 1u);
-            }
-            if (less == r - 1) {
-                const uint64_t kap = K + 1ull;
-                a.kappa[b] = kap;
-                window_next(a.win + (size_t)b * 4, kap, 1, (uint32_t)nb);
+            for (int i = lane; i < nb; i += 32) less += keys[i] < K ? 1u : 0u;
+            less = __reduce_add_sync(0xFFFFFFFFu, less);
+            if (lane == 0) {
+                const bool kept = less < r;
+                a.cfate[(size_t)b * WIN_CAP + j] = kept ? 1 : 0;
+                if (kept) {
+                    const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
+                    atomicAdd(head_kept_of(a, cx) + (int64_t)b * a.LH + cl, 1u);
+                }
+                if (less == r - 1) {
+                    const uint64_t kap = K + 1ull;
+                    a.kappa[b] = kap;
+                    window_next(a.win + (size_t)b * 4, kap, 1, (uint32_t)nb);
+                }
             }
         }
         __syncthreads();
     }
-    if (blockIdx.x == 0 && tid < a.B && (sm.fl[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap[tid];
+    if (blockIdx.x == 0 && tid < a.B && (sm.fl()[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap()[tid];
     return true;
 }
 
@@ -758,7 +803,7 @@ __device__ __forceinline__ void for_range_keys(const StepArgs &a, const Sm &sm, 
             bool ok = false;
             if (ld[u]) {
                 const int b = hc[u] / a.LH;
-                ok = entry_key(sm.t[b], (uint32_t)(hc[u] - b * a.LH), pos[u], lbv[u], a.ibits, &K);
+                ok = entry_key(sm.t()[b], (uint32_t)(hc[u] - b * a.LH), pos[u], lbv[u], a.ibits, &K);
                 if (!ok) set_status(a.status, RKV_DEV_BAD_INPUT);
             }
             f(hc[u], pidx[u], r, K, ok);
@@ -767,8 +812,8 @@ __device__ __forceinline__ void for_range_keys(const StepArgs &a, const Sm &sm, 
 }
 
 // This call's largest kept key of sequence b (uint64 in the counter half).
-__device__ __forceinline__ unsigned long long *kmax_of(const Ctx &cx, int b) {
-    return reinterpret_cast<unsigned long long *>(cx.seqc + (size_t)b * 4 + 2);
+__device__ __forceinline__ unsigned long long *kmax_of(const StepArgs &a, const Ctx &cx, int b) {
+    return reinterpret_cast<unsigned long long *>(seqc_of(a, cx) + (size_t)b * 4 + 2);
 }
 
 // Digit p of sequence b's threshold from its completed global histogram
@@ -784,39 +829,39 @@ __device__ void scan_digit(const StepArgs &a, const Sm &sm, int b, int p) {
         v[j] = i < NBINS ? __ldcg(gh + i) : 0u;
         loc += v[j];
     }
-    if (tid == 0) sm.misc[MS_FOUND] = 0;
+    if (tid == 0) sm.misc()[MS_FOUND] = 0;
     uint32_t total;
-    const uint32_t ex = block_exclusive_scan(loc, sm.scan, &total);
-    const uint32_t rank = sm.rank[b];
+    const uint32_t ex = block_exclusive_scan(loc, sm.scan(), &total);
+    const uint32_t rank = sm.rank()[b];
     if (ex < rank && rank <= ex + loc) {
         uint32_t cum = ex;
 #pragma unroll
         for (int j = 0; j < PER; j++) {
             if (cum < rank && rank <= cum + v[j]) {
-                sm.misc[MS_DIG] = tid * PER + j;
-                sm.misc[MS_NR] = (int)(rank - cum);
-                sm.misc[MS_H] = (int)v[j];
-                sm.misc[MS_FOUND] = 1;
+                sm.misc()[MS_DIG] = tid * PER + j;
+                sm.misc()[MS_NR] = (int)(rank - cum);
+                sm.misc()[MS_H] = (int)v[j];
+                sm.misc()[MS_FOUND] = 1;
             }
             cum += v[j];
         }
     }
     __syncthreads();
     if (tid == 0) {
-        if (!sm.misc[MS_FOUND]) {
+        if (!sm.misc()[MS_FOUND]) {
             // fewer matching keys than the rank (entries rejected as bad input)
             set_status(a.status, RKV_DEV_BAD_INPUT);
-            sm.fl[b] |= SF_DONE;
-            sm.kap[b] = (sm.pk[b] | ~sm.pm[b]) + 1ull;
+            sm.fl()[b] |= SF_DONE;
+            sm.kap()[b] = (sm.pk()[b] | ~sm.pm()[b]) + 1ull;
         } else {
             const int sh = digit_shift(p);
-            const uint64_t d = (uint64_t)sm.misc[MS_DIG];
-            sm.pk[b] |= d << sh;
-            sm.pm[b] |= ((1ull << digit_bits(p)) - 1ull) << sh;
-            sm.rank[b] = (uint32_t)sm.misc[MS_NR];
-            if ((uint32_t)sm.misc[MS_H] == sm.rank[b] || p == NPASS - 1) {
-                sm.fl[b] |= SF_DONE;
-                sm.kap[b] = (sm.pk[b] | ~sm.pm[b]) + 1ull;
+            const uint64_t d = (uint64_t)sm.misc()[MS_DIG];
+            sm.pk()[b] |= d << sh;
+            sm.pm()[b] |= ((1ull << digit_bits(p)) - 1ull) << sh;
+            sm.rank()[b] = (uint32_t)sm.misc()[MS_NR];
+            if ((uint32_t)sm.misc()[MS_H] == sm.rank()[b] || p == NPASS - 1) {
+                sm.fl()[b] |= SF_DONE;
+                sm.kap()[b] = (sm.pk()[b] | ~sm.pm()[b]) + 1ull;
             }
         }
     }
@@ -829,33 +874,37 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
     const int tid = threadIdx.x, lane = tid & 31;
     {
         // page prefix of the heads this CTA's range visits, for page -> head
-        int64_t p = cx.my_pfx;
-        for (int c = cx.h0; c < cx.h1; c++) {
+        const int CS = (a.C + NTH - 1) / NTH;
+        const int h0 = min(a.C, tid * CS), h1 = min(a.C, h0 + CS);
+        uint32_t mine = 0, tot;
+        for (int c = h0; c < h1; c++) mine += (uint32_t)((max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE);
+        int64_t p = block_exclusive_scan(mine, sm.scan(), &tot);
+        for (int c = h0; c < h1; c++) {
             if (c >= cx.c_start && c <= cx.c_last + 1) a.pfx[c] = (int32_t)p;
             p += (max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE;
         }
         if (tid == 0 && cx.c_last + 1 == a.C) a.pfx[a.C] = (int32_t)cx.TP;
     }
     cx.exact = true;
-    if (tid < a.B && !(sm.fl[tid] & SF_TRIVIAL)) {
-        sm.fl[tid] &= ~SF_DONE;
-        sm.rank[tid] = (uint32_t)sm.m[tid];
-        sm.pk[tid] = 0ull;
-        sm.pm[tid] = 0ull;
+    if (tid < a.B && !(sm.fl()[tid] & SF_TRIVIAL)) {
+        sm.fl()[tid] &= ~SF_DONE;
+        sm.rank()[tid] = (uint32_t)sm.m()[tid];
+        sm.pk()[tid] = 0ull;
+        sm.pm()[tid] = 0ull;
     }
-    if (tid < MAXB) sm.kmx[tid] = 0ull;
+    if (tid < MAXB) sm.kmx()[tid] = 0ull;
     __syncthreads();
     const int b_first = cx.c_start < a.C ? cx.c_start / a.LH : 0;
     const int b_last = cx.c_last >= 0 ? cx.c_last / a.LH : -1;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(sm.big);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sm.big());
     for (int p = 0; p < NPASS; p++) {
         if (tid == 0) {
             int act = 0;
-            for (int b = 0; b < a.B; b++) act |= (sm.fl[b] & SF_DONE) ? 0 : 1;
-            sm.misc[MS_ACTIVE] = act;
+            for (int b = 0; b < a.B; b++) act |= (sm.fl()[b] & SF_DONE) ? 0 : 1;
+            sm.misc()[MS_ACTIVE] = act;
         }
         __syncthreads();
-        if (!sm.misc[MS_ACTIVE]) break;
+        if (!sm.misc()[MS_ACTIVE]) break;
         cx.passes = p + 1;
         for (int g0 = b_first; g0 <= b_last; g0 += HGRP) {
             const int g1 = min(b_last + 1, g0 + HGRP);
@@ -864,7 +913,7 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
             for_range_keys(a, sm, cx, [&](int c, int, int, uint64_t K, bool ok) {
                 if (!ok) return;
                 const int b = c / a.LH;
-                if (b < g0 || b >= g1 || (sm.fl[b] & SF_DONE) || ((K ^ sm.pk[b]) & sm.pm[b]) != 0ull) return;
+                if (b < g0 || b >= g1 || (sm.fl()[b] & SF_DONE) || ((K ^ sm.pk()[b]) & sm.pm()[b]) != 0ull) return;
                 atomicAdd(&hist[(b - g0) * NBINS + key_digit((uint32_t)(K >> 32), (uint32_t)K, p)], 1u);
             });
             __syncthreads();
@@ -875,9 +924,9 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
             }
             __syncthreads();
         }
-        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return false;
+        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return false;
         for (int b = 0; b < a.B; b++)
-            if (!(sm.fl[b] & SF_DONE)) scan_digit(a, sm, b, p);
+            if (!(sm.fl()[b] & SF_DONE)) scan_digit(a, sm, b, p);
     }
     // keep masks (half-warp ballots), kept counts and the largest kept key of
     // each sequence (the reported threshold is that key + 1: a radix bucket
@@ -886,10 +935,10 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
     unsigned long long km = 0ull;
     for_range_keys(a, sm, cx, [&](int c, int pidx, int r, uint64_t K, bool ok) {
         const int b = c >= 0 ? c / a.LH : 0;
-        const bool keep = ok && K < sm.kap[b];
+        const bool keep = ok && K < sm.kap()[b];
         if (keep) {
             if (b != kb) {
-                if (kb >= 0) atomicMax(sm.kmx + kb, km);
+                if (kb >= 0) atomicMax(sm.kmx() + kb, km);
                 kb = b;
                 km = K;
             } else if (K > km) {
@@ -900,13 +949,13 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
         if (r == 0 && c >= 0) {
             const uint32_t m16 = (ball >> (lane & 16)) & 0xFFFFu;
             a.keep_mask[(int64_t)c * a.max_pages + pidx] = (uint16_t)m16;
-            if (m16) atomicAdd(cx.head_kept + c, (uint32_t)__popc(m16));
+            if (m16) atomicAdd(head_kept_of(a, cx) + c, (uint32_t)__popc(m16));
         }
     });
-    if (kb >= 0) atomicMax(sm.kmx + kb, km);
+    if (kb >= 0) atomicMax(sm.kmx() + kb, km);
     __syncthreads();
-    if (tid < a.B && sm.kmx[tid]) atomicMax(kmax_of(cx, tid), sm.kmx[tid]);
-    if (blockIdx.x == 0 && tid < a.B && (sm.fl[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap[tid];
+    if (tid < a.B && sm.kmx()[tid]) atomicMax(kmax_of(a, cx, tid), sm.kmx()[tid]);
+    if (blockIdx.x == 0 && tid < a.B && (sm.fl()[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap()[tid];
     __syncthreads();
     return true;
 }
@@ -928,14 +977,14 @@ template <class M, int D, int G>
 __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int64_t pfx, int jf, int jl,
                              uint32_t flag, bool cands) {
     using LY = StepLayout<M, D, G>;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nct = gridDim.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = c / a.LH;
     const int cl = c - b * a.LH;
-    int32_t *clist = reinterpret_cast<int32_t *>(sm.big + T_CL);
+    int32_t *clist = reinterpret_cast<int32_t *>(sm.big() + T_CL);
     int ncl = 0;
     if (cands) {
         if (warp == 0) {
-            const int nb = (int)sm.nc[b];
+            const int nb = (int)sm.nc()[b];
             int cnt = 0;
             for (int base = 0; base < nb; base += 32) {
                 const int i = base + lane;
@@ -948,10 +997,10 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
                 if (mine) clist[cnt + __popc(ball & ((1u << lane) - 1u))] = i;
                 cnt += __popc(ball);
             }
-            if (lane == 0) sm.misc[MS_NCL] = cnt;
+            if (lane == 0) sm.misc()[MS_NCL] = cnt;
         }
         __syncthreads();
-        ncl = sm.misc[MS_NCL];
+        ncl = sm.misc()[MS_NCL];
     }
     const bool split = jf != jl;
     const size_t cb = (size_t)b * WIN_CAP;
@@ -963,8 +1012,8 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
         s.me = -INFINITY;
         if (split) {
             for (int j = jf; j <= jl; j++) {
-                if (!(range_lo(j, cx.TP, nct) < range_lo(j + 1, cx.TP, nct))) continue;
-                const float *r = a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, cx.TP, nct)) ? 0 : 1)) * LY::REC;
+                if (!(sm.rlo()[j] < sm.rlo()[j + 1])) continue;
+                const float *r = a.partial + ((int64_t)j * 2 + ((pfx < sm.rlo()[j]) ? 0 : 1)) * LY::REC;
                 s.mk = fmaxf(s.mk, __ldcg(r + G * D + g));
                 s.me = fmaxf(s.me, __ldcg(r + G * D + 2 * G + g));
             }
@@ -991,8 +1040,8 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
         };
         if (split) {
             for (int j = jf; j <= jl; j++) {
-                if (!(range_lo(j, cx.TP, nct) < range_lo(j + 1, cx.TP, nct))) continue;
-                add(a.partial + ((int64_t)j * 2 + ((pfx < range_lo(j, cx.TP, nct)) ? 0 : 1)) * LY::REC);
+                if (!(sm.rlo()[j] < sm.rlo()[j + 1])) continue;
+                add(a.partial + ((int64_t)j * 2 + ((pfx < sm.rlo()[j]) ? 0 : 1)) * LY::REC);
             }
         } else if (flag & 2u) {
             add(a.hrec + (int64_t)c * LY::REC);
@@ -1040,7 +1089,7 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
     using LY = StepLayout<M, D, G>;
     constexpr int GD = G * D;
     constexpr int EPL = (GD + 31) / 32;
-    const int lane = threadIdx.x & 31, nct = gridDim.x;
+    const int lane = threadIdx.x & 31;
     const int b = c / a.LH;
     const int cl = c - b * a.LH;
     // ---- sources ----
@@ -1048,8 +1097,8 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
     if (lane == 0) {
         if (jf != jl) {
             for (int j = jf; j <= jl; j++) {
-                const int64_t lo = range_lo(j, cx.TP, nct);
-                if (!(lo < range_lo(j + 1, cx.TP, nct))) continue;
+                const int64_t lo = sm.rlo()[j];
+                if (!(lo < sm.rlo()[j + 1])) continue;
                 if (nrec < RCAP) w.recp[nrec] = a.partial + ((int64_t)j * 2 + ((pfx < lo) ? 0 : 1)) * LY::REC;
                 nrec++;
             }
@@ -1063,7 +1112,7 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
     int ncl = 0;
     const size_t cb = (size_t)b * WIN_CAP;
     if (cands) {
-        const int nb = (int)sm.nc[b];
+        const int nb = (int)sm.nc()[b];
         for (int base = 0; base < nb; base += 32) {
             const int i = base + lane;
             bool mine = false;
@@ -1089,6 +1138,14 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
     }
     for (int t = lane; t < ncl * G; t += 32) w.cz[t] = __ldcg(a.cz + (cb + w.cidx[t / G]) * G + (t % G));
     for (int i = lane; i < ncl; i += 32) w.cfate[i] = __ldcg(a.cfate + cb + w.cidx[i]);
+    // the first two records' output values, in the same round
+    float v0[EPL], v1[EPL];
+#pragma unroll
+    for (int u = 0; u < EPL; u++) {
+        const int e = lane + 32 * u;
+        v0[u] = (nrec > 0 && e < GD) ? __ldcg(w.recp[0] + e) : 0.0f;
+        v1[u] = (nrec > 1 && e < GD) ? __ldcg(w.recp[1] + e) : 0.0f;
+    }
     __syncwarp();
     // ---- per query row: merged maxima, sums, lse and dropped mass ----
     if (lane < G) {
@@ -1134,21 +1191,21 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
     // ---- outputs: EPL elements per lane, two records' loads in flight at a time ----
     float av[EPL];
 #pragma unroll
-    for (int u = 0; u < EPL; u++) av[u] = 0.0f;
-    for (int k = 0; k < nrec; k += 2) {
-        const bool two = k + 1 < nrec;
-        float v0[EPL], v1[EPL];
+    for (int u = 0; u < EPL; u++) {
+        const int e = lane + 32 * u;
+        const int g = (e < GD ? e : 0) / D;
+        av[u] = (nrec > 0 ? v0[u] * w.fk[g] : 0.0f) + (nrec > 1 ? v1[u] * w.fk[G + g] : 0.0f);
+    }
+    for (int k = 2; k < nrec; k++) {
 #pragma unroll
         for (int u = 0; u < EPL; u++) {
             const int e = lane + 32 * u;
             v0[u] = e < GD ? __ldcg(w.recp[k] + e) : 0.0f;
-            v1[u] = (two && e < GD) ? __ldcg(w.recp[k + 1] + e) : 0.0f;
         }
 #pragma unroll
         for (int u = 0; u < EPL; u++) {
             const int e = lane + 32 * u;
-            const int g = (e < GD ? e : 0) / D;
-            av[u] += v0[u] * w.fk[k * G + g] + (two ? v1[u] * w.fk[(k + 1) * G + g] : 0.0f);
+            av[u] += v0[u] * w.fk[k * G + (e < GD ? e : 0) / D];
         }
     }
     for (int i = 0; i < ncl; i++) {
@@ -1187,11 +1244,11 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
 __device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int n, int nn, int32_t off) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int mp = a.max_pages;
-    int32_t *tbl = reinterpret_cast<int32_t *>(sm.big + T_TBL);
+    int32_t *tbl = reinterpret_cast<int32_t *>(sm.big() + T_TBL);
     int32_t *src_pfx = tbl + mp;
     int32_t *hole_pfx = src_pfx + mp + 1;
     uint16_t *msk = reinterpret_cast<uint16_t *>(hole_pfx + mp + 1);
-    int2 *pairs = reinterpret_cast<int2 *>(sm.big + T_PAIRS);
+    int2 *pairs = reinterpret_cast<int2 *>(sm.big() + T_PAIRS);
     const int W = (n + PAGE - 1) / PAGE, Wn = (nn + PAGE - 1) / PAGE;
     const int64_t cm = (int64_t)c * mp;
     for (int w = tid; w < W; w += NTH) {
@@ -1203,8 +1260,8 @@ __device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
         hole_pfx[w] = __popc(~m & below & 0xFFFFu);
     }
     __syncthreads();
-    scan_words(src_pfx, W, sm.scan);
-    scan_words(hole_pfx, W, sm.scan);
+    scan_words(src_pfx, W, sm.scan());
+    scan_words(hole_pfx, W, sm.scan());
     const int moves = min(hole_pfx[W], src_pfx[W]);
     const int chunks = a.row_bytes / 16;
     for (int r0 = 0; r0 < moves; r0 += CMP_PAIRS) {
@@ -1270,10 +1327,12 @@ __device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
 
 // Warp-level hole-fill compaction of head c (same result as compact_head)
 // for heads with at most HCAP evicted entries; returns false otherwise and
-// the block-wide compaction runs.  Keep words are read WPL per lane per round
-// (loads issued together); holes (non-kept slots below nn) and sources (kept
-// slots at or above nn) are listed in ascending order with warp scans; rows
-// move four pairs at a time with every load issued before the stores.
+// the block-wide compaction runs.  Keep words and block-table entries are
+// read WPL per lane per round (all loads issued together); holes (non-kept
+// slots below nn) and sources (kept slots at or above nn) are listed in
+// ascending order with warp scans, already as physical rows, and freed pages
+// are pushed from the same registers; rows then move four pairs at a time
+// with every load issued before the stores.
 __device__ bool compact_warp(const StepArgs &a, const Ctx &cx, WarpScr &w, int c, int n, int nn, int32_t off) {
     if (n - nn > HCAP) return false;
     constexpr int WPL = 8;
@@ -1283,10 +1342,12 @@ __device__ bool compact_warp(const StepArgs &a, const Ctx &cx, WarpScr &w, int c
     int nh = 0, ns = 0;
     for (int w0 = 0; w0 < W; w0 += 32 * WPL) {
         uint32_t m[WPL];
+        int32_t pg[WPL];
 #pragma unroll
         for (int u = 0; u < WPL; u++) {
             const int wd = w0 + 32 * u + lane;
             m[u] = wd < W ? ((uint32_t)__ldcg(a.keep_mask + cm + wd) & below_bits(wd, n)) : 0u;
+            pg[u] = wd < W ? __ldcg(a.block_table + cm + wd) : 0;
         }
 #pragma unroll
         for (int u = 0; u < WPL; u++) {
@@ -1310,14 +1371,20 @@ __device__ bool compact_warp(const StepArgs &a, const Ctx &cx, WarpScr &w, int c
             while (hb) {
                 const int bit = __ffs(hb) - 1;
                 hb &= hb - 1;
-                if (hx < HCAP) w.holes[hx] = wd * PAGE + bit;
+                if (hx < HCAP) w.holes[hx] = pg[u] * PAGE + bit;
                 hx++;
             }
             while (sb) {
                 const int bit = __ffs(sb) - 1;
                 sb &= sb - 1;
-                if (sx < HCAP) w.srcs[sx] = wd * PAGE + bit;
+                if (sx < HCAP) w.srcs[sx] = pg[u] * PAGE + bit;
                 sx++;
+            }
+            // pages past ceil(nn/16): pushed at this head's offset in the stack
+            // (the moves below use the rows listed above, not the table)
+            if (wd >= Wn && wd < W) {
+                a.free_stack[cx.top0 + off + (wd - Wn)] = pg[u];
+                a.block_table[cm + wd] = -1;
             }
             nh += htot;
             ns += stot;
@@ -1325,13 +1392,6 @@ __device__ bool compact_warp(const StepArgs &a, const Ctx &cx, WarpScr &w, int c
     }
     __syncwarp();
     const int moves = min(min(nh, ns), HCAP);
-    // physical rows of the pairs (table entries read before any is cleared)
-    for (int p = lane; p < moves; p += 32) {
-        const int hs = w.holes[p], ss = w.srcs[p];
-        w.holes[p] = __ldcg(a.block_table + cm + hs / PAGE) * PAGE + hs % PAGE;
-        w.srcs[p] = __ldcg(a.block_table + cm + ss / PAGE) * PAGE + ss % PAGE;
-    }
-    __syncwarp();
     const int chunks = a.row_bytes / 16;
     for (int p0 = 0; p0 < moves; p0 += 4) {
         uint4 v[4][2];
@@ -1377,22 +1437,16 @@ __device__ bool compact_warp(const StepArgs &a, const Ctx &cx, WarpScr &w, int c
         }
     }
     __syncwarp();
-    // freed pages, ascending table index, at this head's offset in the stack
-    for (int pi = Wn + lane; pi < W; pi += 32) {
-        a.free_stack[cx.top0 + off + (pi - Wn)] = __ldcg(a.block_table + cm + pi);
-        a.block_table[cm + pi] = -1;
-    }
-    __syncwarp();
     return true;
 }
 
 // Bounded wait until every CTA has finished its compactions (pushes).
 __device__ bool wait_pushes(const StepArgs &a, const Ctx &cx) {
     const uint32_t target = gridDim.x;
-    if (ld_acquire_gpu(cx.arrive) >= target) return true;
+    if (ld_acquire_gpu(arrive_of(a, cx)) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
-    while (ld_acquire_gpu(cx.arrive) < target) {
+    while (ld_acquire_gpu(arrive_of(a, cx)) < target) {
         if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
             record_timeout(a.status, 0x200);
             return false;
@@ -1431,7 +1485,7 @@ __device__ void append_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int 
             row = (int64_t)__ldcg(a.block_table + (int64_t)c * a.max_pages + pidx) * PAGE + (k % PAGE);
         }
         if (row >= 0) {
-            a.pos_pool[row] = sm.t[c / a.LH];
+            a.pos_pool[row] = sm.t()[c / a.LH];
             a.lb_pool[row] = __ldg(a.lb_new + c);
         }
         a.len[c] = k + 1;
@@ -1454,7 +1508,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nct = gridDim.x;
     const int C = a.C;
     const int hc0 = (int)((int64_t)blockIdx.x * C / nct), hc1 = (int)((int64_t)(blockIdx.x + 1) * C / nct);
-    int32_t *st_npre = reinterpret_cast<int32_t *>(sm.big + T_STASH);
+    int32_t *st_npre = reinterpret_cast<int32_t *>(sm.big() + T_STASH);
     int32_t *st_nnew = st_npre + NTH, *st_pfx = st_nnew + NTH, *st_plan = st_pfx + NTH, *st_pop = st_plan + NTH;
     // exact-select histograms are no longer read by anyone: clear them
     if (cx.passes > 0) {
@@ -1469,13 +1523,13 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
         uint32_t v[3] = {0u, 0u, 0u};
         if (c < C) {
             np = __ldcg(a.npre + c);
-            nn = cx.evict ? (int32_t)__ldcg(cx.head_kept + c) : np;
+            nn = cx.evict ? (int32_t)__ldcg(head_kept_of(a, cx) + c) : np;
             v[0] = (uint32_t)((np + PAGE - 1) / PAGE);
             v[1] = cx.evict ? v[0] - (uint32_t)((nn + PAGE - 1) / PAGE) : 0u;
             v[2] = (nn % PAGE == 0) ? 1u : 0u;
         }
         uint32_t ex[3], tot[3];
-        block_scan_n<3>(v, ex, tot, sm.scan);
+        block_scan_n<3>(v, ex, tot, sm.scan());
         if (c >= hc0 && c < hc1) {
             const int k = c - hc0;
             st_npre[k] = np;
@@ -1495,12 +1549,12 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
             a.plan[hc0 + k] = st_plan[k];
         }
     }
-    if (cx.exact && blockIdx.x == 0 && tid < a.B && !(sm.fl[tid] & SF_TRIVIAL)) {
+    if (cx.exact && blockIdx.x == 0 && tid < a.B && !(sm.fl()[tid] & SF_TRIVIAL)) {
         // thresholds of the exact selection: largest kept key + 1 (every CTA's
         // final pass is complete), and the window for the next call
-        const uint64_t kap = __ldcg(kmax_of(cx, tid)) + 1ull;
+        const uint64_t kap = __ldcg(kmax_of(a, cx, tid)) + 1ull;
         a.kappa[tid] = kap;
-        window_next(a.win + (size_t)tid * 4, kap, (int)sm.wres[tid], sm.nc[tid]);
+        window_next(a.win + (size_t)tid * 4, kap, (int)sm.wres()[tid], sm.nc()[tid]);
     }
     if (blockIdx.x == nct - 1 && tid == 0) {
         if (cx.evict) {
@@ -1510,26 +1564,57 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
         const int nt = cx.top0 + (int)pushes - (int)pops;
         *a.free_top = nt < 0 ? 0 : nt;
     }
-    // merges, keep-bit patches and compaction: one warp per head; heads too
-    // large for a warp are done block-wide afterwards, one at a time
+    // merges (keep-bit patches included) and compactions are tasks that
+    // warps take from a queue in shared memory; a head's compaction is a task
+    // of its own unless the head holds candidates (then it follows the merge
+    // that patches its keep bits).  Heads too large for a warp are done
+    // block-wide afterwards, one at a time.
+    const int nh = hc1 - hc0;
     int32_t *st_heavy = st_pop + NTH;
-    WarpScr &wsc = *reinterpret_cast<WarpScr *>(sm.big + T_WARP + warp * WARP_SCR);
-    for (int k = warp; k < hc1 - hc0; k += NWARP) {
+    int32_t *tasks = reinterpret_cast<int32_t *>(sm.big() + T_CL);  // [2 * NTH]
+    WarpScr &wsc = *reinterpret_cast<WarpScr *>(sm.big() + T_WARP + warp * WARP_SCR);
+    if (tid == 0) {
+        sm.misc()[MS_QN] = 0;
+        sm.misc()[MS_QH] = 0;
+    }
+    __syncthreads();
+    for (int k = tid; k < nh; k += NTH) {
         const int c = hc0 + k;
         const int np = st_npre[k], nn = st_nnew[k];
         const int pages = (np + PAGE - 1) / PAGE;
-        int heavy = 0;
+        st_heavy[k] = 0;
+        bool merge = false, cands = false;
         if (pages > 0) {
             const int64_t pfx = st_pfx[k];
-            const int jf = owner_of(pfx, cx.TP, nct), jl = owner_of(pfx + pages - 1, cx.TP, nct);
-            const uint32_t flag = __ldcg(cx.head_flag + c);
-            const bool cands = spec && (flag & 1u);
-            if ((jf != jl || (flag & 2u) || cands) &&
-                !combine_warp<M, D, G>(a, sm, cx, wsc, c, pfx, jf, jl, flag, cands))
-                heavy = 3;  // merge, then compaction (after the keep-bit patches), block-wide
+            const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
+            cands = spec && (flag & 1u);
+            merge = owner_rlo(sm.rlo(), nct, pfx) != owner_rlo(sm.rlo(), nct, pfx + pages - 1) || (flag & 2u) || cands;
         }
-        if (!(heavy & 2) && cx.evict && nn < np && !compact_warp(a, cx, wsc, c, np, nn, st_plan[k])) heavy |= 2;
-        if (lane == 0) st_heavy[k] = heavy;
+        const bool comp = cx.evict && nn < np;
+        if (merge) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 1 | ((cands && comp) ? 2 : 0);
+        if (comp && !(cands && merge)) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 2;
+    }
+    __syncthreads();
+    const int ntask = sm.misc()[MS_QN];
+    for (;;) {
+        int t = 0;
+        if (lane == 0) t = atomicAdd(&sm.misc()[MS_QH], 1);
+        t = __shfl_sync(0xFFFFFFFFu, t, 0);
+        if (t >= ntask) break;
+        const int task = tasks[t], k = task >> 2, c = hc0 + k;
+        const int np = st_npre[k], nn = st_nnew[k];
+        bool comp = (task & 2) != 0;
+        if (task & 1) {
+            const int pages = (np + PAGE - 1) / PAGE;
+            const int64_t pfx = st_pfx[k];
+            const int jf = owner_rlo(sm.rlo(), nct, pfx), jl = owner_rlo(sm.rlo(), nct, pfx + pages - 1);
+            const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
+            if (!combine_warp<M, D, G>(a, sm, cx, wsc, c, pfx, jf, jl, flag, spec && (flag & 1u))) {
+                if (lane == 0) atomicOr(st_heavy + k, comp ? 3 : 1);
+                comp = false;
+            }
+        }
+        if (comp && !compact_warp(a, cx, wsc, c, np, nn, st_plan[k]) && lane == 0) atomicOr(st_heavy + k, 2);
     }
     __syncthreads();
     for (int k = 0; k < hc1 - hc0; k++) {
@@ -1540,8 +1625,8 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
         if (heavy & 1) {
             const int pages = (np + PAGE - 1) / PAGE;
             const int64_t pfx = st_pfx[k];
-            const int jf = owner_of(pfx, cx.TP, nct), jl = owner_of(pfx + pages - 1, cx.TP, nct);
-            const uint32_t flag = __ldcg(cx.head_flag + c);
+            const int jf = owner_rlo(sm.rlo(), nct, pfx), jl = owner_rlo(sm.rlo(), nct, pfx + pages - 1);
+            const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
             combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, spec && (flag & 1u));
         }
         if ((heavy & 2) && cx.evict && nn < np) compact_head(a, sm, cx, c, np, nn, st_plan[k]);
@@ -1549,7 +1634,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        atomicAdd(cx.arrive, 1u);
+        atomicAdd(arrive_of(a, cx), 1u);
     }
     for (int k = warp; k < hc1 - hc0; k += NWARP) append_head(a, sm, cx, hc0 + k, st_nnew[k], st_pop[k], pushes);
 }
@@ -1560,55 +1645,31 @@ __global__ void __launch_bounds__(NTH, 1)
     step_kernel(StepArgs a, const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv) {
     using LY = StepLayout<M, D, G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    unsigned char *smem = smem_raw + ((M::STAGE_ALIGN - (smem_u32(smem_raw) & (M::STAGE_ALIGN - 1))) &
-                                      (M::STAGE_ALIGN - 1));
+    unsigned char *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Sm sm;
-    sm.bars = reinterpret_cast<uint64_t *>(smem + LY::OFF_BAR);
-    {
-        unsigned char *p = smem + LY::OFF_SEQ;
-        sm.lo = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
-        sm.hi = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
-        sm.kap = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
-        sm.pk = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
-        sm.pm = reinterpret_cast<uint64_t *>(p); p += MAXB * 8;
-        sm.kmx = reinterpret_cast<unsigned long long *>(p); p += MAXB * 8;
-        sm.m = reinterpret_cast<int64_t *>(p); p += MAXB * 8;
-        sm.t = reinterpret_cast<int32_t *>(p); p += MAXB * 4;
-        sm.n = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
-        sm.rank = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
-        sm.fl = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
-        sm.above = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
-        sm.nc = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
-        sm.off = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
-        sm.wres = reinterpret_cast<uint32_t *>(p); p += MAXB * 4;
-    }
-    sm.spare = nullptr;
-    sm.scan = reinterpret_cast<uint32_t *>(smem + LY::OFF_SCAN);
-    sm.misc = reinterpret_cast<int *>(smem + LY::OFF_MISC);
-    sm.misc64 = reinterpret_cast<int64_t *>(smem + LY::OFF_MISC + 64 * 4);
-    sm.big = smem + LY::OFF_BIG;
+    sm.base = smem;
 
     Ctx cx;
     prologue<M, D, G>(a, sm, cx, &tmk, &tmv);
     bool spec = false;
-    if (cx.evict && !sm.misc[MS_RADIX]) {
+    if (cx.evict && !sm.misc()[MS_RADIX]) {
         attn_pass<M, D, G, true>(a, sm, cx, &tmk, &tmv);
-        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return;
+        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
         if (resolve(a, sm, cx)) {
-            if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return;
+            if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
             spec = true;
             if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(a.status + 2, 1);
         } else {
             // a window missed: drop the speculative counts, select exactly
             for (size_t i = (size_t)blockIdx.x * NTH + threadIdx.x; i < 2 * (size_t)a.C; i += (size_t)gridDim.x * NTH)
-                cx.head_kept[i] = 0u;  // head_kept and head_flag are adjacent
+                head_kept_of(a, cx)[i] = 0u;  // head_kept and head_flag are adjacent
         }
     }
     if (!spec) {
         if (cx.evict && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(a.status + 3, 1);
         if (cx.evict && !exact_select(a, sm, cx)) return;
         attn_pass<M, D, G, false>(a, sm, cx, &tmk, &tmv);
-        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc[MS_BAR])) return;
+        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
     }
     tail<M, D, G>(a, sm, cx, spec);
     // exit ticket: the last CTA resets the barrier counter and flips the half
