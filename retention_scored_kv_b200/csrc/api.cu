@@ -457,6 +457,7 @@ RKV_API int rkv_decode_step(const rkv_cache_t *cache, const int32_t *t, const in
     a.cv = at<unsigned char>(ws, L.cv);
     a.ghist = at<uint32_t>(ws, L.ghist);
     a.partial = at<float>(ws, L.partial);
+    a.head_cnt = at<uint32_t>(ws, L.head_cnt);
     a.hrec = at<float>(ws, L.hrec);
     a.npre = at<int32_t>(ws, L.npre);
     a.pfx = at<int32_t>(ws, L.pfx);

@@ -27,7 +27,11 @@ constexpr int ATTN_THREADS = (NCW + NPW) * 32;
 constexpr int LAUNCH_REGS = 168;
 constexpr int PRODUCER_REGS = 56;
 constexpr int CONSUMER_REGS = 224;
+#ifdef RKV_NO_REG_SPLIT
+constexpr bool REG_SPLIT = false;
+#else
 constexpr bool REG_SPLIT = (NCW % 4 == 0) && (NPW % 4 == 0);
+#endif
 static_assert(!REG_SPLIT || NPW * 32 * PRODUCER_REGS + NCW * 32 * CONSUMER_REGS <= ATTN_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
 

@@ -170,6 +170,7 @@ struct StepArgs {
     unsigned char *cv;
     uint32_t *ghist;
     float *partial;
+    uint32_t *head_cnt;        // [C] cross-CTA merge tickets (self-resetting)
     float *hrec;
     int32_t *npre;
     int32_t *pfx;

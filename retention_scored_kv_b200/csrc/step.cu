@@ -32,10 +32,10 @@
 //    grid barriers), writes the keep masks and kept counts, and the attention
 //    pass then reads the masks.
 //  * Tail.  Heads are dealt to CTAs in contiguous chunks: heads split across
-//    CTAs or holding candidates are merged, candidate keep bits patched, each
-//    head compacted (hole-fill, freed pages pushed at the plan's offsets) and
-//    the new rows appended; a pop waits (bounded) only for a page pushed in
-//    this call.
+//    CTAs or holding candidates are merged (the kept candidates' keep bits
+//    were set when their fates were found), each head compacted (hole-fill,
+//    freed pages pushed at the plan's offsets) and the new rows appended; a
+//    pop waits (bounded) only for a page pushed in this call.
 // Selection, keep masks, block tables, lengths and the free stack come out
 // identical to the separate calls; attention outputs agree within rounding.
 #include <cuda.h>
@@ -731,7 +731,13 @@ __device__ bool resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
                 a.cfate[(size_t)b * WIN_CAP + j] = kept ? 1 : 0;
                 if (kept) {
                     const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
-                    atomicAdd(head_kept_of(a, cx) + (int64_t)b * a.LH + cl, 1u);
+                    const int64_t c = (int64_t)b * a.LH + cl;
+                    atomicAdd(head_kept_of(a, cx) + c, 1u);
+                    // its keep bit (several candidates may share a mask word)
+                    const int slot = __ldcg(a.cslot + (size_t)b * WIN_CAP + j);
+                    const uintptr_t addr = reinterpret_cast<uintptr_t>(a.keep_mask + c * a.max_pages + slot / PAGE);
+                    atomicOr(reinterpret_cast<unsigned int *>(addr & ~(uintptr_t)3),
+                             (1u << (slot % PAGE)) << ((addr & 2) ? 16 : 0));
                 }
                 if (less == r - 1) {
                     const uint64_t kap = K + 1ull;
@@ -1064,16 +1070,6 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
             if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
         }
     }
-    if (cands && tid == 0) {
-        for (int i = 0; i < ncl; i++) {
-            const size_t idx = cb + clist[i];
-            if (__ldcg(a.cfate + idx)) {
-                const int slot = __ldcg(a.cslot + idx);
-                uint16_t *wd = a.keep_mask + (int64_t)c * a.max_pages + slot / PAGE;
-                *wd = (uint16_t)(*wd | (1u << (slot % PAGE)));
-            }
-        }
-    }
     __syncthreads();
 }
 
@@ -1224,15 +1220,6 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
             const float lk = w.lk[e / D];
             a.out[(int64_t)c * GD + e] = lk > 0.0f ? av[u] / lk : 0.0f;
         }
-    }
-    // ---- keep bits of the kept candidates (several may share a mask word) ----
-    for (int i = lane; i < ncl; i += 32) {
-        if (!w.cfate[i]) continue;
-        const int slot = __ldcg(a.cslot + cb + w.cidx[i]);
-        const int64_t idx = (int64_t)c * a.max_pages + slot / PAGE;
-        const uintptr_t addr = reinterpret_cast<uintptr_t>(a.keep_mask + idx);
-        unsigned int *word = reinterpret_cast<unsigned int *>(addr & ~(uintptr_t)3);
-        atomicOr(word, (1u << (slot % PAGE)) << ((addr & 2) ? 16 : 0));
     }
     __syncwarp();
     return true;
@@ -1564,11 +1551,10 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
         const int nt = cx.top0 + (int)pushes - (int)pops;
         *a.free_top = nt < 0 ? 0 : nt;
     }
-    // merges (keep-bit patches included) and compactions are tasks that
-    // warps take from a queue in shared memory; a head's compaction is a task
-    // of its own unless the head holds candidates (then it follows the merge
-    // that patches its keep bits).  Heads too large for a warp are done
-    // block-wide afterwards, one at a time.
+    // merges and compactions are independent tasks (kept candidates' keep
+    // bits were set by the resolve step) that warps take from a queue in
+    // shared memory.  Heads too large for a warp are done block-wide
+    // afterwards, one at a time.
     const int nh = hc1 - hc0;
     int32_t *st_heavy = st_pop + NTH;
     int32_t *tasks = reinterpret_cast<int32_t *>(sm.big() + T_CL);  // [2 * NTH]
@@ -1591,8 +1577,8 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
             merge = owner_rlo(sm.rlo(), nct, pfx) != owner_rlo(sm.rlo(), nct, pfx + pages - 1) || (flag & 2u) || cands;
         }
         const bool comp = cx.evict && nn < np;
-        if (merge) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 1 | ((cands && comp) ? 2 : 0);
-        if (comp && !(cands && merge)) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 2;
+        if (merge) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 1;
+        if (comp) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 2;
     }
     __syncthreads();
     const int ntask = sm.misc()[MS_QN];
@@ -1603,16 +1589,14 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
         if (t >= ntask) break;
         const int task = tasks[t], k = task >> 2, c = hc0 + k;
         const int np = st_npre[k], nn = st_nnew[k];
-        bool comp = (task & 2) != 0;
+        const bool comp = (task & 2) != 0;
         if (task & 1) {
             const int pages = (np + PAGE - 1) / PAGE;
             const int64_t pfx = st_pfx[k];
             const int jf = owner_rlo(sm.rlo(), nct, pfx), jl = owner_rlo(sm.rlo(), nct, pfx + pages - 1);
             const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
-            if (!combine_warp<M, D, G>(a, sm, cx, wsc, c, pfx, jf, jl, flag, spec && (flag & 1u))) {
-                if (lane == 0) atomicOr(st_heavy + k, comp ? 3 : 1);
-                comp = false;
-            }
+            if (!combine_warp<M, D, G>(a, sm, cx, wsc, c, pfx, jf, jl, flag, spec && (flag & 1u)) && lane == 0)
+                atomicOr(st_heavy + k, 1);
         }
         if (comp && !compact_warp(a, cx, wsc, c, np, nn, st_plan[k]) && lane == 0) atomicOr(st_heavy + k, 2);
     }
