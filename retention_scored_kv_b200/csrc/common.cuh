@@ -14,6 +14,15 @@ constexpr int NPASS = 6;           // radix digits of the 64-bit key: 11,11,10 |
 constexpr int NBINS = 2048;        // bins of the widest digit
 constexpr int MAX_ATTN_CTAS = 512; // upper bound of the persistent attention grid
 constexpr int WIN_CAP = 1024;      // threshold-window candidates per sequence
+// A window that resolved its call is halved above WIN_HI candidates and
+// doubled below WIN_LO.
+#ifndef RKV_WIN_LO
+#define RKV_WIN_LO 16
+#endif
+#ifndef RKV_WIN_HI
+#define RKV_WIN_HI 128
+#endif
+constexpr uint32_t WIN_LO = RKV_WIN_LO, WIN_HI = RKV_WIN_HI;
 constexpr uint32_t KEY_INVALID = 0xFFFFFFFFu;  // hi word no valid score maps to (NaN space)
 
 // ---------------------------------------------------------------- keys ----
@@ -98,7 +107,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, in
 // the score-key (high word) range whose keys are ranked individually next
 // call, w[3] its half width.  Centred on this call's threshold score key and
 // resized by how this call went: wres 1 resolved in the window (wn
-// candidates: shrink above WIN_CAP/2, grow below 64), 2 missed (grow 4x),
+// candidates: shrink above WIN_HI, grow below WIN_LO), 2 missed (grow 4x),
 // 3 too many candidates (shrink 4x), 0 no window was used.  Nothing changes
 // when nothing or everything was kept (kappa 0 or ~0).
 __device__ __forceinline__ void window_next(uint32_t *w, uint64_t kappa, int wres, uint32_t wn) {
@@ -107,8 +116,8 @@ __device__ __forceinline__ void window_next(uint32_t *w, uint64_t kappa, int wre
     uint32_t hw = w[3];
     if (hw == 0u) hw = 1u << 14;
     if (wres == 1) {
-        if (wn > WIN_CAP / 2) hw = hw > 1u ? hw >> 1 : 1u;
-        else if (wn < 64u) hw = hw < (1u << 28) ? hw << 1 : hw;
+        if (wn > WIN_HI) hw = hw > 1u ? hw >> 1 : 1u;
+        else if (wn < WIN_LO) hw = hw < (1u << 28) ? hw << 1 : hw;
     } else if (wres == 2) {
         hw = hw < (1u << 26) ? hw << 2 : (1u << 28);
     } else if (wres == 3) {

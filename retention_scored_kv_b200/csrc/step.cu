@@ -96,12 +96,21 @@ constexpr size_t RESOLVE_BYTES = (size_t)WIN_CAP * 8;
 // for every instance): per-sequence state, scan scratch, flags, the CTA range
 // starts and the pipeline barriers; the big region follows at S_BIG.
 constexpr int MAX_NBAR = 2 * NCW * 8 + 2 * QR;
+// Local resolve: every CTA ranks all candidates itself when there are at
+// most RES_CAP of them and at most CADD_CAP heads (their kept-candidate
+// counts are tallied in shared memory), so no second grid barrier is needed.
+#ifndef RKV_RES_CAP
+#define RKV_RES_CAP 1024
+#endif
+constexpr int RES_CAP = RKV_RES_CAP;
+constexpr int CADD_CAP = 8192;
 constexpr int S_LO = 0, S_HI = S_LO + MAXB * 8, S_KAP = S_HI + MAXB * 8, S_PK = S_KAP + MAXB * 8,
               S_PM = S_PK + MAXB * 8, S_KMX = S_PM + MAXB * 8, S_M = S_KMX + MAXB * 8, S_T = S_M + MAXB * 8,
               S_N = S_T + MAXB * 4, S_RANK = S_N + MAXB * 4, S_FL = S_RANK + MAXB * 4, S_ABOVE = S_FL + MAXB * 4,
               S_NC = S_ABOVE + MAXB * 4, S_OFF = S_NC + MAXB * 4, S_WRES = S_OFF + MAXB * 4,
               S_SCAN = S_WRES + MAXB * 4, S_MISC = S_SCAN + 4 * 36 * 4, S_MISC64 = S_MISC + 64 * 4,
-              S_RLO = S_MISC64 + 8 * 8, S_BAR = (S_RLO + (MAX_ATTN_CTAS + 1) * 4 + 15) / 16 * 16,
+              S_RLO = S_MISC64 + 8 * 8, S_FATE = S_RLO + (MAX_ATTN_CTAS + 1) * 4,
+              S_BAR = (S_FATE + (RES_CAP > 0 ? RES_CAP : 1) + 15) / 16 * 16,
               S_BIG = (S_BAR + MAX_NBAR * 8 + 1023) / 1024 * 1024;
 
 // Shared memory: the fixed part (pipeline barriers, per-sequence state, scan
@@ -161,6 +170,7 @@ struct Sm {
     __device__ __forceinline__ int *misc() const { return at<int>(S_MISC); }
     __device__ __forceinline__ int64_t *misc64() const { return at<int64_t>(S_MISC64); }
     __device__ __forceinline__ int32_t *rlo() const { return at<int32_t>(S_RLO); }
+    __device__ __forceinline__ int8_t *fate() const { return at<int8_t>(S_FATE); }
     __device__ __forceinline__ unsigned char *big() const { return base + S_BIG; }
 };
 
@@ -678,11 +688,17 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
 // --------------------------------------------------------------- resolve ----
 // After the speculative pass: per sequence, is the M-th key inside the
 // window with every candidate stored?  If so every candidate's fate is its
-// rank among the candidates (keys are distinct), counted by the CTA that owns
-// its slice; kept candidates are added to their head's kept count and the
-// M-th key gives the exclusive threshold.  Returns false if any sequence
+// rank among the candidates (keys are distinct) and the M-th key gives the
+// exclusive threshold.  Few candidates (RES_MODE_LOCAL): every CTA ranks all
+// of them in shared memory, tallies kept candidates per head (sm.big() +
+// T_WARP + RES_CAP*8, read by the tail's scan), keeps the fates in sm.fate()
+// (indexed by the sequence's candidate offset + index) and sets the keep bits
+// of its own heads; nothing crosses CTAs, so no barrier follows.  Otherwise
+// (RES_MODE_GRID) each CTA ranks a slice, writes fates and kept counts to
+// global memory, and a grid barrier must follow.  RES_MISS: some sequence
 // missed (the exact path runs instead).
-__device__ bool resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
+enum { RES_MISS = 0, RES_MODE_LOCAL = 1, RES_MODE_GRID = 2 };
+__device__ int resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
     const int tid = threadIdx.x, nct = gridDim.x;
     if (tid < a.B) {
         const int b = tid;
@@ -699,7 +715,7 @@ __device__ bool resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
         }
     }
     __syncthreads();
-    if (sm.misc()[MS_MISS]) return false;
+    if (sm.misc()[MS_MISS]) return RES_MISS;
     if (tid == 0) {
         uint32_t o = 0;
         for (int b = 0; b < a.B; b++) {
@@ -710,6 +726,48 @@ __device__ bool resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
     }
     __syncthreads();
     const int64_t total = sm.misc()[MS_TOTAL];
+    if (total <= RES_CAP && a.C <= CADD_CAP) {
+        uint64_t *keys = reinterpret_cast<uint64_t *>(sm.big() + T_WARP);
+        uint32_t *cadd = reinterpret_cast<uint32_t *>(sm.big() + T_WARP + RES_CAP * 8);
+        const int hc0 = (int)((int64_t)blockIdx.x * a.C / nct), hc1 = (int)((int64_t)(blockIdx.x + 1) * a.C / nct);
+        for (int i = tid; i < a.C; i += NTH) cadd[i] = 0u;
+        for (int g = tid; g < total; g += NTH) {
+            int b = 0;
+            while (b + 1 < a.B && (int64_t)sm.off()[b + 1] <= g) b++;
+            keys[g] = __ldcg(a.ckey + (size_t)b * WIN_CAP + (g - sm.off()[b]));
+        }
+        __syncthreads();
+        for (int g = tid; g < total; g += NTH) {
+            int b = 0;
+            while (b + 1 < a.B && (int64_t)sm.off()[b + 1] <= g) b++;
+            const int ob = (int)sm.off()[b], nb = (int)sm.nc()[b];
+            const uint64_t K = keys[g];
+            uint32_t less = 0;
+            for (int i = 0; i < nb; i++) less += keys[ob + i] < K ? 1u : 0u;
+            const uint32_t r = (uint32_t)(sm.m()[b] - (int64_t)sm.above()[b]);
+            const bool kept = less < r;
+            sm.fate()[g] = kept ? 1 : 0;
+            if (kept) {
+                const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
+                const int c = b * a.LH + cl;
+                atomicAdd(cadd + c, 1u);
+                if (c >= hc0 && c < hc1) {
+                    const int slot = __ldcg(a.cslot + (size_t)b * WIN_CAP + (g - ob));
+                    const uintptr_t addr = reinterpret_cast<uintptr_t>(a.keep_mask + (int64_t)c * a.max_pages + slot / PAGE);
+                    atomicOr(reinterpret_cast<unsigned int *>(addr & ~(uintptr_t)3),
+                             (1u << (slot % PAGE)) << ((addr & 2) ? 16 : 0));
+                }
+            }
+            if (blockIdx.x == 0 && less == r - 1) {
+                const uint64_t kap = K + 1ull;
+                a.kappa[b] = kap;
+                window_next(a.win + (size_t)b * 4, kap, 1, (uint32_t)nb);
+            }
+        }
+        if (blockIdx.x == 0 && tid < a.B && (sm.fl()[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap()[tid];
+        __syncthreads();
+        return RES_MODE_LOCAL;
+    }
     const int64_t s0 = (int64_t)blockIdx.x * total / nct, s1 = (int64_t)(blockIdx.x + 1) * total / nct;
     uint64_t *keys = reinterpret_cast<uint64_t *>(sm.big());
     for (int b = 0; b < a.B; b++) {
@@ -749,7 +807,7 @@ __device__ bool resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
         __syncthreads();
     }
     if (blockIdx.x == 0 && tid < a.B && (sm.fl()[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap()[tid];
-    return true;
+    return RES_MODE_GRID;
 }
 
 // --------------------------------------------------------- exact select ----
@@ -976,12 +1034,18 @@ __device__ __forceinline__ float row_elt(const unsigned char *row, int d) {
     }
 }
 
+// Fate (1 = kept) of candidate j of sequence b: from shared memory after a
+// local resolve, else from the workspace.
+__device__ __forceinline__ int cand_fate(const StepArgs &a, const Sm &sm, bool local, int b, int j) {
+    return local ? (int)sm.fate()[sm.off()[b] + j] : __ldcg(a.cfate + (size_t)b * WIN_CAP + j);
+}
+
 // Merge of a head's partial states: the records of the CTAs its pages span
 // (or the record of the one CTA that held candidates of it) and its
 // candidates, each kept (logit z, weight 1, value v) or evicted (logit z).
 template <class M, int D, int G>
 __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int64_t pfx, int jf, int jl,
-                             uint32_t flag, bool cands) {
+                             uint32_t flag, bool cands, bool local) {
     using LY = StepLayout<M, D, G>;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = c / a.LH;
@@ -1031,7 +1095,7 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
         for (int i = 0; i < ncl; i++) {
             const size_t idx = cb + clist[i];
             const float z = __ldcg(a.cz + idx * G + g);
-            if (__ldcg(a.cfate + idx)) s.mk = fmaxf(s.mk, z); else s.me = fmaxf(s.me, z);
+            if (cand_fate(a, sm, local, b, clist[i])) s.mk = fmaxf(s.mk, z); else s.me = fmaxf(s.me, z);
         }
         s.lk = 0.0f;
         s.le = 0.0f;
@@ -1055,7 +1119,7 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
         for (int i = 0; i < ncl; i++) {
             const size_t idx = cb + clist[i];
             const float z = __ldcg(a.cz + idx * G + g);
-            if (__ldcg(a.cfate + idx)) {
+            if (cand_fate(a, sm, local, b, clist[i])) {
                 const float w = ex2(z - s.mk);
                 s.lk += w;
                 if (!is_stat) av += w * row_elt<M>(a.cv + idx * a.row_bytes, e - g * D);
@@ -1081,7 +1145,7 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
 // or CCAP candidates; the block-wide merge handles it then.
 template <class M, int D, int G>
 __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, WarpScr &w, int c, int64_t pfx,
-                             int jf, int jl, uint32_t flag, bool cands) {
+                             int jf, int jl, uint32_t flag, bool cands, bool local) {
     using LY = StepLayout<M, D, G>;
     constexpr int GD = G * D;
     constexpr int EPL = (GD + 31) / 32;
@@ -1133,7 +1197,7 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
         w.st[3][t] = __ldcg(r + 3 * G);
     }
     for (int t = lane; t < ncl * G; t += 32) w.cz[t] = __ldcg(a.cz + (cb + w.cidx[t / G]) * G + (t % G));
-    for (int i = lane; i < ncl; i += 32) w.cfate[i] = __ldcg(a.cfate + cb + w.cidx[i]);
+    for (int i = lane; i < ncl; i += 32) w.cfate[i] = cand_fate(a, sm, local, b, w.cidx[i]);
     // the first two records' output values, in the same round
     float v0[EPL], v1[EPL];
 #pragma unroll
@@ -1491,7 +1555,7 @@ __device__ void append_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int 
 }
 
 template <class M, int D, int G>
-__device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) {
+__device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, bool local) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nct = gridDim.x;
     const int C = a.C;
     const int hc0 = (int)((int64_t)blockIdx.x * C / nct), hc1 = (int)((int64_t)(blockIdx.x + 1) * C / nct);
@@ -1511,6 +1575,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
         if (c < C) {
             np = __ldcg(a.npre + c);
             nn = cx.evict ? (int32_t)__ldcg(head_kept_of(a, cx) + c) : np;
+            if (local) nn += (int32_t)reinterpret_cast<const uint32_t *>(sm.big() + T_WARP + RES_CAP * 8)[c];
             v[0] = (uint32_t)((np + PAGE - 1) / PAGE);
             v[1] = cx.evict ? v[0] - (uint32_t)((nn + PAGE - 1) / PAGE) : 0u;
             v[2] = (nn % PAGE == 0) ? 1u : 0u;
@@ -1595,7 +1660,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
             const int64_t pfx = st_pfx[k];
             const int jf = owner_rlo(sm.rlo(), nct, pfx), jl = owner_rlo(sm.rlo(), nct, pfx + pages - 1);
             const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
-            if (!combine_warp<M, D, G>(a, sm, cx, wsc, c, pfx, jf, jl, flag, spec && (flag & 1u)) && lane == 0)
+            if (!combine_warp<M, D, G>(a, sm, cx, wsc, c, pfx, jf, jl, flag, spec && (flag & 1u), local) && lane == 0)
                 atomicOr(st_heavy + k, 1);
         }
         if (comp && !compact_warp(a, cx, wsc, c, np, nn, st_plan[k]) && lane == 0) atomicOr(st_heavy + k, 2);
@@ -1611,7 +1676,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec) 
             const int64_t pfx = st_pfx[k];
             const int jf = owner_rlo(sm.rlo(), nct, pfx), jl = owner_rlo(sm.rlo(), nct, pfx + pages - 1);
             const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
-            combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, spec && (flag & 1u));
+            combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, spec && (flag & 1u), local);
         }
         if ((heavy & 2) && cx.evict && nn < np) compact_head(a, sm, cx, c, np, nn, st_plan[k]);
     }
@@ -1635,13 +1700,15 @@ __global__ void __launch_bounds__(NTH, 1)
 
     Ctx cx;
     prologue<M, D, G>(a, sm, cx, &tmk, &tmv);
-    bool spec = false;
+    bool spec = false, local = false;
     if (cx.evict && !sm.misc()[MS_RADIX]) {
         attn_pass<M, D, G, true>(a, sm, cx, &tmk, &tmv);
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
-        if (resolve(a, sm, cx)) {
-            if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
+        const int res = resolve(a, sm, cx);
+        if (res != RES_MISS) {
+            if (res == RES_MODE_GRID && !grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
             spec = true;
+            local = res == RES_MODE_LOCAL;
             if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(a.status + 2, 1);
         } else {
             // a window missed: drop the speculative counts, select exactly
@@ -1655,7 +1722,7 @@ __global__ void __launch_bounds__(NTH, 1)
         attn_pass<M, D, G, false>(a, sm, cx, &tmk, &tmv);
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
     }
-    tail<M, D, G>(a, sm, cx, spec);
+    tail<M, D, G>(a, sm, cx, spec, local);
     // exit ticket: the last CTA resets the barrier counter and flips the half
     // of the per-call counters the next call uses
     __syncthreads();

@@ -21,6 +21,7 @@ from tests.oracle_helpers import host_cache
 pytestmark = pytest.mark.gpu
 
 WIN_CAP = 1024
+WIN_LO, WIN_HI = 16, 128   # a window that resolved its call doubles below WIN_LO candidates, halves above WIN_HI
 WIN_OFF = 144   # byte offset of the threshold windows ([B][4] uint32) in the workspace
 
 
@@ -84,9 +85,9 @@ class WindowModel:
                 nc = 0
             hw = self.hw[b] or (1 << 14)
             if wres == 1:
-                if nc > WIN_CAP // 2:
+                if nc > WIN_HI:
                     hw = max(hw >> 1, 1)
-                elif nc < 64 and hw < (1 << 28):
+                elif nc < WIN_LO and hw < (1 << 28):
                     hw <<= 1
             elif wres == 2:
                 hw = hw << 2 if hw < (1 << 26) else (1 << 28)
