@@ -298,12 +298,41 @@ template <class M, int D, int G>
 __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &cx, const CUtensorMap *tmk,
                                          const CUtensorMap *tmv) {
     const int tid = threadIdx.x, nct = gridDim.x;
+    // every independent load first: the counter half, the stack top, this
+    // thread's head lengths (LPT in registers) and its sequence's step inputs
+    // and threshold window
+    constexpr int LPT = 4;
+    cx.evict = a.m_global != nullptr;
     cx.par = __ldcg(a.parity) & 1u;
+    cx.top0 = __ldcg(a.free_top);
+    const int CS = (a.C + NTH - 1) / NTH;
+    const int h0 = min(a.C, tid * CS), h1 = min(a.C, h0 + CS);
+    int32_t nl[LPT];
+#pragma unroll
+    for (int u = 0; u < LPT; u++) nl[u] = h0 + u < h1 ? max(__ldcg(a.len + h0 + u), 0) : 0;
+    auto len_at = [&](int c) -> int32_t {
+        const int u = c - h0;
+        int32_t v = 0;
+#pragma unroll
+        for (int q = 0; q < LPT; q++)
+            if (u == q) v = nl[q];
+        return u < LPT ? v : max(__ldcg(a.len + c), 0);
+    };
+    int32_t seq_t = 0;
+    int64_t seq_m = 0;
+    uint32_t seq_w[3] = {0u, 0u, 0u};
+    if (tid < a.B) {
+        seq_t = __ldg(a.t + tid);
+        if (cx.evict) {
+            seq_m = __ldg(a.m_global + tid);
+            seq_w[0] = __ldcg(a.win + (size_t)tid * 4);
+            seq_w[1] = __ldcg(a.win + (size_t)tid * 4 + 1);
+            seq_w[2] = __ldcg(a.win + (size_t)tid * 4 + 2);
+        }
+    }
     uint32_t *other = a.ctr + (size_t)(cx.par ^ 1u) * a.ctr_words;
     // the other half is the next call's: clear it now
     for (size_t i = (size_t)blockIdx.x * NTH + tid; i < (size_t)a.ctr_words; i += (size_t)nct * NTH) other[i] = 0u;
-    cx.top0 = __ldcg(a.free_top);
-    cx.evict = a.m_global != nullptr;
     cx.epoch = 0;
     cx.exact = false;
     cx.passes = 0;
@@ -321,11 +350,9 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
         prefetch_tensormap(tmv);
     }
     __syncthreads();
-    const int CS = (a.C + NTH - 1) / NTH;
-    const int h0 = min(a.C, tid * CS), h1 = min(a.C, h0 + CS);
     uint32_t my_pages = 0;
     for (int c = h0; c < h1; c++) {
-        const int32_t n = max(__ldcg(a.len + c), 0);
+        const int32_t n = len_at(c);
         my_pages += (uint32_t)((n + PAGE - 1) / PAGE);
         atomicAdd(&sm.n()[c / a.LH], (uint32_t)n);
         if (c % nct == (int)blockIdx.x) {
@@ -349,7 +376,7 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
     {
         int64_t p = my_pfx;
         for (int c = h0; c < h1; c++) {
-            const int64_t pg = (max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE;
+            const int64_t pg = (len_at(c) + PAGE - 1) / PAGE;
             if (first == a.C && p + (pg > 0 ? pg : 1) > cx.x0) {
                 first = c;
                 first_pfx = p;
@@ -365,23 +392,21 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
     // per-sequence setup
     if (tid < a.B) {
         const int b = tid;
-        sm.t()[b] = __ldg(a.t + b);
+        sm.t()[b] = seq_t;
         const int64_t N = sm.n()[b];
         uint32_t fl = SF_TRIVIAL | SF_DONE;
         uint64_t lo = ~0ull, hi = ~0ull, kap = ~0ull;
         int64_t m = N;
         if (cx.evict) {
-            const int64_t mg = __ldg(a.m_global + b);
-            m = mg < 0 ? 0 : (mg > N ? N : mg);
+            m = seq_m < 0 ? 0 : (seq_m > N ? N : seq_m);
             if (m == 0 || m == N) {
                 kap = m == 0 ? 0ull : ~0ull;
                 lo = hi = kap;
             } else {
-                const uint32_t *w = a.win + (size_t)b * 4;
-                if (__ldcg(w) != 0u) {
+                if (seq_w[0] != 0u) {
                     fl = SF_WIN;
-                    lo = (uint64_t)__ldcg(w + 1) << 32;
-                    hi = (uint64_t)__ldcg(w + 2) << 32;
+                    lo = (uint64_t)seq_w[1] << 32;
+                    hi = (uint64_t)seq_w[2] << 32;
                 } else {
                     fl = 0u;
                     atomicOr(&sm.misc()[MS_RADIX], 1);
@@ -1566,15 +1591,30 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
         const size_t nh = (size_t)cx.passes * a.B * NBINS;
         for (size_t i = (size_t)blockIdx.x * NTH + tid; i < nh; i += (size_t)nct * NTH) a.ghist[i] = 0u;
     }
-    // per head: pre-step pages, freed pages, pops -- prefixes over all heads
+    // per head: pre-step pages, freed pages, pops -- prefixes over all heads.
+    // The same pass queues this CTA's tail tasks: merges (heads split across
+    // CTAs or holding candidates) and compactions are independent tasks (kept
+    // candidates' keep bits were set by the resolve step) that warps take from
+    // a queue in shared memory; heads too large for a warp are done
+    // block-wide afterwards, one at a time.
+    const int nh = hc1 - hc0;
+    int32_t *st_heavy = st_pop + NTH;
+    int32_t *tasks = reinterpret_cast<int32_t *>(sm.big() + T_CL);  // [2 * NTH]
+    if (tid == 0) {
+        sm.misc()[MS_QN] = 0;  // ordered before the queue's atomics by the scan's barriers
+        sm.misc()[MS_QH] = 0;
+    }
     uint32_t carry[3] = {0u, 0u, 0u};
     for (int base = 0; base < C; base += NTH) {
         const int c = base + tid;
+        const bool mine = c >= hc0 && c < hc1;
         int32_t np = 0, nn = 0;
+        uint32_t flag = 0u;
         uint32_t v[3] = {0u, 0u, 0u};
         if (c < C) {
             np = __ldcg(a.npre + c);
             nn = cx.evict ? (int32_t)__ldcg(head_kept_of(a, cx) + c) : np;
+            if (mine) flag = __ldcg(head_flag_of(a, cx) + c);
             if (local) nn += (int32_t)reinterpret_cast<const uint32_t *>(sm.big() + T_WARP + RES_CAP * 8)[c];
             v[0] = (uint32_t)((np + PAGE - 1) / PAGE);
             v[1] = cx.evict ? v[0] - (uint32_t)((nn + PAGE - 1) / PAGE) : 0u;
@@ -1582,13 +1622,20 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
         }
         uint32_t ex[3], tot[3];
         block_scan_n<3>(v, ex, tot, sm.scan());
-        if (c >= hc0 && c < hc1) {
+        if (mine) {
             const int k = c - hc0;
+            const int64_t pfx = carry[0] + ex[0];
             st_npre[k] = np;
             st_nnew[k] = nn;
-            st_pfx[k] = (int32_t)(carry[0] + ex[0]);
+            st_pfx[k] = (int32_t)pfx;
             st_plan[k] = (int32_t)(carry[1] + ex[1]);
             st_pop[k] = (int32_t)(carry[2] + ex[2]);
+            st_heavy[k] = 0;
+            const int pages = (int)v[0];
+            const bool merge = pages > 0 && (owner_rlo(sm.rlo(), nct, pfx) != owner_rlo(sm.rlo(), nct, pfx + pages - 1) ||
+                                             (flag & 2u) || (spec && (flag & 1u)));
+            if (merge) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 1;
+            if (cx.evict && nn < np) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 2;
         }
 #pragma unroll
         for (int s = 0; s < 3; s++) carry[s] += tot[s];
@@ -1616,36 +1663,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
         const int nt = cx.top0 + (int)pushes - (int)pops;
         *a.free_top = nt < 0 ? 0 : nt;
     }
-    // merges and compactions are independent tasks (kept candidates' keep
-    // bits were set by the resolve step) that warps take from a queue in
-    // shared memory.  Heads too large for a warp are done block-wide
-    // afterwards, one at a time.
-    const int nh = hc1 - hc0;
-    int32_t *st_heavy = st_pop + NTH;
-    int32_t *tasks = reinterpret_cast<int32_t *>(sm.big() + T_CL);  // [2 * NTH]
     WarpScr &wsc = *reinterpret_cast<WarpScr *>(sm.big() + T_WARP + warp * WARP_SCR);
-    if (tid == 0) {
-        sm.misc()[MS_QN] = 0;
-        sm.misc()[MS_QH] = 0;
-    }
-    __syncthreads();
-    for (int k = tid; k < nh; k += NTH) {
-        const int c = hc0 + k;
-        const int np = st_npre[k], nn = st_nnew[k];
-        const int pages = (np + PAGE - 1) / PAGE;
-        st_heavy[k] = 0;
-        bool merge = false, cands = false;
-        if (pages > 0) {
-            const int64_t pfx = st_pfx[k];
-            const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
-            cands = spec && (flag & 1u);
-            merge = owner_rlo(sm.rlo(), nct, pfx) != owner_rlo(sm.rlo(), nct, pfx + pages - 1) || (flag & 2u) || cands;
-        }
-        const bool comp = cx.evict && nn < np;
-        if (merge) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 1;
-        if (comp) tasks[atomicAdd(&sm.misc()[MS_QN], 1)] = (k << 2) | 2;
-    }
-    __syncthreads();
     const int ntask = sm.misc()[MS_QN];
     for (;;) {
         int t = 0;
