@@ -155,6 +155,85 @@ def run_workload(rkv, name, steps, seqs=None, sample=6, seed=0):
     return dc
 
 
+def run_workload_fused(rkv, name, steps, seqs=None, sample=6, seed=0):
+    """As run_workload, through the single-launch rkv_decode_step: the oracle
+    state, the sampled heads' rows and their attention inputs are taken before
+    the call (the launch compacts and appends in place)."""
+    cfg = workloads.CONFIGS[name]
+    dc = workloads.prefill_cache(cfg, seed, device="cuda", n_steps=steps + 1)
+    cache = rkv_cache(rkv, dc)
+    sel = rkv.Selection.empty(cache)
+    ws = rkv.Workspace(cache)
+    outs = rkv.StepOutputs.empty(cache)
+    rng = np.random.default_rng(seed)
+    check_seqs = list(range(cfg.B)) if seqs is None else seqs
+    full = len(check_seqs) == cfg.B
+    for s in range(steps):
+        inp = workloads.step_inputs(cfg, seed, s, "cuda")
+        host, heads = meta_host(dc, check_seqs)
+        sampled = sorted(int(x) for x in rng.choice(heads, size=min(sample, len(heads)), replace=False))
+        before = {c: head_rows(dc, c) for c in sampled}
+        mini, maxp = mini_cache(dc, sampled)
+        len_pre = host.len.copy()
+        rkv.decode_step(cache, inp["t"], inp["m_global"] if inp["evict"] else None, inp["q"], cfg.scale,
+                        inp["k_new"], inp["v_new"], inp["lb_new"], sel if inp["evict"] else None, outs.out, outs.lse,
+                        outs.dropped, ws)
+        sync()
+        assert ws.status() == 0, f"{name} step {s}: {ws.counters()}"
+        qs = inp["q"].reshape(cfg.C, cfg.G, cfg.D)[sampled].cpu().numpy()
+        if inp["evict"]:
+            t_sub = inp["t"].cpu().numpy()[check_seqs]
+            m_sub = inp["m_global"].cpu().numpy()[check_seqs]
+            keep_o, kept_o = oracle.select(host, t_sub, m_sub)
+            keep_g = masked_keep(keep_flags(sel, dc.max_pages)[heads], len_pre)
+            assert np.array_equal(sel.kept.cpu().numpy()[heads], kept_o), f"{name} step {s}: kept"
+            assert np.array_equal(keep_g, keep_o), f"{name} step {s}: keep flags"
+            pos_idx = {c: j for j, c in enumerate(heads)}
+            kk = np.zeros((len(sampled), maxp * 16), np.uint8)
+            for j, c in enumerate(sampled):
+                kk[j, :len_pre[pos_idx[c]]] = keep_o[pos_idx[c]][:len_pre[pos_idx[c]]]
+        else:
+            kk = None
+        o_ref, lse_ref, dm_ref = oracle.attention(mini, qs, cfg.scale, kk)
+        kept_any = np.array([bool(kk[j, : mini.len[j]].any()) if kk is not None else mini.len[j] > 0
+                             for j in range(len(sampled))])
+        assert_outputs_close(outs.out.reshape(cfg.C, cfg.G, cfg.D)[sampled].cpu().numpy(),
+                             outs.lse.reshape(cfg.C, cfg.G)[sampled].cpu().numpy(),
+                             outs.dropped.reshape(cfg.C, cfg.G)[sampled].cpu().numpy(), o_ref, lse_ref, dm_ref,
+                             kept_any)
+        if inp["evict"]:
+            oracle.compact(host, keep_o)
+        rc = oracle.append(host, inp["t"].cpu().numpy()[check_seqs],
+                           np.zeros((len(heads), 1), np.uint16), np.zeros((len(heads), 1), np.uint16),
+                           inp["lb_new"].cpu().numpy()[heads])
+        assert np.array_equal(dc.len.cpu().numpy()[heads], host.len), f"{name} step {s}: len"
+        tb = dc.block_table.cpu().numpy()[heads]
+        if not full:
+            # a page popped by the append comes from the stack shared by every
+            # head (pops in ascending head order): only full runs can check it
+            for j in range(len(heads)):
+                k = int(host.len[j]) - 1
+                if k % 16 == 0:
+                    tb[j, k // 16] = host.block_table[j, k // 16]
+        assert np.array_equal(tb, host.block_table), f"{name} step {s}: tables"
+        if full:
+            assert rc == oracle.OK
+            top = int(host.free_top[0])
+            assert int(dc.free_top.item()) == top
+            assert np.array_equal(dc.free_stack.cpu().numpy()[:top], host.free_stack[:top])
+            assert np.array_equal(dc.pos_pool.cpu().numpy(), host.pos_pool)
+            assert np.array_equal(dc.lb_pool.cpu().numpy().view(np.uint32), host.lb_pool.view(np.uint32))
+        for c in sampled:  # kept rows moved whole, the new row appended last
+            K0, V0, P0, _ = before[c]
+            K1, V1, P1, _ = head_rows(dc, c)
+            where = {int(p): i for i, p in enumerate(P0.cpu().numpy())}
+            old_pos = P1.cpu().numpy()[:-1]
+            idx = torch.tensor([where[int(p)] for p in old_pos], device="cuda", dtype=torch.long)
+            assert torch.equal(K1[:-1], K0[idx]) and torch.equal(V1[:-1], V0[idx])
+            assert torch.equal(K1[-1], inp["k_new"][c]) and torch.equal(V1[-1], inp["v_new"][c])
+    return ws.counters()
+
+
 def test_llama32k_prefill_eviction_and_steady_steps(rkv):
     run_workload(rkv, "llama32k", steps=3)
 
@@ -169,3 +248,20 @@ def test_qwen8k_batched_subset(rkv):
 
 def test_vlm16k_evicting_and_non_evicting_steps(rkv):
     run_workload(rkv, "vlm16k", steps=3, seqs=[0, 7], sample=4)
+
+
+def test_fused_llama32k_prefill_eviction_and_steady_steps(rkv):
+    ctr = run_workload_fused(rkv, "llama32k", steps=4)
+    assert ctr["exact_steps"] >= 1 and ctr["window_steps"] >= 2, ctr   # prefill eviction exact, then mostly the window
+
+
+def test_fused_long128k_prefill_eviction_and_steady_steps(rkv):
+    run_workload_fused(rkv, "long128k", steps=3, sample=4)
+
+
+def test_fused_qwen8k_batched_subset(rkv):
+    run_workload_fused(rkv, "qwen8k", steps=3, seqs=[0, 15], sample=4)
+
+
+def test_fused_vlm16k_evicting_and_non_evicting_steps(rkv):
+    run_workload_fused(rkv, "vlm16k", steps=3, seqs=[0, 7], sample=4)
