@@ -305,6 +305,7 @@ def run_rkv(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    sel0 = ws.counters()
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             t_start.record(stream)
@@ -323,6 +324,10 @@ def run_rkv(args, world, rank, local):
     status = ws.status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed steps")
+    sel1 = ws.counters()
+    # how the timed steps selected: inside the threshold window kept from the
+    # previous step, or by the exact radix fallback
+    selection = {k: sel1[k] - sel0[k] for k in ("window_steps", "exact_steps")}
     kern = {k: [] for k in kernel_names}
     for i in range(K):
         e = evs[i]
@@ -408,6 +413,7 @@ def run_rkv(args, world, rank, local):
         "retained_kv": {"gbs": retained / step_s / 1e9, "frac_of_peak": retained / step_s / 1e9 / peaks["hbm_gbs"]},
         "kernels_us": kern_us, "us_per_step": 1000.0 * ms_max / K, "step0_ms": step0_ms,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": len(kernel_names) * K, "clocks": clocks, "path": args.path,
+        "selection": selection,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

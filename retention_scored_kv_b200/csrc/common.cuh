@@ -103,30 +103,41 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, in
     return *smem_flag != 0;
 }
 
-// Threshold window kept across calls, per sequence: w[0] valid, [w[1], w[2])
-// the score-key (high word) range whose keys are ranked individually next
-// call, w[3] its half width.  Centred on this call's threshold score key and
+// Threshold window kept across calls, per sequence: w[0] bit 0 valid and
+// bits 8.. log2(floor) + 1 (0: no floor), [w[1], w[2]) the score-key (high
+// word) range whose keys are ranked individually next call, w[3] its half
+// width (a power of two).  Centred on this call's threshold score key and
 // resized by how this call went: wres 1 resolved in the window (wn
-// candidates: shrink above WIN_HI, grow below WIN_LO), 2 missed (grow 4x),
-// 3 too many candidates (shrink 4x), 0 no window was used.  Nothing changes
-// when nothing or everything was kept (kappa 0 or ~0).
+// candidates: shrink above WIN_HI, but never below the floor; grow below
+// WIN_LO), 2 missed (grow 4x; the floor becomes twice the half width that
+// missed, so the window does not shrink back into the step-to-step drift of
+// the threshold that it could not hold), 3 too many candidates (shrink 4x,
+// drop the floor), 0 no window was used.  Nothing changes when nothing or
+// everything was kept (kappa 0 or ~0).
 __device__ __forceinline__ void window_next(uint32_t *w, uint64_t kappa, int wres, uint32_t wn) {
     if (kappa == 0ull || kappa == ~0ull) return;
     const uint32_t center = (uint32_t)((kappa - 1ull) >> 32);
     uint32_t hw = w[3];
     if (hw == 0u) hw = 1u << 14;
+    const uint32_t fe = w[0] >> 8;
+    uint32_t floor = fe ? 1u << (fe - 1u) : 0u;
     if (wres == 1) {
-        if (wn > WIN_HI) hw = hw > 1u ? hw >> 1 : 1u;
-        else if (wn < WIN_LO) hw = hw < (1u << 28) ? hw << 1 : hw;
+        if (wn > WIN_HI) {
+            if (hw > 1u && (hw >> 1) >= floor) hw >>= 1;
+        } else if (wn < WIN_LO && hw < (1u << 28)) {
+            hw <<= 1;
+        }
     } else if (wres == 2) {
+        floor = hw < (1u << 27) ? hw << 1 : (1u << 28);
         hw = hw < (1u << 26) ? hw << 2 : (1u << 28);
     } else if (wres == 3) {
+        floor = 0u;
         hw = hw > 4u ? hw >> 2 : 1u;
     }
     w[1] = center > hw ? center - hw : 0u;
     w[2] = center < 0xFFFFFFFFu - hw ? center + hw : 0xFFFFFFFFu;
     w[3] = hw;
-    w[0] = 1u;
+    w[0] = 1u | (floor ? (uint32_t)__ffs(floor) << 8 : 0u);
 }
 
 // ------------------------------------------------ mbarrier / bulk copy ----

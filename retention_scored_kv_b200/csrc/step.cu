@@ -175,7 +175,7 @@ struct Sm {
 };
 
 // misc slots
-enum { MS_CSTART = 0, MS_CLAST, MS_RADIX, MS_MISS, MS_BAR, MS_TOTAL, MS_FOUND, MS_DIG, MS_NR, MS_H, MS_NCL,
+enum { MS_CSTART = 0, MS_CLAST, MS_RADIX, MS_MISS, MS_BAR, MS_TOTAL, MS_NCL,
        MS_ACTIVE, MS_QN, MS_QH };
 
 struct Ctx {
@@ -905,50 +905,62 @@ __device__ __forceinline__ unsigned long long *kmax_of(const StepArgs &a, const 
     return reinterpret_cast<unsigned long long *>(seqc_of(a, cx) + (size_t)b * 4 + 2);
 }
 
-// Digit p of sequence b's threshold from its completed global histogram
-// (every CTA computes the same result).
-__device__ void scan_digit(const StepArgs &a, const Sm &sm, int b, int p) {
-    const int tid = threadIdx.x;
-    constexpr int PER = (NBINS + NTH - 1) / NTH;
-    const uint32_t *gh = a.ghist + ((size_t)p * a.B + b) * NBINS;
-    uint32_t v[PER], loc = 0;
-#pragma unroll
-    for (int j = 0; j < PER; j++) {
-        const int i = tid * PER + j;
-        v[j] = i < NBINS ? __ldcg(gh + i) : 0u;
-        loc += v[j];
-    }
-    if (tid == 0) sm.misc()[MS_FOUND] = 0;
-    uint32_t total;
-    const uint32_t ex = block_exclusive_scan(loc, sm.scan(), &total);
-    const uint32_t rank = sm.rank()[b];
-    if (ex < rank && rank <= ex + loc) {
-        uint32_t cum = ex;
-#pragma unroll
-        for (int j = 0; j < PER; j++) {
-            if (cum < rank && rank <= cum + v[j]) {
-                sm.misc()[MS_DIG] = tid * PER + j;
-                sm.misc()[MS_NR] = (int)(rank - cum);
-                sm.misc()[MS_H] = (int)v[j];
-                sm.misc()[MS_FOUND] = 1;
-            }
-            cum += v[j];
+// Digit p of every unfinished sequence's threshold from its completed global
+// histogram, one warp per sequence (every CTA computes the same result):
+// lane l sums bins [64 l, 64 l + 64), a warp scan of the sums finds the lane
+// whose bins hold the rank, and that lane reads its bins again to find the bin.
+__device__ void scan_digits(const StepArgs &a, const Sm &sm, int p) {
+    constexpr int PER = NBINS / 32;
+    static_assert(NBINS % 128 == 0, "bins per lane in 16-byte loads");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int b = warp; b < a.B; b += NWARP) {
+        if (sm.fl()[b] & SF_DONE) continue;
+        const uint4 *gh = reinterpret_cast<const uint4 *>(a.ghist + ((size_t)p * a.B + b) * NBINS + lane * PER);
+        uint32_t loc = 0;
+#pragma unroll 4
+        for (int j = 0; j < PER / 4; j++) {
+            const uint4 q = __ldcg(gh + j);
+            loc += q.x + q.y + q.z + q.w;
         }
-    }
-    __syncthreads();
-    if (tid == 0) {
-        if (!sm.misc()[MS_FOUND]) {
+        uint32_t inc = loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        const uint32_t rank = sm.rank()[b];
+        const bool mine = inc - loc < rank && rank <= inc;
+        if (__ballot_sync(0xFFFFFFFFu, mine) == 0u) {
             // fewer matching keys than the rank (entries rejected as bad input)
-            set_status(a.status, RKV_DEV_BAD_INPUT);
-            sm.fl()[b] |= SF_DONE;
-            sm.kap()[b] = (sm.pk()[b] | ~sm.pm()[b]) + 1ull;
-        } else {
+            if (lane == 0) {
+                set_status(a.status, RKV_DEV_BAD_INPUT);
+                sm.fl()[b] |= SF_DONE;
+                sm.kap()[b] = (sm.pk()[b] | ~sm.pm()[b]) + 1ull;
+            }
+            continue;
+        }
+        if (mine) {
+            uint32_t cum = inc - loc, nr = 0, h = 0;
+            int dig = 0;
+#pragma unroll 2
+            for (int j = 0; j < PER / 4; j++) {
+                const uint4 q = __ldcg(gh + j);
+                const uint32_t e[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    if (cum < rank && rank <= cum + e[u]) {
+                        dig = lane * PER + 4 * j + u;
+                        nr = rank - cum;
+                        h = e[u];
+                    }
+                    cum += e[u];
+                }
+            }
             const int sh = digit_shift(p);
-            const uint64_t d = (uint64_t)sm.misc()[MS_DIG];
-            sm.pk()[b] |= d << sh;
+            sm.pk()[b] |= (uint64_t)dig << sh;
             sm.pm()[b] |= ((1ull << digit_bits(p)) - 1ull) << sh;
-            sm.rank()[b] = (uint32_t)sm.misc()[MS_NR];
-            if ((uint32_t)sm.misc()[MS_H] == sm.rank()[b] || p == NPASS - 1) {
+            sm.rank()[b] = nr;
+            if (h == nr || p == NPASS - 1) {
                 sm.fl()[b] |= SF_DONE;
                 sm.kap()[b] = (sm.pk()[b] | ~sm.pm()[b]) + 1ull;
             }
@@ -1014,8 +1026,7 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
             __syncthreads();
         }
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return false;
-        for (int b = 0; b < a.B; b++)
-            if (!(sm.fl()[b] & SF_DONE)) scan_digit(a, sm, b, p);
+        scan_digits(a, sm, p);
     }
     // keep masks (half-warp ballots), kept counts and the largest kept key of
     // each sequence (the reported threshold is that key + 1: a radix bucket

@@ -22,6 +22,7 @@ pytestmark = pytest.mark.gpu
 
 WIN_CAP = 1024
 WIN_LO, WIN_HI = 16, 128   # a window that resolved its call doubles below WIN_LO candidates, halves above WIN_HI
+                            # (not below a floor: twice the half width of its last miss)
 WIN_OFF = 144   # byte offset of the threshold windows ([B][4] uint32) in the workspace
 
 
@@ -61,6 +62,7 @@ class WindowModel:
     def __init__(self, B):
         self.w = [None] * B        # (lo, hi) score-key range, or None
         self.hw = [0] * B
+        self.floor = [0] * B       # half width the window does not shrink below
 
     def call(self, keys_by_seq, m):
         hits = []
@@ -84,19 +86,30 @@ class WindowModel:
                 hits.append(False)
                 nc = 0
             hw = self.hw[b] or (1 << 14)
+            fl = self.floor[b]
             if wres == 1:
                 if nc > WIN_HI:
-                    hw = max(hw >> 1, 1)
+                    if hw > 1 and (hw >> 1) >= fl:
+                        hw >>= 1
                 elif nc < WIN_LO and hw < (1 << 28):
                     hw <<= 1
             elif wres == 2:
+                fl = hw << 1 if hw < (1 << 27) else (1 << 28)
                 hw = hw << 2 if hw < (1 << 26) else (1 << 28)
             elif wres == 3:
+                fl = 0
                 hw = hw >> 2 if hw > 4 else 1
+            self.floor[b] = fl
             center = (kap - 1) >> 32
             self.w[b] = (center - hw if center > hw else 0, center + hw if center < 0xFFFFFFFF - hw else 0xFFFFFFFF)
             self.hw[b] = hw
         return hits
+
+    def words(self, b):
+        """The four window words the kernel keeps for sequence b."""
+        lo, hi = self.w[b]
+        fl = self.floor[b]
+        return [1 | ((fl.bit_length() << 8) if fl else 0), lo, hi, self.hw[b]]
 
 
 def run_fused(rkv, cfg, seed, steps, *, budgets=None, model=True, mutate=None):
@@ -143,6 +156,10 @@ def run_fused(rkv, cfg, seed, steps, *, budgets=None, model=True, mutate=None):
                     info.append(dict(kernel_win=win_before[b].tolist(), model_win=wm_prev[b], n=len(keys), m=int(mg[b]),
                                      above=int((hw_ < lo).sum()), nc=int(((hw_ >= lo) & (hw_ < hi)).sum())))
                 raise AssertionError(f"step {s}: took {took}, model {trace[-1]}: {info}")
+            win_after = ws.buf[WIN_OFF:WIN_OFF + 16 * cfg.B].view(torch.int32).cpu().numpy().view(np.uint32).reshape(cfg.B, 4)
+            for b in range(cfg.B):
+                if wm.w[b] is not None:
+                    assert win_after[b].tolist() == wm.words(b), f"step {s}: window of sequence {b}"
         ref = oracle.step(hc, t, mg, inp["q"].cpu().numpy().reshape(cfg.C, cfg.G, cfg.D),
                           workloads.rows_to_host(inp["k_new"]), workloads.rows_to_host(inp["v_new"]),
                           inp["lb_new"].cpu().numpy(), evict=inp["evict"], scale=cfg.scale)
