@@ -1615,14 +1615,50 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
         sm.misc()[MS_QN] = 0;  // ordered before the queue's atomics by the scan's barriers
         sm.misc()[MS_QH] = 0;
     }
-    uint32_t carry[3] = {0u, 0u, 0u};
-    for (int base = 0; base < C; base += NTH) {
+    uint32_t carry[3] = {0u, 0u, 0u}, total[3] = {0u, 0u, 0u};
+    int base0 = 0;
+    if (C > NTH) {
+        // many heads: each thread sums a contiguous chunk (its loads in flight
+        // together), one block scan gives the prefixes at this CTA's first
+        // head and the totals; the scan below then covers this CTA's heads only
+        const int CS = (C + NTH - 1) / NTH;
+        const int c0 = min(C, tid * CS), c1 = min(C, c0 + CS);
+        uint32_t sum[3] = {0u, 0u, 0u}, pre[3] = {0u, 0u, 0u};
+#pragma unroll 4
+        for (int c = c0; c < c1; c++) {
+            const int32_t np = __ldcg(a.npre + c);
+            int32_t nn = cx.evict ? (int32_t)__ldcg(head_kept_of(a, cx) + c) : np;
+            if (local) nn += (int32_t)reinterpret_cast<const uint32_t *>(sm.big() + T_WARP + RES_CAP * 8)[c];
+            const uint32_t pg = (uint32_t)((np + PAGE - 1) / PAGE);
+            const uint32_t v[3] = {pg, cx.evict ? pg - (uint32_t)((nn + PAGE - 1) / PAGE) : 0u,
+                                   (nn % PAGE == 0) ? 1u : 0u};
+#pragma unroll
+            for (int q = 0; q < 3; q++) {
+                sum[q] += v[q];
+                if (c < hc0) pre[q] += v[q];
+            }
+        }
+        uint32_t ex[3];
+        block_scan_n<3>(sum, ex, total, sm.scan());
+        uint32_t *at_hc0 = sm.scan() + 3 * 36;
+        if (c0 <= hc0 && hc0 < c1) {
+#pragma unroll
+            for (int q = 0; q < 3; q++) at_hc0[q] = ex[q] + pre[q];
+        }
+        __syncthreads();
+        if (hc0 < C) {
+#pragma unroll
+            for (int q = 0; q < 3; q++) carry[q] = at_hc0[q];
+        }
+        base0 = hc0;
+    }
+    for (int base = base0; base < (C > NTH ? hc1 : C); base += NTH) {
         const int c = base + tid;
         const bool mine = c >= hc0 && c < hc1;
         int32_t np = 0, nn = 0;
         uint32_t flag = 0u;
         uint32_t v[3] = {0u, 0u, 0u};
-        if (c < C) {
+        if (c < (C > NTH ? hc1 : C)) {
             np = __ldcg(a.npre + c);
             nn = cx.evict ? (int32_t)__ldcg(head_kept_of(a, cx) + c) : np;
             if (mine) flag = __ldcg(head_flag_of(a, cx) + c);
@@ -1651,7 +1687,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
 #pragma unroll
         for (int s = 0; s < 3; s++) carry[s] += tot[s];
     }
-    const uint32_t pushes = carry[1], pops = carry[2];
+    const uint32_t pushes = C > NTH ? total[1] : carry[1], pops = C > NTH ? total[2] : carry[2];
     __syncthreads();
     if (cx.evict) {
         for (int k = tid; k < hc1 - hc0; k += NTH) {
