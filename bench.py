@@ -56,8 +56,8 @@ METRIC = "evict+paged-decode steps/s"
 # only while the attention kernel's sources are the ones that were captured.
 ATTN_TRAFFIC = {"sources_sha256": "6e67ee544df2f78e", "workload": "llama32k", "bytes_per_launch": 2 * 139.574528e6}
 # The same for the fused step kernel: the 16-layer capture in
-# profiles/step_kernel_llama32k_16L.md (read 137.73 MB + write 7.44 MB) x2.
-STEP_TRAFFIC = {"sources_sha256": "9cd74d2b164e43ff", "workload": "llama32k", "bytes_per_launch": 2 * 145.165568e6}
+# profiles/step_kernel_llama32k_16L.md (read 137.71 MB + write 4.15 MB) x2.
+STEP_TRAFFIC = {"sources_sha256": "f4c114055eede79d", "workload": "llama32k", "bytes_per_launch": 2 * 141.859584e6}
 UNIT = "steps/s"
 SAMPLE_LAYERS = 2  # CPU oracle sample: 2 of the workload's layers, time scaled by L / 2
 
