@@ -30,8 +30,8 @@ def _declared_symbols():
 def test_header_declares_the_boundary():
     names = set(_declared_symbols())
     for want in ("rkv_score_select", "rkv_compact_pages", "rkv_paged_decode_attn", "rkv_dropped_mass",
-                 "rkv_append", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status", "rkv_version",
-                 "rkv_last_error"):
+                 "rkv_append", "rkv_decode_step", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status",
+                 "rkv_version", "rkv_last_error"):
         assert want in names
 
 
@@ -114,3 +114,44 @@ def test_unsupported_attention_shape(lib):
     rc = so.rkv_paged_decode_attn(ctypes.byref(cs), ctypes.c_void_p(16), ctypes.c_float(0.1), None,
                                   ctypes.c_void_p(16), None, None, ctypes.c_void_p(16), need, None)
     assert rc == rkv.ERR_UNSUPPORTED
+
+
+def _decode_step(rkv, so, cs, *, q=16, m_global=16, sel=None, ws_bytes=None):
+    """One rkv_decode_step call with placeholder device pointers.  Every case
+    below must be rejected before the first CUDA call: a call that passed
+    validation would launch on those pointers."""
+    sel = rkv.SelectStruct(16, 16, 16, 16, 16) if sel is None else sel
+    need = so.rkv_workspace_size(ctypes.byref(cs))
+    return so.rkv_decode_step(ctypes.byref(cs), 16, m_global, q, 0.1, 16, 16, 16, ctypes.byref(sel), 16, 16, 16,
+                              16, need if ws_bytes is None else ws_bytes, None)
+
+
+def test_decode_step_rejects_bad_arguments_before_cuda(lib):
+    rkv, so = lib
+    cs = _cache(rkv)
+    assert _decode_step(rkv, so, cs, q=None) == rkv.ERR_INVALID_ARG
+    assert "non-NULL" in so.rkv_last_error().decode()
+    assert _decode_step(rkv, so, cs, q=8) == rkv.ERR_INVALID_ARG
+    assert "aligned" in so.rkv_last_error().decode()
+    # a budget needs every selection buffer; without one (no eviction) the
+    # selection is not read, and the call proceeds to the workspace check
+    bad_sel = rkv.SelectStruct(16, 16, 16, None, 16)
+    assert _decode_step(rkv, so, cs, sel=bad_sel) == rkv.ERR_INVALID_ARG
+    assert "selection" in so.rkv_last_error().decode()
+    assert _decode_step(rkv, so, cs, m_global=None, sel=bad_sel, ws_bytes=1) == rkv.ERR_WORKSPACE_TOO_SMALL
+    assert _decode_step(rkv, so, cs, ws_bytes=1) == rkv.ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.parametrize("kw,needle", [
+    (dict(B=65), "at most 64"),          # one launch holds at most 64 sequences
+    (dict(H=2, Hq=6), "not built"),      # GQA group 3
+    (dict(D=96), "not built"),
+    (dict(dtype="F32", H=2, Hq=16), "not built"),  # fp32 pools with G = 8
+])
+def test_decode_step_unsupported_shapes(lib, kw, needle):
+    rkv, so = lib
+    if kw.get("dtype") == "F32":
+        kw = dict(kw, dtype=rkv.F32)
+    cs = _cache(rkv, **kw)
+    assert _decode_step(rkv, so, cs) == rkv.ERR_UNSUPPORTED
+    assert needle in so.rkv_last_error().decode()
