@@ -56,7 +56,9 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        # RKV_ORACLE_LIB: another build of oracle.c (the pin tests' planted-
+        # mistake check runs them against altered copies)
+        lib = ctypes.CDLL(os.environ.get("RKV_ORACLE_LIB") or build())
         P = ctypes.c_void_p
         lib.orc_score.restype = ctypes.c_float
         lib.orc_score.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_float]
