@@ -30,15 +30,16 @@
  *               - Methodology 3 / main contributions: dropped mass, the
  *                 summed dense attention weight of the discarded keys.
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent:
  *   - score s = fl32(float(t - i) * log(beta_i)), one IEEE binary32 multiply
  *     (log beta^(t-i) = (t-i) log beta); -0 is the same score as +0;
  *   - ties broken by ascending (layer, kv head, position);
  *   - entries present at step t are those with position < t;
  *   - logits use scale = 1/sqrt(D) (passed in); K/V bf16 values are widened
  *     exactly; attention is accumulated in binary64;
- *   - the paged layout, hole-fill compaction and free-page stack below are
- *     this build's own specification.
+ *   - the pages fix no paged layout: the hole-fill compaction and the
+ *     free-page stack below are a layout rule of this implementation, stated
+ *     so that tables and pools can be compared bit for bit.
  *
  * Build: gcc -O2 -std=c99 -ffp-contract=off -fexcess-precision=standard
  *        -fno-fast-math -shared -fPIC (no FMA contraction: the score must be
@@ -253,7 +254,7 @@ int orc_attention(const orc_cache *cc, const float *q, float scale, const uint8_
 /* ------------------------------------------------------------ compaction ---
  * [ContourKV] Methodology 2: the kept set is stored physically (ragged
  * storage); evicted rows are really removed.  [DBTrimKV] Methodology 4: each
- * head keeps its own length in a paged layout.  This build's layout rule:
+ * head keeps its own length in a paged layout.  The layout rule used here:
  * heads in ascending c; in head c with n entries and n_new kept,
  *   holes   = slots k < n_new that are not kept, ascending;
  *   sources = slots k >= n_new that are kept, ascending;
