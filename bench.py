@@ -175,6 +175,20 @@ def oracle_steady_state(cfg_s: workloads.Config, n_steps: int, seed: int):
     return oracle.HostCache(**workloads.to_host(dc))
 
 
+def host_cpu() -> dict:
+    """The host the oracle runs on: logical CPUs and the CPU model name."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "model": model}
+
+
 def time_oracle(cfg: workloads.Config, steps: int, warmup: int, seed: int) -> dict:
     """Seconds per oracle step on the sample, and the full-step throughput it implies."""
     import oracle
@@ -395,7 +409,8 @@ def run_rkv(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         o = time_oracle(cfg, steps=args.cpu_steps, warmup=1, seed=seed)
-        cpu = {"value": o["value"], "unit": UNIT, "cores": o["cores"], "kind": "oracle", "sample": o["sample"]}
+        cpu = {"value": o["value"], "unit": UNIT, "cores": o["cores"], "kind": "oracle", "sample": o["sample"],
+               "host": host_cpu()}
 
     peaks = _peaks()
     s_bytes = step_bytes(cfg, n_pre, kept, pages)
@@ -514,7 +529,8 @@ def run_reference(args, world, rank):
         "config": {"workload": f"{cfg.name}: L{cfg.L} H{cfg.H} Hq{cfg.Hq} D{cfg.D} B{cfg.B} T0 {cfg.T0} "
                                f"M {cfg.M} bf16 K/V, steady-state evicting steps",
                    "kv_dtype": cfg.kv_dtype, "batch": cfg.B, "context": cfg.T0, "budget": cfg.M},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": o["cores"], "kind": "oracle", "sample": o["sample"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": o["cores"], "kind": "oracle", "sample": o["sample"],
+                         "host": host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
