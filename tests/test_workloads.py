@@ -1,0 +1,128 @@
+"""The seeded input generators follow the stated recipe.
+
+- Each Beta component of the retention mixtures is checked against scipy's
+  Beta distribution (Kolmogorov-Smirnov).
+- The mixture weights and the clamp to [1e-4, 1 - 1e-6] are checked.
+- The log-retention must be the fp32 log of the draw.
+- Planted keys must lie along the stated query direction, and values are
+  never planted.
+- The workload shapes and budgets are checked.
+- The generators must be deterministic per seed.
+
+The generators hold none of the method's arithmetic; both the oracle and the
+CUDA path read what they produce.
+"""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+from scipy import stats
+
+import workloads as W
+
+N = 200_000
+
+
+def _u(mix, n, *keys):
+    return W.sample_u(mix, n, W._gen("cpu", 0, "test", *keys), "cpu").numpy()
+
+
+@pytest.mark.parametrize("a,b", [(2.0, 2.0), (2.0, 8.0), (8.0, 2.0), (2.0, 10.0), (10.0, 1.5), (1.5, 6.0),
+                                 (6.0, 2.0)])
+def test_beta_components_follow_the_beta_distribution(a, b):
+    u = _u(((1.0, ("beta", a, b)),), N, "beta", a, b)
+    assert stats.kstest(u, stats.beta(a, b).cdf).pvalue > 1e-3
+    assert abs(u.mean() - a / (a + b)) < 5 * math.sqrt(a * b / ((a + b) ** 2 * (a + b + 1)) / N)
+
+
+def test_mixture_weights_of_the_8b_workloads():
+    # 70% Beta(2,8), 25% Beta(8,2), 5% the constant 1 - 1e-4
+    u = _u(W.MIX_8B, N, "mix8b")
+    const = u == 1.0 - 1e-4
+    assert abs(const.mean() - 0.05) < 5 * math.sqrt(0.05 * 0.95 / N)
+    rest = u[~const]
+    cdf = lambda x: (0.70 * stats.beta(2, 8).cdf(x) + 0.25 * stats.beta(8, 2).cdf(x)) / 0.95
+    assert stats.kstest(rest, cdf).pvalue > 1e-3
+
+
+def test_mixture_weights_of_the_long_context_workload():
+    # 80% Beta(2,10), 20% Beta(10,1.5)
+    u = _u(W.MIX_LONG, N, "mixlong")
+    cdf = lambda x: 0.80 * stats.beta(2, 10).cdf(x) + 0.20 * stats.beta(10, 1.5).cdf(x)
+    assert stats.kstest(u, cdf).pvalue > 1e-3
+
+
+def test_draws_are_clamped():
+    u = _u(((0.5, ("const", 0.0)), (0.5, ("const", 1.0))), 1000, "clamp")
+    assert set(np.unique(u).tolist()) == {W.U_LO, W.U_HI}
+    v = _u(W.MIX_8B, N, "range")
+    assert v.min() >= 1e-4 and v.max() <= 1.0 - 1e-6
+
+
+def test_log_retention_is_the_fp32_log_of_the_draw():
+    mix = W.MIX_LONG
+    u = W.sample_u(mix, 20_000, W._gen("cpu", 3, "lr"), "cpu").numpy()
+    lb = W.log_retention(mix, 20_000, W._gen("cpu", 3, "lr"), "cpu").numpy()
+    assert lb.dtype == np.float32
+    np.testing.assert_array_max_ulp(lb, np.log(u).astype(np.float32), maxulp=1)
+    assert np.all(np.isfinite(lb)) and np.all(lb < 0)
+
+
+def _rows(pool, cfg, P0):
+    return pool[: cfg.C * P0].view(cfg.C, P0 * cfg.P, cfg.D)[:, : cfg.T0].double()
+
+
+def test_planted_keys_lie_along_the_summed_query_direction():
+    # a 10% rate for a clear signal; the mechanism is the one the 1% workloads
+    # use.  32,768 rows: planting along one query head's direction instead of
+    # the group's sum (mean 0.3 x cos ~ 0.21) fails by ~3x the tolerance
+    cfg = dataclasses.replace(W.small_config(L=1, H=4, G=2, D=64, B=1, T0=8192, M=1000, kv_dtype="f32"),
+                              planted=0.10)
+    dc = W.prefill_cache(cfg, 7, n_steps=1)
+    P0 = -(-cfg.T0 // cfg.P)
+    q0 = W.queries(cfg, 7, 0).reshape(cfg.C, cfg.G, cfg.D).sum(dim=1).double()
+    d = q0 / q0.norm(dim=-1, keepdim=True)
+    k = _rows(dc.k_pool, cfg, P0)
+    v = _rows(dc.v_pool, cfg, P0)
+    n = cfg.C * cfg.T0
+    proj_k = torch.einsum("ctd,cd->ct", k, d)
+    proj_v = torch.einsum("ctd,cd->ct", v, d)
+    # planted rows add 3 along d: the mean projection is 3 x the rate
+    assert abs(proj_k.mean().item() - 3 * 0.10) < 5 / math.sqrt(n)
+    assert abs(proj_v.mean().item()) < 5 / math.sqrt(n)
+    # and only along d: a direction orthogonal to d sees nothing
+    r = torch.randn(cfg.C, cfg.D, generator=torch.Generator().manual_seed(1), dtype=torch.float64)
+    r = r - (r * d).sum(-1, keepdim=True) * d
+    r = r / r.norm(dim=-1, keepdim=True)
+    assert abs(torch.einsum("ctd,cd->ct", k, r).mean().item()) < 5 / math.sqrt(n)
+
+
+def test_workload_shapes_and_budgets():
+    c = W.CONFIGS
+    assert (c["tiny"].L, c["tiny"].H, c["tiny"].G, c["tiny"].D, c["tiny"].T0, c["tiny"].M) == (2, 4, 1, 64, 512, 1024)
+    assert c["tiny"].kv_dtype == "f32" and c["tiny"].C * c["tiny"].T0 == 4096
+    for name in ("llama32k", "long128k"):
+        assert (c[name].L, c[name].H, c[name].G, c[name].D, c[name].B) == (32, 8, 4, 128, 1)
+    assert c["llama32k"].T0 == 32 * 1024 and c["llama32k"].M == 32 * 8 * 2048
+    assert c["long128k"].T0 == 128 * 1024 and c["long128k"].M == math.floor(0.1 * 32 * 8 * 128 * 1024)
+    q = c["qwen8k"]
+    assert (q.L, q.H, q.G, q.D, q.B, q.T0, q.M) == (36, 8, 4, 128, 16, 8192, 36 * 8 * 512)
+    v = c["vlm16k"]
+    assert (v.L, v.H, v.Hq, v.D, v.B, v.T0, v.vision, v.M) == (28, 4, 28, 128, 8, 16384, 12288, 28 * 4 * 512)
+    assert v.evict_every == 16 and v.slack == 16
+    assert [s for s in range(33) if v.evicts(s)] == [0, 16, 32]
+    for name in ("llama32k", "qwen8k", "long128k"):
+        assert c[name].planted == 0.01 and c[name].evict_every == 1
+
+
+def test_generators_are_deterministic_per_seed():
+    cfg = W.CONFIGS["tiny"]
+    a, b, other = (W.prefill_cache(cfg, s, n_steps=2) for s in (0, 0, 1))
+    for f in ("k_pool", "v_pool", "lb_pool", "pos_pool", "block_table"):
+        assert torch.equal(getattr(a, f), getattr(b, f)), f
+    assert not torch.equal(a.k_pool, other.k_pool) and not torch.equal(a.lb_pool, other.lb_pool)
+    s0, s0b, s1 = W.step_inputs(cfg, 0, 0), W.step_inputs(cfg, 0, 0), W.step_inputs(cfg, 0, 1)
+    assert torch.equal(s0["q"], s0b["q"]) and not torch.equal(s0["q"], s1["q"])
+    assert int(s1["t"][0]) == cfg.T0 + 1 and int(s1["m_global"][0]) == cfg.M
