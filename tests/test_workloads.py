@@ -126,3 +126,23 @@ def test_generators_are_deterministic_per_seed():
     s0, s0b, s1 = W.step_inputs(cfg, 0, 0), W.step_inputs(cfg, 0, 0), W.step_inputs(cfg, 0, 1)
     assert torch.equal(s0["q"], s0b["q"]) and not torch.equal(s0["q"], s1["q"])
     assert int(s1["t"][0]) == cfg.T0 + 1 and int(s1["m_global"][0]) == cfg.M
+
+
+@pytest.mark.parametrize("lengths", [[0, 1, 15, 16, 17, 33], [200, 0, 0, 48, 5, 160]])
+def test_ragged_cache_is_a_valid_layout(lengths):
+    cfg = W.small_config(L=1, H=3, G=2, D=64, B=2, T0=200, M=100, kv_dtype="f32")
+    dc = W.ragged_cache(cfg, 5, lengths)
+    table, pos = dc.block_table.numpy(), dc.pos_pool.numpy()
+    assert dc.len.tolist() == lengths
+    owned = []
+    for c, n in enumerate(lengths):
+        np_ = -(-n // cfg.P)
+        assert (table[c, :np_] >= 0).all() and (table[c, np_:] == -1).all()
+        owned += table[c, :np_].tolist()
+        slots = [pos[table[c, s // cfg.P], s % cfg.P] for s in range(n)]
+        assert len(set(slots)) == n and all(0 <= p < cfg.T0 for p in slots)
+    top = int(dc.free_top[0])
+    free = dc.free_stack[:top].tolist()
+    # every page is in exactly one head's table or on the free stack
+    assert sorted(owned + free) == list(range(dc.n_pages))
+    assert (dc.free_stack[top:] == -1).all()
