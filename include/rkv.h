@@ -85,7 +85,9 @@ extern "C" {
  *   len             [C] int32, entries per head
  *   free_stack      [n_pages] int32, free_top [1] int32
  * Positions within one head must be distinct.  Pools must be 16-byte
- * aligned (row bytes D*elt are a multiple of 16). */
+ * aligned (row bytes D*elt are a multiple of 16).  A len outside
+ * [0, max_pages*16] is read as the nearest bound and recorded as
+ * RKV_DEV_BAD_INPUT. */
 typedef struct rkv_cache {
     void *k_pool;
     void *v_pool;
@@ -253,7 +255,9 @@ RKV_API int rkv_compact_pages(const rkv_cache_t *cache, const rkv_select_t *sel,
  *   k_new, v_new [C][D] of the pool dtype
  *   lb_new    [C] float
  * Errors: RKV_ERR_INVALID_ARG, RKV_ERR_WORKSPACE_TOO_SMALL, RKV_ERR_CUDA.
- * Device: RKV_DEV_POOL_EXHAUSTED, RKV_DEV_TABLE_OVERFLOW (head skipped).
+ * Device: RKV_DEV_POOL_EXHAUSTED, RKV_DEV_TABLE_OVERFLOW, RKV_DEV_BAD_INPUT
+ * (negative len): the head is skipped and keeps its length; a head whose
+ * table is full takes no page, so later heads still pop in order.
  */
 RKV_API int rkv_append(const rkv_cache_t *cache, const int32_t *t, const void *k_new,
                        const void *v_new, const float *lb_new, void *ws, size_t ws_bytes,

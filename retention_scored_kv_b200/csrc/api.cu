@@ -42,6 +42,7 @@ int check_cache(const rkv_cache_t *c, bool need_pools) {
     if (c->P != PAGE) return fail(RKV_ERR_UNSUPPORTED, "page size must be 16 (got %d)", c->P);
     if (c->n_pages <= 0 || c->max_pages <= 0) return fail(RKV_ERR_INVALID_ARG, "n_pages and max_pages must be positive");
     if ((int64_t)c->n_pages * PAGE >= (1ll << 31)) return fail(RKV_ERR_UNSUPPORTED, "n_pages*16 must be < 2^31");
+    if ((int64_t)c->max_pages * PAGE >= (1ll << 31)) return fail(RKV_ERR_UNSUPPORTED, "max_pages*16 must be < 2^31");
     const int64_t C = (int64_t)c->B * c->L * c->H;
     if (C >= (1ll << 31) || C * c->max_pages >= (1ll << 40)) return fail(RKV_ERR_UNSUPPORTED, "too many heads");
     const int eb = elt_bytes(c->dtype);

@@ -97,7 +97,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     const int CS = (a.C + ATTN_THREADS - 1) / ATTN_THREADS;
     const int h0 = min(a.C, tid * CS), h1 = min(a.C, h0 + CS);
     uint32_t my_pages = 0;
-    for (int c = h0; c < h1; c++) my_pages += (uint32_t)((max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE);
+    for (int c = h0; c < h1; c++)
+        my_pages += (uint32_t)((clamp_len(__ldcg(a.len + c), a.max_pages, a.status) + PAGE - 1) / PAGE);
     if (tid == 0) misc[0] = a.C;
     if (tid < LY::NBAR) {
         // full: producer; empty: the owning consumer warp; qfull: producer 0; qempty: every consumer warp
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     {
         int64_t p = my_pfx;
         for (int c = h0; c < h1; c++) {
-            const int64_t pg = (max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE;
+            const int64_t pg = (clamp_len(__ldcg(a.len + c), a.max_pages, nullptr) + PAGE - 1) / PAGE;
             if (p + (pg > 0 ? pg : 1) > x0) { cand = c; cand_pfx = p; break; }
             p += pg;
         }
@@ -136,7 +137,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if constexpr (REG_SPLIT) setmaxnreg_dec<PRODUCER_REGS>();
         const int pw = warp - NCW;
         Walker w;
-        w.init(a.len, a.C, x1, last, c_start, pfx_start);
+        w.init(a.len, a.C, a.max_pages, x1, last, c_start, pfx_start);
         const uint64_t pol_kv = policy_evict_first();
         const uint64_t pol_q = policy_evict_last();
         int nq = 0;
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     // ================================ consumers ================================
     if constexpr (REG_SPLIT) setmaxnreg_inc<CONSUMER_REGS>();
     Walker w;
-    w.init(a.len, a.C, x1, last, c_start, pfx_start);
+    w.init(a.len, a.C, a.max_pages, x1, last, c_start, pfx_start);
     int nq = 0;
     int c, pages, n;
     int64_t pfx;

@@ -11,14 +11,8 @@ namespace rkv {
 namespace core {
 
 
-#ifndef RKV_NCW
-#define RKV_NCW 8
-#endif
-#ifndef RKV_NPW
-#define RKV_NPW 4
-#endif
-constexpr int NCW = RKV_NCW;           // consumer warps
-constexpr int NPW = RKV_NPW;           // producer warps (one issuing lane each)
+constexpr int NCW = 8;                 // consumer warps
+constexpr int NPW = 4;                 // producer warps (one issuing lane each)
 constexpr int ATTN_THREADS = (NCW + NPW) * 32;
 // Register split between warpgroups (consumers: warps 0..NCW-1, producers:
 // the last NPW warps).  The block launches with LAUNCH_REGS per thread; the
@@ -27,11 +21,7 @@ constexpr int ATTN_THREADS = (NCW + NPW) * 32;
 constexpr int LAUNCH_REGS = 168;
 constexpr int PRODUCER_REGS = 56;
 constexpr int CONSUMER_REGS = 224;
-#ifdef RKV_NO_REG_SPLIT
-constexpr bool REG_SPLIT = false;
-#else
 constexpr bool REG_SPLIT = (NCW % 4 == 0) && (NPW % 4 == 0);
-#endif
 static_assert(!REG_SPLIT || NPW * 32 * PRODUCER_REGS + NCW * 32 * CONSUMER_REGS <= ATTN_THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
 
@@ -479,10 +469,12 @@ struct MmaMath {
 // Walks the heads this CTA owns, in order.  A head c with pages = ceil(len/16)
 // occupies flattened pages [pfx, pfx + pages).  The CTA owns every head whose
 // pages intersect [x0, x1), every empty head with x0 <= pfx < x1, and (last
-// CTA only) the trailing empty heads.  Lengths are fetched 32 at a time.
+// CTA only) the trailing empty heads.  Lengths are fetched 32 at a time and
+// clamped to [0, max_pages*16] (the kernels' prologues record a length past
+// that as bad input).
 struct Walker {
     const int32_t *len;
-    int C;
+    int C, maxlen;
     int64_t x1;
     bool last;
     int c;
@@ -490,8 +482,10 @@ struct Walker {
     int cbuf;
     int32_t lbuf;
 
-    __device__ void init(const int32_t *len_, int C_, int64_t x1_, bool last_, int c0, int64_t pfx0) {
-        len = len_; C = C_; x1 = x1_; last = last_; c = c0; pfx = pfx0; cbuf = -64; lbuf = 0;
+    __device__ void init(const int32_t *len_, int C_, int max_pages, int64_t x1_, bool last_, int c0,
+                         int64_t pfx0) {
+        len = len_; C = C_; maxlen = max_pages * PAGE; x1 = x1_; last = last_; c = c0; pfx = pfx0;
+        cbuf = -64; lbuf = 0;
     }
     __device__ bool next(int *hc, int64_t *hpfx, int *hpages, int *hlen) {
         if (c >= C) return false;
@@ -501,7 +495,7 @@ struct Walker {
             lbuf = (cbuf + lane < C) ? __ldcg(len + cbuf + lane) : 0;
         }
         int32_t n = __shfl_sync(0xFFFFFFFFu, lbuf, c - cbuf);
-        if (n < 0) n = 0;
+        n = n < 0 ? 0 : (n > maxlen ? maxlen : n);
         const int pages = (n + PAGE - 1) / PAGE;
         if (pfx >= x1 && !last) return false;
         *hc = c; *hpfx = pfx; *hpages = pages; *hlen = n;

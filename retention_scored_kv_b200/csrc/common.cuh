@@ -16,13 +16,7 @@ constexpr int MAX_ATTN_CTAS = 512; // upper bound of the persistent attention gr
 constexpr int WIN_CAP = 1024;      // threshold-window candidates per sequence
 // A window that resolved its call is halved above WIN_HI candidates and
 // doubled below WIN_LO.
-#ifndef RKV_WIN_LO
-#define RKV_WIN_LO 16
-#endif
-#ifndef RKV_WIN_HI
-#define RKV_WIN_HI 128
-#endif
-constexpr uint32_t WIN_LO = RKV_WIN_LO, WIN_HI = RKV_WIN_HI;
+constexpr uint32_t WIN_LO = 16, WIN_HI = 128;
 constexpr uint32_t KEY_INVALID = 0xFFFFFFFFu;  // hi word no valid score maps to (NaN space)
 
 // ---------------------------------------------------------------- keys ----
@@ -51,6 +45,19 @@ __host__ __device__ __forceinline__ int digit_shift(int p) {
 // ------------------------------------------------------------ status ----
 __device__ __forceinline__ void set_status(int32_t *status, int32_t bits) {
     if ((__ldcg(status) & bits) != bits) atomicOr(status, bits);
+}
+
+// A head length as the kernels use it: a negative length counts as 0, and a
+// length past the head's block-table row (max_pages * 16 slots) is cut to it
+// and recorded as RKV_DEV_BAD_INPUT (status may be NULL at sites that re-read
+// a length already checked), so no read leaves the head's row of the table.
+__device__ __forceinline__ int32_t clamp_len(int32_t n, int max_pages, int32_t *status) {
+    const int32_t cap = max_pages * PAGE;
+    if (n > cap) {
+        if (status) set_status(status, RKV_DEV_BAD_INPUT);
+        return cap;
+    }
+    return n < 0 ? 0 : n;
 }
 
 // A bounded wait that gave up: RKV_DEV_TIMEOUT in status[0] and, if no
@@ -110,17 +117,50 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, in
 // resized by how this call went: wres 1 resolved in the window (wn
 // candidates: shrink above WIN_HI, but never below the floor; grow below
 // WIN_LO), 2 missed (grow 4x; the floor becomes twice the half width that
-// missed, so the window does not shrink back into the step-to-step drift of
-// the threshold that it could not hold), 3 too many candidates (shrink 4x,
-// drop the floor), 0 no window was used.  Nothing changes when nothing or
-// everything was kept (kappa 0 or ~0).
-__device__ __forceinline__ void window_next(uint32_t *w, uint64_t kappa, int wres, uint32_t wn) {
+// missed), 3 too many candidates (shrink 4x, drop the floor), 0 no window was
+// used.  The floor also follows the threshold's own movement: after every
+// call but an overflowing one it is at least DRIFT_MARGIN times the distance
+// between this call's threshold score key and the previous window's centre
+// (rounded up to a power of two; capped where the key density this call saw
+// would put more than WIN_CAP/2 keys inside), and the half width is raised to
+// the floor, so the window does not shrink into the step-to-step drift of the
+// threshold.  A sequence's
+// first window is sized from the density of keys around its threshold when
+// the exact selection measured it (h1: keys in the threshold's 1024-wide
+// bucket of score keys, 0 if unknown) so that about WIN_INIT keys fall
+// inside, else 2^14.  Nothing changes when nothing or everything was kept
+// (kappa 0 or ~0).
+constexpr uint32_t DRIFT_MARGIN = 4, WIN_INIT = 256;
+__device__ __forceinline__ void window_next(uint32_t *w, uint64_t kappa, int wres, uint32_t wn, uint32_t h1 = 0u) {
     if (kappa == 0ull || kappa == ~0ull) return;
     const uint32_t center = (uint32_t)((kappa - 1ull) >> 32);
+    const bool had = (w[0] & 1u) != 0u;
     uint32_t hw = w[3];
-    if (hw == 0u) hw = 1u << 14;
+    if (hw == 0u) {
+        hw = 1u << 14;
+        if (h1) {
+            hw = 1u;
+            while (hw < (1u << 20) && (uint64_t)hw * h1 < (uint64_t)WIN_INIT * 512u) hw <<= 1;
+        }
+    }
     const uint32_t fe = w[0] >> 8;
     uint32_t floor = fe ? 1u << (fe - 1u) : 0u;
+    if (had && wres != 3) {
+        const uint32_t old = w[1] > 0u ? w[1] + w[3] : w[2] - w[3];
+        const uint64_t d = center > old ? center - old : old - center;
+        // no higher than the half width at which about WIN_CAP/2 keys would
+        // fall inside, at the density this call's window saw (wn keys when it
+        // resolved the call)
+        uint64_t lim = 1u << 26;
+        if (wres == 1 && wn > 0u) {
+            const uint64_t dl = (uint64_t)w[3] * (WIN_CAP / 2) / wn;
+            if (dl < lim) lim = dl;
+        }
+        uint32_t fd = 1u;
+        while ((uint64_t)fd * 2u <= lim && (uint64_t)fd < DRIFT_MARGIN * d) fd <<= 1;
+        if (fd > floor) floor = fd;
+        if (hw < floor) hw = floor;
+    }
     if (wres == 1) {
         if (wn > WIN_HI) {
             if (hw > 1u && (hw >> 1) >= floor) hw >>= 1;

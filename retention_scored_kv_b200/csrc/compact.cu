@@ -16,11 +16,12 @@
 // result does not depend on scheduling order.
 //
 // Append: 32 heads per CTA; each CTA counts the page-needing heads before its
-// slice (len % 16 == 0), scans its own slice, pops pages from the top of the
-// stack in ascending head order, and warps store the new rows (loaded into
-// registers at kernel start).  The last CTA to finish (atomic ticket, no
-// waiting) bumps every length and the stack top, so no CTA ever reads a
-// length another CTA already changed.
+// slice (len % 16 == 0 with room left in the head's table), scans its own
+// slice, pops pages from the top of the stack in ascending head order, and
+// warps store the new rows (loaded into registers at kernel start).  The last
+// CTA to finish (atomic ticket, no waiting) bumps the length of every head
+// that appended and lowers the stack top, so no CTA ever reads a length
+// another CTA already changed; a head that could not append keeps its length.
 #include "common.cuh"
 #include "internal.h"
 
@@ -33,6 +34,12 @@ constexpr int CMP_PAIRS = 1024;   // hole/source pairs resolved per round
 constexpr int APP_THREADS = 128;  // 4 warps
 constexpr int APP_HEADS = 32;     // heads per append CTA (8 per warp)
 constexpr int MAX_ROW_CHUNKS = 32; // 16-byte chunks of one K (or V) row: D*elt <= 512 bytes
+
+// A head of length n pops a page on append: n is a multiple of 16 and the
+// new page's table index n/16 is inside the head's table row.
+__device__ __forceinline__ bool pops_page(int32_t n, int max_pages) {
+    return n >= 0 && n % PAGE == 0 && n / PAGE < max_pages;
+}
 
 __device__ __forceinline__ uint32_t below_bits(int w, int nn) {
     const int lo = w * PAGE;
@@ -164,7 +171,7 @@ __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
     constexpr int HPW = APP_HEADS / (APP_THREADS / 32);  // heads per warp
     const int top = __ldcg(a.free_top);
     uint32_t before = 0;
-    for (int cc = tid; cc < c0; cc += blockDim.x) before += (__ldcg(a.len + cc) % PAGE == 0) ? 1u : 0u;
+    for (int cc = tid; cc < c0; cc += blockDim.x) before += pops_page(__ldcg(a.len + cc), a.max_pages) ? 1u : 0u;
     int k = 0, tb = 0;
     float lbn = 0.0f;
     const int c = c0 + lane;
@@ -192,7 +199,7 @@ __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
     }
     uint32_t tot_before;
     block_exclusive_scan(before, scan, &tot_before);
-    const uint32_t need = (mine && k % PAGE == 0) ? 1u : 0u;
+    const uint32_t need = (mine && pops_page(k, a.max_pages)) ? 1u : 0u;
     uint32_t ex = 0;
     {
         // exclusive scan of need over warp 0
@@ -208,7 +215,9 @@ __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
         int64_t row = -1;
         if (mine) {
             const int pidx = k / PAGE;
-            if (pidx >= a.max_pages) {
+            if (k < 0) {
+                set_status(a.status, RKV_DEV_BAD_INPUT);
+            } else if (pidx >= a.max_pages) {
                 set_status(a.status, RKV_DEV_TABLE_OVERFLOW);
             } else if (need) {
                 const int idx = top - 1 - (int)(tot_before + ex);
@@ -245,23 +254,29 @@ __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
             }
         }
     }
-    // last CTA to finish: every length +1, stack top lowered by the pops
+    // last CTA to finish: the length of every head whose append succeeded
+    // +1 and the stack top lowered by the pops that found a page.  Success is
+    // decided as above: a length in [0, max_pages*16) and, when the head pops,
+    // a pop rank (ascending heads) below the stack top.
     __threadfence();
     __syncthreads();
     if (tid == 0) last_flag = (atomicAdd(a.done, 1u) == gridDim.x - 1) ? 1 : 0;
     __syncthreads();
     if (!last_flag) return;
     __threadfence();
-    uint32_t pops = 0;
-    for (int cc = tid; cc < a.C; cc += blockDim.x) {
-        const int32_t nl = __ldcg(a.len + cc);
-        pops += (nl % PAGE == 0) ? 1u : 0u;
-        a.len[cc] = nl + 1;
+    uint32_t rank0 = 0;
+    for (int base = 0; base < a.C; base += blockDim.x) {
+        const int cc = base + tid;
+        const int32_t nl = cc < a.C ? __ldcg(a.len + cc) : -1;
+        const bool pops = cc < a.C && pops_page(nl, a.max_pages);
+        uint32_t tot;
+        const uint32_t ex = block_exclusive_scan(pops ? 1u : 0u, scan, &tot);
+        const bool ok = nl >= 0 && nl / PAGE < a.max_pages && (!pops || (int64_t)rank0 + ex < (int64_t)top);
+        if (cc < a.C && ok) a.len[cc] = nl + 1;
+        rank0 += tot;
     }
-    uint32_t tot_pops;
-    block_exclusive_scan(pops, scan, &tot_pops);
     if (tid == 0) {
-        const int nt = top - (int)tot_pops;
+        const int nt = top - (int)min((int64_t)rank0, (int64_t)(top > 0 ? top : 0));
         *a.free_top = nt < 0 ? 0 : nt;
         *a.done = 0u;
     }

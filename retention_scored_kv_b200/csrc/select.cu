@@ -397,8 +397,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
             int64_t nsum = 0;
             for (int base = 0; base < a.LH; base += blockDim.x) {
                 const int cl = base + threadIdx.x;
-                int32_t n = cl < a.LH ? __ldcg(a.len + (int64_t)st.b * a.LH + cl) : 0;
-                if (n < 0) n = 0;
+                const int32_t n =
+                    cl < a.LH ? clamp_len(__ldcg(a.len + (int64_t)st.b * a.LH + cl), a.max_pages, a.status) : 0;
                 if (cl < a.LH) { sm.lens[cl] = n; sm.kc[cl] = 0; }
                 uint32_t tot;
                 const uint32_t ex = block_exclusive_scan((uint32_t)((n + PAGE - 1) / PAGE), sm.scan, &tot);

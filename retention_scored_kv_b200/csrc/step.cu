@@ -99,18 +99,15 @@ constexpr int MAX_NBAR = 2 * NCW * 8 + 2 * QR;
 // Local resolve: every CTA ranks all candidates itself when there are at
 // most RES_CAP of them and at most CADD_CAP heads (their kept-candidate
 // counts are tallied in shared memory), so no second grid barrier is needed.
-#ifndef RKV_RES_CAP
-#define RKV_RES_CAP 1024
-#endif
-constexpr int RES_CAP = RKV_RES_CAP;
+constexpr int RES_CAP = 1024;
 constexpr int CADD_CAP = 8192;
 constexpr int S_LO = 0, S_HI = S_LO + MAXB * 8, S_KAP = S_HI + MAXB * 8, S_PK = S_KAP + MAXB * 8,
               S_PM = S_PK + MAXB * 8, S_KMX = S_PM + MAXB * 8, S_M = S_KMX + MAXB * 8, S_T = S_M + MAXB * 8,
               S_N = S_T + MAXB * 4, S_RANK = S_N + MAXB * 4, S_FL = S_RANK + MAXB * 4, S_ABOVE = S_FL + MAXB * 4,
               S_NC = S_ABOVE + MAXB * 4, S_OFF = S_NC + MAXB * 4, S_WRES = S_OFF + MAXB * 4,
-              S_SCAN = S_WRES + MAXB * 4, S_MISC = S_SCAN + 4 * 36 * 4, S_MISC64 = S_MISC + 64 * 4,
+              S_H1 = S_WRES + MAXB * 4, S_SCAN = S_H1 + MAXB * 4, S_MISC = S_SCAN + 4 * 36 * 4, S_MISC64 = S_MISC + 64 * 4,
               S_RLO = S_MISC64 + 8 * 8, S_FATE = S_RLO + (MAX_ATTN_CTAS + 1) * 4,
-              S_BAR = (S_FATE + (RES_CAP > 0 ? RES_CAP : 1) + 15) / 16 * 16,
+              S_BAR = (S_FATE + RES_CAP + 15) / 16 * 16,
               S_BIG = (S_BAR + MAX_NBAR * 8 + 1023) / 1024 * 1024;
 
 // Shared memory: the fixed part (pipeline barriers, per-sequence state, scan
@@ -166,6 +163,8 @@ struct Sm {
     __device__ __forceinline__ uint32_t *nc() const { return at<uint32_t>(S_NC); }
     __device__ __forceinline__ uint32_t *off() const { return at<uint32_t>(S_OFF); }
     __device__ __forceinline__ uint32_t *wres() const { return at<uint32_t>(S_WRES); }
+    // keys in the threshold's 1024-wide score-key bucket (second radix pass)
+    __device__ __forceinline__ uint32_t *h1() const { return at<uint32_t>(S_H1); }
     __device__ __forceinline__ uint32_t *scan() const { return at<uint32_t>(S_SCAN); }
     __device__ __forceinline__ int *misc() const { return at<int>(S_MISC); }
     __device__ __forceinline__ int64_t *misc64() const { return at<int64_t>(S_MISC64); }
@@ -309,14 +308,14 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
     const int h0 = min(a.C, tid * CS), h1 = min(a.C, h0 + CS);
     int32_t nl[LPT];
 #pragma unroll
-    for (int u = 0; u < LPT; u++) nl[u] = h0 + u < h1 ? max(__ldcg(a.len + h0 + u), 0) : 0;
+    for (int u = 0; u < LPT; u++) nl[u] = h0 + u < h1 ? clamp_len(__ldcg(a.len + h0 + u), a.max_pages, a.status) : 0;
     auto len_at = [&](int c) -> int32_t {
         const int u = c - h0;
         int32_t v = 0;
 #pragma unroll
         for (int q = 0; q < LPT; q++)
             if (u == q) v = nl[q];
-        return u < LPT ? v : max(__ldcg(a.len + c), 0);
+        return u < LPT ? v : clamp_len(__ldcg(a.len + c), a.max_pages, a.status);
     };
     int32_t seq_t = 0;
     int64_t seq_m = 0;
@@ -466,7 +465,7 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
         if constexpr (REG_SPLIT) setmaxnreg_dec<PRODUCER_REGS>();
         const int pw = warp - NCW;
         Walker w;
-        w.init(a.len, a.C, cx.x1, cx.last, cx.c_start, cx.pfx_start);
+        w.init(a.len, a.C, a.max_pages, cx.x1, cx.last, cx.c_start, cx.pfx_start);
         const uint64_t pol_kv = policy_evict_first();
         const uint64_t pol_keep = policy_evict_last();
         int nq = cx.qbase;
@@ -527,7 +526,7 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
         // ================================ consumers ================================
         if constexpr (REG_SPLIT) setmaxnreg_inc<CONSUMER_REGS>();
         Walker w;
-        w.init(a.len, a.C, cx.x1, cx.last, cx.c_start, cx.pfx_start);
+        w.init(a.len, a.C, a.max_pages, cx.x1, cx.last, cx.c_start, cx.pfx_start);
         int nq = cx.qbase;
         int c, pages, n;
         int64_t pfx;
@@ -869,7 +868,7 @@ __device__ __forceinline__ void for_range_keys(const StepArgs &a, const Sm &sm, 
                 while (cur < cx.c_last && a.pfx[cur + 1] <= x) cur++;
                 hc[u] = cur;
                 pidx[u] = (int)(x - a.pfx[cur]);
-                if (pidx[u] * PAGE + r < max(__ldcg(a.len + cur), 0)) {
+                if (pidx[u] * PAGE + r < clamp_len(__ldcg(a.len + cur), a.max_pages, nullptr)) {
                     ld[u] = true;
                     pg[u] = __ldcg(a.block_table + (int64_t)cur * a.max_pages + pidx[u]);
                 }
@@ -956,6 +955,7 @@ __device__ void scan_digits(const StepArgs &a, const Sm &sm, int p) {
                     cum += e[u];
                 }
             }
+            if (p == 1) sm.h1()[b] = h;
             const int sh = digit_shift(p);
             sm.pk()[b] |= (uint64_t)dig << sh;
             sm.pm()[b] |= ((1ull << digit_bits(p)) - 1ull) << sh;
@@ -978,11 +978,12 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
         const int CS = (a.C + NTH - 1) / NTH;
         const int h0 = min(a.C, tid * CS), h1 = min(a.C, h0 + CS);
         uint32_t mine = 0, tot;
-        for (int c = h0; c < h1; c++) mine += (uint32_t)((max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE);
+        for (int c = h0; c < h1; c++)
+            mine += (uint32_t)((clamp_len(__ldcg(a.len + c), a.max_pages, nullptr) + PAGE - 1) / PAGE);
         int64_t p = block_exclusive_scan(mine, sm.scan(), &tot);
         for (int c = h0; c < h1; c++) {
             if (c >= cx.c_start && c <= cx.c_last + 1) a.pfx[c] = (int32_t)p;
-            p += (max(__ldcg(a.len + c), 0) + PAGE - 1) / PAGE;
+            p += (clamp_len(__ldcg(a.len + c), a.max_pages, nullptr) + PAGE - 1) / PAGE;
         }
         if (tid == 0 && cx.c_last + 1 == a.C) a.pfx[a.C] = (int32_t)cx.TP;
     }
@@ -992,6 +993,7 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
         sm.rank()[tid] = (uint32_t)sm.m()[tid];
         sm.pk()[tid] = 0ull;
         sm.pm()[tid] = 0ull;
+        sm.h1()[tid] = 0u;
     }
     if (tid < MAXB) sm.kmx()[tid] = 0ull;
     __syncthreads();
@@ -1545,6 +1547,9 @@ __device__ bool wait_pushes(const StepArgs &a, const Ctx &cx) {
 // Append of the new token to head c (one warp): slot k (the post-compaction
 // length) takes K, V, position t and log-retention; a page is popped when k
 // is a multiple of 16 (the pop-th pop of this call, ascending head order).
+// A head whose table is full takes no pop rank (the tail's scan counts pops
+// of heads with k < max_pages*16 only); a head that cannot append (full
+// table, empty stack, a timed-out wait) is skipped with its length unchanged.
 __device__ void append_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int k, int pop, uint32_t pushes) {
     const int lane = threadIdx.x & 31;
     const int chunks = a.row_bytes / 16;
@@ -1574,8 +1579,8 @@ __device__ void append_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int 
         if (row >= 0) {
             a.pos_pool[row] = sm.t()[c / a.LH];
             a.lb_pool[row] = __ldg(a.lb_new + c);
+            a.len[c] = k + 1;  // a skipped head keeps its length
         }
-        a.len[c] = k + 1;
     }
     row = __shfl_sync(0xFFFFFFFFu, row, 0);
     if (row >= 0) {
@@ -1631,7 +1636,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
             if (local) nn += (int32_t)reinterpret_cast<const uint32_t *>(sm.big() + T_WARP + RES_CAP * 8)[c];
             const uint32_t pg = (uint32_t)((np + PAGE - 1) / PAGE);
             const uint32_t v[3] = {pg, cx.evict ? pg - (uint32_t)((nn + PAGE - 1) / PAGE) : 0u,
-                                   (nn % PAGE == 0) ? 1u : 0u};
+                                   (nn % PAGE == 0 && nn / PAGE < a.max_pages) ? 1u : 0u};
 #pragma unroll
             for (int q = 0; q < 3; q++) {
                 sum[q] += v[q];
@@ -1665,7 +1670,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
             if (local) nn += (int32_t)reinterpret_cast<const uint32_t *>(sm.big() + T_WARP + RES_CAP * 8)[c];
             v[0] = (uint32_t)((np + PAGE - 1) / PAGE);
             v[1] = cx.evict ? v[0] - (uint32_t)((nn + PAGE - 1) / PAGE) : 0u;
-            v[2] = (nn % PAGE == 0) ? 1u : 0u;
+            v[2] = (nn % PAGE == 0 && nn / PAGE < a.max_pages) ? 1u : 0u;
         }
         uint32_t ex[3], tot[3];
         block_scan_n<3>(v, ex, tot, sm.scan());
@@ -1700,7 +1705,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
         // final pass is complete), and the window for the next call
         const uint64_t kap = __ldcg(kmax_of(a, cx, tid)) + 1ull;
         a.kappa[tid] = kap;
-        window_next(a.win + (size_t)tid * 4, kap, (int)sm.wres()[tid], sm.nc()[tid]);
+        window_next(a.win + (size_t)tid * 4, kap, (int)sm.wres()[tid], sm.nc()[tid], sm.h1()[tid]);
     }
     if (blockIdx.x == nct - 1 && tid == 0) {
         if (cx.evict) {

@@ -22,7 +22,6 @@ pytestmark = pytest.mark.gpu
 
 WIN_CAP = 1024
 WIN_LO, WIN_HI = 16, 128   # a window that resolved its call doubles below WIN_LO candidates, halves above WIN_HI
-                            # (not below a floor: twice the half width of its last miss)
 WIN_OFF = 144   # byte offset of the threshold windows ([B][4] uint32) in the workspace
 
 
@@ -57,12 +56,40 @@ def score_keys(hc, t):
 
 class WindowModel:
     """The per-sequence threshold window of the fused kernel, replayed from
-    the oracle's keys: predicts whether a call resolves in the window."""
+    the oracle's keys: predicts whether a call resolves in the window.
+
+    Mirrors the kernel's rule: a resolved call halves the half width above
+    WIN_HI candidates (not below the floor) and doubles it below WIN_LO; a
+    miss quadruples it and sets the floor to twice the half width that
+    missed; too many candidates quarter it and drop the floor.  After every
+    call but an overflowing one the floor is also at least DRIFT_MARGIN times
+    the threshold's move from the previous window's centre (power of two,
+    capped at the half width where WIN_CAP/2 keys would fall inside at the
+    density this call saw), and the half width is raised to the floor.  A
+    first window is sized from the keys in the threshold's 1024-wide bucket
+    of score keys (the exact selection's second radix pass) to hold about
+    WIN_INIT keys, or 2^14 when the selection ended after one pass."""
+
+    DRIFT_MARGIN, WIN_INIT = 4, 256
 
     def __init__(self, B):
         self.w = [None] * B        # (lo, hi) score-key range, or None
         self.hw = [0] * B
         self.floor = [0] * B       # half width the window does not shrink below
+
+    @staticmethod
+    def _h1(keys, thr, m):
+        """Keys in the threshold's 1024-wide score-key bucket, or 0 when the
+        radix selection ends after its first 11-bit digit (the threshold's
+        bucket of that digit is kept whole)."""
+        hi = (keys >> np.uint64(32)).astype(np.int64)
+        t_hi = int(thr >> 32)
+        d0 = hi >> 21
+        h0 = int((d0 == (t_hi >> 21)).sum())
+        below = int((d0 < (t_hi >> 21)).sum())
+        if h0 == m - below:
+            return 0
+        return int(((hi >> 10) == (t_hi >> 10)).sum())
 
     def call(self, keys_by_seq, m):
         hits = []
@@ -75,7 +102,8 @@ class WindowModel:
             kap = int(np.sort(keys)[mb - 1]) + 1
             hi_words = (keys >> np.uint64(32)).astype(np.int64)
             wres = 0
-            if self.w[b] is not None:
+            had = self.w[b] is not None
+            if had:
                 lo, hi = self.w[b]
                 above = int((hi_words < lo).sum())
                 nc = int(((hi_words >= lo) & (hi_words < hi)).sum())
@@ -85,8 +113,28 @@ class WindowModel:
             else:
                 hits.append(False)
                 nc = 0
-            hw = self.hw[b] or (1 << 14)
+            center = (kap - 1) >> 32
+            hw = self.hw[b]
+            if hw == 0:
+                hw = 1 << 14
+                h1 = self._h1(keys, kap - 1, mb)
+                if h1:
+                    hw = 1
+                    while hw < (1 << 20) and hw * h1 < self.WIN_INIT * 512:
+                        hw <<= 1
             fl = self.floor[b]
+            if had and wres != 3:
+                lo, hi = self.w[b]
+                old = lo + self.hw[b] if lo > 0 else hi - self.hw[b]
+                d = abs(center - old)
+                lim = 1 << 26
+                if wres == 1 and nc > 0:
+                    lim = min(lim, self.hw[b] * (WIN_CAP // 2) // nc)
+                fd = 1
+                while fd * 2 <= lim and fd < self.DRIFT_MARGIN * d:
+                    fd <<= 1
+                fl = max(fl, fd)
+                hw = max(hw, fl)
             if wres == 1:
                 if nc > WIN_HI:
                     if hw > 1 and (hw >> 1) >= fl:
@@ -100,7 +148,6 @@ class WindowModel:
                 fl = 0
                 hw = hw >> 2 if hw > 4 else 1
             self.floor[b] = fl
-            center = (kap - 1) >> 32
             self.w[b] = (center - hw if center > hw else 0, center + hw if center < 0xFFFFFFFF - hw else 0xFFFFFFFF)
             self.hw[b] = hw
         return hits
