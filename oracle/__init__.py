@@ -25,6 +25,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_LIB_OMP_PATH = os.path.join(_HERE, "liboracle_omp.so")
 
 GCC_FLAGS = ["-O2", "-std=c99", "-ffp-contract=off", "-fexcess-precision=standard",
              "-fno-fast-math", "-shared", "-fPIC"]
@@ -32,13 +33,16 @@ GCC_FLAGS = ["-O2", "-std=c99", "-ffp-contract=off", "-fexcess-precision=standar
 OK, ERR_INPUT, ERR_POOL, ERR_TABLE = 0, -1, -2, -3
 
 
-def build(force: bool = False) -> str:
-    """Compile oracle.c into liboracle.so next to it (gcc, no FMA contraction)."""
-    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", *GCC_FLAGS, _SRC, "-o", tmp, "-lm"])
-        os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile oracle.c next to it (gcc, no FMA contraction): liboracle.so,
+    or with ``openmp`` liboracle_omp.so, whose attention spreads independent
+    heads over threads (same per-head arithmetic, same results)."""
+    path = _LIB_OMP_PATH if openmp else _LIB_PATH
+    if force or not os.path.exists(path) or os.path.getmtime(path) < os.path.getmtime(_SRC):
+        tmp = path + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *GCC_FLAGS, *(["-fopenmp"] if openmp else []), _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, path)
+    return path
 
 
 class _Cache(ctypes.Structure):
@@ -50,16 +54,30 @@ class _Cache(ctypes.Structure):
     ]
 
 
-_lib = None
+_libs: dict = {}
+_use_openmp = False
+
+
+def use_threads(n: int) -> int:
+    """Run the following oracle calls on the OpenMP build with n threads
+    (n <= 0: every core; n == 1 or no call: the plain single-threaded build).
+    Returns the number of threads in effect."""
+    global _use_openmp
+    _use_openmp = n != 1
+    lib = _load()
+    return int(lib.orc_threads(n if n > 1 else 0)) if _use_openmp else 1
 
 
 def _load():
-    global _lib
-    if _lib is None:
+    key = "omp" if _use_openmp else "plain"
+    if key not in _libs:
         # RKV_ORACLE_LIB: another build of oracle.c (the pin tests' planted-
         # mistake check runs them against altered copies)
-        lib = ctypes.CDLL(os.environ.get("RKV_ORACLE_LIB") or build())
+        path = os.environ.get("RKV_ORACLE_LIB") or build(openmp=_use_openmp)
+        lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
+        lib.orc_threads.restype = ctypes.c_int
+        lib.orc_threads.argtypes = [ctypes.c_int]
         lib.orc_score.restype = ctypes.c_float
         lib.orc_score.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_float]
         lib.orc_entry_ok.restype = ctypes.c_int
@@ -70,12 +88,14 @@ def _load():
         lib.orc_select.argtypes = [ctypes.POINTER(_Cache), P, P, P, P]
         lib.orc_attention.restype = ctypes.c_int
         lib.orc_attention.argtypes = [ctypes.POINTER(_Cache), P, ctypes.c_float, P, P, P, P]
+        lib.orc_eviction_error.restype = ctypes.c_int
+        lib.orc_eviction_error.argtypes = [ctypes.POINTER(_Cache), P, ctypes.c_float, P, P, P]
         lib.orc_compact.restype = ctypes.c_int
         lib.orc_compact.argtypes = [ctypes.POINTER(_Cache), P]
         lib.orc_append.restype = ctypes.c_int
         lib.orc_append.argtypes = [ctypes.POINTER(_Cache), P, P, P, P]
-        _lib = lib
-    return _lib
+        _libs[key] = lib
+    return _libs[key]
 
 
 def _ptr(a: np.ndarray | None):
@@ -183,6 +203,25 @@ def attention(cache: HostCache, q: np.ndarray, scale: float, keep: np.ndarray | 
     if rc != OK:
         raise ValueError(f"oracle attention failed (code {rc})")
     return out, lse, dm
+
+
+def eviction_error(cache: HostCache, q: np.ndarray, scale: float, keep: np.ndarray | None,
+                   with_dense: bool = False):
+    """Per query head, the distance ||mu - m_A|| between the dense output mu
+    (softmax over every entry present) and the forced-weight output m_A over
+    the kept set.  Returns err float32 [C, G], and with ``with_dense`` also mu
+    [C, G, D]."""
+    q = np.ascontiguousarray(q, np.float32).reshape(cache.C, cache.G, cache.D)
+    err = np.zeros((cache.C, cache.G), np.float32)
+    mu = np.zeros((cache.C, cache.G, cache.D), np.float32) if with_dense else None
+    if keep is not None:
+        keep = np.ascontiguousarray(keep, np.uint8)
+    st = cache._struct()
+    rc = _load().orc_eviction_error(ctypes.byref(st), _ptr(q), ctypes.c_float(scale), _ptr(keep), _ptr(err),
+                                    _ptr(mu))
+    if rc != OK:
+        raise ValueError(f"oracle eviction error failed (code {rc})")
+    return (err, mu) if with_dense else err
 
 
 def compact(cache: HostCache, keep: np.ndarray) -> None:

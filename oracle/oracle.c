@@ -29,6 +29,8 @@
  *                 storage), not as a mask over the full cache.
  *               - Methodology 3 / main contributions: dropped mass, the
  *                 summed dense attention weight of the discarded keys.
+ *               - Methodology 1: the eviction error ||mu - m_A|| between
+ *                 the dense output and the forced-weight output.
  *
  * Readings where the pages are silent:
  *   - score s = fl32(float(t - i) * log(beta_i)), one IEEE binary32 multiply
@@ -43,12 +45,18 @@
  *
  * Build: gcc -O2 -std=c99 -ffp-contract=off -fexcess-precision=standard
  *        -fno-fast-math -shared -fPIC (no FMA contraction: the score must be
- *        exactly one rounded multiply).
+ *        exactly one rounded multiply).  The same source built with -fopenmp
+ *        runs the attention's independent heads on several threads (each
+ *        head's sums keep their order, so the results are the same bits);
+ *        only the CPU timing of the benchmark uses that build.
  */
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_OK 0
 #define ORC_ERR_INPUT (-1) /* NaN log-retention, age outside [1, 2^24), bad layout */
@@ -73,6 +81,18 @@ typedef struct {
 } orc_cache;
 
 static int64_t n_heads(const orc_cache *cc) { return (int64_t)cc->B * cc->L * cc->H; }
+
+/* Threads the attention may use: sets them when n > 0 (OpenMP builds only)
+ * and returns the number in effect (1 in a build without OpenMP). */
+int orc_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 static int64_t phys_row(const orc_cache *cc, int64_t c, int32_t k) {
     int32_t page = cc->block_table[c * cc->max_pages + k / cc->P];
@@ -181,6 +201,24 @@ int orc_select(const orc_cache *cc, const int32_t *t, const int64_t *m_global,
     return ORC_OK;
 }
 
+/* Query row of query head g of KV head c (grouped-query attention: query
+ * head h*G + g of a layer reads KV head h). */
+static const float *query_of(const float *q, int64_t c, int32_t g, int32_t G, int32_t D) {
+    return q + (c * G + g) * D;
+}
+
+/* Logits z_k = scale * <q, k_k> of every entry (slot order) of head c, in
+ * binary64 over the exactly widened K elements. */
+static void head_logits(const orc_cache *cc, int64_t c, const float *qv, float scale, double *z) {
+    const int32_t n = cc->len[c], D = cc->D;
+    for (int32_t k = 0; k < n; k++) {
+        int64_t row = phys_row(cc, c, k);
+        double dot = 0.0;
+        for (int32_t d = 0; d < D; d++) dot += (double)qv[d] * kv_elem(cc, cc->k_pool, row, d);
+        z[k] = (double)scale * dot;
+    }
+}
+
 /* ------------------------------------------------------------ attention ---
  * [ContourKV] Problem definition: once the subset is chosen, the weights are
  * the softmax renormalised over the kept set (forced weights):
@@ -200,55 +238,138 @@ int orc_attention(const orc_cache *cc, const float *q, float scale, const uint8_
     const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
     const int32_t D = cc->D, G = cc->G;
     int32_t max_len = 0;
+    int failed = 0;
     for (int64_t c = 0; c < C; c++) if (cc->len[c] > max_len) max_len = cc->len[c];
-    double *z = (double *)malloc((size_t)(max_len > 0 ? max_len : 1) * sizeof(double));
-    double *acc = (double *)malloc((size_t)D * sizeof(double));
-    if (!z || !acc) { free(z); free(acc); return ORC_ERR_INPUT; }
-    for (int64_t c = 0; c < C; c++) {
-        const int32_t n = cc->len[c];
-        for (int32_t g = 0; g < G; g++) {
-            const float *qv = q + (c * G + g) * D;
-            for (int32_t k = 0; k < n; k++) {
-                int64_t row = phys_row(cc, c, k);
-                double dot = 0.0;
-                for (int32_t d = 0; d < D; d++) dot += (double)qv[d] * kv_elem(cc, cc->k_pool, row, d);
-                z[k] = (double)scale * dot;
-            }
-            /* dense over all entries present before eviction */
-            double m_all = -INFINITY;
-            for (int32_t k = 0; k < n; k++) if (z[k] > m_all) m_all = z[k];
-            double z_all = 0.0, z_ev = 0.0;
-            for (int32_t k = 0; k < n; k++) {
-                double p = exp(z[k] - m_all);
-                z_all += p;
-                if (keep && !keep[c * slots_per_head + k]) z_ev += p;
-            }
-            if (dropped) dropped[c * G + g] = (float)(n > 0 ? z_ev / z_all : 0.0);
-            /* forced weights over the kept set */
-            double m_k = -INFINITY;
-            int32_t n_kept = 0;
-            for (int32_t k = 0; k < n; k++) {
-                if (keep && !keep[c * slots_per_head + k]) continue;
-                n_kept++;
-                if (z[k] > m_k) m_k = z[k];
-            }
-            double zk = 0.0;
-            for (int32_t d = 0; d < D; d++) acc[d] = 0.0;
-            for (int32_t k = 0; k < n; k++) {
-                if (keep && !keep[c * slots_per_head + k]) continue;
-                double p = exp(z[k] - m_k);
-                int64_t row = phys_row(cc, c, k);
-                zk += p;
-                for (int32_t d = 0; d < D; d++) acc[d] += p * kv_elem(cc, cc->v_pool, row, d);
-            }
-            float *o = out + (c * G + g) * D;
-            for (int32_t d = 0; d < D; d++) o[d] = (float)(n_kept > 0 ? acc[d] / zk : 0.0);
-            if (lse_kept) lse_kept[c * G + g] = (float)(n_kept > 0 ? m_k + log(zk) : -INFINITY);
+    /* heads are independent: each thread has its own logit and sum buffers */
+#pragma omp parallel
+    {
+        double *z = (double *)malloc((size_t)(max_len > 0 ? max_len : 1) * sizeof(double));
+        double *acc = (double *)malloc((size_t)D * sizeof(double));
+        if (!z || !acc) {
+#pragma omp atomic write
+            failed = 1;
         }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t c = 0; c < C; c++) {
+            if (!z || !acc) continue;
+            const int32_t n = cc->len[c];
+            for (int32_t g = 0; g < G; g++) {
+                head_logits(cc, c, query_of(q, c, g, G, D), scale, z);
+                /* dense over all entries present before eviction */
+                double m_all = -INFINITY;
+                for (int32_t k = 0; k < n; k++) if (z[k] > m_all) m_all = z[k];
+                double z_all = 0.0, z_ev = 0.0;
+                for (int32_t k = 0; k < n; k++) {
+                    double p = exp(z[k] - m_all);
+                    z_all += p;
+                    if (keep && !keep[c * slots_per_head + k]) z_ev += p;
+                }
+                if (dropped) dropped[c * G + g] = (float)(n > 0 ? z_ev / z_all : 0.0);
+                /* forced weights over the kept set */
+                double m_k = -INFINITY;
+                int32_t n_kept = 0;
+                for (int32_t k = 0; k < n; k++) {
+                    if (keep && !keep[c * slots_per_head + k]) continue;
+                    n_kept++;
+                    if (z[k] > m_k) m_k = z[k];
+                }
+                double zk = 0.0;
+                for (int32_t d = 0; d < D; d++) acc[d] = 0.0;
+                for (int32_t k = 0; k < n; k++) {
+                    if (keep && !keep[c * slots_per_head + k]) continue;
+                    double p = exp(z[k] - m_k);
+                    int64_t row = phys_row(cc, c, k);
+                    zk += p;
+                    for (int32_t d = 0; d < D; d++) acc[d] += p * kv_elem(cc, cc->v_pool, row, d);
+                }
+                float *o = out + (c * G + g) * D;
+                for (int32_t d = 0; d < D; d++) o[d] = (float)(n_kept > 0 ? acc[d] / zk : 0.0);
+                if (lse_kept) lse_kept[c * G + g] = (float)(n_kept > 0 ? m_k + log(zk) : -INFINITY);
+            }
+        }
+        free(z);
+        free(acc);
     }
-    free(z);
-    free(acc);
-    return ORC_OK;
+    return failed ? ORC_ERR_INPUT : ORC_OK;
+}
+
+/* ------------------------------------------------------- eviction error ---
+ * [ContourKV] Methodology 1 (theoretical analysis and enumeration): a kept
+ * subset A is judged by the distance between the dense attention output mu
+ * and the forced-weight output m_A over A:
+ *   e(A) = || mu - m_A ||,
+ *   mu  = sum_{j all}  exp(z_j) v_j / sum_{j all}  exp(z_j),
+ *   m_A = sum_{j in A} exp(z_j) v_j / sum_{j in A} exp(z_j),
+ * "all" = every entry of the head present before this step's eviction.
+ * Readings: the norm is the Euclidean norm over the head dimension, per
+ * query head; a head with no entries has e = 0; with nothing kept m_A = 0 (as
+ * in orc_attention), so e = ||mu||; keep == NULL means A is every entry.
+ * err [C][G]; mu_out [C][G][D] receives mu (may be NULL). */
+int orc_eviction_error(const orc_cache *cc, const float *q, float scale, const uint8_t *keep,
+                       float *err, float *mu_out) {
+    const int64_t C = n_heads(cc);
+    const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
+    const int32_t D = cc->D, G = cc->G;
+    int32_t max_len = 0;
+    int failed = 0;
+    for (int64_t c = 0; c < C; c++) if (cc->len[c] > max_len) max_len = cc->len[c];
+#pragma omp parallel
+    {
+        double *z = (double *)malloc((size_t)(max_len > 0 ? max_len : 1) * sizeof(double));
+        double *mu = (double *)malloc((size_t)D * sizeof(double));
+        double *ma = (double *)malloc((size_t)D * sizeof(double));
+        if (!z || !mu || !ma) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t c = 0; c < C; c++) {
+            if (!z || !mu || !ma) continue;
+            const int32_t n = cc->len[c];
+            for (int32_t g = 0; g < G; g++) {
+                head_logits(cc, c, query_of(q, c, g, G, D), scale, z);
+                /* mu: softmax over every entry */
+                double m_all = -INFINITY;
+                for (int32_t k = 0; k < n; k++) if (z[k] > m_all) m_all = z[k];
+                double s_all = 0.0;
+                for (int32_t d = 0; d < D; d++) mu[d] = 0.0;
+                for (int32_t k = 0; k < n; k++) {
+                    double p = exp(z[k] - m_all);
+                    int64_t row = phys_row(cc, c, k);
+                    s_all += p;
+                    for (int32_t d = 0; d < D; d++) mu[d] += p * kv_elem(cc, cc->v_pool, row, d);
+                }
+                for (int32_t d = 0; d < D; d++) mu[d] = n > 0 ? mu[d] / s_all : 0.0;
+                /* m_A: softmax over the kept entries only */
+                double m_k = -INFINITY;
+                int32_t n_kept = 0;
+                for (int32_t k = 0; k < n; k++) {
+                    if (keep && !keep[c * slots_per_head + k]) continue;
+                    n_kept++;
+                    if (z[k] > m_k) m_k = z[k];
+                }
+                double s_k = 0.0;
+                for (int32_t d = 0; d < D; d++) ma[d] = 0.0;
+                for (int32_t k = 0; k < n; k++) {
+                    if (keep && !keep[c * slots_per_head + k]) continue;
+                    double p = exp(z[k] - m_k);
+                    int64_t row = phys_row(cc, c, k);
+                    s_k += p;
+                    for (int32_t d = 0; d < D; d++) ma[d] += p * kv_elem(cc, cc->v_pool, row, d);
+                }
+                for (int32_t d = 0; d < D; d++) ma[d] = n_kept > 0 ? ma[d] / s_k : 0.0;
+                double sq = 0.0;
+                for (int32_t d = 0; d < D; d++) sq += (mu[d] - ma[d]) * (mu[d] - ma[d]);
+                err[c * G + g] = (float)sqrt(sq);
+                if (mu_out)
+                    for (int32_t d = 0; d < D; d++) mu_out[(c * G + g) * D + d] = (float)mu[d];
+            }
+        }
+        free(z);
+        free(mu);
+        free(ma);
+    }
+    return failed ? ORC_ERR_INPUT : ORC_OK;
 }
 
 /* ------------------------------------------------------------ compaction ---

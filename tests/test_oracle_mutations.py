@@ -16,7 +16,7 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = ["tests/test_oracle_score.py", "tests/test_oracle_select.py", "tests/test_oracle_layout.py",
-        "tests/test_oracle_attention.py"]
+        "tests/test_oracle_attention.py", "tests/test_oracle_error.py"]
 
 # name: (text in oracle.c, replacement)
 MUTATIONS = {
@@ -40,7 +40,7 @@ MUTATIONS = {
     # attention: logits without the scale
     "no_scale": ("z[k] = (double)scale * dot;", "z[k] = dot;"),
     # attention: query of the wrong head in a GQA group
-    "gqa_wrong_query": ("const float *qv = q + (c * G + g) * D;", "const float *qv = q + ((c * G + g) % G) * D;"),
+    "gqa_wrong_query": ("return q + (c * G + g) * D;", "return q + ((c * G + g) % G) * D;"),
     # attention: values read from the K pool
     "values_from_keys": ("acc[d] += p * kv_elem(cc, cc->v_pool, row, d);",
                          "acc[d] += p * kv_elem(cc, cc->k_pool, row, d);"),
@@ -51,6 +51,16 @@ MUTATIONS = {
                              "if (keep && keep[c * slots_per_head + k]) z_ev += p;"),
     # dropped mass: relative to the kept mass, not the dense total
     "dropped_mass_over_kept": ("z_ev / z_all", "z_ev / (z_all - z_ev)"),
+    # eviction error: squared distance (no square root)
+    "error_no_sqrt": ("err[c * G + g] = (float)sqrt(sq);", "err[c * G + g] = (float)sq;"),
+    # eviction error: dense output built from the keys
+    "error_dense_from_keys": ("for (int32_t d = 0; d < D; d++) mu[d] += p * kv_elem(cc, cc->v_pool, row, d);",
+                              "for (int32_t d = 0; d < D; d++) mu[d] += p * kv_elem(cc, cc->k_pool, row, d);"),
+    # eviction error: dense normaliser over the kept entries only
+    "error_dense_sum_over_kept": ("            s_all += p;\n",
+                                  "            if (!keep || keep[c * slots_per_head + k]) s_all += p;\n"),
+    # eviction error: kept output not normalised
+    "error_kept_unnormalised": ("ma[d] = n_kept > 0 ? ma[d] / s_k : 0.0;", "ma[d] = n_kept > 0 ? ma[d] : 0.0;"),
     # compaction: freed pages pushed in descending table order
     "pushes_descending": ("for (int32_t pi = keep_pages; pi < old_pages; pi++) {",
                           "for (int32_t pi = old_pages - 1; pi >= keep_pages; pi--) {"),
