@@ -88,6 +88,11 @@ def _load():
         lib.orc_select.argtypes = [ctypes.POINTER(_Cache), P, P, P, P]
         lib.orc_attention.restype = ctypes.c_int
         lib.orc_attention.argtypes = [ctypes.POINTER(_Cache), P, ctypes.c_float, P, P, P, P]
+        lib.orc_select_per_head.restype = ctypes.c_int
+        lib.orc_select_per_head.argtypes = [ctypes.POINTER(_Cache), P, P, P, P]
+        lib.orc_select_contour.restype = ctypes.c_int
+        lib.orc_select_contour.argtypes = [ctypes.POINTER(_Cache), P, P, P, ctypes.c_float, ctypes.c_int32,
+                                           ctypes.c_int32, P, P, P]
         lib.orc_eviction_error.restype = ctypes.c_int
         lib.orc_eviction_error.argtypes = [ctypes.POINTER(_Cache), P, ctypes.c_float, P, P, P]
         lib.orc_compact.restype = ctypes.c_int
@@ -184,6 +189,39 @@ def select(cache: HostCache, t, m_global):
     if rc != OK:
         raise ValueError(f"oracle select refused its input (code {rc})")
     return keep, kept
+
+
+def select_per_head(cache: HostCache, t, m_head):
+    """Top-m_head[c] entries of every head c by score (equal scores by
+    ascending position).  Returns (keep uint8 [C, max_pages*P], kept int32 [C])."""
+    t = np.ascontiguousarray(t, np.int32).reshape(cache.B)
+    m = np.ascontiguousarray(m_head, np.int32).reshape(cache.C)
+    keep = np.zeros((cache.C, cache.max_pages * cache.P), np.uint8)
+    kept = np.zeros(cache.C, np.int32)
+    st = cache._struct()
+    rc = _load().orc_select_per_head(ctypes.byref(st), _ptr(t), _ptr(m), _ptr(keep), _ptr(kept))
+    if rc != OK:
+        raise ValueError(f"oracle per-head select refused its input (code {rc})")
+    return keep, kept
+
+
+def select_contour(cache: HostCache, t, m_global, dm_prev, tau: float, flat_budget: int, floor: int):
+    """ContourKV allocation: recency floor in every head, a fixed budget for
+    heads whose mean previous dropped mass exceeds tau, the rest of M_global
+    by the global order over the other heads.  dm_prev float32 [C, G].
+    Returns (keep, kept, flat uint8 [C])."""
+    t = np.ascontiguousarray(t, np.int32).reshape(cache.B)
+    m = np.ascontiguousarray(m_global, np.int64).reshape(cache.B)
+    dm = np.ascontiguousarray(dm_prev, np.float32).reshape(cache.C, cache.G)
+    keep = np.zeros((cache.C, cache.max_pages * cache.P), np.uint8)
+    kept = np.zeros(cache.C, np.int32)
+    flat = np.zeros(cache.C, np.uint8)
+    st = cache._struct()
+    rc = _load().orc_select_contour(ctypes.byref(st), _ptr(t), _ptr(m), _ptr(dm), ctypes.c_float(tau),
+                                    int(flat_budget), int(floor), _ptr(keep), _ptr(kept), _ptr(flat))
+    if rc != OK:
+        raise ValueError(f"oracle ContourKV select refused its input (code {rc})")
+    return keep, kept, flat
 
 
 def attention(cache: HostCache, q: np.ndarray, scale: float, keep: np.ndarray | None):

@@ -219,6 +219,156 @@ static void head_logits(const orc_cache *cc, int64_t c, const float *qv, float s
     }
 }
 
+/* ------------------------------------------------------- per-head budget ---
+ * [TRIM-KV] core mechanism 4 (inference eviction) with a budget for each
+ * head: a head over its budget drops the entries with the lowest current
+ * retention beta^(t-i) (the pages' analogy, section 3: a backpack of fixed
+ * size drops its least valuable item).  [DBTrimKV] Methodology 3 names this
+ * fixed per-head allocation as what its single global budget replaces.
+ * Head c keeps its top m_head[c] entries by score (negative = 0); equal
+ * scores by ascending position. */
+typedef struct {
+    float s;
+    int32_t i;
+    int32_t slot;
+} orc_head_entry;
+
+static int cmp_head_rank(const void *pa, const void *pb) {
+    const orc_head_entry *a = (const orc_head_entry *)pa, *b = (const orc_head_entry *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    if (a->i != b->i) return a->i < b->i ? -1 : 1;
+    return 0;
+}
+
+static int cmp_recent(const void *pa, const void *pb) {
+    const orc_head_entry *a = (const orc_head_entry *)pa, *b = (const orc_head_entry *)pb;
+    if (a->i != b->i) return a->i > b->i ? -1 : 1;
+    return 0;
+}
+
+/* The entries of head c (sequence b) with their scores; NULL on bad input. */
+static orc_head_entry *head_entries(const orc_cache *cc, int64_t c, int32_t t, int32_t *n_out) {
+    const int32_t n = cc->len[c];
+    orc_head_entry *e = (orc_head_entry *)malloc((size_t)(n > 0 ? n : 1) * sizeof(orc_head_entry));
+    if (!e) return NULL;
+    for (int32_t k = 0; k < n; k++) {
+        int64_t row = phys_row(cc, c, k);
+        int32_t pos = cc->pos_pool[row];
+        float lb = cc->lb_pool[row];
+        if (!orc_entry_ok(t, pos, lb)) { free(e); return NULL; }
+        e[k].s = orc_score(t, pos, lb);
+        e[k].i = pos;
+        e[k].slot = k;
+    }
+    *n_out = n;
+    return e;
+}
+
+int orc_select_per_head(const orc_cache *cc, const int32_t *t, const int32_t *m_head, uint8_t *keep,
+                        int32_t *kept) {
+    const int64_t C = n_heads(cc);
+    const int64_t LH = (int64_t)cc->L * cc->H;
+    const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
+    memset(keep, 0, (size_t)(C * slots_per_head));
+    for (int64_t c = 0; c < C; c++) {
+        int32_t n = 0;
+        orc_head_entry *e = head_entries(cc, c, t[c / LH], &n);
+        if (!e) return ORC_ERR_INPUT;
+        qsort(e, (size_t)n, sizeof(orc_head_entry), cmp_head_rank);
+        int32_t m = m_head[c] < 0 ? 0 : m_head[c];
+        if (m > n) m = n;
+        for (int32_t r = 0; r < m; r++) keep[c * slots_per_head + e[r].slot] = 1;
+        kept[c] = m;
+        free(e);
+    }
+    return ORC_OK;
+}
+
+/* --------------------------------------------------- ContourKV allocation ---
+ * [ContourKV] Methodology 3: the dropped-mass statistic predicts the cells
+ * (attention heads) whose top-mass selection stays far from the dense
+ * output; those "flat" cells get a fixed budget directly, every cell keeps a
+ * recency floor, and the importance scores of an existing method are reused
+ * with this allocation in place of its own (here the retention scores and
+ * the global order of [DBTrimKV] Methodology 3).  Readings:
+ *   - a cell is a KV head c; its statistic is the mean of its G query
+ *     heads' dropped mass at the previous evicting step, dm_prev[c][g],
+ *     summed in ascending g and divided by G in binary32; flat iff > tau;
+ *   - 1. every head keeps its floor: its min(r, len) most recent entries
+ *     (largest positions; positions within a head are distinct);
+ *   - 2. a flat head also keeps the top flat_budget of its other entries
+ *     (score descending, equal scores by ascending position);
+ *   - 3. the rest of the sequence's budget, M_rest = max(0, M_global -
+ *     entries kept by 1 and 2), goes to the global order (score descending,
+ *     equal scores by ascending (layer, head, position)) over the remaining
+ *     entries of the non-flat heads.
+ * Floors and flat budgets are kept even when they exceed M_global.
+ * flat_out[C] (may be NULL) receives 1 for the flat heads. */
+int orc_select_contour(const orc_cache *cc, const int32_t *t, const int64_t *m_global, const float *dm_prev,
+                       float tau, int32_t flat_budget, int32_t floor_r, uint8_t *keep, int32_t *kept,
+                       uint8_t *flat_out) {
+    const int64_t C = n_heads(cc);
+    const int64_t LH = (int64_t)cc->L * cc->H;
+    const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
+    memset(keep, 0, (size_t)(C * slots_per_head));
+    for (int64_t c = 0; c < C; c++) kept[c] = 0;
+    for (int32_t b = 0; b < cc->B; b++) {
+        int64_t forced = 0, rest_n = 0;
+        for (int64_t cl = 0; cl < LH; cl++) rest_n += cc->len[b * LH + cl];
+        orc_entry *rest = (orc_entry *)malloc((size_t)(rest_n > 0 ? rest_n : 1) * sizeof(orc_entry));
+        if (!rest) return ORC_ERR_INPUT;
+        int64_t w = 0;
+        for (int64_t cl = 0; cl < LH; cl++) {
+            const int64_t c = b * LH + cl;
+            float sum = 0.0f;
+            for (int32_t g = 0; g < cc->G; g++) sum += dm_prev[c * cc->G + g];
+            const float mean = sum / (float)cc->G;
+            const int flat = mean > tau;
+            if (flat_out) flat_out[c] = (uint8_t)flat;
+            int32_t n = 0;
+            orc_head_entry *e = head_entries(cc, c, t[b], &n);
+            if (!e) { free(rest); return ORC_ERR_INPUT; }
+            /* 1. the floor: the most recent entries */
+            qsort(e, (size_t)n, sizeof(orc_head_entry), cmp_recent);
+            int32_t nf = floor_r < 0 ? 0 : (floor_r > n ? n : floor_r);
+            for (int32_t r = 0; r < nf; r++) keep[c * slots_per_head + e[r].slot] = 1;
+            kept[c] += nf;
+            /* 2. a flat head's fixed budget over its other entries */
+            if (flat) {
+                qsort(e + nf, (size_t)(n - nf), sizeof(orc_head_entry), cmp_head_rank);
+                int32_t m = flat_budget < 0 ? 0 : flat_budget;
+                if (m > n - nf) m = n - nf;
+                for (int32_t r = nf; r < nf + m; r++) keep[c * slots_per_head + e[r].slot] = 1;
+                kept[c] += m;
+            } else {
+                for (int32_t r = nf; r < n; r++) {
+                    rest[w].s = e[r].s;
+                    rest[w].l = (int32_t)(cl / cc->H);
+                    rest[w].h = (int32_t)(cl % cc->H);
+                    rest[w].i = e[r].i;
+                    rest[w].c = c;
+                    rest[w].slot = e[r].slot;
+                    w++;
+                }
+            }
+            forced += kept[c];
+            free(e);
+        }
+        /* 3. the rest of the budget, globally over the non-flat heads */
+        qsort(rest, (size_t)w, sizeof(orc_entry), cmp_rank);
+        int64_t m = m_global[b] - forced;
+        if (m < 0) m = 0;
+        if (m > w) m = w;
+        for (int64_t r = 0; r < m; r++) {
+            keep[rest[r].c * slots_per_head + rest[r].slot] = 1;
+            kept[rest[r].c] += 1;
+        }
+        free(rest);
+    }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------------ attention ---
  * [ContourKV] Problem definition: once the subset is chosen, the weights are
  * the softmax renormalised over the kept set (forced weights):

@@ -16,7 +16,7 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = ["tests/test_oracle_score.py", "tests/test_oracle_select.py", "tests/test_oracle_layout.py",
-        "tests/test_oracle_attention.py", "tests/test_oracle_error.py"]
+        "tests/test_oracle_attention.py", "tests/test_oracle_error.py", "tests/test_oracle_budget.py"]
 
 # name: (text in oracle.c, replacement)
 MUTATIONS = {
@@ -25,18 +25,19 @@ MUTATIONS = {
     # score: -0 left as -0 (it must rank equal to +0)
     "negative_zero_kept": ("if (s == 0.0f) s = 0.0f;", ""),
     # order: lower scores first
-    "score_ascending": ("if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
-                        "if (a->s < b->s) return -1;\n    if (a->s > b->s) return 1;"),
+    "score_ascending": ("(const orc_entry *)pb;\n    if (a->s > b->s) return -1;\n    if (a->s < b->s) return 1;",
+                        "(const orc_entry *)pb;\n    if (a->s < b->s) return -1;\n    if (a->s > b->s) return 1;"),
     # ties: later positions first
-    "ties_descending_position": ("if (a->i != b->i) return a->i < b->i ? -1 : 1;",
-                                 "if (a->i != b->i) return a->i > b->i ? -1 : 1;"),
+    "ties_descending_position": ("return a->h < b->h ? -1 : 1;\n    if (a->i != b->i) return a->i < b->i ? -1 : 1;",
+                                 "return a->h < b->h ? -1 : 1;\n    if (a->i != b->i) return a->i > b->i ? -1 : 1;"),
     # ties: head before layer
     "ties_head_before_layer": ("if (a->l != b->l) return a->l < b->l ? -1 : 1;\n"
                                "    if (a->h != b->h) return a->h < b->h ? -1 : 1;",
                                "if (a->h != b->h) return a->h < b->h ? -1 : 1;\n"
                                "    if (a->l != b->l) return a->l < b->l ? -1 : 1;"),
     # select: one entry over the budget
-    "budget_plus_one": ("for (int64_t r = 0; r < m; r++) {", "for (int64_t r = 0; r < m + (m < n); r++) {"),
+    "budget_plus_one": ("for (int64_t r = 0; r < m; r++) {\n            keep[e[r].c",
+                        "for (int64_t r = 0; r < m + (m < n); r++) {\n            keep[e[r].c"),
     # attention: logits without the scale
     "no_scale": ("z[k] = (double)scale * dot;", "z[k] = dot;"),
     # attention: query of the wrong head in a GQA group
@@ -61,6 +62,18 @@ MUTATIONS = {
                                   "            if (!keep || keep[c * slots_per_head + k]) s_all += p;\n"),
     # eviction error: kept output not normalised
     "error_kept_unnormalised": ("ma[d] = n_kept > 0 ? ma[d] / s_k : 0.0;", "ma[d] = n_kept > 0 ? ma[d] : 0.0;"),
+    # per-head budget: one entry over the budget
+    "per_head_budget_plus_one": ("for (int32_t r = 0; r < m; r++) keep[c * slots_per_head + e[r].slot] = 1;",
+                                 "for (int32_t r = 0; r < m + (m < n); r++) keep[c * slots_per_head + e[r].slot] = 1;"),
+    # per-head budget: ties by descending position
+    "per_head_ties_descending": ("if (a->i != b->i) return a->i < b->i ? -1 : 1;\n    return 0;\n}\n\nstatic int cmp_recent",
+                                 "if (a->i != b->i) return a->i > b->i ? -1 : 1;\n    return 0;\n}\n\nstatic int cmp_recent"),
+    # ContourKV: the floor holds the oldest entries
+    "floor_oldest": ("if (a->i != b->i) return a->i > b->i ? -1 : 1;", "if (a->i != b->i) return a->i < b->i ? -1 : 1;"),
+    # ContourKV: a head at the threshold counts as flat
+    "flat_not_strict": ("const int flat = mean > tau;", "const int flat = mean >= tau;"),
+    # ContourKV: the global part ignores what the floors and flat heads took
+    "m_rest_ignores_forced": ("int64_t m = m_global[b] - forced;", "int64_t m = m_global[b];"),
     # compaction: freed pages pushed in descending table order
     "pushes_descending": ("for (int32_t pi = keep_pages; pi < old_pages; pi++) {",
                           "for (int32_t pi = old_pages - 1; pi >= keep_pages; pi--) {"),
