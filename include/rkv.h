@@ -171,6 +171,55 @@ RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const i
                              const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
+ * rkv_score_select_budget -- the selection under another budget allocation,
+ * with the same outputs as rkv_score_select (so attention, dropped mass,
+ * compaction and append follow unchanged).
+ *
+ * RKV_BUDGET_PER_HEAD ([TRIM-KV] core mechanism 4 with a budget for each
+ * head; [DBTrimKV] Methodology 3 names this fixed per-head allocation as
+ * what its global budget replaces): head c keeps its top m_head[c] entries
+ * by score (negative = 0), equal scores by ascending position.  kappa = 0
+ * (there is no sequence-wide threshold).
+ *
+ * RKV_BUDGET_CONTOUR ([ContourKV] Methodology 3: the dropped-mass statistic
+ * marks "flat" cells, which get a fixed budget; every cell keeps a recency
+ * floor; the scores are reused with this allocation).  This library's
+ * reading, per sequence:
+ *   - a cell is a KV head c; it is flat iff the binary32 mean of its query
+ *     heads' dropped mass at the previous evicting step, dm_prev[c][0..G-1]
+ *     summed in ascending order and divided by G, exceeds flat_threshold;
+ *   - every head keeps its min(recency_floor, len) most recent entries
+ *     (largest positions);
+ *   - a flat head also keeps the top flat_budget of its other entries by
+ *     score (equal scores by ascending position);
+ *   - the rest of the budget, max(0, m_global[b] - entries kept so far), goes
+ *     to the global order of rkv_score_select over the other entries of the
+ *     non-flat heads; kappa[b] is that part's threshold.
+ *   Floors and flat budgets are kept even when they exceed m_global.
+ *
+ *   budget    host pointer to the parameters below (device arrays inside)
+ * Errors: RKV_ERR_INVALID_ARG (unknown mode, missing array, NaN threshold),
+ * RKV_ERR_WORKSPACE_TOO_SMALL, RKV_ERR_UNSUPPORTED, RKV_ERR_CUDA.  Device:
+ * RKV_DEV_BAD_INPUT (entry ignored), RKV_DEV_TIMEOUT.  One launch per head
+ * plus a plan launch (per head) or the global selection (ContourKV); the
+ * threshold window of the decode step is not used or changed.
+ */
+#define RKV_BUDGET_PER_HEAD 0
+#define RKV_BUDGET_CONTOUR 1
+typedef struct rkv_budget {
+    int32_t mode;            /* RKV_BUDGET_PER_HEAD or RKV_BUDGET_CONTOUR */
+    const int32_t *m_head;   /* [C] per-head budgets (PER_HEAD) */
+    const int64_t *m_global; /* [B] budget per sequence (CONTOUR) */
+    const float *dm_prev;    /* [C][G] dropped mass of the previous evicting step (CONTOUR) */
+    float flat_threshold;    /* a head is flat iff its mean dropped mass > this (CONTOUR) */
+    int32_t flat_budget;     /* entries a flat head keeps beyond its floor (CONTOUR) */
+    int32_t recency_floor;   /* most recent entries every head keeps (CONTOUR) */
+} rkv_budget_t;
+
+RKV_API int rkv_score_select_budget(const rkv_cache_t *cache, const int32_t *t, const rkv_budget_t *budget,
+                                    const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
  * rkv_score_select_noalloc -- rkv_score_select without a workspace argument,
  * for callers that cannot allocate device memory themselves (for example
  * code running where cudaMalloc is not permitted, such as inside a host
@@ -229,6 +278,30 @@ RKV_API int rkv_paged_decode_attn(const rkv_cache_t *cache, const float *q, floa
 RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float scale,
                              const rkv_select_t *sel, float *dropped, void *ws, size_t ws_bytes,
                              void *stream);
+
+/* ---------------------------------------------------------------------------
+ * rkv_eviction_error -- per query head, the distance between the dense
+ * attention output mu (softmax over every entry present before this step's
+ * eviction) and the forced-weight output m_A over the kept set:
+ *   err[c,g] = || mu - m_A ||   (Euclidean norm over the head dimension)
+ * ([ContourKV] Methodology 1, theoretical analysis: the eviction error of a
+ * kept subset A).  Computed as dm * || m_ev - m_A ||, with m_ev the
+ * forced-weight output over the evicted entries (mu is the dm-weighted mix
+ * of m_ev and m_A): the evicted rows' K and V are read, pages with no
+ * evicted row are not.  Call it after rkv_paged_decode_attn of the same step
+ * (whose out and dropped it takes) and before rkv_compact_pages.
+ *   q, scale    as rkv_paged_decode_attn
+ *   sel         the step's selection (keep masks), non-NULL
+ *   out_kept    [C][G][D] float: m_A, rkv_paged_decode_attn's out
+ *   dropped     [C][G] float: that call's dropped mass
+ *   err         [C][G] float   written (0 where nothing is evicted; ||mu||
+ *               where nothing is kept)
+ * Uses the workspace's scratch (an evicted-set output of C*G*D floats).
+ * Errors as rkv_paged_decode_attn.
+ */
+RKV_API int rkv_eviction_error(const rkv_cache_t *cache, const float *q, float scale,
+                               const rkv_select_t *sel, const float *out_kept, const float *dropped,
+                               float *err, void *ws, size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------
  * rkv_compact_pages -- physically remove the evicted entries

@@ -6,7 +6,8 @@ no CPU fallback: if the library is missing or fails to load, every call
 raises.
 
 Entry points (same names as the C ABI, without the ``rkv_`` prefix):
-``score_select``, ``paged_decode_attn``, ``dropped_mass``, ``compact_pages``,
+``score_select``, ``score_select_budget`` (as ``score_select_per_head`` and
+``score_select_contour``), ``paged_decode_attn``, ``dropped_mass``, ``eviction_error``, ``compact_pages``,
 ``append``, ``decode_step``, ``workspace_size``, ``workspace_init``,
 ``device_status``, ``version``, ``last_error``.  ``Cache``/``Selection``/
 ``Workspace`` hold the tensors and build the C structs; ``step`` runs one
@@ -31,8 +32,9 @@ BF16, F32 = 0, 1
 PAGE = 16
 
 EXPORTS = ("rkv_version", "rkv_last_error", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status",
-           "rkv_score_select", "rkv_paged_decode_attn", "rkv_dropped_mass", "rkv_compact_pages", "rkv_append",
-           "rkv_decode_step")
+           "rkv_score_select", "rkv_score_select_budget", "rkv_paged_decode_attn", "rkv_dropped_mass",
+           "rkv_eviction_error", "rkv_compact_pages", "rkv_append", "rkv_decode_step")
+BUDGET_PER_HEAD, BUDGET_CONTOUR = 0, 1
 
 
 class RkvError(RuntimeError):
@@ -51,6 +53,12 @@ class CacheStruct(ctypes.Structure):
 class SelectStruct(ctypes.Structure):
     _fields_ = [("kappa", ctypes.c_void_p), ("kept", ctypes.c_void_p), ("n_pre", ctypes.c_void_p),
                 ("keep_mask", ctypes.c_void_p), ("plan", ctypes.c_void_p)]
+
+
+class BudgetStruct(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("m_head", ctypes.c_void_p), ("m_global", ctypes.c_void_p),
+                ("dm_prev", ctypes.c_void_p), ("flat_threshold", ctypes.c_float), ("flat_budget", ctypes.c_int32),
+                ("recency_floor", ctypes.c_int32)]
 
 
 _lib = None
@@ -75,8 +83,10 @@ def load(path: str | None = None):
         "rkv_workspace_init": (I, [P, SZ, P]),
         "rkv_device_status": (P, [P]),
         "rkv_score_select": (I, [CP, P, P, SP, P, SZ, P]),
+        "rkv_score_select_budget": (I, [CP, P, ctypes.POINTER(BudgetStruct), SP, P, SZ, P]),
         "rkv_paged_decode_attn": (I, [CP, P, ctypes.c_float, SP, P, P, P, P, SZ, P]),
         "rkv_dropped_mass": (I, [CP, P, ctypes.c_float, SP, P, P, SZ, P]),
+        "rkv_eviction_error": (I, [CP, P, ctypes.c_float, SP, P, P, P, P, SZ, P]),
         "rkv_compact_pages": (I, [CP, SP, P, SZ, P]),
         "rkv_append": (I, [CP, P, P, P, P, P, SZ, P]),
         "rkv_decode_step": (I, [CP, P, P, P, ctypes.c_float, P, P, P, SP, P, P, P, P, SZ, P]),
@@ -236,6 +246,28 @@ def score_select(cache: Cache, t: torch.Tensor, m_global: torch.Tensor, sel: Sel
                                    ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
 
 
+def score_select_per_head(cache: Cache, t: torch.Tensor, m_head: torch.Tensor, sel: Selection, ws: Workspace,
+                          stream=None):
+    """Each head keeps its top m_head[c] entries (int32 [C])."""
+    cs, ss = cache.struct(), sel.struct()
+    bs = BudgetStruct(BUDGET_PER_HEAD, _ptr(m_head), None, None, 0.0, 0, 0)
+    _check(load().rkv_score_select_budget(ctypes.byref(cs), _ptr(t), ctypes.byref(bs), ctypes.byref(ss),
+                                          ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
+def score_select_contour(cache: Cache, t: torch.Tensor, m_global: torch.Tensor, dm_prev: torch.Tensor,
+                         flat_threshold: float, flat_budget: int, recency_floor: int, sel: Selection,
+                         ws: Workspace, stream=None):
+    """ContourKV allocation: dm_prev float32 [B, L, Hq] (the previous
+    evicting step's dropped mass), recency floor, flat heads' budget, the
+    rest of m_global ranked globally (see rkv.h)."""
+    cs, ss = cache.struct(), sel.struct()
+    bs = BudgetStruct(BUDGET_CONTOUR, None, _ptr(m_global), _ptr(dm_prev), float(flat_threshold), int(flat_budget),
+                      int(recency_floor))
+    _check(load().rkv_score_select_budget(ctypes.byref(cs), _ptr(t), ctypes.byref(bs), ctypes.byref(ss),
+                                          ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
 def paged_decode_attn(cache: Cache, q: torch.Tensor, scale: float, sel: Selection | None, out: torch.Tensor,
                       lse: torch.Tensor | None, dropped: torch.Tensor | None, ws: Workspace, stream=None):
     cs = cache.struct()
@@ -250,6 +282,14 @@ def dropped_mass(cache: Cache, q: torch.Tensor, scale: float, sel: Selection, dr
     cs, ss = cache.struct(), sel.struct()
     _check(load().rkv_dropped_mass(ctypes.byref(cs), _ptr(q), ctypes.c_float(scale), ctypes.byref(ss),
                                    _ptr(dropped), ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
+def eviction_error(cache: Cache, q: torch.Tensor, scale: float, sel: Selection, out_kept: torch.Tensor,
+                   dropped: torch.Tensor, err: torch.Tensor, ws: Workspace, stream=None):
+    cs, ss = cache.struct(), sel.struct()
+    _check(load().rkv_eviction_error(ctypes.byref(cs), _ptr(q), ctypes.c_float(scale), ctypes.byref(ss),
+                                     _ptr(out_kept), _ptr(dropped), _ptr(err), ctypes.c_void_p(ws.ptr), ws.nbytes,
+                                     _stream(stream)))
 
 
 def compact_pages(cache: Cache, sel: Selection, ws: Workspace, stream=None):
@@ -291,13 +331,19 @@ class StepOutputs:
 
 
 def step(cache: Cache, sel: Selection, ws: Workspace, outs: StepOutputs, *, q, t, m_global, k_new, v_new,
-         lb_new, evict: bool = True, scale: float | None = None, fused: bool = False, stream=None):
-    """One decode step: [select] -> attention + dropped mass -> [compaction] -> append.
+         lb_new, evict: bool = True, scale: float | None = None, fused: bool = False, stream=None,
+         err: torch.Tensor | None = None):
+    """One decode step: [select] -> attention + dropped mass -> [eviction
+    error] -> [compaction] -> append.
 
     On a non-evicting step every entry is kept and the dropped mass is 0.
-    ``fused`` runs the whole step as one ``decode_step`` launch."""
+    ``fused`` runs the whole step as one ``decode_step`` launch; ``err``
+    ([B, L, Hq] float32) asks for the eviction error of an evicting step,
+    which the separate calls provide (not the fused launch)."""
     if scale is None:
         scale = 1.0 / math.sqrt(cache.D)
+    if err is not None and fused:
+        raise ValueError("the eviction error comes from the separate calls (fused=False)")
     if fused:
         decode_step(cache, t, m_global if evict else None, q, scale, k_new, v_new, lb_new, sel if evict else None,
                     outs.out, outs.lse, outs.dropped, ws, stream)
@@ -305,6 +351,8 @@ def step(cache: Cache, sel: Selection, ws: Workspace, outs: StepOutputs, *, q, t
     if evict:
         score_select(cache, t, m_global, sel, ws, stream)
         paged_decode_attn(cache, q, scale, sel, outs.out, outs.lse, outs.dropped, ws, stream)
+        if err is not None:
+            eviction_error(cache, q, scale, sel, outs.out, outs.dropped, err, ws, stream)
         compact_pages(cache, sel, ws, stream)
     else:
         paged_decode_attn(cache, q, scale, None, outs.out, outs.lse, outs.dropped, ws, stream)

@@ -113,6 +113,12 @@ void layout_for(const rkv_cache_t &c, int sel_groups_x_waves, WsLayout *L) {
     L->hrec = take((size_t)SC * attn_partial_rec_floats(c.D, G) * 4, 256);
     L->npre = take((size_t)SC * 4, 256);
     L->pfx = take((size_t)(SC + 1) * 4, 256);
+    L->ev_out = take((size_t)C * G * c.D * 4, 256);
+    L->bmask = take((size_t)C * c.max_pages * 2, 256);
+    L->bkept = take((size_t)C * 4, 256);
+    L->bfloor = take((size_t)C * 4, 256);
+    L->bskip = take((size_t)C, 256);
+    L->bseq = take((size_t)c.B * 16, 256);
     L->total = take(0, 256);
 }
 
@@ -325,7 +331,7 @@ RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t,
 
 static int attn_common(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
                        float *out, float *lse, float *dropped, void *ws, size_t ws_bytes, void *stream,
-                       const char *what) {
+                       const char *what, bool invert = false) {
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if (!q) return fail(RKV_ERR_INVALID_ARG, "%s: q is NULL", what);
@@ -354,6 +360,7 @@ static int attn_common(const rkv_cache_t *cache, const float *q, float scale, co
     a.C = cache->B * cache->L * cache->H;
     a.max_pages = cache->max_pages;
     a.qscale = scale * 1.4426950408889634f;
+    a.invert = invert ? 1 : 0;
     CUtensorMap tk{}, tv{};
     if (attn_uses_tensor_maps(cache->dtype)) {
         if ((rc = encode_pool_map(&tk, cache->k_pool, cache->D, cache->n_pages))) return rc;
@@ -376,6 +383,130 @@ RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float sca
     if (!dropped) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: dropped is NULL");
     if (!sel) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: sel is NULL");
     return attn_common(cache, q, scale, sel, nullptr, nullptr, dropped, ws, ws_bytes, stream, "rkv_dropped_mass");
+}
+
+RKV_API int rkv_score_select_budget(const rkv_cache_t *cache, const int32_t *t, const rkv_budget_t *budget,
+                                    const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if ((rc = check_sel(sel))) return rc;
+    if (!t || !budget) return fail(RKV_ERR_INVALID_ARG, "rkv_score_select_budget: t / budget is NULL");
+    const bool contour = budget->mode == RKV_BUDGET_CONTOUR;
+    if (!contour && budget->mode != RKV_BUDGET_PER_HEAD)
+        return fail(RKV_ERR_INVALID_ARG, "rkv_score_select_budget: unknown mode %d", budget->mode);
+    if (!contour && !budget->m_head) return fail(RKV_ERR_INVALID_ARG, "rkv_score_select_budget: m_head is NULL");
+    if (contour && (!budget->m_global || !budget->dm_prev))
+        return fail(RKV_ERR_INVALID_ARG, "rkv_score_select_budget: m_global / dm_prev is NULL");
+    if (contour && budget->flat_threshold != budget->flat_threshold)
+        return fail(RKV_ERR_INVALID_ARG, "rkv_score_select_budget: flat_threshold is NaN");
+    WsLayout L;
+    if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
+    const int64_t LH = (int64_t)cache->L * cache->H;
+    const int lb = lh_bits(LH);
+    if (lb > 24) return fail(RKV_ERR_UNSUPPORTED, "L*H must be <= 2^24");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    BudgetArgs b{};
+    b.pos_pool = cache->pos_pool;
+    b.lb_pool = cache->lb_pool;
+    b.block_table = cache->block_table;
+    b.len = cache->len;
+    b.t = t;
+    b.LH = (int)LH;
+    b.C = (int)(cache->B * LH);
+    b.G = cache->Hq / cache->H;
+    b.max_pages = cache->max_pages;
+    b.mode = budget->mode;
+    b.m_head = budget->m_head;
+    b.dm_prev = budget->dm_prev;
+    b.tau = budget->flat_threshold;
+    b.flat_budget = budget->flat_budget;
+    b.floor_r = budget->recency_floor;
+    b.status = at<int32_t>(ws, L.status);
+    cudaError_t e;
+    if (!contour) {
+        // every head's own top-m: masks, counts and lengths, then the plan
+        b.mask = sel->keep_mask;
+        b.kept = sel->kept;
+        b.n_pre = sel->n_pre;
+        if ((e = launch_head_budget(b, s)) != cudaSuccess) return cuda_fail(e, "budget kernel launch");
+        if ((e = launch_plan(sel->n_pre, sel->kept, sel->plan, cache->free_top, sel->kappa, b.C, cache->B, s)) !=
+            cudaSuccess)
+            return cuda_fail(e, "plan kernel launch");
+        return RKV_OK;
+    }
+    // ContourKV: floors and flat heads' budgets first, then the global
+    // selection over what is left with the rest of the budget
+    b.mask = at<uint16_t>(ws, L.bmask);
+    b.kept = at<int32_t>(ws, L.bkept);
+    b.floor_pos = at<int32_t>(ws, L.bfloor);
+    b.skip = at<uint8_t>(ws, L.bskip);
+    b.seq = at<unsigned long long>(ws, L.bseq);
+    if ((e = cudaMemsetAsync(b.seq, 0, (size_t)cache->B * 16, s)) != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync(budget counters)");
+    if ((e = launch_head_budget(b, s)) != cudaSuccess) return cuda_fail(e, "budget kernel launch");
+    int sms = 0;
+    if ((rc = sm_count_now(&sms))) return rc;
+    SelectGrid g = select_grid_for(*cache, sms < MAX_SEL_CTAS ? sms : MAX_SEL_CTAS);
+    if (g.cache_pages < 0) return fail(RKV_ERR_UNSUPPORTED, "L*H too large for the selection kernel");
+    SelectArgs a{};
+    a.pos_pool = cache->pos_pool;
+    a.lb_pool = cache->lb_pool;
+    a.block_table = cache->block_table;
+    a.len = cache->len;
+    a.free_top = cache->free_top;
+    a.B = cache->B;
+    a.LH = (int)LH;
+    a.C = (int)(cache->B * LH);
+    a.max_pages = cache->max_pages;
+    a.ibits = 32 - lb;
+    a.t = t;
+    a.m_global = budget->m_global;
+    a.kappa = sel->kappa;
+    a.kept = sel->kept;
+    a.n_pre = sel->n_pre;
+    a.keep_mask = sel->keep_mask;
+    a.plan = sel->plan;
+    a.status = at<int32_t>(ws, L.status);
+    a.bar = at<uint32_t>(ws, L.bar);
+    a.leave = at<uint32_t>(ws, L.leave);
+    a.win = at<uint32_t>(ws, L.win);
+    a.cnt = at<uint32_t>(ws, L.cnt);
+    a.kmax = at<unsigned long long>(ws, L.kmax);
+    a.cand = at<uint2>(ws, L.cand);
+    a.more = at<uint32_t>(ws, L.more);
+    a.hist = at<uint32_t>(ws, L.hist);
+    a.n_groups = g.n_groups;
+    a.cta_per_group = g.cta_per_group;
+    a.waves = g.waves;
+    a.cache_pages = g.cache_pages;
+    a.floor_pos = b.floor_pos;
+    a.skip = b.skip;
+    a.pre_mask = b.mask;
+    a.pre_kept = b.kept;
+    a.seq = b.seq;
+    if ((e = launch_select(a, g, s)) != cudaSuccess) return cuda_fail(e, "select kernel launch");
+    return RKV_OK;
+}
+
+RKV_API int rkv_eviction_error(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
+                               const float *out_kept, const float *dropped, float *err, void *ws, size_t ws_bytes,
+                               void *stream) {
+    if (!sel) return fail(RKV_ERR_INVALID_ARG, "rkv_eviction_error: sel is NULL");
+    if (!out_kept || !dropped || !err)
+        return fail(RKV_ERR_INVALID_ARG, "rkv_eviction_error: out_kept, dropped and err must be non-NULL");
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    WsLayout L;
+    if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
+    float *m_ev = at<float>(ws, L.ev_out);
+    // the evicted set's forced-weight output, then err = dm * ||m_ev - m_A||
+    if ((rc = attn_common(cache, q, scale, sel, m_ev, nullptr, nullptr, ws, ws_bytes, stream, "rkv_eviction_error",
+                          true)))
+        return rc;
+    const int64_t rows = (int64_t)cache->B * cache->Hq * cache->L;
+    cudaError_t e = launch_evict_err(m_ev, out_kept, dropped, err, rows, cache->D, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rkv_eviction_error");
+    return RKV_OK;
 }
 
 RKV_API int rkv_decode_step(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global, const float *q,

@@ -41,6 +41,12 @@ struct WsLayout {
     size_t hrec;          // float  [C][rec] state of whole heads that hold candidates
     size_t npre;          // int32  [C] pre-step lengths
     size_t pfx;           // int32  [C+1] page prefix of the pre-step lengths (own range of each CTA)
+    size_t ev_out;        // float  [C][G][D] output of the evicted set (eviction error)
+    size_t bmask;         // uint16 [C][max_pages] forced keep bits (ContourKV)
+    size_t bkept;         // int32  [C] forced counts (ContourKV)
+    size_t bfloor;        // int32  [C] oldest floor position (ContourKV)
+    size_t bskip;         // uint8  [C] flat heads (ContourKV)
+    size_t bseq;          // uint64 [B][2] forced entries, entries left to rank (ContourKV)
     size_t total;
 };
 
@@ -80,8 +86,44 @@ struct SelectArgs {
     uint32_t *more;
     uint32_t *hist;
     int n_groups, cta_per_group, waves, cache_pages;
+    // ContourKV's global part (all NULL otherwise): entries of heads with
+    // skip[c] set and entries at positions >= floor_pos[c] are left out of
+    // the ranking; pre_mask bits are ORed into the keep masks and pre_kept
+    // added to the kept counts; the budget is min(max(0, m_global[b] -
+    // seq[2b]), seq[2b+1]) (forced entries, entries left to rank); the
+    // threshold window is neither read nor updated.
+    const int32_t *floor_pos;
+    const uint8_t *skip;
+    const uint16_t *pre_mask;
+    const int32_t *pre_kept;
+    const unsigned long long *seq;
 };
 cudaError_t launch_select(const SelectArgs &a, const SelectGrid &g, cudaStream_t s);
+
+// Budget variants (budget.cu): one CTA per head.
+struct BudgetArgs {
+    const int32_t *pos_pool;
+    const float *lb_pool;
+    const int32_t *block_table;
+    const int32_t *len;
+    const int32_t *t;
+    int LH, C, G, max_pages;
+    int mode;                  // RKV_BUDGET_PER_HEAD / RKV_BUDGET_CONTOUR
+    const int32_t *m_head;     // [C] (per head)
+    const float *dm_prev;      // [C][G] (ContourKV)
+    float tau;
+    int32_t flat_budget, floor_r;
+    uint16_t *mask;            // keep masks (per head) / forced bits (ContourKV)
+    int32_t *kept;             // kept (per head) / forced counts (ContourKV)
+    int32_t *n_pre;            // per head
+    int32_t *floor_pos;        // ContourKV: [C] oldest floor position (INT_MAX: none)
+    uint8_t *skip;             // ContourKV: [C] flat heads
+    unsigned long long *seq;   // ContourKV: [B][2] forced, entries left to rank (zeroed before)
+    int32_t *status;
+};
+cudaError_t launch_head_budget(const BudgetArgs &a, cudaStream_t s);
+cudaError_t launch_plan(const int32_t *n_pre, const int32_t *kept, int32_t *plan, const int32_t *free_top,
+                        uint64_t *kappa, int C, int B, cudaStream_t s);
 
 // Fixed scratch of the allocation-free selection (a __device__ array in
 // select.cu): word offsets of its fields and its size.
@@ -117,6 +159,7 @@ struct AttnArgs {
     float *partial;
     int C, max_pages;
     float qscale;              // scale * log2(e)
+    int invert;                // 1: attend the evicted rows (keep_mask required, dropped NULL)
 };
 // Returns cudaErrorNotSupported if (dtype, D, G) is not instantiated.  bf16
 // pools are read through the two tensor maps (64-column boxes of 16 rows,
@@ -124,6 +167,9 @@ struct AttnArgs {
 cudaError_t launch_attn(const AttnArgs &a, int dtype, int D, int G, int sm_count, cudaStream_t s,
                         const CUtensorMap &tk, const CUtensorMap &tv);
 bool attn_supported(int dtype, int D, int G);
+// err[r] = dropped[r] * ||m_ev[r] - m_kept[r]|| for rows r < rows of D floats.
+cudaError_t launch_evict_err(const float *m_ev, const float *m_kept, const float *dropped, float *err, int64_t rows,
+                             int D, cudaStream_t s);
 bool attn_uses_tensor_maps(int dtype);
 size_t attn_partial_rec_floats(int D, int G);
 

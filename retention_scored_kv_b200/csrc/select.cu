@@ -83,6 +83,11 @@ __device__ __forceinline__ uint2 make_key(const SelectArgs &a, const SeqState &s
         set_status(a.status, RKV_DEV_BAD_INPUT);
         return make_uint2(KEY_INVALID, 0u);
     }
+    if (a.skip) {
+        // ContourKV's global part: flat heads and floor entries are not ranked
+        const int64_t c = (int64_t)st.b * a.LH + cl;
+        if (__ldg(a.skip + c) || pos >= __ldg(a.floor_pos + c)) return make_uint2(KEY_INVALID, 0u);
+    }
     float s = __fmul_rn((float)(int32_t)age, lb);
     if (s == 0.0f) s = 0.0f;
     return make_uint2(score_key_desc(s), (uint32_t)(((uint64_t)cl << a.ibits) | (uint32_t)pos));
@@ -329,7 +334,8 @@ __device__ void final_pass(const SelectArgs &a, const SelSmem &sm, const SeqStat
             const uint32_t m16 = (ball >> (lane & 16)) & 0xFFFFu;
             const int cl = head_of(a, sm, x, k);
             const int pidx = x - sm.pfx[cl];
-            a.keep_mask[((int64_t)st.b * a.LH + cl) * a.max_pages + pidx] = (uint16_t)m16;
+            const int64_t wi = ((int64_t)st.b * a.LH + cl) * a.max_pages + pidx;
+            a.keep_mask[wi] = (uint16_t)(a.pre_mask ? (m16 | __ldg(a.pre_mask + wi)) : m16);
             if (m16) atomicAdd(&sm.kc[cl], __popc(m16));
         }
     });
@@ -419,10 +425,16 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
             for (int cl = rr * blockDim.x + threadIdx.x; cl < a.LH; cl += a.cta_per_group * blockDim.x) {
                 const int64_t c = (int64_t)st.b * a.LH + cl;
                 a.n_pre[c] = sm.lens[cl];
-                a.kept[c] = 0;
+                a.kept[c] = a.pre_kept ? __ldg(a.pre_kept + c) : 0;
             }
             st.t = __ldg(a.t + st.b);
             int64_t m = __ldg(a.m_global + st.b);
+            if (a.seq) {
+                // the budget left after the forced entries, at most the entries left to rank
+                m -= (int64_t)__ldcg(a.seq + 2 * st.b);
+                const int64_t left = (int64_t)__ldcg(a.seq + 2 * st.b + 1);
+                if (m > left) m = left;
+            }
             st.m = m < 0 ? 0 : (m > st.n ? st.n : m);
             st.rank = (uint32_t)st.m;
             st.pk = 0;
@@ -431,7 +443,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
             st.kappa = st.m == 0 ? 0ull : ~0ull;
             {
                 const uint32_t *w = a.win + (size_t)st.b * 4;
-                st.wv = __ldcg(w) != 0u;
+                st.wv = !a.seq && __ldcg(w) != 0u;
                 st.wlo = __ldcg(w + 1);
                 st.whi = __ldcg(w + 2);
             }
@@ -500,7 +512,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) select_kernel(SelectArgs a) {
         if (wres != 0xFFFFFFFFu) {
             const uint64_t kap = __ldcg(a.kmax + b) + 1ull;
             a.kappa[b] = kap;
-            window_next(a.win + (size_t)b * 4, kap, (int)wres, __ldcg(a.cnt + (size_t)b * 4 + 3));
+            if (!a.seq) window_next(a.win + (size_t)b * 4, kap, (int)wres, __ldcg(a.cnt + (size_t)b * 4 + 3));
         }
         a.kmax[b] = 0ull;
     }

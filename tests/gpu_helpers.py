@@ -57,6 +57,23 @@ def assert_outputs_close(out, lse, dm, o_ref, lse_ref, dm_ref, kept_any):
         assert np.abs(np.asarray(dm, np.float64) - dm_ref.astype(np.float64)).max() <= DM_ATOL
 
 
+def assert_error_close(err, err_ref, dm_ref, m_kept_ref, m_ev_ref):
+    """Eviction error err = ||mu - m_A|| = dm * ||m_ev - m_A|| [C, G] against
+    the oracle.  The library forms it from its own m_ev, m_A (each within
+    OUT_RTOL of its row norm) and dm (within DM_ATOL), so the bound is
+    OUT_RTOL * dm * (||m_ev|| + ||m_A||) + DM_ATOL * ||m_ev - m_A|| (+1e-6)."""
+    err = np.asarray(err, np.float64)
+    ref = np.asarray(err_ref, np.float64)
+    m_k = np.asarray(m_kept_ref, np.float64)
+    m_e = np.asarray(m_ev_ref, np.float64)
+    dm = np.asarray(dm_ref, np.float64)
+    tol = (OUT_RTOL * dm * (np.linalg.norm(m_e, axis=-1) + np.linalg.norm(m_k, axis=-1))
+           + DM_ATOL * np.linalg.norm(m_e - m_k, axis=-1) + 1e-6)
+    bad = np.argwhere(np.abs(err - ref) > tol)
+    assert bad.size == 0, f"{len(bad)} rows out of tolerance, first {bad[:5].tolist()}: " \
+                          f"{[(float(err[tuple(i)]), float(ref[tuple(i)])) for i in bad[:3]]}"
+
+
 def compare_state(dc: workloads.DeviceCache, hc: oracle.HostCache, pools: bool = True):
     """Bit-exact comparison of a device cache with an oracle cache."""
     g = host_cache(dc) if pools else None

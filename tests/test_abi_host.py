@@ -30,6 +30,7 @@ def _declared_symbols():
 def test_header_declares_the_boundary():
     names = set(_declared_symbols())
     for want in ("rkv_score_select", "rkv_compact_pages", "rkv_paged_decode_attn", "rkv_dropped_mass",
+                 "rkv_eviction_error",
                  "rkv_append", "rkv_decode_step", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status",
                  "rkv_version", "rkv_last_error"):
         assert want in names
@@ -98,6 +99,12 @@ def test_small_workspace_and_null_arguments(lib):
     rc = so.rkv_dropped_mass(ctypes.byref(cs), ctypes.c_void_p(16), ctypes.c_float(0.1), None,
                              ctypes.c_void_p(16), ctypes.c_void_p(16), need, None)
     assert rc == rkv.ERR_INVALID_ARG and "sel" in so.rkv_last_error().decode()
+    rc = so.rkv_eviction_error(ctypes.byref(cs), ctypes.c_void_p(16), ctypes.c_float(0.1), None, ctypes.c_void_p(16),
+                               ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), need, None)
+    assert rc == rkv.ERR_INVALID_ARG and "sel" in so.rkv_last_error().decode()
+    rc = so.rkv_eviction_error(ctypes.byref(cs), ctypes.c_void_p(16), ctypes.c_float(0.1), ctypes.byref(sel), None,
+                               ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), need, None)
+    assert rc == rkv.ERR_INVALID_ARG and "out_kept" in so.rkv_last_error().decode()
     rc = so.rkv_append(ctypes.byref(cs), None, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16),
                        ctypes.c_void_p(16), need, None)
     assert rc == rkv.ERR_INVALID_ARG
