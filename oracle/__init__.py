@@ -93,6 +93,10 @@ def _load():
         lib.orc_select_contour.restype = ctypes.c_int
         lib.orc_select_contour.argtypes = [ctypes.POINTER(_Cache), P, P, P, ctypes.c_float, ctypes.c_int32,
                                            ctypes.c_int32, P, P, P]
+        lib.orc_memory_update.restype = ctypes.c_int
+        lib.orc_memory_update.argtypes = [ctypes.POINTER(_Cache), P, P, ctypes.c_double, P, P]
+        lib.orc_memory_read.restype = ctypes.c_int
+        lib.orc_memory_read.argtypes = [ctypes.POINTER(_Cache), P, P, P, P, P, P, P]
         lib.orc_eviction_error.restype = ctypes.c_int
         lib.orc_eviction_error.argtypes = [ctypes.POINTER(_Cache), P, ctypes.c_float, P, P, P]
         lib.orc_compact.restype = ctypes.c_int
@@ -260,6 +264,34 @@ def eviction_error(cache: HostCache, q: np.ndarray, scale: float, keep: np.ndarr
     if rc != OK:
         raise ValueError(f"oracle eviction error failed (code {rc})")
     return (err, mu) if with_dense else err
+
+
+def memory_update(cache: HostCache, keep: np.ndarray, proj: np.ndarray, decay: float, M: np.ndarray,
+                  b: np.ndarray) -> None:
+    """Latent memory update with this step's evicted entries, in place:
+    M [C, D, D], b [C, D] float64; proj [L, D, D] float32."""
+    assert M.dtype == np.float64 and b.dtype == np.float64 and M.flags["C_CONTIGUOUS"] and b.flags["C_CONTIGUOUS"]
+    keep = np.ascontiguousarray(keep, np.uint8)
+    proj = np.ascontiguousarray(proj, np.float32)
+    st = cache._struct()
+    rc = _load().orc_memory_update(ctypes.byref(st), _ptr(keep), _ptr(proj), float(decay), _ptr(M), _ptr(b))
+    if rc != OK:
+        raise ValueError(f"oracle memory update failed (code {rc})")
+
+
+def memory_read(cache: HostCache, q: np.ndarray, proj: np.ndarray, gate_w: np.ndarray, gate_b: np.ndarray,
+                M: np.ndarray, b: np.ndarray, out: np.ndarray) -> np.ndarray:
+    """out + g(q) * m(q) per query head (a new float32 [C, G, D] array);
+    gate_w [L, Hq, D], gate_b [L, Hq] float32."""
+    q = np.ascontiguousarray(q, np.float32).reshape(cache.C, cache.G, cache.D)
+    res = np.array(np.asarray(out, np.float32).reshape(cache.C, cache.G, cache.D), copy=True)
+    st = cache._struct()
+    rc = _load().orc_memory_read(ctypes.byref(st), _ptr(q), _ptr(np.ascontiguousarray(proj, np.float32)),
+                                 _ptr(np.ascontiguousarray(gate_w, np.float32)),
+                                 _ptr(np.ascontiguousarray(gate_b, np.float32)), _ptr(M), _ptr(b), _ptr(res))
+    if rc != OK:
+        raise ValueError(f"oracle memory read failed (code {rc})")
+    return res
 
 
 def compact(cache: HostCache, keep: np.ndarray) -> None:

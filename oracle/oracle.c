@@ -31,6 +31,9 @@
  *                 summed dense attention weight of the discarded keys.
  *               - Methodology 1: the eviction error ||mu - m_A|| between
  *                 the dense output and the forced-weight output.
+ *   [IndexMem]  "learned KV eviction with latent memory", Methodology B:
+ *               evicted tokens folded into a decayed outer-product state
+ *               that a gated read adds back to the attention output.
  *
  * Readings where the pages are silent:
  *   - score s = fl32(float(t - i) * log(beta_i)), one IEEE binary32 multiply
@@ -520,6 +523,102 @@ int orc_eviction_error(const orc_cache *cc, const float *q, float scale, const u
         free(ma);
     }
     return failed ? ORC_ERR_INPUT : ORC_OK;
+}
+
+/* -------------------------------------------------------- latent memory ---
+ * IndexMem ("learned KV eviction with latent memory"), Methodology B: the
+ * evicted tokens update a fixed-size state matrix M and a stabilising
+ * vector b online, by outer-product accumulation with decay (fast
+ * weights); learned projections and a gate g(q) read it (slow weights);
+ * the output is o = o_attn + g(q) * m(q).  Readings (the page gives no
+ * formulas; this is the linear-attention form those words describe):
+ *   - one state per KV head c: M_c [D][D], b_c [D];
+ *   - feature map phi(x) = elu(P_l x) + 1 with a per-layer projection P_l
+ *     [D][D] (D*D*L parameters: 0.5M for an 8B-class model, the size the
+ *     page quotes for the memory), elu(y) = y for y > 0, exp(y) - 1 else;
+ *   - update at an evicting step, with this step's evicted entries j of
+ *     head c:  M_c = decay * M_c + sum_j phi(k_j) v_j^T,
+ *              b_c = decay * b_c + sum_j phi(k_j);
+ *   - read for query head (c, g):  m = phi(q)^T M_c / (phi(q)^T b_c), and
+ *     m = 0 when phi(q)^T b_c = 0 (nothing ever evicted);
+ *   - gate g(q) = sigmoid(w_{l,hq} . q + beta_{l,hq});  out += g * m.
+ * The update runs after the selection and before compaction (the evicted
+ * rows are still in place); the read adds to the attention output. */
+static double phi_of(double y) { return y > 0.0 ? y + 1.0 : exp(y); }
+
+/* Features phi(P_l x) of one D-vector x (float or stored K element). */
+static void features(const float *P, const double *x, int32_t D, double *f) {
+    for (int32_t i = 0; i < D; i++) {
+        double y = 0.0;
+        for (int32_t d = 0; d < D; d++) y += (double)P[(int64_t)i * D + d] * x[d];
+        f[i] = phi_of(y);
+    }
+}
+
+int orc_memory_update(const orc_cache *cc, const uint8_t *keep, const float *proj, double decay, double *M,
+                      double *bvec) {
+    const int64_t C = n_heads(cc);
+    const int64_t LH = (int64_t)cc->L * cc->H;
+    const int64_t slots_per_head = (int64_t)cc->max_pages * cc->P;
+    const int32_t D = cc->D;
+    double *k = (double *)malloc((size_t)D * sizeof(double));
+    double *f = (double *)malloc((size_t)D * sizeof(double));
+    if (!k || !f) { free(k); free(f); return ORC_ERR_INPUT; }
+    for (int64_t c = 0; c < C; c++) {
+        const int32_t l = (int32_t)((c % LH) / cc->H);
+        const float *P = proj + (int64_t)l * D * D;
+        double *Mc = M + c * (int64_t)D * D, *bc = bvec + c * D;
+        for (int64_t e = 0; e < (int64_t)D * D; e++) Mc[e] *= decay;
+        for (int32_t i = 0; i < D; i++) bc[i] *= decay;
+        for (int32_t s = 0; s < cc->len[c]; s++) {
+            if (keep[c * slots_per_head + s]) continue;
+            const int64_t row = phys_row(cc, c, s);
+            for (int32_t d = 0; d < D; d++) k[d] = kv_elem(cc, cc->k_pool, row, d);
+            features(P, k, D, f);
+            for (int32_t i = 0; i < D; i++) {
+                bc[i] += f[i];
+                for (int32_t j = 0; j < D; j++) Mc[(int64_t)i * D + j] += f[i] * kv_elem(cc, cc->v_pool, row, j);
+            }
+        }
+    }
+    free(k);
+    free(f);
+    return ORC_OK;
+}
+
+int orc_memory_read(const orc_cache *cc, const float *q, const float *proj, const float *gate_w,
+                    const float *gate_b, const double *M, const double *bvec, float *out) {
+    const int64_t C = n_heads(cc);
+    const int64_t LH = (int64_t)cc->L * cc->H;
+    const int32_t D = cc->D, G = cc->G;
+    double *x = (double *)malloc((size_t)D * sizeof(double));
+    double *f = (double *)malloc((size_t)D * sizeof(double));
+    if (!x || !f) { free(x); free(f); return ORC_ERR_INPUT; }
+    for (int64_t c = 0; c < C; c++) {
+        const int32_t l = (int32_t)((c % LH) / cc->H);
+        const int32_t h = (int32_t)(c % cc->H);
+        const float *P = proj + (int64_t)l * D * D;
+        const double *Mc = M + c * (int64_t)D * D, *bc = bvec + c * D;
+        for (int32_t g = 0; g < G; g++) {
+            const float *qv = query_of(q, c, g, G, D);
+            const int64_t hq = (int64_t)l * cc->H * G + (int64_t)h * G + g;  /* query head of the layer */
+            for (int32_t d = 0; d < D; d++) x[d] = (double)qv[d];
+            features(P, x, D, f);
+            double den = 0.0, z = (double)gate_b[hq];
+            for (int32_t i = 0; i < D; i++) den += f[i] * bc[i];
+            for (int32_t d = 0; d < D; d++) z += (double)gate_w[hq * D + d] * x[d];
+            const double gate = 1.0 / (1.0 + exp(-z));
+            float *o = out + (c * G + g) * D;
+            for (int32_t j = 0; j < D; j++) {
+                double num = 0.0;
+                for (int32_t i = 0; i < D; i++) num += f[i] * Mc[(int64_t)i * D + j];
+                o[j] = (float)((double)o[j] + (den > 0.0 ? gate * num / den : 0.0));
+            }
+        }
+    }
+    free(x);
+    free(f);
+    return ORC_OK;
 }
 
 /* ------------------------------------------------------------ compaction ---

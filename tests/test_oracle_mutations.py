@@ -16,7 +16,8 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = ["tests/test_oracle_score.py", "tests/test_oracle_select.py", "tests/test_oracle_layout.py",
-        "tests/test_oracle_attention.py", "tests/test_oracle_error.py", "tests/test_oracle_budget.py"]
+        "tests/test_oracle_attention.py", "tests/test_oracle_error.py", "tests/test_oracle_budget.py",
+        "tests/test_oracle_memory.py"]
 
 # name: (text in oracle.c, replacement)
 MUTATIONS = {
@@ -74,6 +75,16 @@ MUTATIONS = {
     "flat_not_strict": ("const int flat = mean > tau;", "const int flat = mean >= tau;"),
     # ContourKV: the global part ignores what the floors and flat heads took
     "m_rest_ignores_forced": ("int64_t m = m_global[b] - forced;", "int64_t m = m_global[b];"),
+    # latent memory: no decay of the state
+    "memory_no_decay": ("        for (int64_t e = 0; e < (int64_t)D * D; e++) Mc[e] *= decay;\n", ""),
+    # latent memory: elu without the +1 (features may vanish or turn negative)
+    "memory_phi_without_one": ("return y > 0.0 ? y + 1.0 : exp(y);", "return y > 0.0 ? y : exp(y) - 1.0;"),
+    # latent memory: read not normalised by phi(q)^T b
+    "memory_read_unnormalised": ("gate * num / den", "gate * num"),
+    # latent memory: kept rows folded in instead of the evicted ones
+    "memory_kept_rows": ("if (keep[c * slots_per_head + s]) continue;", "if (!keep[c * slots_per_head + s]) continue;"),
+    # latent memory: gate without its bias
+    "memory_gate_no_bias": ("double den = 0.0, z = (double)gate_b[hq];", "double den = 0.0, z = 0.0;"),
     # compaction: freed pages pushed in descending table order
     "pushes_descending": ("for (int32_t pi = keep_pages; pi < old_pages; pi++) {",
                           "for (int32_t pi = old_pages - 1; pi >= keep_pages; pi--) {"),
