@@ -9,6 +9,8 @@
  *   [TRIM-KV]   "Cache What Lasts: Token Retention for Memory-Bounded KV
  *               Cache in LLMs"
  *   [ContourKV] "Trust the Mass: Forced Weights in KV-Cache Eviction"
+ *   [IndexMem]  "IndexMem: learned KV eviction with latent memory" (only
+ *               its latent memory for evicted tokens)
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -302,6 +304,47 @@ RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float sca
 RKV_API int rkv_eviction_error(const rkv_cache_t *cache, const float *q, float scale,
                                const rkv_select_t *sel, const float *out_kept, const float *dropped,
                                float *err, void *ws, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------
+ * Latent memory for evicted tokens ([IndexMem] "learned KV eviction with
+ * latent memory", Methodology B: evicted tokens update a fixed-size state M
+ * and a stabilising vector b online by outer-product accumulation with
+ * decay; a learned projection and a gate g(q) read it; the output is
+ * o = o_attn + g(q) * m(q)).  The page gives no formulas; this library's
+ * form, per KV head c of layer l:
+ *   phi(x) = elu(P_l x) + 1   (elu(y) = y for y > 0, exp(y) - 1 else)
+ *   update:  M_c = decay * M_c + sum_{j evicted} phi(k_j) v_j^T
+ *            b_c = decay * b_c + sum_{j evicted} phi(k_j)
+ *   read:    m = phi(q)^T M_c / (phi(q)^T b_c)   (0 when that is 0)
+ *            g = sigmoid(gate_w[l][hq] . q + gate_b[l][hq]);  out += g * m
+ * The slow weights are the caller's (random ones in this repository's
+ * benchmark); the state is the caller's, zero at the start of a sequence. */
+typedef struct rkv_memory {
+    const float *proj;    /* [L][D][D] projection P_l, row i gives feature i */
+    const float *gate_w;  /* [L][Hq][D] gate weights (read only) */
+    const float *gate_b;  /* [L][Hq] gate biases (read only) */
+    float decay;          /* in [0, 1], applied once per update call */
+    float *M;             /* [C][D][D] state, fp32, 16-byte aligned */
+    float *b;             /* [C][D] normaliser */
+} rkv_memory_t;
+
+/* rkv_memory_update -- fold this step's evicted entries (keep-mask bit clear
+ * among the first n_pre[c] slots) into the state.  Call it after the
+ * selection and before rkv_compact_pages (the rows are read in place).
+ *   sel   the step's selection (keep_mask, n_pre)
+ *   mem   host pointer; proj, decay, M, b used
+ * Errors: RKV_ERR_INVALID_ARG (NULL, decay outside [0, 1]), RKV_ERR_UNSUPPORTED
+ * (D not 64/128 or G > 8), RKV_ERR_CUDA.  One launch, one CTA per head. */
+RKV_API int rkv_memory_update(const rkv_cache_t *cache, const rkv_select_t *sel, const rkv_memory_t *mem,
+                              void *stream);
+
+/* rkv_memory_read -- add the gated memory read to the attention output:
+ * out[c][g][:] += g(q) * m(q) for every query row.
+ *   q     [C][G][D] float, the step's queries
+ *   out   [C][G][D] float, rkv_paged_decode_attn's output, updated in place
+ * Errors as rkv_memory_update.  One launch, one CTA per head. */
+RKV_API int rkv_memory_read(const rkv_cache_t *cache, const float *q, const rkv_memory_t *mem, float *out,
+                            void *stream);
 
 /* ---------------------------------------------------------------------------
  * rkv_compact_pages -- physically remove the evicted entries

@@ -7,7 +7,8 @@ raises.
 
 Entry points (same names as the C ABI, without the ``rkv_`` prefix):
 ``score_select``, ``score_select_budget`` (as ``score_select_per_head`` and
-``score_select_contour``), ``paged_decode_attn``, ``dropped_mass``, ``eviction_error``, ``compact_pages``,
+``score_select_contour``), ``paged_decode_attn``, ``dropped_mass``, ``eviction_error``,
+``memory_update``, ``memory_read``, ``compact_pages``,
 ``append``, ``decode_step``, ``workspace_size``, ``workspace_init``,
 ``device_status``, ``version``, ``last_error``.  ``Cache``/``Selection``/
 ``Workspace`` hold the tensors and build the C structs; ``step`` runs one
@@ -33,7 +34,8 @@ PAGE = 16
 
 EXPORTS = ("rkv_version", "rkv_last_error", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status",
            "rkv_score_select", "rkv_score_select_budget", "rkv_paged_decode_attn", "rkv_dropped_mass",
-           "rkv_eviction_error", "rkv_compact_pages", "rkv_append", "rkv_decode_step")
+           "rkv_eviction_error", "rkv_memory_update", "rkv_memory_read", "rkv_compact_pages", "rkv_append",
+           "rkv_decode_step")
 BUDGET_PER_HEAD, BUDGET_CONTOUR = 0, 1
 
 
@@ -59,6 +61,11 @@ class BudgetStruct(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("m_head", ctypes.c_void_p), ("m_global", ctypes.c_void_p),
                 ("dm_prev", ctypes.c_void_p), ("flat_threshold", ctypes.c_float), ("flat_budget", ctypes.c_int32),
                 ("recency_floor", ctypes.c_int32)]
+
+
+class MemoryStruct(ctypes.Structure):
+    _fields_ = [("proj", ctypes.c_void_p), ("gate_w", ctypes.c_void_p), ("gate_b", ctypes.c_void_p),
+                ("decay", ctypes.c_float), ("M", ctypes.c_void_p), ("b", ctypes.c_void_p)]
 
 
 _lib = None
@@ -87,6 +94,8 @@ def load(path: str | None = None):
         "rkv_paged_decode_attn": (I, [CP, P, ctypes.c_float, SP, P, P, P, P, SZ, P]),
         "rkv_dropped_mass": (I, [CP, P, ctypes.c_float, SP, P, P, SZ, P]),
         "rkv_eviction_error": (I, [CP, P, ctypes.c_float, SP, P, P, P, P, SZ, P]),
+        "rkv_memory_update": (I, [CP, SP, ctypes.POINTER(MemoryStruct), P]),
+        "rkv_memory_read": (I, [CP, P, ctypes.POINTER(MemoryStruct), P, P]),
         "rkv_compact_pages": (I, [CP, SP, P, SZ, P]),
         "rkv_append": (I, [CP, P, P, P, P, P, SZ, P]),
         "rkv_decode_step": (I, [CP, P, P, P, ctypes.c_float, P, P, P, SP, P, P, P, P, SZ, P]),
@@ -292,6 +301,39 @@ def eviction_error(cache: Cache, q: torch.Tensor, scale: float, sel: Selection, 
                                      _stream(stream)))
 
 
+@dataclass
+class Memory:
+    """Latent memory of the evicted tokens (rkv.h, rkv_memory_update/read):
+    slow weights (proj [L, D, D], gate_w [L, Hq, D], gate_b [L, Hq]) and the
+    state (M [C, D, D], b [C, D], zero for a fresh sequence), all float32."""
+    proj: torch.Tensor
+    gate_w: torch.Tensor
+    gate_b: torch.Tensor
+    M: torch.Tensor
+    b: torch.Tensor
+    decay: float = 0.99
+
+    @classmethod
+    def zeros(cls, cache: Cache, proj, gate_w, gate_b, decay: float = 0.99) -> "Memory":
+        dev = cache.len.device
+        return cls(proj, gate_w, gate_b, torch.zeros(cache.C, cache.D, cache.D, device=dev),
+                   torch.zeros(cache.C, cache.D, device=dev), decay)
+
+    def struct(self) -> MemoryStruct:
+        return MemoryStruct(_ptr(self.proj), _ptr(self.gate_w), _ptr(self.gate_b), float(self.decay), _ptr(self.M),
+                            _ptr(self.b))
+
+
+def memory_update(cache: Cache, sel: Selection, mem: Memory, stream=None):
+    cs, ss, ms = cache.struct(), sel.struct(), mem.struct()
+    _check(load().rkv_memory_update(ctypes.byref(cs), ctypes.byref(ss), ctypes.byref(ms), _stream(stream)))
+
+
+def memory_read(cache: Cache, q: torch.Tensor, mem: Memory, out: torch.Tensor, stream=None):
+    cs, ms = cache.struct(), mem.struct()
+    _check(load().rkv_memory_read(ctypes.byref(cs), _ptr(q), ctypes.byref(ms), _ptr(out), _stream(stream)))
+
+
 def compact_pages(cache: Cache, sel: Selection, ws: Workspace, stream=None):
     cs, ss = cache.struct(), sel.struct()
     _check(load().rkv_compact_pages(ctypes.byref(cs), ctypes.byref(ss), ctypes.c_void_p(ws.ptr), ws.nbytes,
@@ -332,30 +374,38 @@ class StepOutputs:
 
 def step(cache: Cache, sel: Selection, ws: Workspace, outs: StepOutputs, *, q, t, m_global, k_new, v_new,
          lb_new, evict: bool = True, scale: float | None = None, fused: bool = False, stream=None,
-         err: torch.Tensor | None = None):
+         err: torch.Tensor | None = None, mem: Memory | None = None):
     """One decode step: [select] -> attention + dropped mass -> [eviction
     error] -> [compaction] -> append.
 
     On a non-evicting step every entry is kept and the dropped mass is 0.
     ``fused`` runs the whole step as one ``decode_step`` launch; ``err``
     ([B, L, Hq] float32) asks for the eviction error of an evicting step,
-    which the separate calls provide (not the fused launch)."""
+    which the separate calls provide (not the fused launch); ``mem`` folds
+    the evicted tokens into the latent memory and adds its gated read to
+    the output (separate calls as well)."""
     if scale is None:
         scale = 1.0 / math.sqrt(cache.D)
-    if err is not None and fused:
-        raise ValueError("the eviction error comes from the separate calls (fused=False)")
+    if (err is not None or mem is not None) and fused:
+        raise ValueError("the eviction error and the latent memory come from the separate calls (fused=False)")
     if fused:
         decode_step(cache, t, m_global if evict else None, q, scale, k_new, v_new, lb_new, sel if evict else None,
                     outs.out, outs.lse, outs.dropped, ws, stream)
         return
     if evict:
         score_select(cache, t, m_global, sel, ws, stream)
+        if mem is not None:
+            memory_update(cache, sel, mem, stream)
         paged_decode_attn(cache, q, scale, sel, outs.out, outs.lse, outs.dropped, ws, stream)
         if err is not None:
             eviction_error(cache, q, scale, sel, outs.out, outs.dropped, err, ws, stream)
+        if mem is not None:
+            memory_read(cache, q, mem, outs.out, stream)
         compact_pages(cache, sel, ws, stream)
     else:
         paged_decode_attn(cache, q, scale, None, outs.out, outs.lse, outs.dropped, ws, stream)
+        if mem is not None:
+            memory_read(cache, q, mem, outs.out, stream)
     append(cache, t, k_new, v_new, lb_new, ws, stream)
 
 

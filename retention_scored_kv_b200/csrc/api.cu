@@ -488,6 +488,66 @@ RKV_API int rkv_score_select_budget(const rkv_cache_t *cache, const int32_t *t, 
     return RKV_OK;
 }
 
+static int check_memory(const rkv_cache_t *cache, const rkv_memory_t *mem, const char *what) {
+    if (!mem || !mem->proj || !mem->M || !mem->b)
+        return fail(RKV_ERR_INVALID_ARG, "%s: memory, proj, M and b must be non-NULL", what);
+    if (!aligned16(mem->M)) return fail(RKV_ERR_INVALID_ARG, "%s: M must be 16-byte aligned", what);
+    if (!memory_supported(cache->D, cache->Hq / cache->H))
+        return fail(RKV_ERR_UNSUPPORTED, "%s: D %d, G %d not built", what, cache->D, cache->Hq / cache->H);
+    return RKV_OK;
+}
+
+RKV_API int rkv_memory_update(const rkv_cache_t *cache, const rkv_select_t *sel, const rkv_memory_t *mem,
+                              void *stream) {
+    int rc = check_cache(cache, true);
+    if (rc) return rc;
+    if ((rc = check_sel(sel))) return rc;
+    if ((rc = check_memory(cache, mem, "rkv_memory_update"))) return rc;
+    if (!(mem->decay >= 0.0f && mem->decay <= 1.0f))
+        return fail(RKV_ERR_INVALID_ARG, "rkv_memory_update: decay must be in [0, 1]");
+    MemUpdateArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.block_table = cache->block_table;
+    a.n_pre = sel->n_pre;
+    a.keep_mask = sel->keep_mask;
+    a.proj = mem->proj;
+    a.decay = mem->decay;
+    a.M = mem->M;
+    a.b = mem->b;
+    a.C = cache->B * cache->L * cache->H;
+    a.LH = cache->L * cache->H;
+    a.H = cache->H;
+    a.max_pages = cache->max_pages;
+    cudaError_t e = launch_memory_update(a, cache->dtype, cache->D, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rkv_memory_update");
+    return RKV_OK;
+}
+
+RKV_API int rkv_memory_read(const rkv_cache_t *cache, const float *q, const rkv_memory_t *mem, float *out,
+                            void *stream) {
+    int rc = check_cache(cache, false);
+    if (rc) return rc;
+    if (!q || !out) return fail(RKV_ERR_INVALID_ARG, "rkv_memory_read: q / out is NULL");
+    if ((rc = check_memory(cache, mem, "rkv_memory_read"))) return rc;
+    if (!mem->gate_w || !mem->gate_b) return fail(RKV_ERR_INVALID_ARG, "rkv_memory_read: gate_w / gate_b is NULL");
+    MemReadArgs a{};
+    a.q = q;
+    a.proj = mem->proj;
+    a.gate_w = mem->gate_w;
+    a.gate_b = mem->gate_b;
+    a.M = mem->M;
+    a.b = mem->b;
+    a.out = out;
+    a.C = cache->B * cache->L * cache->H;
+    a.LH = cache->L * cache->H;
+    a.H = cache->H;
+    a.Hq = cache->Hq;
+    cudaError_t e = launch_memory_read(a, cache->D, cache->Hq / cache->H, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rkv_memory_read");
+    return RKV_OK;
+}
+
 RKV_API int rkv_eviction_error(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
                                const float *out_kept, const float *dropped, float *err, void *ws, size_t ws_bytes,
                                void *stream) {

@@ -227,6 +227,33 @@ size_t step_smem_bytes(int dtype, int D, int G, int max_pages);
 cudaError_t launch_step(const StepArgs &a, int dtype, int D, int G, int grid, cudaStream_t s,
                         const CUtensorMap &tk, const CUtensorMap &tv);
 
+// Latent memory (memory.cu).
+struct MemUpdateArgs {
+    const void *k_pool;
+    const void *v_pool;
+    const int32_t *block_table;
+    const int32_t *n_pre;
+    const uint16_t *keep_mask;
+    const float *proj;         // [L][D][D]
+    float decay;
+    float *M;                  // [C][D][D]
+    float *b;                  // [C][D]
+    int C, LH, H, max_pages;
+};
+struct MemReadArgs {
+    const float *q;            // [C][G][D]
+    const float *proj;         // [L][D][D]
+    const float *gate_w;       // [L][Hq][D]
+    const float *gate_b;       // [L][Hq]
+    const float *M;
+    const float *b;
+    float *out;                // [C][G][D], added to
+    int C, LH, H, Hq;
+};
+bool memory_supported(int D, int G);
+cudaError_t launch_memory_update(const MemUpdateArgs &a, int dtype, int D, cudaStream_t s);
+cudaError_t launch_memory_read(const MemReadArgs &a, int D, int G, cudaStream_t s);
+
 struct CompactArgs {
     void *k_pool;
     void *v_pool;

@@ -174,6 +174,17 @@ def step_inputs(cfg: Config, seed: int, step: int, device="cpu") -> dict:
     return dict(q=q, k_new=k_new, v_new=v_new, lb_new=lb_new, t=t, m_global=m, evict=cfg.evicts(step))
 
 
+def memory_weights(cfg: Config, seed: int, device="cpu") -> dict:
+    """Synthetic slow weights of the latent memory (no trained ones exist
+    here): proj [L, D, D] ~ N(0, 1/D), gate_w [L, Hq, D] ~ N(0, 1/D),
+    gate_b [L, Hq] ~ N(0, 1), float32."""
+    g = _gen(device, seed, "memory")
+    s = 1.0 / math.sqrt(cfg.D)
+    return dict(proj=torch.randn(cfg.L, cfg.D, cfg.D, generator=g, device=device) * s,
+                gate_w=torch.randn(cfg.L, cfg.Hq, cfg.D, generator=g, device=device) * s,
+                gate_b=torch.randn(cfg.L, cfg.Hq, generator=g, device=device))
+
+
 def pool_geometry(cfg: Config, n_steps: int) -> tuple[int, int, int]:
     """(P0, n_pages, max_pages) for a run of n_steps decode steps."""
     P0 = -(-cfg.T0 // cfg.P)
