@@ -34,7 +34,9 @@ per-kernel CUDA events inside the graph split each step into its kernels.
 The dominant kernel's algorithmic bytes over its duration is the roofline
 entry.  e2e repeats the headline measurement through the public API with
 packed pinned host inputs and outputs (one H2D + graph replay + one D2H per
-step).  cpu_baseline times the CPU oracle on whole steady-state steps of the
+step).  "variants" times the eviction error, the latent memory and the
+per-head / ContourKV selections on steady llama32k steps through the
+separate calls.  cpu_baseline times the CPU oracle on whole steady-state steps of the
 headline workload on the host cores (one step single-threaded, two on every
 core).  ``--impl reference`` times the oracle alone on whole steps, every
 core.
@@ -587,6 +589,115 @@ def run_e2e(runner, per_step, s_next, W, K, stream, world, local, dev):
     return rec, s_next + W + K, clk2.summary()
 
 
+def run_variants(args, world: int, rank: int, local: int) -> dict:
+    """The rows beyond the default step, measured on steady llama32k decode
+    steps through the separate calls (one CUDA graph of K steps with an
+    event after every launch): the eviction error, the latent-memory update
+    and read, and the per-head and ContourKV selections (run on the same
+    pre-step cache into their own selection buffers).  Each reports its
+    device time and its algorithmic bytes against the HBM peak."""
+    import retention_scored_kv_b200 as rkv
+    cfg = workload_config("llama32k", args.layers)
+    dev = torch.device("cuda", local)
+    seed = args.seed + 1000 * rank + 7
+    K, W = args.steps, args.warmup
+    total = 1 + W + K + 2
+    dc = workloads.prefill_cache(cfg, seed, device=dev, n_steps=total)
+    cache = rkv.Cache.from_tensors(dc, cfg.B, cfg.L, cfg.H, cfg.Hq)
+    stream = torch.cuda.Stream(device=dev)
+    sel, ws, outs = rkv.Selection.empty(cache), rkv.Workspace(cache, stream), rkv.StepOutputs.empty(cache)
+    sel_h, sel_c = rkv.Selection.empty(cache), rkv.Selection.empty(cache)
+    wts = workloads.memory_weights(cfg, seed, dev)
+    mem = rkv.Memory.zeros(cache, wts["proj"], wts["gate_w"], wts["gate_b"], 0.99)
+    err = torch.empty(cfg.B, cfg.L, cfg.Hq, device=dev)
+    per_step = [workloads.step_inputs(cfg, seed, s, dev) for s in range(total)]
+    m_head = torch.full((cfg.C,), cfg.M // cfg.C, dtype=torch.int32, device=dev)
+    dm_prev = torch.zeros(cfg.B, cfg.L, cfg.Hq, device=dev)
+    tau, flat_budget, floor = 2e-4, 2048, 64
+    names = ["per_head_select", "contour_select", "select", "memory_update", "attn", "eviction_error",
+             "memory_read", "compact", "append"]
+
+    def enqueue(s, ev=None):
+        i = per_step[s]
+        calls = [
+            lambda: rkv.score_select_per_head(cache, i["t"], m_head, sel_h, ws, stream),
+            lambda: rkv.score_select_contour(cache, i["t"], i["m_global"], dm_prev, tau, flat_budget, floor, sel_c,
+                                             ws, stream),
+            lambda: rkv.score_select(cache, i["t"], i["m_global"], sel, ws, stream),
+            lambda: rkv.memory_update(cache, sel, mem, stream),
+            lambda: rkv.paged_decode_attn(cache, i["q"], cfg.scale, sel, outs.out, outs.lse, outs.dropped, ws,
+                                          stream),
+            lambda: rkv.eviction_error(cache, i["q"], cfg.scale, sel, outs.out, outs.dropped, err, ws, stream),
+            lambda: rkv.memory_read(cache, i["q"], mem, outs.out, stream),
+            lambda: rkv.compact_pages(cache, sel, ws, stream),
+            lambda: rkv.append(cache, i["t"], i["k_new"], i["v_new"], i["lb_new"], ws, stream),
+        ]
+        if ev is not None:
+            ev[0].record(stream)
+        for j, f in enumerate(calls):
+            f()
+            if ev is not None:
+                ev[j + 1].record(stream)
+        dm_prev.copy_(outs.dropped)  # the next step's ContourKV statistic
+
+    with torch.cuda.stream(stream):
+        # step 0 (prefill eviction) and warm-up through the fused launch
+        for s in range(1 + W):
+            i = per_step[s]
+            rkv.decode_step(cache, i["t"], i["m_global"], i["q"], cfg.scale, i["k_new"], i["v_new"], i["lb_new"],
+                            sel, outs.out, outs.lse, outs.dropped, ws, stream)
+        for s in range(1 + W, 1 + W + 2):
+            enqueue(s)   # loads the variants' kernels
+    torch.cuda.synchronize()
+    first = 1 + W + 2
+    Kv = min(K, total - first)
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)] for _ in range(Kv)]
+    graph = capture(lambda: [enqueue(first + i, evs[i]) for i in range(Kv)], stream, args.no_graph)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(Kv):
+                enqueue(first + i, evs[i])
+    torch.cuda.synchronize()
+    if ws.status() != 0:
+        raise RuntimeError(f"variants: device status {ws.counters()}")
+    us = {n: 1000.0 * statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(Kv))
+          for j, n in enumerate(names)}
+    us = {n: max_over_ranks(v, world, dev) for n, v in us.items()}
+    del graph
+    # algorithmic bytes of the last step (steady state)
+    e = elt(cfg)
+    n_pre = int(sel.n_pre.sum().item())
+    kept = int(sel.kept.sum().item())
+    pages = int(((sel.n_pre + 15) // 16).sum().item())
+    evicted = n_pre - kept
+    rows_q = cfg.C * cfg.G
+    state = cfg.C * (cfg.D * cfg.D + cfg.D) * 4
+    proj = cfg.L * cfg.D * cfg.D * 4
+    sel_bytes = 8 * n_pre + 6 * pages + 12 * cfg.C
+    byts = {
+        "per_head_select": sel_bytes,
+        "contour_select": sel_bytes + 4 * rows_q,
+        "eviction_error": 2 * e * cfg.D * evicted + 6 * pages + 2 * 4 * rows_q * cfg.D + 3 * 4 * rows_q,
+        "memory_update": 2 * e * cfg.D * evicted + 6 * pages + 2 * state + proj,
+        "memory_read": state + proj + 3 * 4 * rows_q * cfg.D + 4 * cfg.L * cfg.Hq * (cfg.D + 1),
+    }
+    peak = _peaks()["hbm_gbs"]
+    out = {}
+    for n, b in byts.items():
+        gbs = b / (us[n] * 1e-6) / 1e9
+        out[n] = {"us": us[n], "bytes": b, "achieved_gbs": gbs, "frac": gbs / peak}
+    out["context"] = {"workload": describe(cfg), "evicted_per_step": evicted, "steps": Kv,
+                      "timing": "CUDA events after every launch inside one graph of K separate-call steps",
+                      "other_kernels_us": {n: us[n] for n in ("select", "attn", "compact", "append")},
+                      "contour": {"flat_threshold": tau, "flat_budget": flat_budget, "recency_floor": floor,
+                                  "flat_heads": int((dm_prev.view(cfg.C, cfg.G).mean(dim=1) > tau).sum().item())},
+                      "per_head_budget": cfg.M // cfg.C}
+    return out
+
+
 def describe(cfg: workloads.Config) -> str:
     sched = "every step evicts" if cfg.evict_every == 1 else f"evicts every {cfg.evict_every} steps"
     return (f"{cfg.name}: L{cfg.L} H{cfg.H} Hq{cfg.Hq} D{cfg.D} B{cfg.B} T0 {cfg.T0} M {cfg.M} per sequence, "
@@ -618,6 +729,10 @@ def run_rkv(args, world, rank, local):
         per[name] = summary(r)
         del r
         torch.cuda.empty_cache()
+    variants = None
+    if not args.skip_variants:
+        variants = run_variants(args, world, rank, local)
+        torch.cuda.empty_cache()
     cfg = head["cfg"]
 
     cpu = None
@@ -643,7 +758,7 @@ def run_rkv(args, world, rank, local):
         "step0": head["step0"], "cpu_baseline": cpu, "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
         "clocks": merge_clocks([head["clocks"]] + [p["clocks"] for p in per.values()]),
         "path": args.path, "selection": head["selection"], "head_lengths": head["head_lengths"],
-        "dropped_mass": head["dropped_mass"], "per_config": per,
+        "dropped_mass": head["dropped_mass"], "per_config": per, "variants": variants,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -744,6 +859,8 @@ def main(argv=None):
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-variants", action="store_true",
+                    help="skip the eviction-error, latent-memory and budget-variant timings")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the timed kernel for this workload (null if not measured)")
     args = ap.parse_args(argv)

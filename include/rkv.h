@@ -72,7 +72,7 @@ extern "C" {
 #define RKV_DEV_BAD_INPUT 1      /* NaN log-retention, age t-i outside [1, 2^24), position too wide */
 #define RKV_DEV_POOL_EXHAUSTED 2 /* append found the free-page stack empty */
 #define RKV_DEV_TABLE_OVERFLOW 4 /* append past max_pages of a head */
-#define RKV_DEV_TIMEOUT 8        /* a grid-wide barrier gave up after ~2 s */
+#define RKV_DEV_TIMEOUT 8        /* a bounded wait gave up (2 s, or the workspace's wait limit) */
 
 /* ---- element types of the K/V pools ---- */
 #define RKV_BF16 0
@@ -139,13 +139,24 @@ RKV_API size_t rkv_workspace_size(const rkv_cache_t *cache);
  * allocating it, and again after a nonzero device status. */
 RKV_API int rkv_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
-/* Device address of the status block inside the workspace: int32[4] =
+/* Device address of the status block inside the workspace: int32[5] =
  *   [0] RKV_DEV_* bits (sticky until rkv_workspace_init)
  *   [1] site of the first bounded wait that gave up (0: none), for reports
  *   [2] rkv_decode_step calls whose selection was resolved in the threshold
- *       window, [3] those that ran the exact selection (cumulative counters).
+ *       window, [3] those that ran the exact selection (cumulative counters)
+ *   [4] the wait limit set by rkv_workspace_set_wait_limit (0: default).
  * Pure pointer arithmetic. */
 RKV_API int32_t *rkv_device_status(void *ws);
+
+/* Limit, in microseconds, of the kernels' waits on other CTAs of the same
+ * launch (grid-wide barriers, the fused step's wait for the compactions
+ * before a pop) for calls on this workspace; 0 restores the default of 2 s.
+ * A wait that runs out records RKV_DEV_TIMEOUT and its site, and the CTA
+ * leaves the kernel; the workspace must then be re-initialised and the
+ * cache contents are unspecified.  Waits of a CTA on its own asynchronous
+ * copies keep the 2 s guard.  A tiny limit makes the timeout path run on
+ * purpose, without any hang.  Enqueued on `stream` (one small launch). */
+RKV_API int rkv_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint32_t microseconds, void *stream);
 
 /* ---------------------------------------------------------------------------
  * rkv_score_select -- score every cached entry and find the global top-M.
@@ -289,17 +300,18 @@ RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float sca
  * ([ContourKV] Methodology 1, theoretical analysis: the eviction error of a
  * kept subset A).  Computed as dm * || m_ev - m_A ||, with m_ev the
  * forced-weight output over the evicted entries (mu is the dm-weighted mix
- * of m_ev and m_A): the evicted rows' K and V are read, pages with no
- * evicted row are not.  Call it after rkv_paged_decode_attn of the same step
- * (whose out and dropped it takes) and before rkv_compact_pages.
+ * of m_ev and m_A): only the evicted rows' K and V and the keep words are
+ * read.  Call it after rkv_paged_decode_attn of the same step (whose out
+ * and dropped it takes) and before rkv_compact_pages.
  *   q, scale    as rkv_paged_decode_attn
  *   sel         the step's selection (keep masks), non-NULL
  *   out_kept    [C][G][D] float: m_A, rkv_paged_decode_attn's out
  *   dropped     [C][G] float: that call's dropped mass
  *   err         [C][G] float   written (0 where nothing is evicted; ||mu||
  *               where nothing is kept)
- * Uses the workspace's scratch (an evicted-set output of C*G*D floats).
- * Errors as rkv_paged_decode_attn.
+ * ws, ws_bytes are checked like the other calls' but not written.
+ * Errors: RKV_ERR_INVALID_ARG, RKV_ERR_UNSUPPORTED ((D, G) not built: D 64 or
+ * 128 with G in {1, 2, 4, 7, 8}), RKV_ERR_WORKSPACE_TOO_SMALL, RKV_ERR_CUDA.
  */
 RKV_API int rkv_eviction_error(const rkv_cache_t *cache, const float *q, float scale,
                                const rkv_select_t *sel, const float *out_kept, const float *dropped,

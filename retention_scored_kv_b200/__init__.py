@@ -33,6 +33,7 @@ BF16, F32 = 0, 1
 PAGE = 16
 
 EXPORTS = ("rkv_version", "rkv_last_error", "rkv_workspace_size", "rkv_workspace_init", "rkv_device_status",
+           "rkv_workspace_set_wait_limit",
            "rkv_score_select", "rkv_score_select_budget", "rkv_paged_decode_attn", "rkv_dropped_mass",
            "rkv_eviction_error", "rkv_memory_update", "rkv_memory_read", "rkv_compact_pages", "rkv_append",
            "rkv_decode_step")
@@ -89,6 +90,7 @@ def load(path: str | None = None):
         "rkv_workspace_size": (SZ, [CP]),
         "rkv_workspace_init": (I, [P, SZ, P]),
         "rkv_device_status": (P, [P]),
+        "rkv_workspace_set_wait_limit": (I, [P, SZ, ctypes.c_uint32, P]),
         "rkv_score_select": (I, [CP, P, P, SP, P, SZ, P]),
         "rkv_score_select_budget": (I, [CP, P, ctypes.POINTER(BudgetStruct), SP, P, SZ, P]),
         "rkv_paged_decode_attn": (I, [CP, P, ctypes.c_float, SP, P, P, P, P, SZ, P]),
@@ -242,6 +244,12 @@ def workspace_size(cache: Cache) -> int:
 
 def workspace_init(ws: Workspace, stream=None):
     _check(load().rkv_workspace_init(ctypes.c_void_p(ws.ptr), ws.nbytes, _stream(stream)))
+
+
+def workspace_set_wait_limit(ws: Workspace, microseconds: int, stream=None):
+    """Limit of the waits on other CTAs for calls on this workspace (0: 2 s)."""
+    _check(load().rkv_workspace_set_wait_limit(ctypes.c_void_p(ws.ptr), ws.nbytes, int(microseconds),
+                                               _stream(stream)))
 
 
 def device_status(ws: Workspace) -> int:

@@ -83,7 +83,7 @@ void layout_for(const rkv_cache_t &c, int sel_groups_x_waves, WsLayout *L) {
         off += bytes;
         return at;
     };
-    L->status = take(16, 16);  // bits, first timeout site, fused steps resolved in the window / exactly
+    L->status = take(32, 16);  // bits, first timeout site, fused steps in the window / exact, wait limit
     L->done_compact = take(4, 4);
     L->done_append = take(4, 4);
     L->bar = take(4, 64);
@@ -113,7 +113,6 @@ void layout_for(const rkv_cache_t &c, int sel_groups_x_waves, WsLayout *L) {
     L->hrec = take((size_t)SC * attn_partial_rec_floats(c.D, G) * 4, 256);
     L->npre = take((size_t)SC * 4, 256);
     L->pfx = take((size_t)(SC + 1) * 4, 256);
-    L->ev_out = take((size_t)C * G * c.D * 4, 256);
     L->bmask = take((size_t)C * c.max_pages * 2, 256);
     L->bkept = take((size_t)C * 4, 256);
     L->bfloor = take((size_t)C * 4, 256);
@@ -209,6 +208,15 @@ RKV_API int rkv_workspace_init(void *ws, size_t ws_bytes, void *stream) {
 }
 
 RKV_API int32_t *rkv_device_status(void *ws) { return ws ? reinterpret_cast<int32_t *>(ws) : nullptr; }
+
+RKV_API int rkv_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint32_t microseconds, void *stream) {
+    if (!ws || ws_bytes < 32) return fail(RKV_ERR_INVALID_ARG, "workspace is NULL or too small");
+    if (microseconds > 0x7FFFFFFFu) return fail(RKV_ERR_INVALID_ARG, "wait limit above 2^31 - 1 microseconds");
+    cudaError_t e = launch_set_word(reinterpret_cast<int32_t *>(ws) + 4, (int32_t)microseconds,
+                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "rkv_workspace_set_wait_limit");
+    return RKV_OK;
+}
 
 RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
                              const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream) {
@@ -331,7 +339,7 @@ RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t,
 
 static int attn_common(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
                        float *out, float *lse, float *dropped, void *ws, size_t ws_bytes, void *stream,
-                       const char *what, bool invert = false) {
+                       const char *what) {
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if (!q) return fail(RKV_ERR_INVALID_ARG, "%s: q is NULL", what);
@@ -360,7 +368,6 @@ static int attn_common(const rkv_cache_t *cache, const float *q, float scale, co
     a.C = cache->B * cache->L * cache->H;
     a.max_pages = cache->max_pages;
     a.qscale = scale * 1.4426950408889634f;
-    a.invert = invert ? 1 : 0;
     CUtensorMap tk{}, tv{};
     if (attn_uses_tensor_maps(cache->dtype)) {
         if ((rc = encode_pool_map(&tk, cache->k_pool, cache->D, cache->n_pages))) return rc;
@@ -552,19 +559,28 @@ RKV_API int rkv_eviction_error(const rkv_cache_t *cache, const float *q, float s
                                const float *out_kept, const float *dropped, float *err, void *ws, size_t ws_bytes,
                                void *stream) {
     if (!sel) return fail(RKV_ERR_INVALID_ARG, "rkv_eviction_error: sel is NULL");
-    if (!out_kept || !dropped || !err)
-        return fail(RKV_ERR_INVALID_ARG, "rkv_eviction_error: out_kept, dropped and err must be non-NULL");
+    if (!out_kept || !dropped || !err || !q)
+        return fail(RKV_ERR_INVALID_ARG, "rkv_eviction_error: q, out_kept, dropped and err must be non-NULL");
     int rc = check_cache(cache, true);
     if (rc) return rc;
+    if ((rc = check_sel(sel))) return rc;
     WsLayout L;
     if ((rc = check_ws(cache, ws, ws_bytes, &L))) return rc;
-    float *m_ev = at<float>(ws, L.ev_out);
-    // the evicted set's forced-weight output, then err = dm * ||m_ev - m_A||
-    if ((rc = attn_common(cache, q, scale, sel, m_ev, nullptr, nullptr, ws, ws_bytes, stream, "rkv_eviction_error",
-                          true)))
-        return rc;
-    const int64_t rows = (int64_t)cache->B * cache->Hq * cache->L;
-    cudaError_t e = launch_evict_err(m_ev, out_kept, dropped, err, rows, cache->D, static_cast<cudaStream_t>(stream));
+    const int G = cache->Hq / cache->H;
+    EvictErrArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.block_table = cache->block_table;
+    a.n_pre = sel->n_pre;
+    a.keep_mask = sel->keep_mask;
+    a.q = q;
+    a.out_kept = out_kept;
+    a.dropped = dropped;
+    a.err = err;
+    a.scale = scale;
+    a.C = cache->B * cache->L * cache->H;
+    a.max_pages = cache->max_pages;
+    cudaError_t e = launch_evict_err(a, cache->dtype, cache->D, G, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "rkv_eviction_error");
     return RKV_OK;
 }

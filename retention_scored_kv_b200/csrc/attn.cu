@@ -27,10 +27,6 @@
 // * Head boundaries: warps merge through shared memory; a head split across
 //   CTAs writes partial (max, sum, acc) records and the last CTA to arrive
 //   (atomic counter, no waiting) merges them -- the cross-split combine.
-// * Evicted-set mode (the eviction error): the evicted rows of each page are
-//   attended instead of the kept ones, pages without an evicted row pass
-//   through the ring without a copy, and no dropped mass is formed; a small
-//   kernel then turns the evicted set's output into the error.
 #include <cuda.h>
 
 #include "attn_core.cuh"
@@ -169,9 +165,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                     const uint32_t valid = nv >= PAGE ? 0xFFFFu : ((1u << nv) - 1u);
                     const uint32_t kp = a.keep_mask ? (uint32_t)__ldg(a.keep_mask + (int64_t)c * a.max_pages + pidx)
                                                     : 0xFFFFu;
-                    // evicted-set mode: the evicted rows are the ones attended
-                    // and nothing else is read (no dropped mass)
-                    m = a.invert ? (~kp & valid) : ((kp & valid) | (valid << 16));
+                    m = (kp & valid) | (valid << 16);
                 }
                 uint32_t todo = __ballot_sync(0xFFFFFFFFu, mine);
                 while (todo) {
@@ -186,16 +180,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                         const int sg = cw * LY::NSW + (int)(nw % LY::NSW);
                         mbar_wait(&empty[sg], (uint32_t)((nw / LY::NSW) & 1) ^ 1u, a.status);
                         meta[sg] = mj;
-                        if (mj == 0u) {
-                            // no row of this page is read (evicted-set mode
-                            // only): the stage passes through empty
-                            mbar_arrive(&full[sg]);
-                        } else {
-                            const bool load_v = WITH_V && (mj & 0xFFFFu);
-                            mbar_arrive_expect_tx(&full[sg], M::PAGE_BYTES * (load_v ? 2 : 1));
-                            M::issue(smem + LY::OFF_STAGE + sg * LY::STAGE_BYTES, load_v, pj, &full[sg], a.k_pool,
-                                     a.v_pool, &tmk, &tmv, pol_kv);
-                        }
+                        const bool load_v = WITH_V && (mj & 0xFFFFu);
+                        mbar_arrive_expect_tx(&full[sg], M::PAGE_BYTES * (load_v ? 2 : 1));
+                        M::issue(smem + LY::OFF_STAGE + sg * LY::STAGE_BYTES, load_v, pj, &full[sg], a.k_pool,
+                                 a.v_pool, &tmk, &tmv, pol_kv);
                     }
                     __syncwarp();
                 }
@@ -245,7 +233,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             const uint32_t mt = meta[sg];
             const uint32_t keepm = mt & 0xFFFFu, evm = (mt >> 16) & ~keepm;
             const unsigned char *sk = smem + LY::OFF_STAGE + sg * LY::STAGE_BYTES;
-            if (mt != 0u) M::page(st, sk, sk + M::PAGE_BYTES, keepm, evm, lane);
+            M::page(st, sk, sk + M::PAGE_BYTES, keepm, evm, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[sg]);
         }
@@ -347,27 +335,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     }
 }
 
-// Eviction error per query row: err = dm * ||m_ev - m_A|| (one warp per row
-// of D floats; the norm's partial sums reduced by a butterfly).
-__global__ void __launch_bounds__(256) evict_err_kernel(const float *m_ev, const float *m_kept, const float *dropped,
-                                                         float *err, int64_t rows, int D) {
-    const int lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (r >= rows) return;
-    const float *e = m_ev + r * D, *k = m_kept + r * D;
-    float sq = 0.0f;
-    for (int d = lane; d < D; d += 32) {
-        const float x = __ldg(e + d) - __ldg(k + d);
-        sq = fmaf(x, x, sq);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xFFFFFFFFu, sq, o);
-    if (lane == 0) {
-        const float dm = __ldg(dropped + r);
-        err[r] = dm > 0.0f ? dm * sqrtf(sq) : 0.0f;
-    }
-}
-
 template <class M, int D, int G, bool WITH_V>
 cudaError_t launch_one(const AttnArgs &a, int sm_count, cudaStream_t s, const CUtensorMap &tk, const CUtensorMap &tv) {
     using LY = Layout<M, D, G, WITH_V>;
@@ -406,14 +373,6 @@ bool attn_supported(int dtype, int D, int G) {
 }
 
 bool attn_uses_tensor_maps(int dtype) { return dtype == RKV_BF16; }
-
-cudaError_t launch_evict_err(const float *m_ev, const float *m_kept, const float *dropped, float *err, int64_t rows,
-                             int D, cudaStream_t s) {
-    if (rows == 0) return cudaSuccess;
-    const int64_t blocks = (rows + 7) / 8;
-    evict_err_kernel<<<(unsigned)blocks, 256, 0, s>>>(m_ev, m_kept, dropped, err, rows, D);
-    return cudaGetLastError();
-}
 
 size_t attn_partial_rec_floats(int D, int G) { return (size_t)G * (D + 4); }
 

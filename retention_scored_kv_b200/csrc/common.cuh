@@ -73,6 +73,13 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// Limit of a wait on other CTAs (grid barriers, the append's wait for the
+// compactions): status[4] microseconds when set, else 2 s.
+__device__ __forceinline__ uint64_t cross_wait_limit_ns(const int32_t *status) {
+    const int32_t us = __ldcg(status + 4);
+    return us > 0 ? (uint64_t)us * 1000ull : 2000000000ull;
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -82,8 +89,9 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
 // Grid-wide barrier for a cooperative (co-resident) grid.  `count` is a
 // monotonically increasing arrival counter, zero when the launch starts; barrier
 // number `epoch` (1, 2, ...) completes when count reaches epoch*gridDim.x.
-// The wait is bounded (~2 s of globaltimer); on timeout RKV_DEV_TIMEOUT is
-// recorded and false returned, so the caller can leave the kernel.
+// The wait is bounded (2 s of globaltimer, or the workspace's wait limit);
+// on timeout RKV_DEV_TIMEOUT is recorded and false returned, so the caller
+// can leave the kernel.
 __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, int32_t *status,
                                              int *smem_flag, int32_t site = 0x100) {
     __syncthreads();
@@ -93,10 +101,11 @@ __device__ __forceinline__ bool grid_barrier(uint32_t *count, uint32_t epoch, in
         const uint32_t target = epoch * gridDim.x;
         int ok = 1;
         if (ld_acquire_gpu(count) < target) {
-            const uint64_t t0 = globaltimer_ns();
+            const uint64_t t0 = globaltimer_ns(), lim = cross_wait_limit_ns(status);
+            const uint32_t every = lim < 100000ull ? 0u : 255u;  // a short limit is checked on every spin
             uint32_t spins = 0;
             while (ld_acquire_gpu(count) < target) {
-                if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
+                if ((++spins & every) == 0 && globaltimer_ns() - t0 > lim) {
                     record_timeout(status, site + (int32_t)epoch);
                     ok = 0;
                     break;

@@ -284,6 +284,15 @@ __global__ void __launch_bounds__(APP_THREADS) append_kernel(AppendArgs a) {
 
 }  // namespace
 
+namespace {
+__global__ void set_word_kernel(int32_t *p, int32_t v) { *p = v; }
+}  // namespace
+
+cudaError_t launch_set_word(int32_t *p, int32_t v, cudaStream_t s) {
+    set_word_kernel<<<1, 1, 0, s>>>(p, v);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_compact(const CompactArgs &a, cudaStream_t s) {
     if (a.C == 0) return cudaSuccess;
     // page ids, keep words, two prefix arrays

@@ -41,7 +41,6 @@ struct WsLayout {
     size_t hrec;          // float  [C][rec] state of whole heads that hold candidates
     size_t npre;          // int32  [C] pre-step lengths
     size_t pfx;           // int32  [C+1] page prefix of the pre-step lengths (own range of each CTA)
-    size_t ev_out;        // float  [C][G][D] output of the evicted set (eviction error)
     size_t bmask;         // uint16 [C][max_pages] forced keep bits (ContourKV)
     size_t bkept;         // int32  [C] forced counts (ContourKV)
     size_t bfloor;        // int32  [C] oldest floor position (ContourKV)
@@ -53,6 +52,9 @@ struct WsLayout {
 // Per-call counters of the fused step: head_kept[C], head_flag[C],
 // seq[B][4] (keys above the window, candidates), misc[16] (compaction arrivals).
 inline size_t step_ctr_words(int64_t C, int B) { return (size_t)(2 * C + 4 * (int64_t)B + 16 + 63) / 64 * 64; }
+
+// One int32 written on the device (compact.cu).
+cudaError_t launch_set_word(int32_t *p, int32_t v, cudaStream_t s);
 
 struct SelectGrid {
     int n_groups, cta_per_group, waves, threads, smem_bytes, cache_pages;
@@ -159,7 +161,6 @@ struct AttnArgs {
     float *partial;
     int C, max_pages;
     float qscale;              // scale * log2(e)
-    int invert;                // 1: attend the evicted rows (keep_mask required, dropped NULL)
 };
 // Returns cudaErrorNotSupported if (dtype, D, G) is not instantiated.  bf16
 // pools are read through the two tensor maps (64-column boxes of 16 rows,
@@ -167,9 +168,22 @@ struct AttnArgs {
 cudaError_t launch_attn(const AttnArgs &a, int dtype, int D, int G, int sm_count, cudaStream_t s,
                         const CUtensorMap &tk, const CUtensorMap &tv);
 bool attn_supported(int dtype, int D, int G);
-// err[r] = dropped[r] * ||m_ev[r] - m_kept[r]|| for rows r < rows of D floats.
-cudaError_t launch_evict_err(const float *m_ev, const float *m_kept, const float *dropped, float *err, int64_t rows,
-                             int D, cudaStream_t s);
+// Eviction error (evict_err.cu): per head, the forced-weight output of the
+// evicted rows against the kept output: err = dropped * ||m_ev - out_kept||.
+struct EvictErrArgs {
+    const void *k_pool;
+    const void *v_pool;
+    const int32_t *block_table;
+    const int32_t *n_pre;
+    const uint16_t *keep_mask;
+    const float *q;            // [C][G][D]
+    const float *out_kept;     // [C][G][D]
+    const float *dropped;      // [C][G]
+    float *err;                // [C][G]
+    float scale;
+    int C, max_pages;
+};
+cudaError_t launch_evict_err(const EvictErrArgs &a, int dtype, int D, int G, cudaStream_t s);
 bool attn_uses_tensor_maps(int dtype);
 size_t attn_partial_rec_floats(int D, int G);
 

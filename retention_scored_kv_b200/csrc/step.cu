@@ -1533,10 +1533,11 @@ __device__ bool compact_warp(const StepArgs &a, const Ctx &cx, WarpScr &w, int c
 __device__ bool wait_pushes(const StepArgs &a, const Ctx &cx) {
     const uint32_t target = gridDim.x;
     if (ld_acquire_gpu(arrive_of(a, cx)) >= target) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = globaltimer_ns(), lim = cross_wait_limit_ns(a.status);
+    const uint32_t every = lim < 100000ull ? 0u : 255u;
     uint32_t spins = 0;
     while (ld_acquire_gpu(arrive_of(a, cx)) < target) {
-        if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
+        if ((++spins & every) == 0 && globaltimer_ns() - t0 > lim) {
             record_timeout(a.status, 0x200);
             return false;
         }

@@ -6,7 +6,8 @@ lengths, free stack -- with one-element stand-in K/V rows, since none of those
 steps reads K or V values); for batched workloads the oracle runs on a subset
 of the independent sequences and the shared free stack is checked by its
 invariants.  Attention and dropped mass are compared on sampled heads, whose
-rows are gathered into a small oracle cache.  K/V row moves are checked on
+rows are gathered into a small oracle cache, and on every head of one steady
+step of llama32k and of two qwen8k sequences.  K/V row moves are checked on
 sampled heads against the pre-compaction rows of the same positions.
 """
 import numpy as np
@@ -155,10 +156,12 @@ def run_workload(rkv, name, steps, seqs=None, sample=6, seed=0):
     return dc
 
 
-def run_workload_fused(rkv, name, steps, seqs=None, sample=6, seed=0):
+def run_workload_fused(rkv, name, steps, seqs=None, sample=6, seed=0, all_heads_at=()):
     """As run_workload, through the single-launch rkv_decode_step: the oracle
     state, the sampled heads' rows and their attention inputs are taken before
-    the call (the launch compacts and appends in place)."""
+    the call (the launch compacts and appends in place).  At the steps in
+    all_heads_at every head of the checked sequences is compared, not a
+    sample (heads split across CTAs, merged by warps or block-wide)."""
     cfg = workloads.CONFIGS[name]
     dc = workloads.prefill_cache(cfg, seed, device="cuda", n_steps=steps + 1)
     cache = rkv_cache(rkv, dc)
@@ -172,6 +175,8 @@ def run_workload_fused(rkv, name, steps, seqs=None, sample=6, seed=0):
         inp = workloads.step_inputs(cfg, seed, s, "cuda")
         host, heads = meta_host(dc, check_seqs)
         sampled = sorted(int(x) for x in rng.choice(heads, size=min(sample, len(heads)), replace=False))
+        if s in all_heads_at:
+            sampled = [int(c) for c in heads]
         before = {c: head_rows(dc, c) for c in sampled}
         mini, maxp = mini_cache(dc, sampled)
         len_pre = host.len.copy()
@@ -253,6 +258,16 @@ def test_vlm16k_evicting_and_non_evicting_steps(rkv):
 def test_fused_llama32k_prefill_eviction_and_steady_steps(rkv):
     ctr = run_workload_fused(rkv, "llama32k", steps=4)
     assert ctr["exact_steps"] >= 1 and ctr["window_steps"] >= 2, ctr   # prefill eviction exact, then mostly the window
+
+
+def test_fused_llama32k_every_head_on_a_steady_step(rkv):
+    # all 256 KV heads (1,024 query rows) of a steady evicting step, in the
+    # launch configuration the benchmark times
+    run_workload_fused(rkv, "llama32k", steps=3, sample=4, all_heads_at={2})
+
+
+def test_fused_qwen8k_every_head_of_two_sequences_on_a_steady_step(rkv):
+    run_workload_fused(rkv, "qwen8k", steps=3, seqs=[0, 15], sample=4, all_heads_at={2})
 
 
 def test_fused_long128k_prefill_eviction_and_steady_steps(rkv):
