@@ -65,6 +65,12 @@ constexpr int T_STASH = 0;                       // int32 [6][NTH]
 constexpr int T_CL = 6 * NTH * 4;                // int32 [WIN_CAP] candidate list of one head
 constexpr int T_PAIRS = T_CL + WIN_CAP * 4;      // int2 [CMP_PAIRS]
 constexpr int T_TBL = T_PAIRS + CMP_PAIRS * 8;   // int32 [mp], src [mp+1], hole [mp+1], uint16 msk [mp]
+// Candidates of this CTA's own tail heads, listed once after the resolve
+// ((head - first own head) << 16 | index in its sequence's list), in the
+// block-wide compaction's pair buffer (unused until the heavy tasks); more
+// than OWN_CAP and the warp merges scan their sequence's list instead.
+constexpr int T_OWN = T_PAIRS;
+constexpr int OWN_CAP = CMP_PAIRS * 8 / 4;
 // Per-warp scratch of the warp-level merge and compaction (used before the
 // block-wide fallbacks, which reuse the same bytes from T_TBL on).
 constexpr int RCAP = 16;    // partial records a warp merges (CTAs a head spans)
@@ -100,6 +106,7 @@ constexpr int MAX_NBAR = 2 * NCW * 8 + 2 * QR;
 // most RES_CAP of them and at most CADD_CAP heads (their kept-candidate
 // counts are tallied in shared memory), so no second grid barrier is needed.
 constexpr int RES_CAP = 1024;
+
 constexpr int CADD_CAP = 8192;
 constexpr int S_LO = 0, S_HI = S_LO + MAXB * 8, S_KAP = S_HI + MAXB * 8, S_PK = S_KAP + MAXB * 8,
               S_PM = S_PK + MAXB * 8, S_KMX = S_PM + MAXB * 8, S_M = S_KMX + MAXB * 8, S_T = S_M + MAXB * 8,
@@ -170,12 +177,13 @@ struct Sm {
     __device__ __forceinline__ int64_t *misc64() const { return at<int64_t>(S_MISC64); }
     __device__ __forceinline__ int32_t *rlo() const { return at<int32_t>(S_RLO); }
     __device__ __forceinline__ int8_t *fate() const { return at<int8_t>(S_FATE); }
+    __device__ __forceinline__ int32_t *own() const { return reinterpret_cast<int32_t *>(base + S_BIG + T_OWN); }
     __device__ __forceinline__ unsigned char *big() const { return base + S_BIG; }
 };
 
 // misc slots
 enum { MS_CSTART = 0, MS_CLAST, MS_RADIX, MS_MISS, MS_BAR, MS_TOTAL, MS_NCL,
-       MS_ACTIVE, MS_QN, MS_QH };
+       MS_ACTIVE, MS_QN, MS_QH, MS_NOWN };
 
 struct Ctx {
     int32_t TP, x0, x1, pfx_start;  // flattened pages (< 2^27)
@@ -761,16 +769,37 @@ __device__ int resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
             keys[g] = __ldcg(a.ckey + (size_t)b * WIN_CAP + (g - sm.off()[b]));
         }
         __syncthreads();
+        if (tid == 0) sm.misc()[MS_NOWN] = 0;
+        __syncthreads();
         for (int g = tid; g < total; g += NTH) {
             int b = 0;
             while (b + 1 < a.B && (int64_t)sm.off()[b + 1] <= g) b++;
             const int ob = (int)sm.off()[b], nb = (int)sm.nc()[b];
             const uint64_t K = keys[g];
-            uint32_t less = 0;
-            for (int i = 0; i < nb; i++) less += keys[ob + i] < K ? 1u : 0u;
+            // rank among the sequence's candidates: four independent counts
+            // so the shared-memory loads overlap
+            const uint64_t *kb = keys + ob;
+            uint32_t l0 = 0, l1 = 0, l2 = 0, l3 = 0;
+            int i = 0;
+            for (; i + 4 <= nb; i += 4) {
+                l0 += kb[i] < K ? 1u : 0u;
+                l1 += kb[i + 1] < K ? 1u : 0u;
+                l2 += kb[i + 2] < K ? 1u : 0u;
+                l3 += kb[i + 3] < K ? 1u : 0u;
+            }
+            for (; i < nb; i++) l0 += kb[i] < K ? 1u : 0u;
+            const uint32_t less = (l0 + l1) + (l2 + l3);
             const uint32_t r = (uint32_t)(sm.m()[b] - (int64_t)sm.above()[b]);
             const bool kept = less < r;
             sm.fate()[g] = kept ? 1 : 0;
+            {
+                const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
+                const int c = b * a.LH + cl;
+                if (c >= hc0 && c < hc1) {
+                    const int at = atomicAdd(&sm.misc()[MS_NOWN], 1);
+                    if (at < OWN_CAP) sm.own()[at] = ((c - hc0) << 16) | (g - ob);
+                }
+            }
             if (kept) {
                 const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
                 const int c = b * a.LH + cl;
@@ -832,6 +861,31 @@ __device__ int resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
     }
     if (blockIdx.x == 0 && tid < a.B && (sm.fl()[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap()[tid];
     return RES_MODE_GRID;
+}
+
+// After a grid-mode resolve: the candidates of this CTA's own tail heads,
+// read from the sequences those heads belong to (see OWN_CAP).
+__device__ void own_list_grid(const StepArgs &a, const Sm &sm) {
+    const int tid = threadIdx.x, nct = gridDim.x;
+    const int hc0 = (int)((int64_t)blockIdx.x * a.C / nct), hc1 = (int)((int64_t)(blockIdx.x + 1) * a.C / nct);
+    if (tid == 0) sm.misc()[MS_NOWN] = 0;
+    __syncthreads();
+    if (hc0 < hc1) {
+        const int b0 = hc0 / a.LH, b1 = (hc1 - 1) / a.LH;
+        const int g0 = (int)sm.off()[b0], g1 = (int)(sm.off()[b1] + sm.nc()[b1]);
+        for (int g = g0 + tid; g < g1; g += NTH) {
+            int b = b0;
+            while (b < b1 && (int)sm.off()[b + 1] <= g) b++;
+            const int j = g - (int)sm.off()[b];
+            const uint64_t K = __ldcg(a.ckey + (size_t)b * WIN_CAP + j);
+            const int c = b * a.LH + (a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits));
+            if (c >= hc0 && c < hc1) {
+                const int at = atomicAdd(&sm.misc()[MS_NOWN], 1);
+                if (at < OWN_CAP) sm.own()[at] = ((c - hc0) << 16) | j;
+            }
+        }
+    }
+    __syncthreads();
 }
 
 // --------------------------------------------------------- exact select ----
@@ -1210,18 +1264,33 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
     int ncl = 0;
     const size_t cb = (size_t)b * WIN_CAP;
     if (cands) {
-        const int nb = (int)sm.nc()[b];
-        for (int base = 0; base < nb; base += 32) {
-            const int i = base + lane;
-            bool mine = false;
-            if (i < nb) {
-                const uint64_t K = __ldcg(a.ckey + cb + i);
-                mine = (a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits)) == cl;
+        const int nown = sm.misc()[MS_NOWN];
+        if (nown <= OWN_CAP) {
+            // this CTA's list of its own heads' candidates (shared memory)
+            const int kk = c - (int)((int64_t)blockIdx.x * a.C / gridDim.x);
+            for (int base = 0; base < nown; base += 32) {
+                const int i = base + lane;
+                const int32_t e = i < nown ? sm.own()[i] : -1;
+                const bool mine = i < nown && (e >> 16) == kk;
+                const uint32_t ball = __ballot_sync(0xFFFFFFFFu, mine);
+                const int k = ncl + __popc(ball & ((1u << lane) - 1u));
+                if (mine && k < CCAP) w.cidx[k] = e & 0xFFFF;
+                ncl += __popc(ball);
             }
-            const uint32_t ball = __ballot_sync(0xFFFFFFFFu, mine);
-            const int k = ncl + __popc(ball & ((1u << lane) - 1u));
-            if (mine && k < CCAP) w.cidx[k] = i;
-            ncl += __popc(ball);
+        } else {
+            const int nb = (int)sm.nc()[b];
+            for (int base = 0; base < nb; base += 32) {
+                const int i = base + lane;
+                bool mine = false;
+                if (i < nb) {
+                    const uint64_t K = __ldcg(a.ckey + cb + i);
+                    mine = (a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits)) == cl;
+                }
+                const uint32_t ball = __ballot_sync(0xFFFFFFFFu, mine);
+                const int k = ncl + __popc(ball & ((1u << lane) - 1u));
+                if (mine && k < CCAP) w.cidx[k] = i;
+                ncl += __popc(ball);
+            }
         }
         if (ncl > CCAP) return false;
     }
@@ -1777,7 +1846,10 @@ __global__ void __launch_bounds__(NTH, 1)
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
         const int res = resolve(a, sm, cx);
         if (res != RES_MISS) {
-            if (res == RES_MODE_GRID && !grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
+            if (res == RES_MODE_GRID) {
+                if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
+                own_list_grid(a, sm);
+            }
             spec = true;
             local = res == RES_MODE_LOCAL;
             if (blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(a.status + 2, 1);
