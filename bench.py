@@ -67,10 +67,11 @@ PER_CONFIG = "llama32k,qwen8k,vlm16k"
 SPLIT_STEPS = 32  # event-timed steps for the evicting / non-evicting split
 
 # DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of one
-# launch of the fused step kernel on a steady llama32k step: the 16-layer
-# capture (read 137.71 MB + write 4.15 MB) x2 to the full launch.  Reported
-# only while the kernel's sources hash to the captured version.
-STEP_TRAFFIC = {"sources_sha256": "f4c114055eede79d", "workload": "llama32k", "bytes_per_launch": 2 * 141.859584e6}
+# launch of the fused step kernel on a steady long128k step: the 4-layer
+# capture (read 218.83 MB + write 5.03 MB) x8 to the full 32-layer launch
+# (pages, hence traffic, grow with the layer count).  Reported only while the
+# kernel's sources hash to the captured version.
+STEP_TRAFFIC = {"sources_sha256": "77fd4020ee5329e1", "workload": "long128k", "bytes_per_launch": 8 * 223.860224e6}
 
 
 # ------------------------------------------------------------------ ranks ---

@@ -238,17 +238,21 @@ RKV_API int rkv_score_select_budget(const rkv_cache_t *cache, const int32_t *t, 
  * code running where cudaMalloc is not permitted, such as inside a host
  * callback or under an allocator they do not control).  It has no
  * counterpart in the papers: it is a deployment convenience.  Same inputs,
- * outputs, results and errors as rkv_score_select; its scratch (status word,
- * barrier counters, radix histograms, window candidates) is a fixed __device__ array of about
- * 0.9 MiB inside the library, which every GPU that loads the library holds
- * until the process exits.  Limits: at most 16 sequences (B <= 16), else
- * RKV_ERR_UNSUPPORTED.  The first call on a device looks up that array's
- * device address (cudaGetSymbolAddress), so make the first call on each
- * device before any stream capture.  Each call clears the scratch it uses
- * (an async memset on `stream`) and allocates nothing.  All calls share the
- * one array: calls that overlap on the GPU (different streams, or other
- * threads) race and must be serialised by the caller.  Device-side input
- * errors are not reported by this variant (its status word is private).
+ * outputs and results as rkv_score_select, and the same host-side errors;
+ * device-side RKV_DEV_* errors and timeouts are not reported (the status
+ * word lives in the private scratch).  Its scratch (status word, barrier
+ * counters, radix histograms, window candidates) is a fixed __device__ array
+ * of about 0.9 MiB inside the library, which every GPU that loads the
+ * library holds until the process exits.  Limits: at most 16 sequences
+ * (B <= 16), else RKV_ERR_UNSUPPORTED.  The first call on a device looks up
+ * that array's device address (cudaGetSymbolAddress), so make the first
+ * call on each device before any stream capture.  Each call clears the
+ * scratch it uses (an async memset on `stream`), threshold window included:
+ * no window is carried between calls, so every call runs the exact radix
+ * passes (its cost is that of a first call of rkv_score_select).  It
+ * allocates nothing.  All calls share the one array: calls that overlap on
+ * the GPU (different streams, or other threads) race and must be serialised
+ * by the caller.
  */
 RKV_API int rkv_score_select_noalloc(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
                                      const rkv_select_t *sel, void *stream);
