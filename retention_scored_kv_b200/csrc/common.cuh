@@ -226,10 +226,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Bounded wait on an mbarrier phase.  Every producer of the phase is in the
 // same CTA and always arrives, so the bound is a guard, not a protocol:
-// after ~2 s the wait records RKV_DEV_TIMEOUT and returns false.
+// after ~2 s the wait records RKV_DEV_TIMEOUT and returns false.  A timeout
+// recorded elsewhere (another CTA's wait on the grid) does not end this
+// wait: the phase still completes, and leaving early could let the CTA exit
+// while bulk copies are still landing in its shared memory.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status, int32_t site = 1) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (__ldcg(status) & RKV_DEV_TIMEOUT) return false;  // an earlier wait already gave up
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
     while (!mbar_try_wait(bar, parity)) {

@@ -53,7 +53,7 @@ using namespace core;
 constexpr int NTH = ATTN_THREADS;
 constexpr int NWARP = NTH / 32;
 constexpr int MAXB = STEP_MAX_B;
-constexpr int UNR = 4;           // pages per half-warp per round of the exact select
+constexpr int PPT = 1;           // pages per thread per round of the exact select's sweeps
 constexpr int HGRP = 8;          // sequences histogrammed together in the exact select
 constexpr int CMP_PAIRS = 1024;  // hole/source pairs resolved per compaction round
 static_assert(STEP_HEADS_PER_CTA == NTH, "tail chunk = one head per thread");
@@ -96,6 +96,8 @@ __host__ __device__ constexpr size_t tail_bytes(int mp) {
     return cmp > wrp ? cmp : wrp;
 }
 constexpr size_t RADIX_BYTES = (size_t)HGRP * NBINS * 4;
+constexpr int KT = NTH * PPT;                // pages per round of the exact select's sweeps
+constexpr int T_SPFX = (int)RADIX_BYTES;     // int32 [KT + 1] page-prefix chunk, after the histograms
 constexpr size_t RESOLVE_BYTES = (size_t)WIN_CAP * 8;
 
 // Fixed part of shared memory (offsets from the 1024-aligned base, the same
@@ -141,7 +143,7 @@ struct StepLayout {
     static_assert(QBYTES % 16 == 0, "query block must be a 16-byte multiple");
     static_assert(NBAR <= NTH && NBAR <= MAX_NBAR, "barrier init");
     static_assert(M::STAGE_ALIGN <= 1024, "big region alignment");
-    static_assert(BIG_ATTN >= (int)RADIX_BYTES && BIG_ATTN >= (int)RESOLVE_BYTES, "scratch");
+    static_assert(BIG_ATTN >= T_SPFX + (KT + 1) * 4 && BIG_ATTN >= (int)RESOLVE_BYTES, "scratch");
     static size_t smem(int mp) {
         const size_t big = tail_bytes(mp) > (size_t)BIG_ATTN ? tail_bytes(mp) : (size_t)BIG_ATTN;
         return (size_t)S_BIG + big + 1024;
@@ -183,7 +185,7 @@ struct Sm {
 
 // misc slots
 enum { MS_CSTART = 0, MS_CLAST, MS_RADIX, MS_MISS, MS_BAR, MS_TOTAL, MS_NCL,
-       MS_ACTIVE, MS_QN, MS_QH, MS_NOWN };
+       MS_ACTIVE, MS_QN, MS_QH, MS_NOWN, MS_HNEXT };
 
 struct Ctx {
     int32_t TP, x0, x1, pfx_start;  // flattened pages (< 2^27)
@@ -275,17 +277,30 @@ __device__ __forceinline__ uint32_t below_bits(int w, int nn) {
     return (1u << (nn - lo)) - 1u;
 }
 
-__device__ void scan_words(int32_t *v, int W, uint32_t *scratch) {
-    uint32_t carry = 0;
-    for (int base = 0; base < W; base += blockDim.x) {
-        const int w = base + threadIdx.x;
-        const uint32_t x = w < W ? (uint32_t)v[w] : 0u;
-        uint32_t tot;
-        const uint32_t ex = block_exclusive_scan(x, scratch, &tot);
-        if (w < W) v[w] = (int32_t)(carry + ex);
-        carry += tot;
+// Exclusive prefix sums of two word arrays in place (va[W], vb[W] receive
+// the totals): each thread sums a contiguous chunk, one block scan of the
+// chunk sums, then the chunks are rewritten as running prefixes.
+__device__ void scan_words2(int32_t *va, int32_t *vb, int W, uint32_t *scratch) {
+    const int CH = (W + NTH - 1) / NTH;
+    const int w0 = min(W, (int)threadIdx.x * CH), w1 = min(W, w0 + CH);
+    uint32_t sum[2] = {0u, 0u};
+    for (int w = w0; w < w1; w++) {
+        sum[0] += (uint32_t)va[w];
+        sum[1] += (uint32_t)vb[w];
     }
-    if (threadIdx.x == 0) v[W] = (int32_t)carry;
+    uint32_t ex[2], tot[2];
+    block_scan_n<2>(sum, ex, tot, scratch);
+    for (int w = w0; w < w1; w++) {
+        const uint32_t xa = (uint32_t)va[w], xb = (uint32_t)vb[w];
+        va[w] = (int32_t)ex[0];
+        vb[w] = (int32_t)ex[1];
+        ex[0] += xa;
+        ex[1] += xb;
+    }
+    if (threadIdx.x == 0) {
+        va[W] = (int32_t)tot[0];
+        vb[W] = (int32_t)tot[1];
+    }
     __syncthreads();
 }
 
@@ -489,20 +504,30 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                 bulk_g2s(qring + slot * G * D, a.q + (int64_t)c * G * D, LY::QBYTES, &qfull[slot], pol_keep);
             }
             nq++;
+            // block-table entries (and keep words) of the next 32 pages are
+            // loaded while this block's copies are issued
+            int32_t phys_n = 0;
+            uint32_t kp_n = 0xFFFFu;
+            auto load_block = [&](int64_t base) {
+                const int64_t i = base + lane;
+                if (i < pb && ((int)((i - cx.x0 + pb0) % NCW)) % NPW == pw) {
+                    phys_n = __ldg(a.block_table + (int64_t)c * a.max_pages + (i - pfx));
+                    if (masks) kp_n = (uint32_t)__ldcg(a.keep_mask + (int64_t)c * a.max_pages + (i - pfx));
+                }
+            };
+            load_block(pa);
             for (int64_t base = pa; base < pb; base += 32) {
                 const int64_t i = base + lane;
-                int32_t phys = 0;
-                uint32_t m = 0;
                 const bool mine = i < pb && ((int)((i - cx.x0 + pb0) % NCW)) % NPW == pw;
+                const int32_t phys = phys_n;
+                uint32_t m = 0;
                 if (mine) {
                     const int64_t pidx = i - pfx;
-                    phys = __ldg(a.block_table + (int64_t)c * a.max_pages + pidx);
                     const int nv = min(PAGE, n - (int)pidx * PAGE);
                     const uint32_t valid = nv >= PAGE ? 0xFFFFu : ((1u << nv) - 1u);
-                    const uint32_t kp =
-                        masks ? (uint32_t)__ldcg(a.keep_mask + (int64_t)c * a.max_pages + pidx) : 0xFFFFu;
-                    m = SPEC ? (valid << 16) : ((kp & valid) | (valid << 16));
+                    m = SPEC ? (valid << 16) : ((kp_n & valid) | (valid << 16));
                 }
+                if (base + 32 < pb) load_block(base + 32);
                 uint32_t todo = __ballot_sync(0xFFFFFFFFu, mine);
                 while (todo) {
                     const int j = __ffs(todo) - 1;
@@ -889,68 +914,123 @@ __device__ void own_list_grid(const StepArgs &a, const Sm &sm) {
 }
 
 // --------------------------------------------------------- exact select ----
-// Calls f(c, pidx, r, K, ok) for slot r of every page of this CTA's range
-// (c = -1 past the range end), half a warp per page, UNR pages per half-warp
-// per round with their loads issued together.  Heads are found through the
-// range's page prefix in a.pfx.  Loop bounds are warp-uniform.
-template <typename F>
-__device__ __forceinline__ void for_range_keys(const StepArgs &a, const Sm &sm, const Ctx &cx, F &&f) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int r = lane & 15;
-    constexpr int STEP = 2 * NWARP;
-    int cur = -1;
-    for (int64_t xb = cx.x0 + 2 * warp; xb < cx.x1; xb += (int64_t)STEP * UNR) {
-        int32_t pg[UNR];
-        int hc[UNR], pidx[UNR];
-        bool ld[UNR];
-#pragma unroll
-        for (int u = 0; u < UNR; u++) {
-            const int64_t x = xb + (lane >> 4) + (int64_t)u * STEP;
-            ld[u] = false;
-            hc[u] = -1;
-            pidx[u] = 0;
-            pg[u] = 0;
-            if (x < cx.x1) {
-                if (cur < 0) {
-                    int lo = cx.c_start, hi = cx.c_last;  // last c with pfx[c] <= x
-                    while (lo < hi) {
-                        const int mid = (lo + hi + 1) >> 1;
-                        if (a.pfx[mid] <= x) lo = mid; else hi = mid - 1;
-                    }
-                    cur = lo;
-                }
-                while (cur < cx.c_last && a.pfx[cur + 1] <= x) cur++;
-                hc[u] = cur;
-                pidx[u] = (int)(x - a.pfx[cur]);
-                if (pidx[u] * PAGE + r < clamp_len(__ldcg(a.len + cur), a.max_pages, nullptr)) {
-                    ld[u] = true;
-                    pg[u] = __ldcg(a.block_table + (int64_t)cur * a.max_pages + pidx[u]);
-                }
-            }
+// Calls f(c, pidx, n, key) for every page of this CTA's range, one page per
+// thread per round (lanes of a warp hold consecutive pages).  c = head (-1 for
+// a thread without a page), pidx = page index in the head, n = valid slots of
+// the page, key(r, K) = the entry key of slot r < n (false, with the status
+// flagged, for an entry rejected as bad input).  Every thread calls f, so f
+// may use warp collectives.  Loads are pipelined across rounds: a round's 16
+// positions and 16 log-retentions per page (16-byte vectors) are in flight
+// together with the next round's head lengths and block-table entries.  The
+// head of a page comes from a binary search in a chunk of the range's page
+// prefix (a.pfx) staged in shared memory, reloaded when a round leaves it.
+__device__ __forceinline__ void range_page_head(const StepArgs &a, const Ctx &cx, const int32_t *spfx, int hcur,
+                                                int32_t x, int &c, int &pidx) {
+    c = -1;
+    pidx = 0;
+    if (x >= cx.x1) return;
+    int32_t base;
+    if (spfx[KT] > x) {
+        int lo = 0, hi = KT - 1;  // last j with spfx[j] <= x
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (spfx[mid] <= x) lo = mid; else hi = mid - 1;
         }
-        int32_t pos[UNR];
-        float lbv[UNR];
-#pragma unroll
-        for (int u = 0; u < UNR; u++) {
-            pos[u] = 0;
-            lbv[u] = 0.0f;
-            if (ld[u]) {
-                pos[u] = __ldcg(a.pos_pool + (int64_t)pg[u] * PAGE + r);
-                lbv[u] = __ldcg(a.lb_pool + (int64_t)pg[u] * PAGE + r);
-            }
+        c = hcur + lo;
+        base = spfx[lo];
+    } else {
+        // more heads start here than the chunk holds (empty heads): search
+        // the prefix in global memory
+        int lo = hcur + KT, hi = cx.c_last;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (__ldcg(a.pfx + mid) <= x) lo = mid; else hi = mid - 1;
         }
-#pragma unroll
-        for (int u = 0; u < UNR; u++) {
-            uint64_t K = 0ull;
-            bool ok = false;
-            if (ld[u]) {
-                const int b = hc[u] / a.LH;
-                ok = entry_key(sm.t()[b], (uint32_t)(hc[u] - b * a.LH), pos[u], lbv[u], a.ibits, &K);
-                if (!ok) set_status(a.status, RKV_DEV_BAD_INPUT);
-            }
-            f(hc[u], pidx[u], r, K, ok);
-        }
+        c = lo;
+        base = __ldcg(a.pfx + c);
     }
+    pidx = x - base;
+}
+
+template <typename F>
+__device__ __forceinline__ void for_range_pages(const StepArgs &a, const Sm &sm, const Ctx &cx, F &&f) {
+    const int tid = threadIdx.x;
+    int32_t *spfx = reinterpret_cast<int32_t *>(sm.big() + T_SPFX);
+    int *hnext = &sm.misc()[MS_HNEXT];
+    int hcur = cx.c_start;
+    auto load_chunk = [&]() {
+        for (int j = tid; j <= KT; j += NTH) {
+            const int c = hcur + j;
+            spfx[j] = c <= cx.c_last + 1 ? __ldcg(a.pfx + c) : 0x7FFFFFFF;
+        }
+        __syncthreads();
+    };
+    load_chunk();
+    int c, pidx;
+    range_page_head(a, cx, spfx, hcur, cx.x0 + tid, c, pidx);
+    int32_t ln = 0, pg = 0;
+    if (c >= 0) {
+        ln = __ldcg(a.len + c);
+        pg = __ldcg(a.block_table + (int64_t)c * a.max_pages + pidx);
+    }
+    for (int32_t X0 = cx.x0; X0 < cx.x1; X0 += KT) {
+        // this round's positions and log-retentions
+        const int n = c >= 0 ? min(PAGE, max(0, clamp_len(ln, a.max_pages, nullptr) - pidx * PAGE)) : 0;
+        int4 pv[4];
+        float4 lv[4];
+        {
+            const int4 *pp = reinterpret_cast<const int4 *>(a.pos_pool + (int64_t)pg * PAGE);
+            const float4 *lp = reinterpret_cast<const float4 *>(a.lb_pool + (int64_t)pg * PAGE);
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                pv[q] = make_int4(0, 0, 0, 0);
+                lv[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (4 * q < n) {
+                    pv[q] = __ldcg(pp + q);
+                    lv[q] = __ldcg(lp + q);
+                }
+            }
+        }
+        // the next round's heads and pages (the chunk is reloaded from this
+        // round's last head when it does not reach the next round's end)
+        const int32_t Xn = X0 + KT;
+        int cn = -1, pn = 0;
+        int32_t lnn = 0, pgn = 0;
+        if (Xn < cx.x1) {
+            if (spfx[KT] <= min(Xn + KT, cx.x1) - 1) {
+                if (tid == NTH - 1) *hnext = c >= 0 ? c : hcur;
+                __syncthreads();
+                hcur = *hnext;
+                __syncthreads();
+                load_chunk();
+            }
+            range_page_head(a, cx, spfx, hcur, Xn + tid, cn, pn);
+            if (cn >= 0) {
+                lnn = __ldcg(a.len + cn);
+                pgn = __ldcg(a.block_table + (int64_t)cn * a.max_pages + pn);
+            }
+        }
+        {
+            const int b = c >= 0 ? c / a.LH : 0;
+            const int32_t tb = sm.t()[b];
+            const uint32_t cl = (uint32_t)(c - b * a.LH);
+            auto key = [&](int r, uint64_t &K) -> bool {
+                const int4 &pq = pv[r >> 2];
+                const float4 &lq = lv[r >> 2];
+                const int32_t ps = (r & 3) == 0 ? pq.x : (r & 3) == 1 ? pq.y : (r & 3) == 2 ? pq.z : pq.w;
+                const float ls = (r & 3) == 0 ? lq.x : (r & 3) == 1 ? lq.y : (r & 3) == 2 ? lq.z : lq.w;
+                if (entry_key(tb, cl, ps, ls, a.ibits, &K)) return true;
+                set_status(a.status, RKV_DEV_BAD_INPUT);
+                return false;
+            };
+            f(c, pidx, n, key);
+        }
+        c = cn;
+        pidx = pn;
+        ln = lnn;
+        pg = pgn;
+    }
+    __syncthreads();
 }
 
 // This call's largest kept key of sequence b (uint64 in the counter half).
@@ -1067,11 +1147,28 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
             const int g1 = min(b_last + 1, g0 + HGRP);
             for (int i = tid; i < (g1 - g0) * NBINS; i += NTH) hist[i] = 0u;
             __syncthreads();
-            for_range_keys(a, sm, cx, [&](int c, int, int, uint64_t K, bool ok) {
-                if (!ok) return;
+            for_range_pages(a, sm, cx, [&](int c, int, int n, auto &key) {
+                if (c < 0) return;
                 const int b = c / a.LH;
-                if (b < g0 || b >= g1 || (sm.fl()[b] & SF_DONE) || ((K ^ sm.pk()[b]) & sm.pm()[b]) != 0ull) return;
-                atomicAdd(&hist[(b - g0) * NBINS + key_digit((uint32_t)(K >> 32), (uint32_t)K, p)], 1u);
+                if (b < g0 || b >= g1 || (sm.fl()[b] & SF_DONE)) return;
+                const uint64_t pk = sm.pk()[b], pm = sm.pm()[b];
+                uint32_t *hb = hist + (b - g0) * NBINS;
+                // a page's neighbouring entries mostly share a bin: add runs
+                uint32_t run_bin = 0u, run_n = 0u;
+#pragma unroll
+                for (int r = 0; r < PAGE; r++) {
+                    uint64_t K;
+                    if (r >= n || !key(r, K) || ((K ^ pk) & pm) != 0ull) continue;
+                    const uint32_t bin = key_digit((uint32_t)(K >> 32), (uint32_t)K, p);
+                    if (run_n && bin == run_bin) {
+                        run_n++;
+                    } else {
+                        if (run_n) atomicAdd(hb + run_bin, run_n);
+                        run_bin = bin;
+                        run_n = 1u;
+                    }
+                }
+                if (run_n) atomicAdd(hb + run_bin, run_n);
             });
             __syncthreads();
             for (int i = tid; i < (g1 - g0) * NBINS; i += NTH) {
@@ -1084,31 +1181,44 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return false;
         scan_digits(a, sm, p);
     }
-    // keep masks (half-warp ballots), kept counts and the largest kept key of
-    // each sequence (the reported threshold is that key + 1: a radix bucket
-    // kept whole only bounds it)
+    // keep masks, kept counts (summed over each run of lanes holding the same
+    // head) and the largest kept key of each sequence (the reported threshold
+    // is that key + 1: a radix bucket kept whole only bounds it)
     int kb = -1;
     unsigned long long km = 0ull;
-    for_range_keys(a, sm, cx, [&](int c, int pidx, int r, uint64_t K, bool ok) {
-        const int b = c >= 0 ? c / a.LH : 0;
-        const bool keep = ok && K < sm.kap()[b];
-        if (keep) {
+    for_range_pages(a, sm, cx, [&](int c, int pidx, int n, auto &key) {
+        uint32_t m16 = 0u;
+        if (c >= 0) {
+            const int b = c / a.LH;
+            const uint64_t kap = sm.kap()[b];
             if (b != kb) {
                 if (kb >= 0) atomicMax(sm.kmx() + kb, km);
                 kb = b;
-                km = K;
-            } else if (K > km) {
-                km = K;
+                km = 0ull;
             }
-        }
-        const uint32_t ball = __ballot_sync(0xFFFFFFFFu, keep);
-        if (r == 0 && c >= 0) {
-            const uint32_t m16 = (ball >> (lane & 16)) & 0xFFFFu;
+#pragma unroll
+            for (int r = 0; r < PAGE; r++) {
+                uint64_t K;
+                if (r < n && key(r, K) && K < kap) {
+                    m16 |= 1u << r;
+                    km = K > km ? K : km;
+                }
+            }
             a.keep_mask[(int64_t)c * a.max_pages + pidx] = (uint16_t)m16;
-            if (m16) atomicAdd(head_kept_of(a, cx) + c, (uint32_t)__popc(m16));
         }
+        // lanes hold consecutive pages, so a head's lanes are contiguous:
+        // suffix sums within runs of equal c, the run's first lane adds
+        uint32_t sum = (uint32_t)__popc(m16);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xFFFFFFFFu, sum, o);
+            const int cy = __shfl_down_sync(0xFFFFFFFFu, c, o);
+            if (lane + o < 32 && cy == c) sum += y;
+        }
+        const int cprev = __shfl_up_sync(0xFFFFFFFFu, c, 1);
+        if (c >= 0 && (lane == 0 || cprev != c) && sum) atomicAdd(head_kept_of(a, cx) + c, sum);
     });
-    if (kb >= 0) atomicMax(sm.kmx() + kb, km);
+    if (kb >= 0 && km) atomicMax(sm.kmx() + kb, km);
     __syncthreads();
     if (tid < a.B && sm.kmx()[tid]) atomicMax(kmax_of(a, cx, tid), sm.kmx()[tid]);
     if (blockIdx.x == 0 && tid < a.B && (sm.fl()[tid] & SF_TRIVIAL)) a.kappa[tid] = sm.kap()[tid];
@@ -1397,9 +1507,18 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
 }
 
 // Hole-fill compaction of head c (n entries, nn kept): the j-th non-kept
-// slot below nn takes the j-th kept slot at or above nn; pages past
-// ceil(nn/16) go to the free stack at this head's plan offset.
-__device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int n, int nn, int32_t off) {
+// slot below nn takes the j-th kept slot at or above nn.  This call moves the
+// ranks [moves * part / parts, moves * (part + 1) / parts), so several CTAs
+// can share a head; with push, pages past ceil(nn/16) go to the free stack at
+// this head's plan offset (only once every part of the head has moved).
+// Pairs are resolved CMP_PAIRS at a time; each warp then moves CPW rows with
+// all their loads issued before the stores.
+template <int ROWB>
+__device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int c, int n, int nn, int32_t off,
+                             int part, int parts, bool push) {
+    constexpr int E = (2 * ROWB / 16 + 31) / 32;  // 16-byte pieces per lane of a row's K and V
+    constexpr int CPW = 8 / E;                    // rows a warp moves at a time
+    static_assert(2 * ROWB / 16 <= 64, "row bytes");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int mp = a.max_pages;
     int32_t *tbl = reinterpret_cast<int32_t *>(sm.big() + T_TBL);
@@ -1409,76 +1528,134 @@ __device__ void compact_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
     int2 *pairs = reinterpret_cast<int2 *>(sm.big() + T_PAIRS);
     const int W = (n + PAGE - 1) / PAGE, Wn = (nn + PAGE - 1) / PAGE;
     const int64_t cm = (int64_t)c * mp;
-    for (int w = tid; w < W; w += NTH) {
-        tbl[w] = __ldcg(a.block_table + cm + w);
-        const uint32_t m = (uint32_t)__ldcg(a.keep_mask + cm + w) & below_bits(w, n);
-        msk[w] = (uint16_t)m;
-        const uint32_t below = below_bits(w, nn);
-        src_pfx[w] = __popc(m & ~below);
-        hole_pfx[w] = __popc(~m & below & 0xFFFFu);
+    // table and keep words, LDW per thread per round with their loads issued
+    // together; per word its sources (kept slots at or above nn) and holes
+    // (non-kept slots below nn)
+    constexpr int LDW = 8;
+    for (int w0 = 0; w0 < W; w0 += NTH * LDW) {
+        int32_t tv[LDW];
+        uint32_t mv[LDW];
+#pragma unroll
+        for (int k = 0; k < LDW; k++) {
+            const int w = w0 + k * NTH + tid;
+            tv[k] = 0;
+            mv[k] = 0u;
+            if (w < W) {
+                tv[k] = __ldcg(a.block_table + cm + w);
+                mv[k] = (uint32_t)__ldcg(a.keep_mask + cm + w);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < LDW; k++) {
+            const int w = w0 + k * NTH + tid;
+            if (w < W) {
+                const uint32_t m = mv[k] & below_bits(w, n);
+                tbl[w] = tv[k];
+                msk[w] = (uint16_t)m;
+                const uint32_t below = below_bits(w, nn);
+                src_pfx[w] = __popc(m & ~below);
+                hole_pfx[w] = __popc(~m & below & 0xFFFFu);
+            }
+        }
     }
     __syncthreads();
-    scan_words(src_pfx, W, sm.scan());
-    scan_words(hole_pfx, W, sm.scan());
+    scan_words2(src_pfx, hole_pfx, W, sm.scan());
     const int moves = min(hole_pfx[W], src_pfx[W]);
-    const int chunks = a.row_bytes / 16;
-    for (int r0 = 0; r0 < moves; r0 += CMP_PAIRS) {
-        const int r1 = min(moves, r0 + CMP_PAIRS);
-        for (int w = tid; w < Wn; w += NTH) {
-            int rank = hole_pfx[w];
-            if (rank >= r1 || hole_pfx[w + 1] <= r0) continue;
-            uint32_t hb = ~(uint32_t)msk[w] & below_bits(w, nn) & 0xFFFFu;
-            while (hb) {
-                const int bit = __ffs(hb) - 1;
-                hb &= hb - 1;
-                if (rank >= r0 && rank < r1) {
-                    int lo = 0, hi = W - 1;  // word of the rank-th source: last w' with src_pfx[w'] <= rank
-                    while (lo < hi) {
-                        const int mid = (lo + hi + 1) >> 1;
-                        if (src_pfx[mid] <= rank) lo = mid; else hi = mid - 1;
-                    }
-                    uint32_t sb = (uint32_t)msk[lo] & ~below_bits(lo, nn);
-                    for (int i = rank - src_pfx[lo]; i > 0; i--) sb &= sb - 1;
-                    const int hslot = w * PAGE + bit, sslot = lo * PAGE + (__ffs(sb) - 1);
-                    pairs[rank - r0] = make_int2((int)((int64_t)tbl[hslot / PAGE] * PAGE + hslot % PAGE),
-                                                 (int)((int64_t)tbl[sslot / PAGE] * PAGE + sslot % PAGE));
+    const int ra = (int)((int64_t)moves * part / parts), rb = (int)((int64_t)moves * (part + 1) / parts);
+    constexpr int chunks = ROWB / 16;
+    // last word w in [0, W) with pfx[w] <= r (pfx[0] = 0 <= r)
+    auto word_of = [&](const int32_t *pfx, int r) {
+        int lo = 0, hi = W - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (pfx[mid] <= r) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
+    for (int r0 = ra; r0 < rb; r0 += CMP_PAIRS) {
+        const int r1 = min(rb, r0 + CMP_PAIRS);
+        // the rank-th hole and the rank-th source for every rank of the
+        // round: each thread expands whole words of the words holding them
+        {
+            const int h0 = word_of(hole_pfx, r0), h1 = word_of(hole_pfx, r1 - 1);
+            for (int w = h0 + tid; w <= h1; w += NTH) {
+                uint32_t hb = ~(uint32_t)msk[w] & below_bits(w, nn) & 0xFFFFu;
+                int rank = hole_pfx[w];
+                const int64_t pbase = (int64_t)tbl[w] * PAGE;
+                while (hb) {
+                    const int bit = __ffs(hb) - 1;
+                    hb &= hb - 1;
+                    if (rank >= r0 && rank < r1) pairs[rank - r0].x = (int)(pbase + bit);
+                    rank++;
                 }
-                rank++;
+            }
+            const int s0 = word_of(src_pfx, r0), s1 = word_of(src_pfx, r1 - 1);
+            for (int w = s0 + tid; w <= s1; w += NTH) {
+                uint32_t sb = (uint32_t)msk[w] & ~below_bits(w, nn);
+                int rank = src_pfx[w];
+                const int64_t pbase = (int64_t)tbl[w] * PAGE;
+                while (sb) {
+                    const int bit = __ffs(sb) - 1;
+                    sb &= sb - 1;
+                    if (rank >= r0 && rank < r1) pairs[rank - r0].y = (int)(pbase + bit);
+                    rank++;
+                }
             }
         }
         __syncthreads();
-        for (int pi = warp; pi < r1 - r0; pi += NWARP) {
-            const int64_t dst = pairs[pi].x, src = pairs[pi].y;
-            const int i0 = lane, i1 = lane + 32;
-            uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-            const uint4 *ks = reinterpret_cast<const uint4 *>((const unsigned char *)a.k_pool + src * a.row_bytes);
-            const uint4 *vs = reinterpret_cast<const uint4 *>((const unsigned char *)a.v_pool + src * a.row_bytes);
-            if (i0 < 2 * chunks) v0 = i0 < chunks ? __ldcg(ks + i0) : __ldcg(vs + i0 - chunks);
-            if (i1 < 2 * chunks) v1 = i1 < chunks ? __ldcg(ks + i1) : __ldcg(vs + i1 - chunks);
+        const int np_ = r1 - r0;
+        for (int p0 = warp * CPW; p0 < np_; p0 += NWARP * CPW) {
+            uint4 v[CPW][E];
             int32_t pos = 0;
             float lbv = 0.0f;
-            if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < CPW; j++) {
+#pragma unroll
+                for (int e = 0; e < E; e++) v[j][e] = make_uint4(0, 0, 0, 0);
+                if (p0 + j < np_) {
+                    const int64_t src = pairs[p0 + j].y;
+                    const uint4 *ks = reinterpret_cast<const uint4 *>((const unsigned char *)a.k_pool + src * ROWB);
+                    const uint4 *vs = reinterpret_cast<const uint4 *>((const unsigned char *)a.v_pool + src * ROWB);
+#pragma unroll
+                    for (int e = 0; e < E; e++) {
+                        const int i = lane + 32 * e;
+                        if (i < 2 * chunks) v[j][e] = i < chunks ? __ldcg(ks + i) : __ldcg(vs + i - chunks);
+                    }
+                }
+            }
+            if (lane < CPW && p0 + lane < np_) {
+                const int64_t src = pairs[p0 + lane].y;
                 pos = __ldcg(a.pos_pool + src);
                 lbv = __ldcg(a.lb_pool + src);
             }
-            uint4 *kd = reinterpret_cast<uint4 *>((unsigned char *)a.k_pool + dst * a.row_bytes);
-            uint4 *vd = reinterpret_cast<uint4 *>((unsigned char *)a.v_pool + dst * a.row_bytes);
-            if (i0 < 2 * chunks) {
-                if (i0 < chunks) kd[i0] = v0; else vd[i0 - chunks] = v0;
+#pragma unroll
+            for (int j = 0; j < CPW; j++) {
+                if (p0 + j < np_) {
+                    const int64_t dst = pairs[p0 + j].x;
+                    uint4 *kd = reinterpret_cast<uint4 *>((unsigned char *)a.k_pool + dst * ROWB);
+                    uint4 *vd = reinterpret_cast<uint4 *>((unsigned char *)a.v_pool + dst * ROWB);
+#pragma unroll
+                    for (int e = 0; e < E; e++) {
+                        const int i = lane + 32 * e;
+                        if (i < 2 * chunks) {
+                            if (i < chunks) kd[i] = v[j][e]; else vd[i - chunks] = v[j][e];
+                        }
+                    }
+                }
             }
-            if (i1 < 2 * chunks) {
-                if (i1 < chunks) kd[i1] = v1; else vd[i1 - chunks] = v1;
-            }
-            if (lane == 0) {
+            if (lane < CPW && p0 + lane < np_) {
+                const int64_t dst = pairs[p0 + lane].x;
                 a.pos_pool[dst] = pos;
                 a.lb_pool[dst] = lbv;
             }
         }
         __syncthreads();
     }
-    for (int pi = Wn + tid; pi < W; pi += NTH) {
-        a.free_stack[cx.top0 + off + (pi - Wn)] = tbl[pi];
-        a.block_table[cm + pi] = -1;
+    if (push) {
+        for (int pi = Wn + tid; pi < W; pi += NTH) {
+            a.free_stack[cx.top0 + off + (pi - Wn)] = tbl[pi];
+            a.block_table[cm + pi] = -1;
+        }
     }
     __syncthreads();
 }
@@ -1666,7 +1843,7 @@ __device__ void append_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int 
 }
 
 template <class M, int D, int G>
-__device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, bool local) {
+__device__ bool tail(const StepArgs &a, const Sm &sm, Ctx &cx, bool spec, bool local) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nct = gridDim.x;
     const int C = a.C;
     const int hc0 = (int)((int64_t)blockIdx.x * C / nct), hc1 = (int)((int64_t)(blockIdx.x + 1) * C / nct);
@@ -1806,19 +1983,55 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
         if (comp && !compact_warp(a, cx, wsc, c, np, nn, st_plan[k]) && lane == 0) atomicOr(st_heavy + k, 2);
     }
     __syncthreads();
+    // A large eviction (an exact selection that frees many pages, e.g. the
+    // prefill eviction) spreads the moves of the heads too large for a warp
+    // over every CTA, parts per head; their owners push the freed pages after
+    // a grid barrier.  The decision is the same in every CTA.
+    const bool spread = cx.exact && cx.evict && pushes >= (uint32_t)nct * 4u;
     for (int k = 0; k < hc1 - hc0; k++) {
-        const int heavy = st_heavy[k];
-        if (!heavy) continue;
+        if (!(st_heavy[k] & 1)) continue;
         const int c = hc0 + k;
-        const int np = st_npre[k], nn = st_nnew[k];
-        if (heavy & 1) {
-            const int pages = (np + PAGE - 1) / PAGE;
-            const int64_t pfx = st_pfx[k];
-            const int jf = owner_rlo(sm.rlo(), nct, pfx), jl = owner_rlo(sm.rlo(), nct, pfx + pages - 1);
-            const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
-            combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, spec && (flag & 1u), local);
+        const int pages = (st_npre[k] + PAGE - 1) / PAGE;
+        const int64_t pfx = st_pfx[k];
+        const int jf = owner_rlo(sm.rlo(), nct, pfx), jl = owner_rlo(sm.rlo(), nct, pfx + pages - 1);
+        const uint32_t flag = __ldcg(head_flag_of(a, cx) + c);
+        combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, spec && (flag & 1u), local);
+    }
+    // heavy compactions: this CTA's own heads, or (spread) its share of every
+    // head's parts
+    const int parts = spread ? min(64, max(1, (4 * nct + C - 1) / C)) : 1;
+    const int njobs = spread ? (int)(((int64_t)C * parts - blockIdx.x + nct - 1) / nct) : hc1 - hc0;
+    for (int j = 0; j < njobs; j++) {
+        int c, part = 0, np, nn;
+        int32_t off = 0;
+        if (spread) {
+            const int64_t id = blockIdx.x + (int64_t)j * nct;
+            c = (int)(id / parts);
+            part = (int)(id % parts);
+            np = __ldcg(a.npre + c);
+            nn = (int)__ldcg(head_kept_of(a, cx) + c);
+            if (!(nn < np && np - nn > HCAP)) continue;
+        } else {
+            if (!(st_heavy[j] & 2)) continue;
+            c = hc0 + j;
+            np = st_npre[j];
+            nn = st_nnew[j];
+            off = st_plan[j];
+            if (!(cx.evict && nn < np)) continue;
         }
-        if ((heavy & 2) && cx.evict && nn < np) compact_head(a, sm, cx, c, np, nn, st_plan[k]);
+        compact_head<M::PAGE_BYTES / PAGE>(a, sm, cx, c, np, nn, off, part, parts, !spread);
+    }
+    if (spread) {
+        if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return false;
+        for (int k = 0; k < hc1 - hc0; k++) {
+            if (!(st_heavy[k] & 2)) continue;
+            const int64_t cm = (int64_t)(hc0 + k) * a.max_pages;
+            const int W = (st_npre[k] + PAGE - 1) / PAGE, Wn = (st_nnew[k] + PAGE - 1) / PAGE;
+            for (int pi = Wn + tid; pi < W; pi += NTH) {
+                a.free_stack[cx.top0 + st_plan[k] + (pi - Wn)] = __ldcg(a.block_table + cm + pi);
+                a.block_table[cm + pi] = -1;
+            }
+        }
     }
     __syncthreads();
     if (tid == 0) {
@@ -1826,6 +2039,7 @@ __device__ void tail(const StepArgs &a, const Sm &sm, const Ctx &cx, bool spec, 
         atomicAdd(arrive_of(a, cx), 1u);
     }
     for (int k = warp; k < hc1 - hc0; k += NWARP) append_head(a, sm, cx, hc0 + k, st_nnew[k], st_pop[k], pushes);
+    return true;
 }
 
 // ---------------------------------------------------------------- kernel ----
@@ -1865,7 +2079,7 @@ __global__ void __launch_bounds__(NTH, 1)
         attn_pass<M, D, G, false>(a, sm, cx, &tmk, &tmv);
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
     }
-    tail<M, D, G>(a, sm, cx, spec, local);
+    if (!tail<M, D, G>(a, sm, cx, spec, local)) return;
     // exit ticket: the last CTA resets the barrier counter and flips the half
     // of the per-call counters the next call uses
     __syncthreads();
