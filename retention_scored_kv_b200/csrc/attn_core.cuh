@@ -281,17 +281,15 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                  : "r"(addr));
 }
 
-// D(rows 0-7) += A(rows 0-7) * B for m16n8k16 bf16 -> fp32; rows 8-15 of A
-// are zero, so only c0/c1 are carried (the other two outputs are dropped).
-__device__ __forceinline__ void mma_rows8(float &c0, float &c1, uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-    float d2, d3;
-    const uint32_t z = 0u;
-    const float fz = 0.0f;
+// D += A * B for m16n8k16 bf16 -> fp32 with all four accumulators: rows 0-7
+// of A in a0/a2 (outputs c0/c1), rows 8-15 in a1/a3 (outputs c2/c3).
+__device__ __forceinline__ void mma_rows16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%10,%11,%12,%13};"
-        : "=f"(c0), "=f"(c1), "=f"(d2), "=f"(d3)
-        : "r"(a0), "r"(z), "r"(a2), "r"(z), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(fz), "f"(fz));
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 template <int D, int G, bool WITH_V>
@@ -348,22 +346,21 @@ struct MmaMath {
                                 uint32_t evm, int lane, uint32_t candm = 0u, float *zdst = nullptr, int zcap = 0) {
         const int t = lane & 3, mi = lane >> 3, r8 = lane & 7;
         // ---- S = Q K^T for the 16 rows of the page (two n-tiles of 8 rows) ----
-        // four independent accumulation chains (high/low query parts x two
-        // 8-row halves of the page), summed at the end
-        float s0h[2] = {0.0f, 0.0f}, s0l[2] = {0.0f, 0.0f}, s1h[2] = {0.0f, 0.0f}, s1l[2] = {0.0f, 0.0f};
+        // the high query parts fill MMA rows 0-7 and the low parts rows 8-15,
+        // so one MMA carries both; two accumulation chains (the 8-row halves
+        // of the page), high and low parts summed at the end
+        float s0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, s1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         const uint32_t kbase = smem_u32(sk);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS; ks++) {
             const int r = (mi >> 1) * 8 + r8, ch = (ks & 3) * 2 + (mi & 1);
             uint32_t b[4];
             ldsm_x4(kbase + swz(r, ks >> 2, ch), b);
-            mma_rows8(s0h[0], s0h[1], s.qh[ks][0], s.qh[ks][1], b[0], b[1]);
-            mma_rows8(s1h[0], s1h[1], s.qh[ks][0], s.qh[ks][1], b[2], b[3]);
-            mma_rows8(s0l[0], s0l[1], s.ql[ks][0], s.ql[ks][1], b[0], b[1]);
-            mma_rows8(s1l[0], s1l[1], s.ql[ks][0], s.ql[ks][1], b[2], b[3]);
+            mma_rows16(s0, s.qh[ks][0], s.ql[ks][0], s.qh[ks][1], s.ql[ks][1], b[0], b[1]);
+            mma_rows16(s1, s.qh[ks][0], s.ql[ks][0], s.qh[ks][1], s.ql[ks][1], b[2], b[3]);
         }
         // this lane holds row g = lane/4 at page rows j = 2t, 2t+1, 2t+8, 2t+9
-        const float y[4] = {s0h[0] + s0l[0], s0h[1] + s0l[1], s1h[0] + s1l[0], s1h[1] + s1l[1]};
+        const float y[4] = {s0[0] + s0[2], s0[1] + s0[3], s1[0] + s1[2], s1[1] + s1[3]};
         const int jr[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
         if constexpr (CAND) {
             if (candm && (lane >> 2) < G) {
@@ -416,10 +413,15 @@ struct MmaMath {
                 const int r = (mi & 1) * 8 + r8, ch = (np & 3) * 2 + (mi >> 1);
                 uint32_t b[4];
                 ldsm_x4_t(vbase + swz(r, np >> 2, ch), b);
-                mma_rows8(s.o[2 * np][0], s.o[2 * np][1], ph0, ph2, b[0], b[1]);
-                mma_rows8(s.o[2 * np][0], s.o[2 * np][1], pl0, pl2, b[0], b[1]);
-                mma_rows8(s.o[2 * np + 1][0], s.o[2 * np + 1][1], ph0, ph2, b[2], b[3]);
-                mma_rows8(s.o[2 * np + 1][0], s.o[2 * np + 1][1], pl0, pl2, b[2], b[3]);
+                // high weights in MMA rows 0-7, low weights in rows 8-15
+                float d0[4] = {s.o[2 * np][0], s.o[2 * np][1], 0.0f, 0.0f};
+                float d1[4] = {s.o[2 * np + 1][0], s.o[2 * np + 1][1], 0.0f, 0.0f};
+                mma_rows16(d0, ph0, pl0, ph2, pl2, b[0], b[1]);
+                mma_rows16(d1, ph0, pl0, ph2, pl2, b[2], b[3]);
+                s.o[2 * np][0] = d0[0] + d0[2];
+                s.o[2 * np][1] = d0[1] + d0[3];
+                s.o[2 * np + 1][0] = d1[0] + d1[2];
+                s.o[2 * np + 1][1] = d1[1] + d1[3];
             }
         }
     }

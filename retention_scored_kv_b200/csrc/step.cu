@@ -1134,7 +1134,32 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
     const int b_first = cx.c_start < a.C ? cx.c_start / a.LH : 0;
     const int b_last = cx.c_last >= 0 ? cx.c_last / a.LH : -1;
     uint32_t *hist = reinterpret_cast<uint32_t *>(sm.big());
-    for (int p = 0; p < NPASS; p++) {
+    // digit p's histogram of the sequences [g0, g1) this sweep counts
+    int p = 0, g0 = 0, g1 = 0;
+    auto count = [&](int c, int, int n, auto &key) {
+        if (c < 0) return;
+        const int b = c / a.LH;
+        if (b < g0 || b >= g1 || (sm.fl()[b] & SF_DONE)) return;
+        const uint64_t pk = sm.pk()[b], pm = sm.pm()[b];
+        uint32_t *hb = hist + (b - g0) * NBINS;
+        // a page's neighbouring entries mostly share a bin: add runs
+        uint32_t run_bin = 0u, run_n = 0u;
+#pragma unroll
+        for (int r = 0; r < PAGE; r++) {
+            uint64_t K;
+            if (r >= n || !key(r, K) || ((K ^ pk) & pm) != 0ull) continue;
+            const uint32_t bin = key_digit((uint32_t)(K >> 32), (uint32_t)K, p);
+            if (run_n && bin == run_bin) {
+                run_n++;
+            } else {
+                if (run_n) atomicAdd(hb + run_bin, run_n);
+                run_bin = bin;
+                run_n = 1u;
+            }
+        }
+        if (run_n) atomicAdd(hb + run_bin, run_n);
+    };
+    for (p = 0; p < NPASS; p++) {
         if (tid == 0) {
             int act = 0;
             for (int b = 0; b < a.B; b++) act |= (sm.fl()[b] & SF_DONE) ? 0 : 1;
@@ -1143,33 +1168,11 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
         __syncthreads();
         if (!sm.misc()[MS_ACTIVE]) break;
         cx.passes = p + 1;
-        for (int g0 = b_first; g0 <= b_last; g0 += HGRP) {
-            const int g1 = min(b_last + 1, g0 + HGRP);
+        for (g0 = b_first; g0 <= b_last; g0 += HGRP) {
+            g1 = min(b_last + 1, g0 + HGRP);
             for (int i = tid; i < (g1 - g0) * NBINS; i += NTH) hist[i] = 0u;
             __syncthreads();
-            for_range_pages(a, sm, cx, [&](int c, int, int n, auto &key) {
-                if (c < 0) return;
-                const int b = c / a.LH;
-                if (b < g0 || b >= g1 || (sm.fl()[b] & SF_DONE)) return;
-                const uint64_t pk = sm.pk()[b], pm = sm.pm()[b];
-                uint32_t *hb = hist + (b - g0) * NBINS;
-                // a page's neighbouring entries mostly share a bin: add runs
-                uint32_t run_bin = 0u, run_n = 0u;
-#pragma unroll
-                for (int r = 0; r < PAGE; r++) {
-                    uint64_t K;
-                    if (r >= n || !key(r, K) || ((K ^ pk) & pm) != 0ull) continue;
-                    const uint32_t bin = key_digit((uint32_t)(K >> 32), (uint32_t)K, p);
-                    if (run_n && bin == run_bin) {
-                        run_n++;
-                    } else {
-                        if (run_n) atomicAdd(hb + run_bin, run_n);
-                        run_bin = bin;
-                        run_n = 1u;
-                    }
-                }
-                if (run_n) atomicAdd(hb + run_bin, run_n);
-            });
+            for_range_pages(a, sm, cx, count);
             __syncthreads();
             for (int i = tid; i < (g1 - g0) * NBINS; i += NTH) {
                 const uint32_t v = hist[i];
@@ -1186,7 +1189,7 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
     // is that key + 1: a radix bucket kept whole only bounds it)
     int kb = -1;
     unsigned long long km = 0ull;
-    for_range_pages(a, sm, cx, [&](int c, int pidx, int n, auto &key) {
+    auto mark = [&](int c, int pidx, int n, auto &key) {
         uint32_t m16 = 0u;
         if (c >= 0) {
             const int b = c / a.LH;
@@ -1217,7 +1220,8 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
         }
         const int cprev = __shfl_up_sync(0xFFFFFFFFu, c, 1);
         if (c >= 0 && (lane == 0 || cprev != c) && sum) atomicAdd(head_kept_of(a, cx) + c, sum);
-    });
+    };
+    for_range_pages(a, sm, cx, mark);
     if (kb >= 0 && km) atomicMax(sm.kmx() + kb, km);
     __syncthreads();
     if (tid < a.B && sm.kmx()[tid]) atomicMax(kmax_of(a, cx, tid), sm.kmx()[tid]);
