@@ -110,6 +110,10 @@ constexpr int MAX_NBAR = 2 * NCW * 8 + 2 * QR;
 constexpr int RES_CAP = 1024;
 
 constexpr int CADD_CAP = 8192;
+// Radix select of the local resolve (sequences, state, histograms; big region).
+constexpr int RSEL_MAXB = 16;
+constexpr int T_RSEL = T_WARP + RES_CAP * 8 + CADD_CAP * 4;  // [RSEL_MAXB] 32-byte states
+constexpr int T_RHIST = T_RSEL + RSEL_MAXB * 32;             // uint32 [RSEL_MAXB][256]
 constexpr int S_LO = 0, S_HI = S_LO + MAXB * 8, S_KAP = S_HI + MAXB * 8, S_PK = S_KAP + MAXB * 8,
               S_PM = S_PK + MAXB * 8, S_KMX = S_PM + MAXB * 8, S_M = S_KMX + MAXB * 8, S_T = S_M + MAXB * 8,
               S_N = S_T + MAXB * 4, S_RANK = S_N + MAXB * 4, S_FL = S_RANK + MAXB * 4, S_ABOVE = S_FL + MAXB * 4,
@@ -144,6 +148,7 @@ struct StepLayout {
     static_assert(NBAR <= NTH && NBAR <= MAX_NBAR, "barrier init");
     static_assert(M::STAGE_ALIGN <= 1024, "big region alignment");
     static_assert(BIG_ATTN >= T_SPFX + (KT + 1) * 4 && BIG_ATTN >= (int)RESOLVE_BYTES, "scratch");
+    static_assert(BIG_ATTN >= T_RHIST + RSEL_MAXB * 256 * 4, "local resolve scratch");
     static size_t smem(int mp) {
         const size_t big = tail_bytes(mp) > (size_t)BIG_ATTN ? tail_bytes(mp) : (size_t)BIG_ATTN;
         return (size_t)S_BIG + big + 1024;
@@ -755,6 +760,121 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
 // global memory, and a grid barrier must follow.  RES_MISS: some sequence
 // missed (the exact path runs instead).
 enum { RES_MISS = 0, RES_MODE_LOCAL = 1, RES_MODE_GRID = 2 };
+
+// Local resolve, up to RSEL_MAXB sequences: the threshold of each sequence
+// (its r-th smallest candidate key, r = m - above, 1 <= r <= nc) by a radix
+// select in shared memory.  Digits of 8 bits start at the highest bit in
+// which the sequence's candidates differ; each pass histograms the
+// candidates still matching the chosen prefix and keeps the bucket holding
+// the remaining rank, until that bucket holds one key (keys are distinct).
+// Afterwards a candidate K is kept iff (K & mask) <= prefix, and is the
+// threshold iff (K & mask) == prefix.
+struct RselSeq {
+    uint64_t prefix, mask;
+    uint32_t rank, shift, done, pad;
+};
+static_assert(sizeof(RselSeq) == 32, "radix select state");
+
+__device__ __forceinline__ int cand_seq(const Sm &sm, int B, int g) {
+    int b = 0;
+    while (b + 1 < B && (int)sm.off()[b + 1] <= g) b++;
+    return b;
+}
+
+__device__ void resolve_radix(const StepArgs &a, const Sm &sm, const uint64_t *keys, int total) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    RselSeq *rs = reinterpret_cast<RselSeq *>(sm.big() + T_RSEL);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sm.big() + T_RHIST);
+    // bits in which each sequence's candidates differ from its first one
+    if (tid < 2 * a.B) hist[tid] = 0u;
+    __syncthreads();
+    for (int g = tid; g < total; g += NTH) {
+        const int b = cand_seq(sm, a.B, g);
+        const uint64_t d = keys[g] ^ keys[sm.off()[b]];
+        if (d >> 32) atomicOr(&hist[2 * b], (uint32_t)(d >> 32));
+        if ((uint32_t)d) atomicOr(&hist[2 * b + 1], (uint32_t)d);
+    }
+    __syncthreads();
+    if (tid < a.B) {
+        const int b = tid;
+        const uint32_t nb = sm.nc()[b];
+        RselSeq r{};
+        r.done = nb <= 1u ? 1u : 0u;
+        r.rank = nb ? (uint32_t)(sm.m()[b] - (int64_t)sm.above()[b]) : 0u;
+        const uint64_t d = ((uint64_t)hist[2 * b] << 32) | hist[2 * b + 1];
+        const int hb = d ? 63 - __clzll((long long)d) : 0;  // highest differing bit
+        r.shift = hb >= 7 ? (uint32_t)(hb - 7) : 0u;
+        r.mask = hb >= 63 ? 0ull : ~((2ull << hb) - 1ull);    // bits above hb are common
+        r.prefix = nb ? (keys[sm.off()[b]] & (r.done ? ~0ull : r.mask)) : 0ull;
+        if (r.done) r.mask = ~0ull;
+        rs[b] = r;
+    }
+    __syncthreads();
+    for (int pass = 0; pass < 9; pass++) {
+        if (tid == 0) {
+            int act = 0;
+            for (int b = 0; b < a.B; b++) act |= rs[b].done ? 0 : 1;
+            sm.misc()[MS_ACTIVE] = act;
+        }
+        for (int i = tid; i < a.B * 256; i += NTH) hist[i] = 0u;
+        __syncthreads();
+        if (!sm.misc()[MS_ACTIVE]) break;
+        for (int g = tid; g < total; g += NTH) {
+            const int b = cand_seq(sm, a.B, g);
+            const RselSeq &r = rs[b];
+            const uint64_t K = keys[g];
+            if (!r.done && (K & r.mask) == r.prefix) atomicAdd(&hist[b * 256 + (uint32_t)((K >> r.shift) & 255u)], 1u);
+        }
+        __syncthreads();
+        for (int b = warp; b < a.B; b += NWARP) {
+            RselSeq &r = rs[b];
+            if (r.done) continue;
+            const uint32_t *hb = hist + b * 256 + lane * 8;
+            uint32_t loc = 0;
+#pragma unroll
+            for (int j = 0; j < 8; j++) loc += hb[j];
+            uint32_t inc = loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            const uint32_t rank = r.rank;
+            const bool mine = inc - loc < rank && rank <= inc;
+            __syncwarp();
+            if (mine) {
+                // the bucket holding the rank, and the keys below it
+                uint32_t cum = inc - loc, below = 0, h = 0;
+                int dig = -1;
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const uint32_t e = hb[j];
+                    if (dig < 0) {
+                        if (rank <= cum + e) {
+                            dig = lane * 8 + j;
+                            h = e;
+                            below = cum;
+                        } else {
+                            cum += e;
+                        }
+                    }
+                }
+                const uint32_t sh = r.shift;
+                r.prefix = (r.prefix & ~(255ull << sh)) | ((uint64_t)dig << sh);
+                r.mask |= 255ull << sh;
+                r.rank = rank - below;
+                if (h <= 1u || sh == 0u) {
+                    r.done = 1u;
+                } else {
+                    r.shift = sh >= 8u ? sh - 8u : 0u;
+                }
+            }
+            __syncwarp();
+        }
+        __syncthreads();
+    }
+}
+
 __device__ int resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
     const int tid = threadIdx.x, nct = gridDim.x;
     if (tid < a.B) {
@@ -794,28 +914,38 @@ __device__ int resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
             keys[g] = __ldcg(a.ckey + (size_t)b * WIN_CAP + (g - sm.off()[b]));
         }
         __syncthreads();
+        const bool radix = a.B <= RSEL_MAXB;
+        if (radix) resolve_radix(a, sm, keys, (int)total);
+        const RselSeq *rs = reinterpret_cast<const RselSeq *>(sm.big() + T_RSEL);
         if (tid == 0) sm.misc()[MS_NOWN] = 0;
         __syncthreads();
         for (int g = tid; g < total; g += NTH) {
-            int b = 0;
-            while (b + 1 < a.B && (int64_t)sm.off()[b + 1] <= g) b++;
+            const int b = cand_seq(sm, a.B, g);
             const int ob = (int)sm.off()[b], nb = (int)sm.nc()[b];
             const uint64_t K = keys[g];
-            // rank among the sequence's candidates: four independent counts
-            // so the shared-memory loads overlap
-            const uint64_t *kb = keys + ob;
-            uint32_t l0 = 0, l1 = 0, l2 = 0, l3 = 0;
-            int i = 0;
-            for (; i + 4 <= nb; i += 4) {
-                l0 += kb[i] < K ? 1u : 0u;
-                l1 += kb[i + 1] < K ? 1u : 0u;
-                l2 += kb[i + 2] < K ? 1u : 0u;
-                l3 += kb[i + 3] < K ? 1u : 0u;
+            bool kept, thr;
+            if (radix) {
+                const uint64_t km = K & rs[b].mask;
+                kept = km <= rs[b].prefix;
+                thr = km == rs[b].prefix;
+            } else {
+                // rank among the sequence's candidates: four independent
+                // counts so the shared-memory loads overlap
+                const uint64_t *kb = keys + ob;
+                uint32_t l0 = 0, l1 = 0, l2 = 0, l3 = 0;
+                int i = 0;
+                for (; i + 4 <= nb; i += 4) {
+                    l0 += kb[i] < K ? 1u : 0u;
+                    l1 += kb[i + 1] < K ? 1u : 0u;
+                    l2 += kb[i + 2] < K ? 1u : 0u;
+                    l3 += kb[i + 3] < K ? 1u : 0u;
+                }
+                for (; i < nb; i++) l0 += kb[i] < K ? 1u : 0u;
+                const uint32_t less = (l0 + l1) + (l2 + l3);
+                const uint32_t r = (uint32_t)(sm.m()[b] - (int64_t)sm.above()[b]);
+                kept = less < r;
+                thr = less == r - 1;
             }
-            for (; i < nb; i++) l0 += kb[i] < K ? 1u : 0u;
-            const uint32_t less = (l0 + l1) + (l2 + l3);
-            const uint32_t r = (uint32_t)(sm.m()[b] - (int64_t)sm.above()[b]);
-            const bool kept = less < r;
             sm.fate()[g] = kept ? 1 : 0;
             {
                 const int cl = a.ibits >= 32 ? 0 : (int)((uint32_t)K >> a.ibits);
@@ -836,7 +966,7 @@ __device__ int resolve(const StepArgs &a, const Sm &sm, const Ctx &cx) {
                              (1u << (slot % PAGE)) << ((addr & 2) ? 16 : 0));
                 }
             }
-            if (blockIdx.x == 0 && less == r - 1) {
+            if (blockIdx.x == 0 && thr) {
                 const uint64_t kap = K + 1ull;
                 a.kappa[b] = kap;
                 window_next(a.win + (size_t)b * 4, kap, 1, (uint32_t)nb);
