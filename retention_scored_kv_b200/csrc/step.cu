@@ -141,7 +141,9 @@ struct StepLayout {
     static constexpr int B_POSLB = NST * STAGE_BYTES;         // [NST][16 positions, 16 log-retentions]
     static constexpr int B_Q = B_POSLB + NST * 128;
     static constexpr int B_MERGE = B_Q + QR * QBYTES;
-    static constexpr int B_META = B_MERGE + 2 * NCW * WSLOT * 4;
+    static constexpr int MFAC = G * NCW + G;                  // per parity: weights [G][NCW], kept sums [G]
+    static constexpr int B_MFAC = B_MERGE + 2 * NCW * WSLOT * 4;
+    static constexpr int B_META = B_MFAC + 2 * MFAC * 4;
     static constexpr int BIG_ATTN = B_META + NST * 4;
     static_assert(STAGE_BYTES % M::STAGE_ALIGN == 0, "stage alignment");
     static_assert(QBYTES % 16 == 0, "query block must be a 16-byte multiple");
@@ -687,7 +689,11 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
             named_bar_sync(1, NCW * 32);
 
             // ---- merge the warps (consumer threads) ----
+            // per query row (one thread each): merged statistics, and each
+            // warp's weight 2^(mk_w - mk) in a table; then every output
+            // element is the weighted sum of the warps' parts
             const float *mb = merge + par * NCW * LY::WSLOT;
+            float *fac = reinterpret_cast<float *>(sm.big() + LY::B_MFAC) + par * LY::MFAC;
             float hc = 0.0f;
 #pragma unroll
             for (int wi = 0; wi < NCW; wi++) hc += mb[wi * LY::WSLOT + G * D + 4 * G];
@@ -695,9 +701,8 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
             const int dest = whole ? (hc > 0.0f ? 1 : 0) : 2;
             float *rec = dest == 1 ? a.hrec + (int64_t)c * LY::REC
                                    : a.partial + ((int64_t)blockIdx.x * 2 + ((pfx < cx.x0) ? 0 : 1)) * LY::REC;
-            for (int e = tid; e < G * D + G; e += NCW * 32) {
-                const bool is_stat = e >= G * D;
-                const int g = is_stat ? e - G * D : e / D;
+            if (tid < G) {
+                const int g = tid;
                 Merged s;
                 s.mk = -INFINITY;
                 s.me = -INFINITY;
@@ -708,7 +713,6 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                 }
                 s.lk = 0.0f;
                 s.le = 0.0f;
-                float av = 0.0f;
 #pragma unroll
                 for (int wi = 0; wi < NCW; wi++) {
                     const float *src = mb + wi * LY::WSLOT;
@@ -717,22 +721,30 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                     const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
                     s.lk += src[G * D + G + g] * fk;
                     s.le += src[G * D + 3 * G + g] * fe;
-                    if (!is_stat) av += src[e] * fk;
+                    fac[g * NCW + wi] = fk;
                 }
+                fac[G * NCW + g] = s.lk;
                 if (dest == 0) {
-                    if (!is_stat) {
-                        a.out[(int64_t)c * G * D + e] = s.lk > 0.0f ? av / s.lk : 0.0f;
-                    } else {
-                        if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
-                        if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
-                    }
-                } else if (!is_stat) {
-                    rec[e] = av;
+                    if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
+                    if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
                 } else {
                     rec[G * D + g] = s.mk;
                     rec[G * D + G + g] = s.lk;
                     rec[G * D + 2 * G + g] = s.me;
                     rec[G * D + 3 * G + g] = s.le;
+                }
+            }
+            named_bar_sync(1, NCW * 32);
+            for (int e = tid; e < G * D; e += NCW * 32) {
+                const int g = e / D;
+                float av = 0.0f;
+#pragma unroll
+                for (int wi = 0; wi < NCW; wi++) av += mb[wi * LY::WSLOT + e] * fac[g * NCW + wi];
+                if (dest == 0) {
+                    const float lk = fac[G * NCW + g];
+                    a.out[(int64_t)c * G * D + e] = lk > 0.0f ? av / lk : 0.0f;
+                } else {
+                    rec[e] = av;
                 }
             }
             if (dest == 1 && tid == 0) atomicOr(head_flag_of(a, cx) + c, 2u);
