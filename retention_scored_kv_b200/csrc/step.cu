@@ -204,11 +204,16 @@ struct Ctx {
     int passes;      // exact-select passes run (histograms to clear)
     int attn_runs;   // attention passes run
     // The pipeline barriers are initialised once per launch; a later
-    // attention pass continues their phases: its page indices start after
-    // the pages of the earlier passes (pbase) and its query slots after
-    // their heads (qbase).  Producer and consumer count both alike.
+    // attention pass continues their phases.  Round-robin passes number
+    // their pages after the earlier passes' (pbase) and their query slots
+    // after the earlier passes' heads (qbase); head-per-warp passes count
+    // every consumer warp's pages over the launch (wcnt[0] in a consumer
+    // warp; in a producer warp wcnt[0] and wcnt[1] for the two consumer
+    // warps it feeds).  Every pass of a launch takes the same mode, and
+    // producer and consumer count alike.
     int32_t pbase;
     int qbase;
+    uint32_t wcnt[2];
 };
 
 // This call's half of the per-call counters: head_kept[C], head_flag[C],
@@ -368,6 +373,7 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
     cx.attn_runs = 0;
     cx.pbase = 0;
     cx.qbase = 0;
+    cx.wcnt[0] = cx.wcnt[1] = 0u;
     if (tid < MAXB) sm.n()[tid] = 0u;
     if (tid < 64) sm.misc()[tid] = 0;
     if (tid == 0) {
@@ -459,6 +465,48 @@ __device__ __forceinline__ void prologue(const StepArgs &a, const Sm &sm, Ctx &c
 }
 
 // -------------------------------------------------------- attention pass ----
+// Head-per-warp mode: when this CTA's range holds at least NCW heads and
+// they are short (at most HPW_PAGES pages per head on average), each head
+// goes to one consumer warp whole (head c_start + j to warp j mod NCW), so no
+// head needs a merge across warps; otherwise pages are dealt to the warps
+// round-robin.
+constexpr int HPW_PAGES = 64;
+__device__ __forceinline__ bool head_per_warp(const Ctx &cx) {
+    const int64_t heads = (int64_t)cx.c_last - cx.c_start + 1;
+    return heads >= NCW && (int64_t)(cx.x1 - cx.x0) <= (int64_t)HPW_PAGES * heads;
+}
+
+// The heads of one consumer warp in the head-per-warp mode: c_start + w,
+// then every NCW-th head while c <= c_last, each with its page prefix (the
+// pages of the heads stepped over are summed from one warp-wide round of
+// length loads).  Every lane of the calling warp runs it.
+struct HeadCursor {
+    int c, n, pages;
+    int64_t pfx;
+    __device__ void step(const StepArgs &a, int from, int64_t pfx_from, int skip) {
+        const int lane = threadIdx.x & 31;
+        const int h = from + lane;
+        const int32_t ln = (lane <= skip && h < a.C) ? clamp_len(__ldcg(a.len + h), a.max_pages, nullptr) : 0;
+        int pg = lane < skip ? (ln + PAGE - 1) / PAGE : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pg += __shfl_xor_sync(0xFFFFFFFFu, pg, o);
+        c = from + skip;
+        pfx = pfx_from + pg;
+        n = __shfl_sync(0xFFFFFFFFu, ln, skip);
+        pages = (n + PAGE - 1) / PAGE;
+    }
+    __device__ void init(const StepArgs &a, const Ctx &cx, int w) { step(a, cx.c_start, cx.pfx_start, w); }
+    __device__ void next(const StepArgs &a) { step(a, c, pfx, NCW); }
+    __device__ bool valid(const Ctx &cx) const { return c <= cx.c_last; }
+};
+
+// Warms L1 with a head's query block (G*D floats), 128 bytes per lane.
+template <int G, int D>
+__device__ __forceinline__ void prefetch_q(const float *q, int lane) {
+    constexpr int LINES = (G * D * 4 + 127) / 128;
+    if (lane < LINES) asm volatile("prefetch.global.L1 [%0];" ::"l"(q + lane * 32));
+}
+
 // Pages are dealt to consumer warps round-robin (page li -> warp li % NCW);
 // each consumer warp owns a private ring filled in order by producer warp
 // (warp % NPW), so every mbarrier has one producer and one consumer.  SPEC
@@ -758,6 +806,305 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
         if constexpr (REG_SPLIT) setmaxnreg_inc<LAUNCH_REGS>();
     }
 }
+
+template <class M, int D, int G, bool SPEC>
+__device__ __forceinline__ void attn_pass_hpw(const StepArgs &a, const Sm &sm, Ctx &cx, const CUtensorMap *tmk,
+                                          const CUtensorMap *tmv) {
+    using LY = StepLayout<M, D, G>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint64_t *full = sm.bars(), *empty = full + LY::NST, *qfull = empty + LY::NST, *qempty = qfull + QR;
+    unsigned char *stage = sm.big() + LY::B_STAGE;
+    unsigned char *poslb = sm.big() + LY::B_POSLB;
+    float *qring = reinterpret_cast<float *>(sm.big() + LY::B_Q);
+    float *merge = reinterpret_cast<float *>(sm.big() + LY::B_MERGE);
+    uint32_t *meta = reinterpret_cast<uint32_t *>(sm.big() + LY::B_META);
+    __syncthreads();
+    if (cx.attn_runs == 0) {
+        if (tid < LY::NBAR) {
+            // full: producer; empty: the owning consumer warp; qfull: producer 0; qempty: every consumer warp
+            mbar_init(full + tid, tid >= 2 * LY::NST + QR ? NCW : 1);
+        }
+        fence_mbar_init();
+        __syncthreads();
+    }
+    // timeout site codes: 0x10 (speculative pass) / 0x20 (mask pass) + wait kind
+    const int32_t site = SPEC ? 0x10 : 0x20;
+    cx.attn_runs++;
+    const bool masks = !SPEC && cx.evict;
+
+    if (warp >= NCW) {
+        // =============================== producers ===============================
+        if constexpr (REG_SPLIT) setmaxnreg_dec<PRODUCER_REGS>();
+        const int pw = warp - NCW;
+        const uint64_t pol_kv = policy_evict_first();
+        const uint64_t pol_keep = policy_evict_last();
+        uint32_t cnt0 = cx.wcnt[0], cnt1 = cx.wcnt[1];  // pages issued to consumer warps pw, pw + NPW
+        // one page to consumer warp cw (lane 0): its next stage, once free
+        auto issue = [&](int cw, uint32_t k, int32_t pj, uint32_t mj) {
+            const int sg = cw * LY::NSW + (int)(k % LY::NSW);
+            mbar_wait(&empty[sg], ((k / LY::NSW) & 1u) ^ 1u, a.status, site + 2);
+            meta[sg] = mj;
+            const bool load_v = SPEC || (mj & 0xFFFFu);
+            mbar_arrive_expect_tx(&full[sg], M::PAGE_BYTES * (load_v ? 2 : 1) + (SPEC ? 128u : 0u));
+            M::issue(stage + sg * LY::STAGE_BYTES, load_v, pj, &full[sg], a.k_pool, a.v_pool, tmk, tmv, pol_kv);
+            if (SPEC) {
+                bulk_g2s(poslb + sg * 128, a.pos_pool + (int64_t)pj * PAGE, 64, &full[sg], pol_keep);
+                bulk_g2s(poslb + sg * 128 + 64, a.lb_pool + (int64_t)pj * PAGE, 64, &full[sg], pol_keep);
+            }
+        };
+        // the keep word (bit 16+ valid slots) of page pidx of a head of n entries
+        auto page_meta = [&](int n, int64_t pidx, uint32_t kp) -> uint32_t {
+            const int nv = min(PAGE, n - (int)pidx * PAGE);
+            const uint32_t valid = nv >= PAGE ? 0xFFFFu : ((1u << nv) - 1u);
+            return SPEC ? (valid << 16) : ((kp & valid) | (valid << 16));
+        };
+        {
+            // head per warp: two cursors (the heads of consumer warps pw and
+            // pw + NPW); a page is issued to whichever warp has a free stage,
+            // so one warp's head end does not hold up the other
+            HeadCursor hc[2];
+            int64_t ip[2], pe[2], bb[2];
+            int32_t bph[2];
+            uint32_t bkp[2];
+            bool on[2];
+            // first page of the cursor's next head with pages in this range
+            // (the consumer warp finishes the others by itself)
+            auto seek = [&](int k) {
+                for (;;) {
+                    on[k] = hc[k].valid(cx);
+                    if (!on[k]) break;
+                    ip[k] = max(hc[k].pfx, (int64_t)cx.x0);
+                    pe[k] = min(hc[k].pfx + hc[k].pages, (int64_t)cx.x1);
+                    if (ip[k] < pe[k]) break;
+                    hc[k].next(a);
+                }
+            };
+            auto load_blk = [&](int k) {
+                bb[k] = ip[k];
+                const int64_t i = ip[k] + lane;
+                bph[k] = 0;
+                bkp[k] = 0xFFFFu;
+                if (i < pe[k]) {
+                    const int64_t pidx = i - hc[k].pfx;
+                    bph[k] = __ldg(a.block_table + (int64_t)hc[k].c * a.max_pages + pidx);
+                    if (masks) bkp[k] = (uint32_t)__ldcg(a.keep_mask + (int64_t)hc[k].c * a.max_pages + pidx);
+                }
+            };
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                hc[k].init(a, cx, pw + k * NPW);
+                seek(k);
+                if (on[k]) load_blk(k);
+            }
+            const uint64_t t0 = globaltimer_ns();
+            uint32_t spins = 0;
+            while (on[0] || on[1]) {
+                bool moved = false;
+#pragma unroll
+                for (int k = 0; k < 2; k++) {
+                    if (!on[k]) continue;
+                    const int cw = pw + k * NPW;
+                    const uint32_t kk = k == 0 ? cnt0 : cnt1;
+                    const int sg = cw * LY::NSW + (int)(kk % LY::NSW);
+                    int ok = 0;
+                    if (lane == 0) ok = mbar_try_wait(&empty[sg], ((kk / LY::NSW) & 1u) ^ 1u) ? 1 : 0;
+                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                    if (!ok) continue;
+                    const int j = (int)(ip[k] - bb[k]);
+                    const int32_t pj = __shfl_sync(0xFFFFFFFFu, bph[k], j);
+                    const uint32_t kp = __shfl_sync(0xFFFFFFFFu, bkp[k], j);
+                    const uint32_t mj = page_meta(hc[k].n, ip[k] - hc[k].pfx, kp);
+                    if (lane == 0) issue(cw, kk, pj, mj);  // the stage is free: no wait
+                    __syncwarp();
+                    if (k == 0) cnt0 = kk + 1u; else cnt1 = kk + 1u;
+                    moved = true;
+                    if (++ip[k] >= pe[k]) {
+                        hc[k].next(a);
+                        seek(k);
+                        if (on[k]) load_blk(k);
+                    } else if (ip[k] - bb[k] == 32) {
+                        load_blk(k);
+                    }
+                }
+                if (!moved && (++spins & 255u) == 0 && globaltimer_ns() - t0 > 2000000000ull) {
+                    if (lane == 0) record_timeout(a.status, site + 5);
+                    break;
+                }
+            }
+        }
+        cx.wcnt[0] = cnt0;
+        cx.wcnt[1] = cnt1;
+    } else {
+        // ================================ consumers ================================
+        if constexpr (REG_SPLIT) setmaxnreg_inc<CONSUMER_REGS>();
+        uint32_t cnt = cx.wcnt[0];  // pages this warp has taken in the launch
+        typename M::State st;
+        // per head: the window classification inputs, kept count and
+        // candidate count of this warp's share of the head
+        int c = 0, b = 0, n = 0;
+        int64_t pfx = 0;
+        uint32_t cl = 0;
+        uint64_t wlo = 0, whi = 0;
+        int32_t tb = 0;
+        uint32_t kc = 0, ncw = 0;
+        auto head_setup = [&]() {
+            if constexpr (SPEC) {
+                b = c / a.LH;
+                cl = (uint32_t)(c - b * a.LH);
+                wlo = sm.lo()[b];
+                whi = sm.hi()[b];
+                tb = sm.t()[b];
+            }
+            kc = 0;
+            ncw = 0;
+        };
+        // page li of the range in stage sg, the k-th page of this warp
+        auto take_page = [&](int64_t li, int sg, uint32_t k) {
+            mbar_wait(&full[sg], (k / LY::NSW) & 1u, a.status, site + 4);
+            const uint32_t mt = meta[sg];
+            const unsigned char *sk = stage + sg * LY::STAGE_BYTES;
+            uint32_t keepm, evm, candm = 0u, cbase = 0u;
+            float *zdst = nullptr;
+            int zcap = 0;
+            if constexpr (SPEC) {
+                const uint32_t valid = mt >> 16;
+                const int r = lane & 15;
+                const unsigned char *pl = poslb + sg * 128;
+                const int32_t pos = reinterpret_cast<const int32_t *>(pl)[r];
+                const float lbv = reinterpret_cast<const float *>(pl + 64)[r];
+                bool kept = false, cand = false, bad = false;
+                uint64_t K = 0ull;
+                if ((valid >> r) & 1u) {
+                    bad = !entry_key(tb, cl, pos, lbv, a.ibits, &K);
+                    kept = !bad && K < wlo;
+                    cand = !bad && !kept && K < whi;
+                }
+                keepm = __ballot_sync(0xFFFFFFFFu, kept) & 0xFFFFu;
+                candm = __ballot_sync(0xFFFFFFFFu, cand) & 0xFFFFu;
+                if (__ballot_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, RKV_DEV_BAD_INPUT);
+                evm = valid & ~keepm & ~candm;
+                const int64_t pidx = li + cx.x0 - pfx;
+                if (lane == 0) a.keep_mask[(int64_t)c * a.max_pages + pidx] = (uint16_t)keepm;
+                kc += (uint32_t)__popc(keepm);
+                if (candm) {
+                    if (lane == 0) {
+                        cbase = atomicAdd(seqc_of(a, cx) + (size_t)b * 4 + 1, (uint32_t)__popc(candm));
+                        atomicOr(head_flag_of(a, cx) + c, 1u);
+                    }
+                    cbase = __shfl_sync(0xFFFFFFFFu, cbase, 0);
+                    if (lane < 16 && cand) {
+                        const uint32_t idx = cbase + (uint32_t)__popc(candm & ((1u << r) - 1u));
+                        if (idx < (uint32_t)WIN_CAP) {
+                            a.ckey[(size_t)b * WIN_CAP + idx] = K;
+                            a.cslot[(size_t)b * WIN_CAP + idx] = (int32_t)(pidx * PAGE + r);
+                        }
+                    }
+                    zdst = a.cz + ((size_t)b * WIN_CAP + cbase) * G;
+                    zcap = cbase < (uint32_t)WIN_CAP ? (int)(WIN_CAP - cbase) : 0;
+                    ncw += (uint32_t)__popc(candm);
+                }
+            } else {
+                keepm = mt & 0xFFFFu;
+                evm = (mt >> 16) & ~keepm;
+            }
+            M::template page<SPEC>(st, sk, sk + M::PAGE_BYTES, keepm, evm, lane, candm, zdst, zcap);
+            if constexpr (SPEC) {
+                if (candm) {
+                    // set the candidates' V rows aside
+                    uint32_t bits = candm;
+                    uint32_t ck = cbase;
+                    while (bits) {
+                        const int j = __ffs(bits) - 1;
+                        bits &= bits - 1;
+                        if (ck < (uint32_t)WIN_CAP)
+                            M::copy_row(sk + M::PAGE_BYTES, j, a.cv + ((size_t)b * WIN_CAP + ck) * a.row_bytes, lane);
+                        ck++;
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[sg]);
+        };
+        auto zero_head = [&]() {
+            // a head with no entries: o = 0, lse = -inf, dropped = 0
+            for (int e = lane; e < G * D; e += 32) a.out[(int64_t)c * G * D + e] = 0.0f;
+            if (lane < G) {
+                if (a.lse) a.lse[(int64_t)c * G + lane] = -INFINITY;
+                if (a.dropped) a.dropped[(int64_t)c * G + lane] = 0.0f;
+            }
+        };
+        {
+            HeadCursor hcur;
+            hcur.init(a, cx, warp);
+            for (; hcur.valid(cx); hcur.next(a)) {
+                c = hcur.c;
+                n = hcur.n;
+                pfx = hcur.pfx;
+                const int pages = hcur.pages;
+                if (pages == 0) {
+                    zero_head();
+                    continue;
+                }
+                const int64_t pa = max(pfx, (int64_t)cx.x0), pb = min(pfx + pages, (int64_t)cx.x1);
+                const bool whole = (pfx >= cx.x0) && (pfx + pages <= cx.x1);
+                M::load_q(st, a.q + (int64_t)c * G * D, a.qscale, lane);
+                if (c + NCW <= cx.c_last) prefetch_q<G, D>(a.q + (int64_t)(c + NCW) * G * D, lane);
+                head_setup();
+                for (int64_t i = pa; i < pb; i++) {
+                    take_page(i - cx.x0, warp * LY::NSW + (int)(cnt % LY::NSW), cnt);
+                    cnt++;
+                }
+                if constexpr (SPEC) {
+                    if (lane == 0 && kc) {
+                        atomicAdd(head_kept_of(a, cx) + c, kc);
+                        atomicAdd(seqc_of(a, cx) + (size_t)b * 4, kc);
+                    }
+                }
+                // this warp holds the whole head (or this CTA's part of it)
+                float *slot = merge + warp * LY::WSLOT;
+                M::flush(st, slot, lane);
+                __syncwarp();
+                const int dest = whole ? (ncw > 0 ? 1 : 0) : 2;
+                float *rec = dest == 1 ? a.hrec + (int64_t)c * LY::REC
+                                       : a.partial + ((int64_t)blockIdx.x * 2 + ((pfx < cx.x0) ? 0 : 1)) * LY::REC;
+                if (lane < G) {
+                    const int g = lane;
+                    Merged s;
+                    s.mk = slot[G * D + g];
+                    s.lk = slot[G * D + G + g];
+                    s.me = slot[G * D + 2 * G + g];
+                    s.le = slot[G * D + 3 * G + g];
+                    if (dest == 0) {
+                        if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
+                        if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
+                    } else {
+                        rec[G * D + g] = s.mk;
+                        rec[G * D + G + g] = s.lk;
+                        rec[G * D + 2 * G + g] = s.me;
+                        rec[G * D + 3 * G + g] = s.le;
+                    }
+                }
+                for (int e = lane; e < G * D; e += 32) {
+                    if (dest == 0) {
+                        const float lk = slot[G * D + G + e / D];
+                        a.out[(int64_t)c * G * D + e] = lk > 0.0f ? slot[e] / lk : 0.0f;
+                    } else {
+                        rec[e] = slot[e];
+                    }
+                }
+                if (dest == 1 && lane == 0) atomicOr(head_flag_of(a, cx) + c, 2u);
+                __syncwarp();
+            }
+        }
+        cx.wcnt[0] = cnt;
+        if constexpr (REG_SPLIT) setmaxnreg_dec<LAUNCH_REGS>();
+    }
+    __syncthreads();
+    if (warp >= NCW) {
+        if constexpr (REG_SPLIT) setmaxnreg_inc<LAUNCH_REGS>();
+    }
+}
+
 
 // --------------------------------------------------------------- resolve ----
 // After the speculative pass: per sequence, is the M-th key inside the
@@ -2202,7 +2549,8 @@ __global__ void __launch_bounds__(NTH, 1)
     prologue<M, D, G>(a, sm, cx, &tmk, &tmv);
     bool spec = false, local = false;
     if (cx.evict && !sm.misc()[MS_RADIX]) {
-        attn_pass<M, D, G, true>(a, sm, cx, &tmk, &tmv);
+        if (head_per_warp(cx)) attn_pass_hpw<M, D, G, true>(a, sm, cx, &tmk, &tmv);
+        else attn_pass<M, D, G, true>(a, sm, cx, &tmk, &tmv);
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
         const int res = resolve(a, sm, cx);
         if (res != RES_MISS) {
@@ -2222,7 +2570,8 @@ __global__ void __launch_bounds__(NTH, 1)
     if (!spec) {
         if (cx.evict && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(a.status + 3, 1);
         if (cx.evict && !exact_select(a, sm, cx)) return;
-        attn_pass<M, D, G, false>(a, sm, cx, &tmk, &tmv);
+        if (head_per_warp(cx)) attn_pass_hpw<M, D, G, false>(a, sm, cx, &tmk, &tmv);
+        else attn_pass<M, D, G, false>(a, sm, cx, &tmk, &tmv);
         if (!grid_barrier(a.bar, ++cx.epoch, a.status, &sm.misc()[MS_BAR])) return;
     }
     if (!tail<M, D, G>(a, sm, cx, spec, local)) return;
