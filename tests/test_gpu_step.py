@@ -259,6 +259,19 @@ def test_fused_batched_sequences(rkv):
     assert _hits(trace) >= 10, trace
 
 
+@pytest.mark.parametrize("dtype,G,D", [("bf16", 4, 128), ("f32", 2, 64)])
+def test_fused_head_per_warp(rkv, dtype, G, D):
+    # enough short heads that every CTA's range holds at least eight of them:
+    # each consumer warp takes whole heads (prefill eviction, evicting and
+    # non-evicting steps, heads split across CTAs)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    L, H = 12, 8
+    B = min(16, -(-10 * sms // (L * H)))
+    cfg = workloads.small_config(L=L, H=H, G=G, D=D, B=B, T0=300, M=L * H * 220, kv_dtype=dtype, steps=6,
+                                 evict_every=2)
+    run_fused(rkv, cfg, 31 + G, 6)
+
+
 def test_fused_non_evicting_steps_between_evictions(rkv):
     cfg = workloads.small_config(L=2, H=2, G=4, D=128, B=2, T0=1000, M=1500, kv_dtype="bf16", steps=12,
                                  evict_every=3)
