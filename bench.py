@@ -269,7 +269,7 @@ def run_config(name: str, args, world: int, rank: int, local: int, *, e2e: bool)
     dc = workloads.prefill_cache(cfg, seed, device=dev, n_steps=total)
     cache = rkv.Cache.from_tensors(dc, cfg.B, cfg.L, cfg.H, cfg.Hq)
     stream = torch.cuda.Stream(device=dev)
-    runner = rkv.StepRunner(cache, scale=cfg.scale, stream=stream, fused=fused)
+    runner = rkv.StepRunner(cache, scale=cfg.scale, stream=stream, fused=fused, buffers=2)
     sel, ws, outs = runner.sel, runner.ws, runner.outs
     per_step = [workloads.step_inputs(cfg, seed, s, dev) for s in range(total)]
     kernel_names = ["step"] if fused else ["select", "attn", "compact", "append"]
@@ -571,6 +571,7 @@ def run_e2e(runner, per_step, s_next, W, K, stream, world, local, dev):
         evict.append(bool(inp["evict"]))
     for i in range(W):
         runner.run_host(host_in[i], host_out[i], evict[i])
+    runner.finish()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
@@ -579,6 +580,7 @@ def run_e2e(runner, per_step, s_next, W, K, stream, world, local, dev):
         a.record(stream)
         for i in range(W, W + K):
             runner.run_host(host_in[i], host_out[i], evict[i])
+        runner.finish()
         b.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -586,7 +588,8 @@ def run_e2e(runner, per_step, s_next, W, K, stream, world, local, dev):
     if runner.ws.status() != 0:
         raise RuntimeError(f"device status {runner.ws.counters()} after the e2e steps")
     rec = {"value": world * K / (e2e_ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": runner.in_bytes,
-           "d2h_bytes_per_step": runner.out_bytes, "graph": bool(runner.graphs)}
+           "d2h_bytes_per_step": runner.out_bytes, "graph": bool(runner.graphs),
+           "copies": "two buffer slots: step s+1's inputs and step s-1's outputs copied on a second stream while step s runs"}
     return rec, s_next + W + K, clk2.summary()
 
 

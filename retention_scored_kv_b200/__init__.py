@@ -431,7 +431,9 @@ class StepRunner:
     offset, shape and dtype so callers can pack pinned host buffers."""
 
     def __init__(self, cache: Cache, *, scale: float | None = None, use_graph: bool = True, fused: bool = True,
-                 stream=None):
+                 stream=None, buffers: int = 1):
+        if buffers not in (1, 2):
+            raise ValueError("buffers must be 1 or 2")
         self.cache = cache
         self.fused = fused
         self.scale = 1.0 / math.sqrt(cache.D) if scale is None else scale
@@ -453,16 +455,27 @@ class StepRunner:
             self.out_layout[name] = (off, shape, torch.float32)
             off = _align(off + math.prod(shape) * 4)
         self.out_bytes = off
-        self.inbuf = torch.zeros(self.in_bytes, dtype=torch.uint8, device=dev)
-        self.outbuf = torch.zeros(self.out_bytes, dtype=torch.uint8, device=dev)
-        self.inp = {k: self._view(self.inbuf, *v) for k, v in self.in_layout.items()}
-        o = {k: self._view(self.outbuf, *v) for k, v in self.out_layout.items()}
-        self.outs = StepOutputs(o["out"], o["lse"], o["dropped"])
+        # one set of device buffers per slot; with two, run_host overlaps a
+        # step's copies with its neighbours' compute (copies on their own stream)
+        self.inbufs = [torch.zeros(self.in_bytes, dtype=torch.uint8, device=dev) for _ in range(buffers)]
+        self.outbufs = [torch.zeros(self.out_bytes, dtype=torch.uint8, device=dev) for _ in range(buffers)]
+        self.inps = [{k: self._view(b, *v) for k, v in self.in_layout.items()} for b in self.inbufs]
+        self.outss = []
+        for b in self.outbufs:
+            o = {k: self._view(b, *v) for k, v in self.out_layout.items()}
+            self.outss.append(StepOutputs(o["out"], o["lse"], o["dropped"]))
+        self.inbuf, self.outbuf, self.inp, self.outs = self.inbufs[0], self.outbufs[0], self.inps[0], self.outss[0]
         self.sel = Selection.empty(cache)
         self.ws = Workspace(cache, self.stream)
         self.use_graph = use_graph
         self.capture_error: str | None = None
-        self.graphs: dict[bool, torch.cuda.CUDAGraph] = {}
+        self.graphs: dict[tuple[int, bool], torch.cuda.CUDAGraph] = {}
+        self.buffers = buffers
+        self.copy_stream = torch.cuda.Stream(device=dev) if buffers > 1 else None
+        self._ev = [{k: torch.cuda.Event() for k in ("in", "done", "out")} for _ in range(buffers)]
+        self._n = 0                # steps submitted through run_host
+        self._pending = None       # (host_out, slot) whose copy-out is not enqueued yet
+        self._restart = True       # the next copy follows the runner's stream
 
     @staticmethod
     def _view(buf: torch.Tensor, off: int, shape, dt) -> torch.Tensor:
@@ -477,9 +490,9 @@ class StepRunner:
     def unpack(self, host: torch.Tensor) -> dict:
         return {k: self._view(host, *v) for k, v in self.out_layout.items()}
 
-    def _enqueue(self, evict: bool) -> None:
-        i = self.inp
-        step(self.cache, self.sel, self.ws, self.outs, q=i["q"], t=i["t"], m_global=i["m_global"],
+    def _enqueue(self, evict: bool, slot: int = 0) -> None:
+        i = self.inps[slot]
+        step(self.cache, self.sel, self.ws, self.outss[slot], q=i["q"], t=i["t"], m_global=i["m_global"],
              k_new=i["k_new"], v_new=i["v_new"], lb_new=i["lb_new"], evict=evict, scale=self.scale,
              fused=self.fused, stream=self.stream)
 
@@ -492,11 +505,12 @@ class StepRunner:
             self.use_graph = False
             return False
         try:
-            for evict in (True, False):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
-                    self._enqueue(evict)
-                self.graphs[evict] = g
+            for slot in range(self.buffers):
+                for evict in (True, False):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
+                        self._enqueue(evict, slot)
+                    self.graphs[(slot, evict)] = g
             return True
         except Exception as ex:
             self.capture_error = f"{type(ex).__name__}: {ex}"
@@ -504,19 +518,64 @@ class StepRunner:
             self.use_graph = False
             return False
 
-    def run(self, evict: bool = True) -> None:
-        """Run one step on the inputs already in the static device buffer."""
-        g = self.graphs.get(evict)
+    def run(self, evict: bool = True, slot: int = 0) -> None:
+        """Run one step on the inputs already in a slot's static device buffer."""
+        g = self.graphs.get((slot, evict))
         if g is not None:
             with torch.cuda.stream(self.stream):
                 g.replay()
         else:
-            self._enqueue(evict)
+            self._enqueue(evict, slot)
 
     def run_host(self, host_in: torch.Tensor, host_out: torch.Tensor, evict: bool = True) -> None:
-        """Copy packed host inputs in, run the step, copy packed outputs out (async)."""
-        with torch.cuda.stream(self.stream):
-            self.inbuf.copy_(host_in, non_blocking=True)
-        self.run(evict)
-        with torch.cuda.stream(self.stream):
-            host_out.copy_(self.outbuf, non_blocking=True)
+        """Copy packed host inputs in, run the step, copy packed outputs out (async).
+
+        With two buffer slots the copies go on a copy stream: step n's inputs
+        are copied while step n - 1 runs, and step n - 1's outputs are copied
+        out after step n's inputs (so they overlap step n).  ``finish()``
+        enqueues the last copy-out and orders it before later work on the
+        runner's stream."""
+        if self.buffers == 1:
+            with torch.cuda.stream(self.stream):
+                self.inbuf.copy_(host_in, non_blocking=True)
+            self.run(evict)
+            with torch.cuda.stream(self.stream):
+                host_out.copy_(self.outbuf, non_blocking=True)
+            return
+        p = self._n % 2
+        cs, ev = self.copy_stream, self._ev[p]
+        if self._restart:
+            cs.wait_stream(self.stream)
+            self._restart = False
+        with torch.cuda.stream(cs):
+            if self._n >= 2:
+                cs.wait_event(ev["done"])      # the slot's previous step has read its inputs
+            self.inbufs[p].copy_(host_in, non_blocking=True)
+            ev["in"].record(cs)
+        self._flush_out()
+        self.stream.wait_event(ev["in"])
+        if self._n >= 2:
+            self.stream.wait_event(ev["out"])  # the slot's previous outputs are copied out
+        self.run(evict, p)
+        ev["done"].record(self.stream)
+        self._pending = (host_out, p)
+        self._n += 1
+
+    def _flush_out(self) -> None:
+        if self._pending is None:
+            return
+        host_out, p = self._pending
+        cs, ev = self.copy_stream, self._ev[p]
+        with torch.cuda.stream(cs):
+            cs.wait_event(ev["done"])
+            host_out.copy_(self.outbufs[p], non_blocking=True)
+            ev["out"].record(cs)
+        self._pending = None
+
+    def finish(self) -> None:
+        """Enqueue the last step's copy-out; later work on the runner's stream follows it."""
+        if self.buffers == 1:
+            return
+        self._flush_out()
+        self.stream.wait_stream(self.copy_stream)
+        self._restart = True

@@ -397,3 +397,39 @@ def test_fused_graph_replay(rkv):
                              ref["dropped"], ref["kept"] > 0)
         compare_state(dc, hc)
     assert runner.ws.status() == 0
+
+
+def test_runner_two_buffer_slots_match_one(rkv):
+    # run_host with two buffer slots (copies overlapped with the neighbouring
+    # steps on a second stream) gives the same outputs and cache as one slot
+    cfg = workloads.small_config(L=2, H=2, G=4, D=128, B=2, T0=1500, M=2500, kv_dtype="bf16", steps=8,
+                                 evict_every=2)
+    dcs = [to_dev(workloads.prefill_cache(cfg, 12, n_steps=9)) for _ in range(2)]
+    runners = [rkv.StepRunner(rkv_cache(rkv, dc), scale=cfg.scale, fused=True, stream=torch.cuda.Stream(),
+                              buffers=nb) for dc, nb in zip(dcs, (1, 2))]
+    steps = [workloads.step_inputs(cfg, 12, s, "cuda") for s in range(8)]
+    outs = [[], []]
+    for r, runner in enumerate(runners):
+        host_in = [torch.empty(runner.in_bytes, dtype=torch.uint8, pin_memory=True) for _ in steps]
+        host_out = [torch.zeros(runner.out_bytes, dtype=torch.uint8, pin_memory=True) for _ in steps]
+        for s, inp in enumerate(steps):
+            runner.pack(host_in[s], q=inp["q"].cpu(), k_new=inp["k_new"].cpu(), v_new=inp["v_new"].cpu(),
+                        lb_new=inp["lb_new"].cpu(), t=inp["t"].cpu(), m_global=inp["m_global"].cpu())
+        runner.run_host(host_in[0], host_out[0], bool(steps[0]["evict"]))   # exact first call, eager
+        runner.finish()
+        sync()
+        assert runner.capture(), runner.capture_error
+        for s in range(1, len(steps)):
+            runner.run_host(host_in[s], host_out[s], bool(steps[s]["evict"]))
+        runner.finish()
+        sync()
+        assert runner.ws.status() == 0
+        outs[r] = [runner.unpack(h) for h in host_out]
+    for s in range(len(steps)):
+        for k in ("out", "lse", "dropped"):
+            # (the order in which candidates enter a merge can differ between
+            # runs, so the sums may differ in the last bits)
+            np.testing.assert_allclose(outs[1][s][k].numpy(), outs[0][s][k].numpy(), rtol=1e-5, atol=1e-6,
+                                       err_msg=f"step {s}: {k}")
+    for name in ("len", "block_table", "k_pool", "v_pool", "pos_pool", "free_top"):
+        assert torch.equal(getattr(dcs[0], name), getattr(dcs[1], name)), name
