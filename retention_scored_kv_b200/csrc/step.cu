@@ -737,9 +737,11 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
             named_bar_sync(1, NCW * 32);
 
             // ---- merge the warps (consumer threads) ----
-            // per query row (one thread each): merged statistics, and each
-            // warp's weight 2^(mk_w - mk) in a table; then every output
-            // element is the weighted sum of the warps' parts
+            // per query row g (eight lanes, one per warp part): merged
+            // statistics by 8-lane shuffles, and each warp's weight
+            // 2^(mk_w - mk) in a table; then every output element is the
+            // weighted sum of the warps' parts
+            static_assert(NCW == 8 && G <= 8, "eight lanes per query row in two warps");
             const float *mb = merge + par * NCW * LY::WSLOT;
             float *fac = reinterpret_cast<float *>(sm.big() + LY::B_MFAC) + par * LY::MFAC;
             float hc = 0.0f;
@@ -749,37 +751,41 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
             const int dest = whole ? (hc > 0.0f ? 1 : 0) : 2;
             float *rec = dest == 1 ? a.hrec + (int64_t)c * LY::REC
                                    : a.partial + ((int64_t)blockIdx.x * 2 + ((pfx < cx.x0) ? 0 : 1)) * LY::REC;
-            if (tid < G) {
-                const int g = tid;
+            if (tid < 64) {
+                const int g = tid >> 3, wi = tid & 7;
+                const bool on = g < G;
+                const float *src = mb + wi * LY::WSLOT;
+                const float mkw = on ? src[G * D + g] : -INFINITY, mew = on ? src[G * D + 2 * G + g] : -INFINITY;
+                const float lkw = on ? src[G * D + G + g] : 0.0f, lew = on ? src[G * D + 3 * G + g] : 0.0f;
                 Merged s;
-                s.mk = -INFINITY;
-                s.me = -INFINITY;
+                s.mk = mkw;
+                s.me = mew;
 #pragma unroll
-                for (int wi = 0; wi < NCW; wi++) {
-                    s.mk = fmaxf(s.mk, mb[wi * LY::WSLOT + G * D + g]);
-                    s.me = fmaxf(s.me, mb[wi * LY::WSLOT + G * D + 2 * G + g]);
+                for (int o = 1; o < 8; o <<= 1) {
+                    s.mk = fmaxf(s.mk, __shfl_xor_sync(0xFFFFFFFFu, s.mk, o));
+                    s.me = fmaxf(s.me, __shfl_xor_sync(0xFFFFFFFFu, s.me, o));
                 }
-                s.lk = 0.0f;
-                s.le = 0.0f;
+                const float fk = (mkw == -INFINITY) ? 0.0f : ex2(mkw - s.mk);
+                const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
+                s.lk = lkw * fk;
+                s.le = lew * fe;
 #pragma unroll
-                for (int wi = 0; wi < NCW; wi++) {
-                    const float *src = mb + wi * LY::WSLOT;
-                    const float mkw = src[G * D + g], mew = src[G * D + 2 * G + g];
-                    const float fk = (mkw == -INFINITY) ? 0.0f : ex2(mkw - s.mk);
-                    const float fe = (mew == -INFINITY) ? 0.0f : ex2(mew - s.me);
-                    s.lk += src[G * D + G + g] * fk;
-                    s.le += src[G * D + 3 * G + g] * fe;
-                    fac[g * NCW + wi] = fk;
+                for (int o = 1; o < 8; o <<= 1) {
+                    s.lk += __shfl_xor_sync(0xFFFFFFFFu, s.lk, o);
+                    s.le += __shfl_xor_sync(0xFFFFFFFFu, s.le, o);
                 }
-                fac[G * NCW + g] = s.lk;
-                if (dest == 0) {
-                    if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
-                    if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
-                } else {
-                    rec[G * D + g] = s.mk;
-                    rec[G * D + G + g] = s.lk;
-                    rec[G * D + 2 * G + g] = s.me;
-                    rec[G * D + 3 * G + g] = s.le;
+                if (on) fac[g * NCW + wi] = fk;
+                if (on && wi == 0) {
+                    fac[G * NCW + g] = s.lk;
+                    if (dest == 0) {
+                        if (a.lse) a.lse[(int64_t)c * G + g] = s.lk > 0.0f ? (s.mk + __log2f(s.lk)) * LN2 : -INFINITY;
+                        if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
+                    } else {
+                        rec[G * D + g] = s.mk;
+                        rec[G * D + G + g] = s.lk;
+                        rec[G * D + 2 * G + g] = s.me;
+                        rec[G * D + 3 * G + g] = s.le;
+                    }
                 }
             }
             named_bar_sync(1, NCW * 32);
