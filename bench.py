@@ -71,7 +71,7 @@ SPLIT_STEPS = 32  # event-timed steps for the evicting / non-evicting split
 # capture (read 218.83 MB + write 5.03 MB) x8 to the full 32-layer launch
 # (pages, hence traffic, grow with the layer count).  Reported only while the
 # kernel's sources hash to the captured version.
-STEP_TRAFFIC = {"sources_sha256": "a616379852524a2f", "workload": "long128k", "bytes_per_launch": 8 * 224.088576e6}
+STEP_TRAFFIC = {"sources_sha256": "029e3e155edfa685", "workload": "long128k", "bytes_per_launch": 8 * 224.378112e6}
 
 
 # ------------------------------------------------------------------ ranks ---
