@@ -448,7 +448,7 @@ int orc_attention(const orc_cache *cc, const float *q, float scale, const uint8_
 
 /* ------------------------------------------------------- eviction error ---
  * [ContourKV] Methodology 1 (theoretical analysis and enumeration): a kept
- * subset A is judged by the distance between the dense attention output mu
+ * subset A is scored by the distance between the dense attention output mu
  * and the forced-weight output m_A over A:
  *   e(A) = || mu - m_A ||,
  *   mu  = sum_{j all}  exp(z_j) v_j / sum_{j all}  exp(z_j),

@@ -1,6 +1,6 @@
 // evict_err.cu -- eviction error of a selection (sm_100a).
 //
-// Trust the Mass (ContourKV), Methodology 1: a kept subset A is judged by
+// Trust the Mass (ContourKV), Methodology 1: a kept subset A is scored by
 // e(A) = ||mu - m_A||, the distance between the dense attention output mu
 // and the forced-weight output m_A over A.  mu mixes the kept and the
 // evicted outputs by the dropped mass dm: mu = (1 - dm) m_A + dm m_ev, so

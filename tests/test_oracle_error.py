@@ -1,7 +1,7 @@
 """Pins of the oracle's eviction error.
 
 Trust the Mass (ContourKV), Methodology 1 (theoretical analysis and
-enumeration): a kept subset A is judged by e(A) = ||mu - m_A||, the distance
+enumeration): a kept subset A is scored by e(A) = ||mu - m_A||, the distance
 between the dense attention output mu and the forced-weight output m_A over
 A.  Readings: Euclidean norm over the head dimension, per query head; a head
 with no entries has e = 0; with nothing kept m_A = 0, so e = ||mu||.
