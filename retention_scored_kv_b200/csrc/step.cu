@@ -1844,12 +1844,57 @@ __device__ void combine_head(const StepArgs &a, const Sm &sm, const Ctx &cx, int
 // accumulates EPL output elements with the records' loads issued together.
 // Returns false (nothing written) when the head has more than RCAP records
 // or CCAP candidates; the block-wide merge handles it then.
+// VW consecutive floats from p (one 16-byte load when VW is 4), zeros when !ok.
+template <int VW>
+__device__ __forceinline__ void load_group(float (&v)[VW], const float *p, bool ok) {
+    if constexpr (VW == 4) {
+        const float4 x = ok ? __ldcg(reinterpret_cast<const float4 *>(p)) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        v[0] = x.x;
+        v[1] = x.y;
+        v[2] = x.z;
+        v[3] = x.w;
+    } else {
+#pragma unroll
+        for (int q = 0; q < VW; q++) v[q] = ok ? __ldcg(p + q) : 0.0f;
+    }
+}
+template <int VW>
+__device__ __forceinline__ void store_group(float *p, const float (&v)[VW]) {
+    if constexpr (VW == 4) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+#pragma unroll
+        for (int q = 0; q < VW; q++) p[q] = v[q];
+    }
+}
+// Elements d .. d + VW - 1 of a V row in the pool dtype, as floats.
+template <class M, int VW>
+__device__ __forceinline__ void row_group(float (&r)[VW], const unsigned char *row, int d) {
+    if constexpr (VW == 4 && M::ROW_BYTES / M::DIM == 2) {
+        const uint2 x = __ldcg(reinterpret_cast<const uint2 *>(row) + d / 4);
+        r[0] = __uint_as_float(x.x << 16);
+        r[1] = __uint_as_float(x.x & 0xFFFF0000u);
+        r[2] = __uint_as_float(x.y << 16);
+        r[3] = __uint_as_float(x.y & 0xFFFF0000u);
+    } else if constexpr (VW == 4) {
+        const float4 x = __ldcg(reinterpret_cast<const float4 *>(row) + d / 4);
+        r[0] = x.x;
+        r[1] = x.y;
+        r[2] = x.z;
+        r[3] = x.w;
+    } else {
+#pragma unroll
+        for (int q = 0; q < VW; q++) r[q] = row_elt<M>(row, d + q);
+    }
+}
+
 template <class M, int D, int G>
 __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, WarpScr &w, int c, int64_t pfx,
                              int jf, int jl, uint32_t flag, bool cands, bool local) {
     using LY = StepLayout<M, D, G>;
     constexpr int GD = G * D;
-    constexpr int EPL = (GD + 31) / 32;
+    constexpr int VW = GD % 128 == 0 ? 4 : 1;
+    constexpr int NU = (GD + 32 * VW - 1) / (32 * VW);
     const int lane = threadIdx.x & 31;
     const int b = c / a.LH;
     const int cl = c - b * a.LH;
@@ -1914,13 +1959,15 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
     }
     for (int t = lane; t < ncl * G; t += 32) w.cz[t] = __ldcg(a.cz + (cb + w.cidx[t / G]) * G + (t % G));
     for (int i = lane; i < ncl; i += 32) w.cfate[i] = cand_fate(a, sm, local, b, w.cidx[i]);
-    // the first two records' output values, in the same round
-    float v0[EPL], v1[EPL];
+    // the first two records' output values, in the same round: each lane
+    // holds NU groups of VW consecutive elements (e = (lane + 32 u) VW + q;
+    // 16-byte loads and stores when the row length allows)
+    float v0[NU][VW], v1[NU][VW];
 #pragma unroll
-    for (int u = 0; u < EPL; u++) {
-        const int e = lane + 32 * u;
-        v0[u] = (nrec > 0 && e < GD) ? __ldcg(w.recp[0] + e) : 0.0f;
-        v1[u] = (nrec > 1 && e < GD) ? __ldcg(w.recp[1] + e) : 0.0f;
+    for (int u = 0; u < NU; u++) {
+        const int e = (lane + 32 * u) * VW;
+        load_group<VW>(v0[u], w.recp[0] + e, nrec > 0 && e < GD);
+        load_group<VW>(v1[u], w.recp[1] + e, nrec > 1 && e < GD);
     }
     __syncwarp();
     // ---- per query row: merged maxima, sums, lse and dropped mass ----
@@ -1964,41 +2011,54 @@ __device__ bool combine_warp(const StepArgs &a, const Sm &sm, const Ctx &cx, War
         if (a.dropped) a.dropped[(int64_t)c * G + g] = dm_of(s);
     }
     __syncwarp();
-    // ---- outputs: EPL elements per lane, two records' loads in flight at a time ----
-    float av[EPL];
+    // ---- outputs: NU groups of VW elements per lane, two records' loads in flight at a time ----
+    float av[NU][VW];
 #pragma unroll
-    for (int u = 0; u < EPL; u++) {
-        const int e = lane + 32 * u;
-        const int g = (e < GD ? e : 0) / D;
-        av[u] = (nrec > 0 ? v0[u] * w.fk[g] : 0.0f) + (nrec > 1 ? v1[u] * w.fk[G + g] : 0.0f);
+    for (int u = 0; u < NU; u++) {
+        const int e = (lane + 32 * u) * VW;
+        const int g = (e < GD ? e : 0) / D;  // (a group never straddles two query rows)
+#pragma unroll
+        for (int q = 0; q < VW; q++)
+            av[u][q] = (nrec > 0 ? v0[u][q] * w.fk[g] : 0.0f) + (nrec > 1 ? v1[u][q] * w.fk[G + g] : 0.0f);
     }
     for (int k = 2; k < nrec; k++) {
 #pragma unroll
-        for (int u = 0; u < EPL; u++) {
-            const int e = lane + 32 * u;
-            v0[u] = e < GD ? __ldcg(w.recp[k] + e) : 0.0f;
+        for (int u = 0; u < NU; u++) {
+            const int e = (lane + 32 * u) * VW;
+            load_group<VW>(v0[u], w.recp[k] + e, e < GD);
         }
 #pragma unroll
-        for (int u = 0; u < EPL; u++) {
-            const int e = lane + 32 * u;
-            av[u] += v0[u] * w.fk[k * G + (e < GD ? e : 0) / D];
+        for (int u = 0; u < NU; u++) {
+            const int e = (lane + 32 * u) * VW;
+            const float f = w.fk[k * G + (e < GD ? e : 0) / D];
+#pragma unroll
+            for (int q = 0; q < VW; q++) av[u][q] += v0[u][q] * f;
         }
     }
     for (int i = 0; i < ncl; i++) {
         if (!w.cfate[i]) continue;
         const unsigned char *row = a.cv + (cb + w.cidx[i]) * a.row_bytes;
 #pragma unroll
-        for (int u = 0; u < EPL; u++) {
-            const int e = lane + 32 * u;
-            if (e < GD) av[u] += w.cz[i * G + e / D] * row_elt<M>(row, e % D);
+        for (int u = 0; u < NU; u++) {
+            const int e = (lane + 32 * u) * VW;
+            if (e < GD) {
+                float r[VW];
+                row_group<M, VW>(r, row, e % D);
+                const float f = w.cz[i * G + e / D];
+#pragma unroll
+                for (int q = 0; q < VW; q++) av[u][q] += f * r[q];
+            }
         }
     }
 #pragma unroll
-    for (int u = 0; u < EPL; u++) {
-        const int e = lane + 32 * u;
+    for (int u = 0; u < NU; u++) {
+        const int e = (lane + 32 * u) * VW;
         if (e < GD) {
             const float lk = w.lk[e / D];
-            a.out[(int64_t)c * GD + e] = lk > 0.0f ? av[u] / lk : 0.0f;
+            float o[VW];
+#pragma unroll
+            for (int q = 0; q < VW; q++) o[q] = lk > 0.0f ? av[u][q] / lk : 0.0f;
+            store_group<VW>(a.out + (int64_t)c * GD + e, o);
         }
     }
     __syncwarp();
