@@ -789,16 +789,28 @@ __device__ __forceinline__ void attn_pass(const StepArgs &a, const Sm &sm, Ctx &
                 }
             }
             named_bar_sync(1, NCW * 32);
-            for (int e = tid; e < G * D; e += NCW * 32) {
+            // four consecutive elements per thread (16-byte loads and stores:
+            // slots, records and rows of outputs are 16-byte multiples)
+            static_assert((G * D) % 4 == 0 && LY::WSLOT % 4 == 0 && LY::REC % 4 == 0, "16-byte groups");
+            for (int e = tid * 4; e < G * D; e += NCW * 32 * 4) {
                 const int g = e / D;
-                float av = 0.0f;
+                float4 av = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-                for (int wi = 0; wi < NCW; wi++) av += mb[wi * LY::WSLOT + e] * fac[g * NCW + wi];
+                for (int wi = 0; wi < NCW; wi++) {
+                    const float4 x = *reinterpret_cast<const float4 *>(mb + wi * LY::WSLOT + e);
+                    const float f = fac[g * NCW + wi];
+                    av.x += x.x * f;
+                    av.y += x.y * f;
+                    av.z += x.z * f;
+                    av.w += x.w * f;
+                }
                 if (dest == 0) {
                     const float lk = fac[G * NCW + g];
-                    a.out[(int64_t)c * G * D + e] = lk > 0.0f ? av / lk : 0.0f;
+                    float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if (lk > 0.0f) o = make_float4(av.x / lk, av.y / lk, av.z / lk, av.w / lk);
+                    *reinterpret_cast<float4 *>(a.out + (int64_t)c * G * D + e) = o;
                 } else {
-                    rec[e] = av;
+                    *reinterpret_cast<float4 *>(rec + e) = av;
                 }
             }
             if (dest == 1 && tid == 0) atomicOr(head_flag_of(a, cx) + c, 2u);
@@ -1090,12 +1102,15 @@ __device__ __forceinline__ void attn_pass_hpw(const StepArgs &a, const Sm &sm, C
                         rec[G * D + 3 * G + g] = s.le;
                     }
                 }
-                for (int e = lane; e < G * D; e += 32) {
+                for (int e = lane * 4; e < G * D; e += 32 * 4) {  // 16-byte groups
+                    const float4 x = *reinterpret_cast<const float4 *>(slot + e);
                     if (dest == 0) {
                         const float lk = slot[G * D + G + e / D];
-                        a.out[(int64_t)c * G * D + e] = lk > 0.0f ? slot[e] / lk : 0.0f;
+                        float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        if (lk > 0.0f) o = make_float4(x.x / lk, x.y / lk, x.z / lk, x.w / lk);
+                        *reinterpret_cast<float4 *>(a.out + (int64_t)c * G * D + e) = o;
                     } else {
-                        rec[e] = slot[e];
+                        *reinterpret_cast<float4 *>(rec + e) = x;
                     }
                 }
                 if (dest == 1 && lane == 0) atomicOr(head_flag_of(a, cx) + c, 2u);
