@@ -435,11 +435,10 @@ struct MmaMath {
         }
         if (g < G) {
             if constexpr (WITH_V) {
+                // (column pairs 2t, 2t + 1: one 8-byte store each; slots are 8-byte aligned)
 #pragma unroll
-                for (int i = 0; i < NT; i++) {
-                    slot[g * D + i * 8 + 2 * t] = s.o[i][0];
-                    slot[g * D + i * 8 + 2 * t + 1] = s.o[i][1];
-                }
+                for (int i = 0; i < NT; i++)
+                    *reinterpret_cast<float2 *>(slot + g * D + i * 8 + 2 * t) = make_float2(s.o[i][0], s.o[i][1]);
             }
             if (t == 0) {
                 slot[G * D + g] = s.mk;
