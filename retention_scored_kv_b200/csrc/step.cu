@@ -282,6 +282,19 @@ __device__ __forceinline__ bool entry_key(int32_t t, uint32_t cl, int32_t pos, f
     return true;
 }
 
+// The same key's hi word alone, under the same rejection rule, in 32-bit
+// arithmetic: plim = 2^ibits (2^31 for ibits = 32), so one unsigned compare
+// rejects negative and out-of-range positions; with pos >= 0, t > pos keeps
+// t - pos from overflowing.  The lo word is (cl << ibits) | pos, truncated to
+// 32 bits.
+__device__ __forceinline__ bool entry_key_hi(int32_t t, int32_t pos, float lb, uint32_t plim, uint32_t *hi) {
+    if ((uint32_t)pos >= plim || t <= pos || (uint32_t)t - (uint32_t)pos >= (1u << 24) || lb != lb) return false;
+    float s = __fmul_rn((float)(int32_t)((uint32_t)t - (uint32_t)pos), lb);
+    if (s == 0.0f) s = 0.0f;
+    *hi = score_key_desc(s);
+    return true;
+}
+
 __device__ __forceinline__ uint32_t below_bits(int w, int nn) {
     const int lo = w * PAGE;
     if (lo + PAGE <= nn) return 0xFFFFu;
@@ -1427,8 +1440,9 @@ __device__ void own_list_grid(const StepArgs &a, const Sm &sm) {
 // Calls f(c, pidx, n, key) for every page of this CTA's range, one page per
 // thread per round (lanes of a warp hold consecutive pages).  c = head (-1 for
 // a thread without a page), pidx = page index in the head, n = valid slots of
-// the page, key(r, K) = the entry key of slot r < n (false, with the status
-// flagged, for an entry rejected as bad input).  Every thread calls f, so f
+// the page, khi(r, hi) = the hi word of slot r's entry key (r < n; false,
+// with the status flagged, for an entry rejected as bad input) and klo(r) =
+// its lo word (valid only where khi returned true).  Every thread calls f, so f
 // may use warp collectives.  Loads are pipelined across rounds: a round's 16
 // positions and 16 log-retentions per page (16-byte vectors) are in flight
 // together with the next round's head lengths and block-table entries.  The
@@ -1524,16 +1538,21 @@ __device__ __forceinline__ void for_range_pages(const StepArgs &a, const Sm &sm,
             const int b = c >= 0 ? c / a.LH : 0;
             const int32_t tb = sm.t()[b];
             const uint32_t cl = (uint32_t)(c - b * a.LH);
-            auto key = [&](int r, uint64_t &K) -> bool {
+            const uint32_t plim = a.ibits < 32 ? (1u << a.ibits) : 0x80000000u;
+            const uint32_t clsh = (uint32_t)((uint64_t)cl << a.ibits);
+            auto pos_of = [&](int r) -> int32_t {
                 const int4 &pq = pv[r >> 2];
+                return (r & 3) == 0 ? pq.x : (r & 3) == 1 ? pq.y : (r & 3) == 2 ? pq.z : pq.w;
+            };
+            auto khi = [&](int r, uint32_t &hi) -> bool {
                 const float4 &lq = lv[r >> 2];
-                const int32_t ps = (r & 3) == 0 ? pq.x : (r & 3) == 1 ? pq.y : (r & 3) == 2 ? pq.z : pq.w;
                 const float ls = (r & 3) == 0 ? lq.x : (r & 3) == 1 ? lq.y : (r & 3) == 2 ? lq.z : lq.w;
-                if (entry_key(tb, cl, ps, ls, a.ibits, &K)) return true;
+                if (entry_key_hi(tb, pos_of(r), ls, plim, &hi)) return true;
                 set_status(a.status, RKV_DEV_BAD_INPUT);
                 return false;
             };
-            f(c, pidx, n, key);
+            auto klo = [&](int r) -> uint32_t { return clsh | (uint32_t)pos_of(r); };
+            f(c, pidx, n, khi, klo);
         }
         c = cn;
         pidx = pn;
@@ -1646,19 +1665,30 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
     uint32_t *hist = reinterpret_cast<uint32_t *>(sm.big());
     // digit p's histogram of the sequences [g0, g1) this sweep counts
     int p = 0, g0 = 0, g1 = 0;
-    auto count = [&](int c, int, int n, auto &key) {
+    auto count = [&](int c, int, int n, auto &khi, auto &klo) {
         if (c < 0) return;
         const int b = c / a.LH;
         if (b < g0 || b >= g1 || (sm.fl()[b] & SF_DONE)) return;
         const uint64_t pk = sm.pk()[b], pm = sm.pm()[b];
+        const uint32_t pkh = (uint32_t)(pk >> 32), pmh = (uint32_t)(pm >> 32);
+        const uint32_t pkl = (uint32_t)pk, pml = (uint32_t)pm;
+        // digit p lies in the hi word for p < 3 (the lo word is then not
+        // needed: its prefix bits are still unset), else in the lo word
+        const bool in_lo = p >= 3;
+        const int sh = digit_shift(p) & 31;
+        const uint32_t dmask = (1u << digit_bits(p)) - 1u;
         uint32_t *hb = hist + (b - g0) * NBINS;
         // a page's neighbouring entries mostly share a bin: add runs
         uint32_t run_bin = 0u, run_n = 0u;
 #pragma unroll
         for (int r = 0; r < PAGE; r++) {
-            uint64_t K;
-            if (r >= n || !key(r, K) || ((K ^ pk) & pm) != 0ull) continue;
-            const uint32_t bin = key_digit((uint32_t)(K >> 32), (uint32_t)K, p);
+            uint32_t w;
+            if (r >= n || !khi(r, w) || ((w ^ pkh) & pmh) != 0u) continue;
+            if (in_lo) {
+                w = klo(r);
+                if (((w ^ pkl) & pml) != 0u) continue;
+            }
+            const uint32_t bin = (w >> sh) & dmask;
             if (run_n && bin == run_bin) {
                 run_n++;
             } else {
@@ -1699,11 +1729,12 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
     // is that key + 1: a radix bucket kept whole only bounds it)
     int kb = -1;
     unsigned long long km = 0ull;
-    auto mark = [&](int c, int pidx, int n, auto &key) {
+    auto mark = [&](int c, int pidx, int n, auto &khi, auto &klo) {
         uint32_t m16 = 0u;
         if (c >= 0) {
             const int b = c / a.LH;
             const uint64_t kap = sm.kap()[b];
+            const uint32_t kaph = (uint32_t)(kap >> 32), kapl = (uint32_t)kap;
             if (b != kb) {
                 if (kb >= 0) atomicMax(sm.kmx() + kb, km);
                 kb = b;
@@ -1711,10 +1742,15 @@ __device__ bool exact_select(const StepArgs &a, const Sm &sm, Ctx &cx) {
             }
 #pragma unroll
             for (int r = 0; r < PAGE; r++) {
-                uint64_t K;
-                if (r < n && key(r, K) && K < kap) {
-                    m16 |= 1u << r;
-                    km = K > km ? K : km;
+                // K < kap on the two words: the lo word only on a hi tie
+                uint32_t hi;
+                if (r < n && khi(r, hi) && hi <= kaph) {
+                    const uint32_t lo = klo(r);
+                    if (hi < kaph || lo < kapl) {
+                        m16 |= 1u << r;
+                        const uint64_t K = ((uint64_t)hi << 32) | lo;
+                        km = K > km ? K : km;
+                    }
                 }
             }
             a.keep_mask[(int64_t)c * a.max_pages + pidx] = (uint16_t)m16;
