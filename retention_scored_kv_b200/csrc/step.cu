@@ -843,7 +843,7 @@ __device__ __forceinline__ void attn_pass_hpw(const StepArgs &a, const Sm &sm, C
                                           const CUtensorMap *tmv) {
     using LY = StepLayout<M, D, G>;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t *full = sm.bars(), *empty = full + LY::NST, *qfull = empty + LY::NST, *qempty = qfull + QR;
+    uint64_t *full = sm.bars(), *empty = full + LY::NST;
     unsigned char *stage = sm.big() + LY::B_STAGE;
     unsigned char *poslb = sm.big() + LY::B_POSLB;
     float *qring = reinterpret_cast<float *>(sm.big() + LY::B_Q);
@@ -2470,7 +2470,6 @@ __device__ bool tail(const StepArgs &a, const Sm &sm, Ctx &cx, bool spec, bool l
     // candidates' keep bits were set by the resolve step) that warps take from
     // a queue in shared memory; heads too large for a warp are done
     // block-wide afterwards, one at a time.
-    const int nh = hc1 - hc0;
     int32_t *st_heavy = st_pop + NTH;
     int32_t *tasks = reinterpret_cast<int32_t *>(sm.big() + T_CL);  // [2 * NTH]
     if (tid == 0) {
