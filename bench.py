@@ -68,10 +68,10 @@ SPLIT_STEPS = 32  # event-timed steps for the evicting / non-evicting split
 
 # DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of one
 # launch of the fused step kernel on a steady long128k step: the 4-layer
-# capture (read 218.83 MB + write 5.03 MB) x8 to the full 32-layer launch
+# capture (read 218.89 MB + write 5.14 MB) x8 to the full 32-layer launch
 # (pages, hence traffic, grow with the layer count).  Reported only while the
 # kernel's sources hash to the captured version.
-STEP_TRAFFIC = {"sources_sha256": "029e3e155edfa685", "workload": "long128k", "bytes_per_launch": 8 * 224.378112e6}
+STEP_TRAFFIC = {"sources_sha256": "7f8ca828d20beef2", "workload": "long128k", "bytes_per_launch": 8 * 224.028416e6}
 
 
 # ------------------------------------------------------------------ ranks ---
