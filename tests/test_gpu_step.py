@@ -368,6 +368,90 @@ def test_fused_empty_and_ragged_heads(rkv):
         compare_state(dc, hc)
 
 
+def _edge_cache(rkv, seed):
+    """L=1, H=3 (position field 30 bits wide), heads of 40, 150 and 300
+    entries; the 300-entry head holds every position in [0, 300)."""
+    cfg = workloads.small_config(L=1, H=3, G=2, D=64, B=1, T0=300, kv_dtype="bf16")
+    dc = to_dev(workloads.ragged_cache(cfg, seed, [40, 150, 300], n_pages=64))
+    return cfg, dc
+
+
+def _set_pos(dc, c, k, pos):
+    dc.pos_pool[int(dc.block_table[c, k // 16]), k % 16] = pos
+
+
+@pytest.mark.parametrize("case", ["ages", "positions"])
+def test_fused_exact_path_key_edges(rkv, case):
+    # entries exactly at the edges of the scorable range are scored, on the
+    # first call (the exact selection): ages 1 and 2^24 - 1 with position 0,
+    # or positions up to 2^30 - 1, the widest that fits beside the head
+    # index when L*H = 3
+    cfg, dc = _edge_cache(rkv, 21)
+    if case == "ages":
+        t = (1 << 24) - 1            # the entry at position 0 has age 2^24 - 1
+        _set_pos(dc, 0, 0, t - 1)    # age 1
+    else:
+        dc.pos_pool += (1 << 30) - 300   # the 300-entry head now ends at 2^30 - 1
+        t = (1 << 30) + 5
+    hc = host_cache(dc)
+    cache = rkv_cache(rkv, dc)
+    sel, ws, outs = rkv.Selection.empty(cache), rkv.Workspace(cache), rkv.StepOutputs.empty(cache)
+    inp = workloads.step_inputs(cfg, 21, 0, "cuda")
+    tt = np.array([t], np.int32)
+    len_before = hc.len.copy()
+    rkv.decode_step(cache, torch.tensor(tt, device="cuda"), torch.tensor([200], dtype=torch.int64, device="cuda"),
+                    inp["q"], cfg.scale, inp["k_new"], inp["v_new"], inp["lb_new"], sel, outs.out, outs.lse,
+                    outs.dropped, ws)
+    sync()
+    c = ws.counters()
+    assert c["status"] == 0 and c["exact_steps"] == 1, c
+    ref = oracle.step(hc, tt, np.array([200]), inp["q"].cpu().numpy().reshape(cfg.C, cfg.G, cfg.D),
+                      workloads.rows_to_host(inp["k_new"]), workloads.rows_to_host(inp["v_new"]),
+                      inp["lb_new"].cpu().numpy(), evict=True, scale=cfg.scale)
+    assert np.array_equal(sel.kept.cpu().numpy(), ref["kept"])
+    assert np.array_equal(masked_keep(keep_flags(sel, dc.max_pages), len_before), ref["keep"])
+    assert_outputs_close(outs.out.cpu().numpy().reshape(cfg.C, cfg.G, cfg.D),
+                         outs.lse.cpu().numpy().reshape(cfg.C, cfg.G),
+                         outs.dropped.cpu().numpy().reshape(cfg.C, cfg.G), ref["out"], ref["lse"],
+                         ref["dropped"], ref["kept"] > 0)
+    compare_state(dc, hc)
+
+
+@pytest.mark.parametrize("kind", ["nan", "age0", "age2^24", "negative", "past_field"])
+def test_fused_exact_path_flags_unscorable_entry(rkv, kind):
+    # one entry the method cannot score (head 1, slot 5), every other entry
+    # valid: the first call's exact selection flags RKV_DEV_BAD_INPUT,
+    # finishes, and keeps nothing of that entry
+    cfg, dc = _edge_cache(rkv, 22)
+    t = cfg.T0 + 5
+    if kind == "nan":
+        dc.lb_pool[int(dc.block_table[1, 0]), 5] = float("nan")
+    elif kind == "age0":
+        _set_pos(dc, 1, 5, t)
+    elif kind == "age2^24":
+        dc.pos_pool += 1000
+        t = (1 << 24) + 999
+        _set_pos(dc, 1, 5, 999)
+    elif kind == "negative":
+        _set_pos(dc, 1, 5, -5)
+    else:
+        dc.pos_pool += (1 << 30) - 300
+        t = (1 << 30) + 5
+        _set_pos(dc, 1, 5, 1 << 30)      # age 5, but past the 30-bit position field
+    cache = rkv_cache(rkv, dc)
+    sel, ws, outs = rkv.Selection.empty(cache), rkv.Workspace(cache), rkv.StepOutputs.empty(cache)
+    inp = workloads.step_inputs(cfg, 22, 0, "cuda")
+    rkv.decode_step(cache, torch.tensor([t], dtype=torch.int32, device="cuda"),
+                    torch.tensor([200], dtype=torch.int64, device="cuda"), inp["q"], cfg.scale, inp["k_new"],
+                    inp["v_new"], inp["lb_new"], sel, outs.out, outs.lse, outs.dropped, ws)
+    sync()
+    assert ws.status() & rkv.DEV_BAD_INPUT
+    assert keep_flags(sel, dc.max_pages)[1, 5] == 0
+    rkv.workspace_init(ws)
+    sync()
+    assert ws.status() == 0
+
+
 def test_fused_graph_replay(rkv):
     # the fused step captured once in a CUDA graph and replayed on new inputs
     cfg = workloads.small_config(L=2, H=2, G=4, D=128, B=1, T0=1500, M=2000, kv_dtype="bf16", steps=6)
