@@ -72,6 +72,9 @@ SPLIT_STEPS = 32  # event-timed steps for the evicting / non-evicting split
 # (pages, hence traffic, grow with the layer count).  Reported only while the
 # kernel's sources hash to the captured version.
 STEP_TRAFFIC = {"sources_sha256": "7f8ca828d20beef2", "workload": "long128k", "bytes_per_launch": 8 * 224.028416e6}
+# The same for the separate path's attention kernel on a steady llama32k
+# step: the 16-layer capture (read 135.23 MB + write 3.43 MB) x2.
+ATTN_TRAFFIC = {"sources_sha256": "095f6c0e7ae6b397", "workload": "llama32k", "bytes_per_launch": 2 * 138.661632e6}
 
 
 # ------------------------------------------------------------------ ranks ---
@@ -417,12 +420,12 @@ def run_config(name: str, args, world: int, rank: int, local: int, *, e2e: bool)
     if fused:
         a_bytes, dom_s = s_bytes, kern_us["step"] * 1e-6
         kernel_desc = "step_kernel (selection + paged decode attention + dropped mass + compaction + append)"
-        traffic = step_traffic(cfg, args.traffic)
+        traffic = kernel_traffic(cfg, args.traffic, STEP_TRAFFIC, TRAFFIC_SOURCES)
     else:
         a_bytes = attn_bytes(cfg, n_pre_ev, kept_ev, pages_ev)
         dom_s = kern_us["attn"] * 1e-6
         kernel_desc = "attn_kernel (paged decode attention + dropped mass)"
-        traffic = None
+        traffic = kernel_traffic(cfg, args.traffic, ATTN_TRAFFIC, ATTN_TRAFFIC_SOURCES)
     achieved = a_bytes / dom_s / 1e9
     retained = elt(cfg) * 2 * cfg.D * kept_ev
     return {
@@ -793,24 +796,25 @@ def _graph_upload(graph, stream):
 
 TRAFFIC_SOURCES = ("retention_scored_kv_b200/csrc/step.cu", "retention_scored_kv_b200/csrc/attn_core.cuh",
                    "retention_scored_kv_b200/csrc/common.cuh")
+ATTN_TRAFFIC_SOURCES = ("retention_scored_kv_b200/csrc/attn.cu", "retention_scored_kv_b200/csrc/attn_core.cuh",
+                        "retention_scored_kv_b200/csrc/common.cuh")
 
 
-def sources_sha() -> str:
+def sources_sha(files=TRAFFIC_SOURCES) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in TRAFFIC_SOURCES:
+    for f in files:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def step_traffic(cfg: workloads.Config, override):
-    """ncu DRAM bytes per launch of the fused step kernel on this workload,
+def kernel_traffic(cfg: workloads.Config, override, rec: dict, files) -> float | None:
+    """ncu DRAM bytes per launch of the kernel `rec` records on this workload,
     or None if not measured for these sources and this workload."""
     if override is not None:
         return override
-    rec = STEP_TRAFFIC
-    if rec and cfg.name == rec["workload"] and sources_sha() == rec["sources_sha256"]:
+    if rec and cfg.name == rec["workload"] and sources_sha(files) == rec["sources_sha256"]:
         return rec["bytes_per_launch"]
     return None
 
