@@ -6,6 +6,8 @@
 #include <cstring>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -187,6 +189,17 @@ bool ws_layout(const rkv_cache_t &c, WsLayout *out) {
 
 using namespace rkv;
 
+// One NVTX range per call that enqueues work, named after the entry point
+// (host side only; a no-op unless a profiler is attached).
+namespace {
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
+}  // namespace
+
 extern "C" {
 
 RKV_API const char *rkv_version(void) { return "librkv 0.1.0 (sm_100a)"; }
@@ -201,6 +214,7 @@ RKV_API size_t rkv_workspace_size(const rkv_cache_t *cache) {
 }
 
 RKV_API int rkv_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    const NvtxRange nvtx_range("rkv_workspace_init");
     if (!ws || ws_bytes == 0) return fail(RKV_ERR_INVALID_ARG, "workspace is NULL or empty");
     cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace)");
@@ -210,6 +224,7 @@ RKV_API int rkv_workspace_init(void *ws, size_t ws_bytes, void *stream) {
 RKV_API int32_t *rkv_device_status(void *ws) { return ws ? reinterpret_cast<int32_t *>(ws) : nullptr; }
 
 RKV_API int rkv_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint32_t microseconds, void *stream) {
+    const NvtxRange nvtx_range("rkv_workspace_set_wait_limit");
     if (!ws || ws_bytes < 32) return fail(RKV_ERR_INVALID_ARG, "workspace is NULL or too small");
     if (microseconds > 0x7FFFFFFFu) return fail(RKV_ERR_INVALID_ARG, "wait limit above 2^31 - 1 microseconds");
     cudaError_t e = launch_set_word(reinterpret_cast<int32_t *>(ws) + 4, (int32_t)microseconds,
@@ -220,6 +235,7 @@ RKV_API int rkv_workspace_set_wait_limit(void *ws, size_t ws_bytes, uint32_t mic
 
 RKV_API int rkv_score_select(const rkv_cache_t *cache, const int32_t *t, const int64_t *m_global,
                              const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream) {
+    const NvtxRange nvtx_range("rkv_score_select");
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if ((rc = check_sel(sel))) return rc;
@@ -381,12 +397,14 @@ static int attn_common(const rkv_cache_t *cache, const float *q, float scale, co
 RKV_API int rkv_paged_decode_attn(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
                                   float *out, float *lse_kept, float *dropped, void *ws, size_t ws_bytes,
                                   void *stream) {
+    const NvtxRange nvtx_range("rkv_paged_decode_attn");
     if (!out) return fail(RKV_ERR_INVALID_ARG, "rkv_paged_decode_attn: out is NULL");
     return attn_common(cache, q, scale, sel, out, lse_kept, dropped, ws, ws_bytes, stream, "rkv_paged_decode_attn");
 }
 
 RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
                              float *dropped, void *ws, size_t ws_bytes, void *stream) {
+    const NvtxRange nvtx_range("rkv_dropped_mass");
     if (!dropped) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: dropped is NULL");
     if (!sel) return fail(RKV_ERR_INVALID_ARG, "rkv_dropped_mass: sel is NULL");
     return attn_common(cache, q, scale, sel, nullptr, nullptr, dropped, ws, ws_bytes, stream, "rkv_dropped_mass");
@@ -394,6 +412,7 @@ RKV_API int rkv_dropped_mass(const rkv_cache_t *cache, const float *q, float sca
 
 RKV_API int rkv_score_select_budget(const rkv_cache_t *cache, const int32_t *t, const rkv_budget_t *budget,
                                     const rkv_select_t *sel, void *ws, size_t ws_bytes, void *stream) {
+    const NvtxRange nvtx_range("rkv_score_select_budget");
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if ((rc = check_sel(sel))) return rc;
@@ -506,6 +525,7 @@ static int check_memory(const rkv_cache_t *cache, const rkv_memory_t *mem, const
 
 RKV_API int rkv_memory_update(const rkv_cache_t *cache, const rkv_select_t *sel, const rkv_memory_t *mem,
                               void *stream) {
+    const NvtxRange nvtx_range("rkv_memory_update");
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if ((rc = check_sel(sel))) return rc;
@@ -533,6 +553,7 @@ RKV_API int rkv_memory_update(const rkv_cache_t *cache, const rkv_select_t *sel,
 
 RKV_API int rkv_memory_read(const rkv_cache_t *cache, const float *q, const rkv_memory_t *mem, float *out,
                             void *stream) {
+    const NvtxRange nvtx_range("rkv_memory_read");
     int rc = check_cache(cache, false);
     if (rc) return rc;
     if (!q || !out) return fail(RKV_ERR_INVALID_ARG, "rkv_memory_read: q / out is NULL");
@@ -558,6 +579,7 @@ RKV_API int rkv_memory_read(const rkv_cache_t *cache, const float *q, const rkv_
 RKV_API int rkv_eviction_error(const rkv_cache_t *cache, const float *q, float scale, const rkv_select_t *sel,
                                const float *out_kept, const float *dropped, float *err, void *ws, size_t ws_bytes,
                                void *stream) {
+    const NvtxRange nvtx_range("rkv_eviction_error");
     if (!sel) return fail(RKV_ERR_INVALID_ARG, "rkv_eviction_error: sel is NULL");
     if (!out_kept || !dropped || !err || !q)
         return fail(RKV_ERR_INVALID_ARG, "rkv_eviction_error: q, out_kept, dropped and err must be non-NULL");
@@ -589,6 +611,7 @@ RKV_API int rkv_decode_step(const rkv_cache_t *cache, const int32_t *t, const in
                             float scale, const void *k_new, const void *v_new, const float *lb_new,
                             const rkv_select_t *sel, float *out, float *lse_kept, float *dropped, void *ws,
                             size_t ws_bytes, void *stream) {
+    const NvtxRange nvtx_range("rkv_decode_step");
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if (!t || !q || !k_new || !v_new || !lb_new || !out)
@@ -681,6 +704,7 @@ RKV_API int rkv_decode_step(const rkv_cache_t *cache, const int32_t *t, const in
 
 RKV_API int rkv_compact_pages(const rkv_cache_t *cache, const rkv_select_t *sel, void *ws, size_t ws_bytes,
                               void *stream) {
+    const NvtxRange nvtx_range("rkv_compact_pages");
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if ((rc = check_sel(sel))) return rc;
@@ -710,6 +734,7 @@ RKV_API int rkv_compact_pages(const rkv_cache_t *cache, const rkv_select_t *sel,
 
 RKV_API int rkv_append(const rkv_cache_t *cache, const int32_t *t, const void *k_new, const void *v_new,
                        const float *lb_new, void *ws, size_t ws_bytes, void *stream) {
+    const NvtxRange nvtx_range("rkv_append");
     int rc = check_cache(cache, true);
     if (rc) return rc;
     if (!t || !k_new || !v_new || !lb_new) return fail(RKV_ERR_INVALID_ARG, "rkv_append: an input is NULL");
