@@ -74,7 +74,7 @@ SPLIT_STEPS = 32  # event-timed steps for the evicting / non-evicting split
 STEP_TRAFFIC = {"sources_sha256": "7f8ca828d20beef2", "workload": "long128k", "bytes_per_launch": 8 * 224.028416e6}
 # The same for the separate path's attention kernel on a steady llama32k
 # step: the 16-layer capture (read 135.23 MB + write 3.43 MB) x2.
-ATTN_TRAFFIC = {"sources_sha256": "095f6c0e7ae6b397", "workload": "llama32k", "bytes_per_launch": 2 * 138.661632e6}
+ATTN_TRAFFIC = {"sources_sha256": "e28da1e460e372cf", "workload": "llama32k", "bytes_per_launch": 2 * 138.661632e6}
 
 
 # ------------------------------------------------------------------ ranks ---

@@ -42,11 +42,7 @@ using namespace core;
 template <class M, int D, int G, bool WITH_V>
 struct Layout {
     static constexpr int STAGE_BYTES = M::PAGE_BYTES * (WITH_V ? 2 : 1);
-#ifdef RKV_STAGE_BYTES_BUDGET
-    static constexpr int BUDGET = RKV_STAGE_BYTES_BUDGET;
-#else
-    static constexpr int BUDGET = 131072;
-#endif
+    static constexpr int BUDGET = 131072;                     // stage-ring bytes per CTA
     static constexpr int NSW0 = BUDGET / (NCW * STAGE_BYTES);
     static constexpr int NSW = NSW0 < 1 ? 1 : (NSW0 > 8 ? 8 : NSW0);   // stages per consumer warp
     static constexpr int NST = NCW * NSW;
