@@ -68,10 +68,10 @@ SPLIT_STEPS = 32  # event-timed steps for the evicting / non-evicting split
 
 # DRAM traffic (ncu dram__bytes_read.sum + dram__bytes_write.sum) of one
 # launch of the fused step kernel on a steady long128k step: the 4-layer
-# capture (read 218.89 MB + write 5.14 MB) x8 to the full 32-layer launch
+# capture (read 218.88 MB + write 8.74 MB) x8 to the full 32-layer launch
 # (pages, hence traffic, grow with the layer count).  Reported only while the
 # kernel's sources hash to the captured version.
-STEP_TRAFFIC = {"sources_sha256": "7f8ca828d20beef2", "workload": "long128k", "bytes_per_launch": 8 * 224.028416e6}
+STEP_TRAFFIC = {"sources_sha256": "84b76a0cbdb33dbf", "workload": "long128k", "bytes_per_launch": 8 * 227.614208e6}
 # The same for the separate path's attention kernel on a steady llama32k
 # step: the 16-layer capture (read 135.23 MB + write 3.43 MB) x2.
 ATTN_TRAFFIC = {"sources_sha256": "e28da1e460e372cf", "workload": "llama32k", "bytes_per_launch": 2 * 138.661632e6}

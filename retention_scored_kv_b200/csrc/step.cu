@@ -2607,8 +2607,9 @@ __device__ bool tail(const StepArgs &a, const Sm &sm, Ctx &cx, bool spec, bool l
         combine_head<M, D, G>(a, sm, cx, c, pfx, jf, jl, flag, spec && (flag & 1u), local);
     }
     // heavy compactions: this CTA's own heads, or (spread) its share of every
-    // head's parts
-    const int parts = spread ? min(64, max(1, (4 * nct + C - 1) / C)) : 1;
+    // head's parts (about two per CTA: each part costs a few microseconds of
+    // loads and scans before its copies, and fewer parts balance worse)
+    const int parts = spread ? min(64, max(1, (2 * nct + C - 1) / C)) : 1;
     const int njobs = spread ? (int)(((int64_t)C * parts - blockIdx.x + nct - 1) / nct) : hc1 - hc0;
     for (int j = 0; j < njobs; j++) {
         int c, part = 0, np, nn;
